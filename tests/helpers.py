@@ -1,0 +1,72 @@
+"""Test helpers: MXFP4-pack a synthetic layer with the oracle's quantizer and call the
+oracle on it. Packed bytes made here are what both the oracle and the CUDA library
+consume in parity tests, so no oracle input comes from the CUDA path."""
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+
+import oracle
+from mxfp4_block_scaled_moe_b200 import inputs
+
+
+@dataclasses.dataclass
+class Packed:
+    lay: inputs.Layer
+    x: np.ndarray          # (T, H) bf16 bits
+    router_w: np.ndarray   # (E, H) bf16 bits
+    router_b: np.ndarray | None
+    gu_blocks: np.ndarray  # (E, 2I, H/2)
+    gu_scales: np.ndarray  # (E, 2I, H/32)
+    gu_bias: np.ndarray    # (E, 2I) fp32
+    d_blocks: np.ndarray   # (E, H, I/2)
+    d_scales: np.ndarray   # (E, H, I/32)
+    d_bias: np.ndarray     # (E, H) fp32
+
+    @property
+    def weights(self):
+        return (self.gu_blocks, self.gu_scales, self.gu_bias, self.d_blocks, self.d_scales,
+                self.d_bias)
+
+    def oracle_forward(self, act_scale=None, dense=False, rows=None):
+        x = self.x if rows is None else self.x[rows]
+        return oracle.moe_forward(x, self.router_w, self.router_b, *self.weights, self.lay.k,
+                                  act_scale=act_scale, dense=dense)
+
+    def oracle_calibrate(self, x_bits):
+        return oracle.calibrate(x_bits, self.router_w, self.router_b, *self.weights, self.lay.k)
+
+
+def pack(lay: inputs.Layer) -> Packed:
+    E, H, I = lay.E, lay.H, lay.I
+    gu_b = np.empty((E, 2 * I, H // 2), np.uint8)
+    gu_s = np.empty((E, 2 * I, H // 32), np.uint8)
+    d_b = np.empty((E, H, I // 2), np.uint8)
+    d_s = np.empty((E, H, I // 32), np.uint8)
+    for e in range(E):
+        gu_b[e], gu_s[e] = oracle.quantize(lay.gate_up(e).cpu().numpy())
+        d_b[e], d_s[e] = oracle.quantize(lay.down(e).cpu().numpy())
+    rb = None if lay.router_b is None else inputs.bits(lay.router_b)
+    return Packed(lay, inputs.bits(lay.x), inputs.bits(lay.router_w), rb, gu_b, gu_s,
+                  lay.gu_bias.cpu().numpy(), d_b, d_s, lay.d_bias.cpu().numpy())
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    return (b.astype(np.uint32) << 16).view(np.float32)
+
+
+def output_tolerance_ok(out_bits: np.ndarray, ref_acc: np.ndarray, rel: float = 2e-3):
+    """The layer-output bar: a bf16 output may differ from the oracle's fp32 accumulator
+    by rel * max|ref| (fp32 arithmetic, accumulation order) plus half a bf16 ulp of the
+    reference element (the single bf16 rounding of the output).
+
+    Returns (ok, max|delta|/max|ref|, worst excess)."""
+    got = bf16_bits_to_f32(out_bits).astype(np.float64)
+    ref = ref_acc.astype(np.float64)
+    scale = float(np.max(np.abs(ref))) if ref.size else 0.0
+    ulp = np.spacing(np.abs(ref).astype(np.float32)).astype(np.float64) * 2.0 ** 16
+    bound = rel * scale + 0.5 * ulp
+    err = np.abs(got - ref)
+    excess = float(np.max(err - bound)) if ref.size else 0.0
+    return bool(np.all(err <= bound)), float(np.max(err) / scale) if scale else 0.0, excess
