@@ -1,0 +1,421 @@
+"""Benchmark of the MXFP4 MoE expert layer on B200 (one JSON line on rank 0).
+
+A step is one moe_mxfp4_forward over one batch of synthetic tokens: router + top-k,
+permute, expert gate_up + SwiGLU, down, weighted combine. Default workload: the
+120B-shaped prefill layer with FP8 activations (E=128, top-4, H=I=2880, T=4096, static
+per-tensor scales from a 256-token calibration batch). Other workloads (--workload):
+decode1/decode8/decode64 (20B shape, E=32, bf16 activations), zipf (T=16384, skewed
+routing).
+
+Metric: MoE-layer tokens/s (whole job = sum over ranks). Inputs are resident in HBM
+when the timed region starts; L2 is flushed (a 512 MiB write) before every timed step,
+outside the step's own events. `e2e` is the same metric through the C ABI with the
+tokens in pinned host memory: host->device copy of x, the forward, device->host copy of
+the output, all inside the timed region.
+
+Multi-GPU (torchrun): every rank runs its own replica of the workload (the layer has no
+cross-GPU exchange on this path), times are the max over ranks, value = total tokens of
+all ranks / that time.
+
+--impl reference: the CPU oracle on a bounded sample of the same workload, timed on the
+host cores (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mxfp4_block_scaled_moe_b200 import inputs  # noqa: E402
+
+METRIC = "MoE-layer tokens/s"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+WORKLOADS = {
+    # name: (constructor, fp8 activations)
+    "prefill": (lambda dev: inputs.prefill_layer(T=4096, E=128, device=dev), True),
+    "zipf": (lambda dev: inputs.zipf_layer(T=16384, E=128, device=dev), True),
+    "decode1": (lambda dev: inputs.decode_layer(T=1, E=32, device=dev), False),
+    "decode8": (lambda dev: inputs.decode_layer(T=8, E=32, device=dev), False),
+    "decode64": (lambda dev: inputs.decode_layer(T=64, E=32, device=dev), False),
+}
+
+PER_EXPERT_PACKED = lambda H, I: 2 * I * H // 2 + 2 * I * H // 32 + H * I // 2 + H * I // 32
+
+
+def peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            return json.load(f), "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- distributed -----
+
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------- setup ----
+
+def build_layer(name, device):
+    from mxfp4_block_scaled_moe_b200 import binding as B
+    make, fp8 = WORKLOADS[name]
+    lay = make(device)
+    E, H, I = lay.E, lay.H, lay.I
+    gu_b = torch.empty(E, 2 * I, H // 2, dtype=torch.uint8, device=device)
+    gu_s = torch.empty(E, 2 * I, H // 32, dtype=torch.uint8, device=device)
+    d_b = torch.empty(E, H, I // 2, dtype=torch.uint8, device=device)
+    d_s = torch.empty(E, H, I // 32, dtype=torch.uint8, device=device)
+    for e in range(E):   # weights: fp32 draws quantized by the library's own kernel
+        B.mxfp4_quantize(lay.gate_up(e), gu_b[e], gu_s[e])
+        B.mxfp4_quantize(lay.down(e), d_b[e], d_s[e])
+    d = dict(x=lay.x, router_w=lay.router_w, router_b=lay.router_b, gu_blocks=gu_b,
+             gu_scales=gu_s, gu_bias=lay.gu_bias, d_blocks=d_b, d_scales=d_s, d_bias=lay.d_bias)
+    act = None
+    if fp8:
+        xc = inputs.calibration_x(H=H, device=device)
+        act = B.moe_mxfp4_calibrate(xc, lay.router_w, lay.router_b, gu_b, gu_s, lay.gu_bias,
+                                    d_b, d_s, lay.d_bias, lay.k).cpu().tolist()
+    torch.cuda.synchronize()
+    return lay, d, act
+
+
+def forward(B, d, k, act, out, stream=None):
+    return B.moe_mxfp4_forward(d["x"], d["router_w"], d["router_b"], d["gu_blocks"],
+                               d["gu_scales"], d["gu_bias"], d["d_blocks"], d["d_scales"],
+                               d["d_bias"], k, act_scale=act, out=out, stream=stream)
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed loop runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [c.strip() for c in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def algorithmic_work(lay, idx):
+    """Bytes and FLOPs the step must move/do: packed weights of the distinct routed experts
+    (+ biases), router weights, x in, out; FLOPs of the routed pairs and the router."""
+    E, k, T, H, I = lay.E, lay.k, lay.T, lay.H, lay.I
+    distinct = len(np.unique(idx.reshape(-1)))
+    w_bytes = distinct * (PER_EXPERT_PACKED(H, I) + (2 * I + H) * 4)
+    bytes_ = w_bytes + E * H * 2 + 2 * T * H * 2
+    flops = T * k * (2 * H * 2 * I + 2 * I * H) + 2 * T * H * E
+    gu_bytes = distinct * (2 * I * H // 2 + 2 * I * H // 32)
+    gu_flops = T * k * 2 * H * 2 * I
+    return dict(bytes=bytes_, flops=flops, distinct=distinct, gu_bytes=gu_bytes, gu_flops=gu_flops)
+
+
+# ------------------------------------------------------------- CPU baseline -----
+
+def oracle_tokens_per_s(lay, d, act, budget_s, host_weights=None):
+    """Time the oracle on a bounded prefix of the workload's tokens on the host cores."""
+    import oracle
+    hw = host_weights or {n: d[n].cpu().numpy() for n in
+                          ("gu_blocks", "gu_scales", "gu_bias", "d_blocks", "d_scales", "d_bias")}
+    xb = inputs.bits(d["x"])
+    rw = inputs.bits(d["router_w"])
+    rb = None if d["router_b"] is None else inputs.bits(d["router_b"])
+    w = (hw["gu_blocks"], hw["gu_scales"], hw["gu_bias"], hw["d_blocks"], hw["d_scales"], hw["d_bias"])
+    t0 = time.perf_counter()
+    oracle.moe_forward(xb[:1], rw, rb, *w, lay.k, act_scale=act)
+    t1 = time.perf_counter() - t0
+    n = int(max(1, min(lay.T, budget_s / max(t1, 1e-6))))
+    t0 = time.perf_counter()
+    oracle.moe_forward(xb[:n], rw, rb, *w, lay.k, act_scale=act)
+    dt = time.perf_counter() - t0
+    return n / dt, n, dt, hw
+
+
+# ------------------------------------------------------------------------ main ----
+
+def run_ours(args, world, rank):
+    from mxfp4_block_scaled_moe_b200 import binding as B
+    pk, pk_kind = peaks()
+    lay, d, act = build_layer(args.workload, "cuda")
+    k, T, H = lay.k, lay.T, lay.H
+    out = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    idx, _ = B.moe_route_topk(d["x"], d["router_w"], d["router_b"], k)
+    work = algorithmic_work(lay, idx.cpu().numpy())
+
+    for _ in range(args.warmup):
+        forward(B, d, k, act, out)
+    B.mxmoe_check()
+    launches_per_step = B.mxmoe_last_launch_count()
+
+    # ---- device-resident timed loop (per-step events, L2 flushed between steps)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    B.mxmoe_profile_enable(True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            ev[i][0].record(stream)
+            forward(B, d, k, act, out)
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    stages = B.mxmoe_profile_read()
+    B.mxmoe_profile_enable(False)
+    B.mxmoe_check()
+    total_ms = sum(a.elapsed_time(b) for a, b in ev)
+    total_ms = max_over_ranks(total_ms, world)
+    ms_per_step = total_ms / args.steps
+    value = T * world * args.steps / (total_ms / 1e3)
+
+    # ---- end to end through the C ABI with host buffers
+    x_host = d["x"].cpu().pin_memory()
+    out_host = torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(d["x"])
+    d_e2e = dict(d, x=x_dev)
+    for _ in range(2):
+        x_dev.copy_(x_host, non_blocking=True)
+        forward(B, d_e2e, k, act, out)
+        out_host.copy_(out, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        forward(B, d_e2e, k, act, out)
+        out_host.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e_value = T * world * args.steps / (e2e_ms / 1e3)
+
+    # ---- roofline of the dominant kernel
+    dom = max((s for s in stages if s not in ("router", "topk", "permute", "act_quant", "combine")),
+              key=lambda s: stages[s][0], default=None)
+    if dom is None:
+        dom = max(stages, key=lambda s: stages[s][0])
+    dom_ms = stages[dom][0] / max(stages[dom][1], 1)
+    fp8 = act is not None
+    if fp8 and lay.T >= 1024:
+        bound, unit = "tensor", "TFLOP/s"
+        # FP8 dense peak = measured bf16 peak x the nominal fp8/bf16 ratio (4.5 / 2.25 = 2)
+        peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"]) * 2.0
+        flops = work["gu_flops"] if dom == "gate_up" else work["flops"] - work["gu_flops"]
+        achieved = flops / (dom_ms / 1e3) / 1e12
+        peak_note = f"{pk_kind} bf16 sustained x 2 (nominal fp8/bf16 ratio)"
+    else:
+        bound, unit = "hbm", "GB/s"
+        peak = pk["hbm_gbs"]
+        b = work["gu_bytes"] if dom == "gate_up" else work["bytes"] - work["gu_bytes"]
+        achieved = b / (dom_ms / 1e3) / 1e9
+        peak_note = f"{pk_kind} hbm copy"
+    roofline = {"bound": bound, "kernel": dom, "achieved": round(achieved, 2), "peak": peak,
+                "unit": unit, "frac": round(achieved / peak, 4), "traffic": None,
+                "peak_source": peak_note, "kernel_ms": round(dom_ms, 5)}
+
+    res = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3 x e2m1 -> f32" if fp8 else "bf16 x e2m1 -> f32",
+        "data": "synthetic (seeded; weights N(0,0.02) quantized to MXFP4 on the GPU)",
+        "config": {"workload": f"{args.workload}: {lay.name}", "E": lay.E, "k": k, "T": T,
+                   "H": H, "I": lay.I, "activations": "fp8_e4m3 static" if fp8 else "bf16",
+                   "l2": "flushed (512 MiB write) before every timed step",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": roofline,
+        "stages_ms_per_step": {s: round(v[0] / max(v[1], 1), 5) for s, v in stages.items()},
+        "algorithmic": {"bytes_per_step": work["bytes"], "flops_per_step": work["flops"],
+                        "distinct_experts": work["distinct"]},
+        "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2},
+        "gpu_launches": launches_per_step * args.steps,
+    }
+    res["clocks"] = clk.summary()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, n, dt, _ = oracle_tokens_per_s(lay, d, act, args.cpu_budget)
+        import oracle
+        res["cpu_baseline"] = {"value": round(v, 4), "unit": "tokens/s",
+                               "cores": oracle.num_threads(), "kind": "oracle",
+                               "sample": f"first {n} of {T} tokens of the same workload, {dt:.1f} s"}
+    return res
+
+
+def run_reference(args, world, rank):
+    """The oracle as it stands, on the host cores, over bounded samples of the workload."""
+    if rank != 0:
+        return None
+    import oracle
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    make, fp8 = WORKLOADS[args.workload]
+    lay = make(dev)
+    # pack with the oracle's own quantizer only the experts the sampled tokens route to
+    xb, rw = inputs.bits(lay.x), inputs.bits(lay.router_w)
+    rb = None if lay.router_b is None else inputs.bits(lay.router_b)
+    E, H, I = lay.E, lay.H, lay.I
+    hw = dict(gu_blocks=np.zeros((E, 2 * I, H // 2), np.uint8),
+              gu_scales=np.full((E, 2 * I, H // 32), 127, np.uint8),
+              gu_bias=lay.gu_bias.cpu().numpy(), d_blocks=np.zeros((E, H, I // 2), np.uint8),
+              d_scales=np.full((E, H, I // 32), 127, np.uint8), d_bias=lay.d_bias.cpu().numpy())
+    packed = set()
+
+    def ensure(x_bits):
+        idx, _ = oracle.topk_softmax(oracle.router_logits(x_bits, rw, rb), lay.k)
+        for e in np.unique(idx):
+            if e not in packed:
+                hw["gu_blocks"][e], hw["gu_scales"][e] = oracle.quantize(lay.gate_up(int(e)).cpu().numpy())
+                hw["d_blocks"][e], hw["d_scales"][e] = oracle.quantize(lay.down(int(e)).cpu().numpy())
+                packed.add(e)
+
+    act = None
+    if fp8:
+        xc = inputs.bits(inputs.calibration_x(H=H, device=dev))
+        ensure(xc)
+        act = oracle.calibrate(xc, rw, rb, hw["gu_blocks"], hw["gu_scales"], hw["gu_bias"],
+                               hw["d_blocks"], hw["d_scales"], hw["d_bias"], lay.k)
+    w = (hw["gu_blocks"], hw["gu_scales"], hw["gu_bias"], hw["d_blocks"], hw["d_scales"], hw["d_bias"])
+    ensure(xb[:1])
+    t0 = time.perf_counter()
+    oracle.moe_forward(xb[:1], rw, rb, *w, lay.k, act_scale=act)
+    t1 = time.perf_counter() - t0
+    n = int(max(1, min(lay.T, args.ref_step_s / max(t1, 1e-6))))
+    steps_rows = [np.arange(i * n, (i + 1) * n) % lay.T for i in range(args.warmup + args.steps)]
+    for r in steps_rows:
+        ensure(xb[r])
+    for r in steps_rows[:args.warmup]:
+        oracle.moe_forward(xb[r], rw, rb, *w, lay.k, act_scale=act)
+    t0 = time.perf_counter()
+    for r in steps_rows[args.warmup:]:
+        oracle.moe_forward(xb[r], rw, rb, *w, lay.k, act_scale=act)
+    dt = time.perf_counter() - t0
+    value = n * args.steps / dt
+    sample = f"{n} tokens per step of the {lay.name} workload ({lay.T} tokens)"
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64 accumulate (CPU oracle)",
+        "data": "synthetic (seeded)",
+        "config": {"workload": f"{args.workload}: {lay.name}", "E": E, "k": lay.k, "T": lay.T,
+                   "H": H, "I": I, "activations": "fp8_e4m3 static" if fp8 else "bf16"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="prefill")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
+    ap.add_argument("--ref-step-s", type=float, default=4.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        res = run_reference(args, world, rank)
+    else:
+        world, rank = dist_init()
+        try:
+            res = run_ours(args, world, rank)
+        finally:
+            if world > 1:
+                import torch.distributed as dist
+                dist.destroy_process_group()
+    if rank == 0 and res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,179 @@
+/*
+ * mxfp4_moe.h -- C ABI of libmxfp4moe.so: the routed Mixture-of-Experts expert layer
+ * with OCP MXFP4 expert weights, for NVIDIA B200 (sm_100a).
+ *
+ * What the operations compute (web pages, cited by title and section):
+ *  - MXFP4: "quantization_mxfp4" (KerasFormers), intro and "Primitives": e2m1 values
+ *    packed two per byte, one e8m0 scale per 32 values along the contracting dim;
+ *    dequantize = codebook[nibble] * 2^(scale - 127); quantize picks the block exponent
+ *    floor(log2(amax)) - 2 and rounds each value to the nearest FP4 grid point.
+ *  - The expert layer: same page, "As GPT-OSS's native format": gate_up_proj (E, 2I, H)
+ *    and down_proj (E, H, I) as blocks + scales, biases in full precision, only the
+ *    top-k routed experts are evaluated on decode.
+ *  - W-MXFP4 / A-FP8: "amd/gpt-oss-20b-MoE-Quant-W-MXFP4-A-FP8-KV-FP8", "Quantization
+ *    schemes": MoE MLP activations in FP8 with a symmetric per-tensor scale, router not
+ *    quantized; "gpt-oss-120b-mxfp4-fp8attn-v2", "Model Details": E4M3 static scales.
+ *
+ * Conventions shared by every entry point
+ *  - Pointers named as device memory must be device (cudaMalloc'd) memory of the current
+ *    device, 16-byte aligned, caller-owned. The library never frees caller memory.
+ *  - bf16 tensors are passed as arrays of uint16_t holding bf16 bit patterns.
+ *  - All tensors are dense row-major with the contracting dimension last.
+ *  - Packed MXFP4: a tensor of logical shape (R, K) is `blocks` (R, K/2) uint8, where
+ *    element 2j is the low nibble of byte j and 2j+1 the high nibble, plus `scales`
+ *    (R, K/32) uint8 e8m0 (value 2^(s-127)). In the expert layer this is
+ *    gu_blocks (E, 2I, H/2) [= (E, 2I, H/32, 16)], gu_scales (E, 2I, H/32),
+ *    d_blocks (E, H, I/2), d_scales (E, H, I/32). gate_up rows [0, I) are the gate
+ *    projection and rows [I, 2I) the up projection.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream). Every
+ *    call is asynchronous on it unless stated; the library never synchronizes the
+ *    device inside a call.
+ *  - Return value: MXMOE_OK (0) or a negative MXMOE_E* code. On error nothing is
+ *    launched and mxmoe_last_error() (thread-local) describes the cause.
+ *  - T == 0 (or rows == 0) is a no-op returning MXMOE_OK.
+ *  - Non-finite inputs give unspecified (but non-faulting) results.
+ *  - The library keeps one grow-only workspace per device (device memory it allocates
+ *    with cudaMalloc on first use, released by mxmoe_release()). A call that must grow
+ *    it allocates, so the first call at a new maximum size must not be inside a CUDA
+ *    graph capture. Calls that share a device must not overlap on the GPU (the
+ *    workspace is shared): issue them on one stream, or order the streams.
+ */
+#ifndef MXFP4_MOE_H
+#define MXFP4_MOE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MXMOE_OK 0
+#define MXMOE_EINVAL (-1)        /* null pointer, negative size, misaligned pointer */
+#define MXMOE_EALIGN (-2)        /* contracting dim (K, H or I) not a multiple of 32 */
+#define MXMOE_EUNSUPPORTED (-3)  /* k > E, k > 8, E > 256, out_dtype unknown, ... */
+#define MXMOE_ECUDA (-4)         /* a CUDA runtime/driver call or a launch failed */
+#define MXMOE_ETIMEOUT (-5)      /* a bounded device wait gave up (reported by mxmoe_check) */
+#define MXMOE_ENOMEM (-6)        /* workspace allocation failed */
+#define MXMOE_EDEVICE (-7)       /* a kernel found bad data, e.g. an expert id out of range */
+
+#define MXMOE_OUT_F32 0
+#define MXMOE_OUT_BF16 1
+
+/* mxfp4_quantize -- "quantization_mxfp4", Primitives (quantize_to_mxfp4).
+ * w: device fp32 (rows, K). Writes blocks: device (rows, K/2) uint8 and scales: device
+ * (rows, K/32) uint8. Per 32-value block: e = clamp(floor(log2(amax)) - 2, -127, 127),
+ * scale byte e + 127 (an all-zero block gets byte 0), each value rounded to the nearest
+ * of +-{0, 0.5, 1, 1.5, 2, 3, 4, 6} * 2^e with ties to the even code, magnitudes past 6
+ * saturating; the sign bit is copied from the input (so -0.0 packs as nibble 8).
+ * Errors: MXMOE_EALIGN if K % 32 != 0 ("As a quantize_model scheme": a clear error);
+ * MXMOE_EINVAL for null pointers or negative sizes. */
+int mxfp4_quantize(const float* w, int64_t rows, int64_t K, uint8_t* blocks, uint8_t* scales,
+                   void* stream);
+
+/* mxfp4_dequantize -- "quantization_mxfp4", Primitives (dequantize_mxfp4).
+ * out[r, k] = codebook[nibble] * 2^(scale - 127), written as fp32 (out_dtype
+ * MXMOE_OUT_F32) or bf16 bits (MXMOE_OUT_BF16) into device memory out (rows, K).
+ * Every finite result is exact in both types (subnormals included); results at or
+ * beyond 2^128 are +-inf (scale bytes 253..255). Errors as mxfp4_quantize, plus
+ * MXMOE_EUNSUPPORTED for an unknown out_dtype. */
+int mxfp4_dequantize(const uint8_t* blocks, const uint8_t* scales, int64_t rows, int64_t K,
+                     void* out, int out_dtype, void* stream);
+
+/* moe_route_topk -- router + top-k softmax (GPT-OSS top-k routing; router kept in bf16:
+ * "gpt-oss-120b-mxfp4-fp8attn-v2", config.json modules_to_not_convert).
+ * x: device bf16 (T, H); router_w: device bf16 (E, H); router_b: device bf16 (E) or NULL.
+ * logits[t, e] = sum_h x*Wr + br in fp32 arithmetic; logits_out: device fp32 (T, E) or
+ * NULL. topk_idx: device int32 (T, k), the k largest logits in descending order, ties to
+ * the lower expert id; topk_w: device fp32 (T, k) = softmax over those k logits.
+ * Limits: 1 <= k <= 8, k <= E <= 256, H % 32 == 0. */
+int moe_route_topk(const uint16_t* x, const uint16_t* router_w, const uint16_t* router_b, int T,
+                   int H, int E, int k, float* logits_out, int32_t* topk_idx, float* topk_w,
+                   void* stream);
+
+/* moe_topk_from_logits -- the top-k + softmax half of moe_route_topk on given fp32
+ * logits (device, (T, E)); same outputs and limits. Lets the selection be checked
+ * bit-exactly on identical logits. */
+int moe_topk_from_logits(const float* logits, int T, int E, int k, int32_t* topk_idx,
+                         float* topk_w, void* stream);
+
+/* moe_permute -- group the T*k (token, slot) pairs by expert (the routed dispatch of
+ * "quantization_mxfp4", As GPT-OSS's native format). topk_idx: device int32 (T, k).
+ * offsets: device int32 (E+1), offsets[e] = first position of expert e; perm_token,
+ * perm_slot: device int32 (T*k): position p holds the pair (perm_token[p], perm_slot[p]).
+ * Within an expert, pairs keep ascending token order (a stable counting sort, the same
+ * result on every run). An expert id outside [0, E) sets MXMOE_EDEVICE in the device
+ * error word (see mxmoe_check) and that pair is dropped. */
+int moe_permute(const int32_t* topk_idx, int T, int E, int k, int32_t* offsets,
+                int32_t* perm_token, int32_t* perm_slot, void* stream);
+
+/* moe_fp8_quantize -- the A-FP8 activation cast ("amd/gpt-oss-20b-MoE-Quant-W-MXFP4-A-
+ * FP8-KV-FP8", Quantization schemes): q[i] = e4m3(fp32(x[i] / s)), IEEE fp32 division,
+ * round-to-nearest-even, saturating to +-448 (E4M3 "fn" has no infinity; NaN stays NaN).
+ * x: device bf16 (n); q: device uint8 (n); s: the static per-tensor scale (> 0). */
+int moe_fp8_quantize(const uint16_t* x, int64_t n, float s, uint8_t* q, void* stream);
+
+/* moe_mxfp4_forward -- the MoE expert layer ("quantization_mxfp4", As GPT-OSS's native
+ * format; A-FP8 option per "amd/gpt-oss-20b-MoE-Quant-W-MXFP4-A-FP8-KV-FP8").
+ * For every token t: route (as moe_route_topk), then for each selected expert e with gate
+ * w: g = s0 * (xin . Wgu[e]^T) + gu_bias[e];  a = silu(g[:I]) * g[I:];
+ * y = s1 * (ain . Wd[e]^T) + d_bias[e];  out[t] = bf16(sum over the k experts of w * y),
+ * accumulated in fp32.
+ *  - act_scale == NULL: bf16 activations, xin = x, ain = bf16(a), s0 = s1 = 1.
+ *  - act_scale != NULL: HOST pointer to two floats {s0, s1} (static per-tensor scales
+ *    read during the call); xin = e4m3(x / s0), ain = e4m3(a / s1).
+ * x: device bf16 (T, H); router_w bf16 (E, H); router_b bf16 (E) or NULL; gu_bias fp32
+ * (E, 2I); d_bias fp32 (E, H); packed weights as described above; out: device bf16 (T, H).
+ * Limits: H, I multiples of 32 (MXMOE_EALIGN), 1 <= k <= 8, k <= E <= 256, T < 2^24.
+ * The weights are read in place (no copy, no re-layout). Uses the library workspace. */
+int moe_mxfp4_forward(const uint16_t* x, const uint16_t* router_w, const uint16_t* router_b,
+                      const uint8_t* gu_blocks, const uint8_t* gu_scales, const float* gu_bias,
+                      const uint8_t* d_blocks, const uint8_t* d_scales, const float* d_bias,
+                      int E, int k, int T, int H, int I, const float* act_scale, uint16_t* out,
+                      void* stream);
+
+/* moe_mxfp4_calibrate -- static per-tensor FP8 scales from a calibration batch with a
+ * min-max observer ("gpt-oss-120b-mxfp4-fp8attn-v2", Quantization Recipe):
+ * act_scale_out[0] = amax|x| / 448; act_scale_out[1] = amax over the routed
+ * (token, expert) pairs of the bf16-path gated activation a (fp32, before rounding) / 448.
+ * Same arguments as moe_mxfp4_forward without act_scale/out; act_scale_out: device fp32 (2). */
+int moe_mxfp4_calibrate(const uint16_t* x, const uint16_t* router_w, const uint16_t* router_b,
+                        const uint8_t* gu_blocks, const uint8_t* gu_scales, const float* gu_bias,
+                        const uint8_t* d_blocks, const uint8_t* d_scales, const float* d_bias,
+                        int E, int k, int T, int H, int I, float* act_scale_out, void* stream);
+
+/* mxmoe_check -- synchronize `stream`, then read and clear the device error word.
+ * Returns MXMOE_OK, MXMOE_EDEVICE (bad data seen by a kernel), MXMOE_ETIMEOUT (a bounded
+ * device wait gave up) or MXMOE_ECUDA (the stream reported an error). */
+int mxmoe_check(void* stream);
+
+/* mxmoe_last_error -- message for the last failing call on this host thread ("" if none).
+ * The string stays valid until the next library call on the same thread. */
+const char* mxmoe_last_error(void);
+
+/* mxmoe_last_launch_count -- number of kernels the last successful moe_mxfp4_forward
+ * on this host thread launched. */
+int mxmoe_last_launch_count(void);
+
+/* mxmoe_profile_enable -- on != 0: from now on every moe_mxfp4_forward on this host
+ * thread records a CUDA event on its stream before its first kernel and after each stage
+ * (router, topk, permute, act_quant, gate_up, down, combine, ...); on == 0 stops. Either
+ * call discards marks not yet read. Timing only: the results are unchanged. Returns
+ * MXMOE_OK. Recording is not allowed while the stream is being captured into a graph. */
+int mxmoe_profile_enable(int on);
+
+/* mxmoe_profile_read -- wait for the recorded events and report, per stage name, the
+ * summed GPU time in milliseconds and the number of calls since profiling was enabled or
+ * last read (then forget them). names: max_entries slots of 32 chars (NUL-terminated);
+ * total_ms, calls: max_entries entries. Returns the number of distinct stages (which may
+ * exceed max_entries; only the first max_entries are written) or a negative error code. */
+int mxmoe_profile_read(char* names, float* total_ms, int* calls, int max_entries);
+
+/* mxmoe_release -- free the workspace of the current device (synchronizes the device).
+ * Returns MXMOE_OK or MXMOE_ECUDA. */
+int mxmoe_release(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MXFP4_MOE_H */

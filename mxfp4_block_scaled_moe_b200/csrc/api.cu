@@ -1,0 +1,502 @@
+// C ABI of libmxfp4moe: argument checks, the per-device workspace, and the launch
+// sequence of the MoE expert layer. Every step of the computation runs in the library's
+// own kernels; this file only validates, sizes buffers and launches.
+#include <mutex>
+#include <string>
+#include <vector>
+#include <cstdio>
+#include <cstdarg>
+#include <cstring>
+
+#include "common.cuh"
+#include "launchers.h"
+
+namespace {
+
+thread_local std::string t_last_error;
+thread_local int t_last_launches = 0;
+
+// ------------------------------------------------------- optional stage timing -----
+// When enabled, run_layer() records a CUDA event on the caller's stream before the first
+// launch and after every stage, so a benchmark can time each kernel inside its own timed
+// region without a profiler. Events come from a per-thread pool reused after each read.
+struct StageMark {
+  const char* name;
+  cudaEvent_t start, stop;
+};
+thread_local bool t_profile = false;
+thread_local std::vector<cudaEvent_t> t_event_pool;
+thread_local size_t t_event_next = 0;
+thread_local std::vector<StageMark> t_marks;
+
+cudaEvent_t next_event() {
+  if (t_event_next == t_event_pool.size()) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    t_event_pool.push_back(e);
+  }
+  return t_event_pool[t_event_next++];
+}
+
+struct StageTimer {
+  cudaStream_t st;
+  cudaEvent_t last = nullptr;
+  explicit StageTimer(cudaStream_t s) : st(s) {
+    if (t_profile && (last = next_event())) cudaEventRecord(last, st);
+  }
+  void mark(const char* name) {
+    if (!t_profile || !last) return;
+    cudaEvent_t e = next_event();
+    if (!e) return;
+    cudaEventRecord(e, st);
+    t_marks.push_back({name, last, e});
+    last = e;
+  }
+};
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(MXMOE_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ------------------------------------------------------------------ workspace ------
+struct Workspace {
+  char* base = nullptr;
+  size_t cap = 0;
+  int* err = nullptr;  // device error word
+  int sms = 0;
+  int smem_K = 0;      // largest K the expert kernels were configured for
+};
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+Workspace g_ws[kMaxDevices];
+
+int current_device_ws(Workspace** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(MXMOE_EUNSUPPORTED, "device %d beyond %d", dev, kMaxDevices);
+  std::lock_guard<std::mutex> lk(g_mu);
+  Workspace& w = g_ws[dev];
+  if (w.err == nullptr) {
+    if ((e = cudaMalloc(&w.err, 256)) != cudaSuccess) return fail(MXMOE_ENOMEM, "error word: %s", cudaGetErrorString(e));
+    if ((e = cudaMemset(w.err, 0, 256)) != cudaSuccess) return cuda_fail(e, "cudaMemset");
+    if ((e = cudaDeviceGetAttribute(&w.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute");
+  }
+  *out = &w;
+  return MXMOE_OK;
+}
+
+int ensure_capacity(Workspace* w, size_t bytes) {
+  if (bytes <= w->cap) return MXMOE_OK;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (bytes <= w->cap) return MXMOE_OK;
+  cudaError_t e;
+  if (w->base) {
+    if ((e = cudaDeviceSynchronize()) != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+    cudaFree(w->base);
+    w->base = nullptr;
+    w->cap = 0;
+  }
+  size_t want = bytes + bytes / 8 + (1u << 20);
+  if ((e = cudaMalloc(&w->base, want)) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(MXMOE_ENOMEM, "workspace of %zu bytes: %s", want, cudaGetErrorString(e));
+  }
+  w->cap = want;
+  return MXMOE_OK;
+}
+
+// Bump layout over the workspace; every slice is 256-byte aligned.
+struct Carve {
+  size_t off = 0;
+  template <class T>
+  size_t take(int64_t count) {
+    size_t o = off;
+    off += (static_cast<size_t>(count) * sizeof(T) + 255) & ~static_cast<size_t>(255);
+    return o;
+  }
+};
+
+struct LayerBuffers {
+  float* logits;
+  int32_t* topk_idx;
+  float* topk_w;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* active;
+  int32_t* n_active;
+  int32_t* perm_token;
+  int32_t* perm_slot;
+  int32_t* inv;
+  uint16_t* xq;        // fp8 path: bf16 values of e4m3(x / s0), (T, H)
+  uint16_t* act_mid;   // (P, I) bf16 bits of the down-projection input
+  float* y;            // (P, H) fp32 expert outputs
+  unsigned* amax;      // 2 x fp32 bits (calibration)
+};
+
+size_t layout(int T, int E, int k, int H, int I, bool fp8, LayerBuffers* b, char* base) {
+  const int64_t P = static_cast<int64_t>(T) * k;
+  Carve c;
+  size_t o_logits = c.take<float>(static_cast<int64_t>(T) * E);
+  size_t o_idx = c.take<int32_t>(P), o_w = c.take<float>(P);
+  size_t o_counts = c.take<int32_t>(static_cast<int64_t>(mxmoe::permute_chunks(P)) * E);
+  size_t o_off = c.take<int32_t>(E + 1), o_act = c.take<int32_t>(E), o_nact = c.take<int32_t>(1);
+  size_t o_pt = c.take<int32_t>(P), o_ps = c.take<int32_t>(P), o_inv = c.take<int32_t>(P);
+  size_t o_xq = c.take<uint16_t>(fp8 ? static_cast<int64_t>(T) * H : 0);
+  size_t o_mid = c.take<uint16_t>(P * I);
+  size_t o_y = c.take<float>(P * H);
+  size_t o_amax = c.take<unsigned>(2);
+  if (b) {
+    b->logits = reinterpret_cast<float*>(base + o_logits);
+    b->topk_idx = reinterpret_cast<int32_t*>(base + o_idx);
+    b->topk_w = reinterpret_cast<float*>(base + o_w);
+    b->counts = reinterpret_cast<int32_t*>(base + o_counts);
+    b->offsets = reinterpret_cast<int32_t*>(base + o_off);
+    b->active = reinterpret_cast<int32_t*>(base + o_act);
+    b->n_active = reinterpret_cast<int32_t*>(base + o_nact);
+    b->perm_token = reinterpret_cast<int32_t*>(base + o_pt);
+    b->perm_slot = reinterpret_cast<int32_t*>(base + o_ps);
+    b->inv = reinterpret_cast<int32_t*>(base + o_inv);
+    b->xq = reinterpret_cast<uint16_t*>(base + o_xq);
+    b->act_mid = reinterpret_cast<uint16_t*>(base + o_mid);
+    b->y = reinterpret_cast<float*>(base + o_y);
+    b->amax = reinterpret_cast<unsigned*>(base + o_amax);
+  }
+  return c.off;
+}
+
+int check_routing_args(int T, int E, int k) {
+  if (T < 0) return fail(MXMOE_EINVAL, "T = %d is negative", T);
+  if (T >= (1 << 24)) return fail(MXMOE_EUNSUPPORTED, "T = %d exceeds 2^24 - 1", T);
+  if (E < 1) return fail(MXMOE_EINVAL, "E = %d must be >= 1", E);
+  if (E > 256) return fail(MXMOE_EUNSUPPORTED, "E = %d exceeds 256", E);
+  if (k < 1 || k > 8) return fail(MXMOE_EUNSUPPORTED, "k = %d outside [1, 8]", k);
+  if (k > E) return fail(MXMOE_EUNSUPPORTED, "k = %d exceeds E = %d", k, E);
+  return MXMOE_OK;
+}
+
+struct LayerArgs {
+  const uint16_t* x;
+  const uint16_t* router_w;
+  const uint16_t* router_b;
+  const uint8_t* gu_blocks;
+  const uint8_t* gu_scales;
+  const float* gu_bias;
+  const uint8_t* d_blocks;
+  const uint8_t* d_scales;
+  const float* d_bias;
+  int E, k, T, H, I;
+};
+
+int check_layer_args(const LayerArgs& a) {
+  if (int rc = check_routing_args(a.T, a.E, a.k)) return rc;
+  if (a.H <= 0 || a.I <= 0) return fail(MXMOE_EINVAL, "H = %d and I = %d must be positive", a.H, a.I);
+  if (a.H % 32 || a.I % 32)
+    return fail(MXMOE_EALIGN, "H = %d and I = %d must be multiples of 32 (MXFP4 block size)", a.H, a.I);
+  const void* ptrs[] = {a.x, a.router_w, a.gu_blocks, a.gu_scales, a.gu_bias,
+                        a.d_blocks, a.d_scales, a.d_bias};
+  const char* names[] = {"x", "router_w", "gu_blocks", "gu_scales", "gu_bias",
+                         "d_blocks", "d_scales", "d_bias"};
+  for (int i = 0; i < 8; ++i) {
+    if (!ptrs[i]) return fail(MXMOE_EINVAL, "%s is NULL", names[i]);
+    if (!aligned16(ptrs[i])) return fail(MXMOE_EINVAL, "%s is not 16-byte aligned", names[i]);
+  }
+  if (a.router_b && !aligned16(a.router_b)) return fail(MXMOE_EINVAL, "router_b is not 16-byte aligned");
+  return MXMOE_OK;
+}
+
+// Runs the layer up to the stage that `calib` needs. Returns a status code.
+int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* calib_out,
+              cudaStream_t st) {
+  using namespace mxmoe;
+  Workspace* ws = nullptr;
+  if (int rc = current_device_ws(&ws)) return rc;
+  const bool fp8 = act_scale != nullptr;
+  const size_t need = layout(a.T, a.E, a.k, a.H, a.I, fp8, nullptr, nullptr);
+  if (int rc = ensure_capacity(ws, need)) return rc;
+  if (std::max(a.H, a.I) > ws->smem_K) {
+    cudaError_t e = expert_mma_set_smem_limits(std::max(a.H, a.I));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    ws->smem_K = std::max(a.H, a.I);
+  }
+  LayerBuffers b;
+  layout(a.T, a.E, a.k, a.H, a.I, fp8, &b, ws->base);
+  const int64_t P = static_cast<int64_t>(a.T) * a.k;
+  int launches = 0;
+  cudaError_t e;
+  const float s0 = fp8 ? act_scale[0] : 1.0f, s1 = fp8 ? act_scale[1] : 1.0f;
+
+  StageTimer tm(st);
+  if ((e = launch_router(a.x, a.router_w, a.router_b, a.T, a.H, a.E, b.logits, st))) return cuda_fail(e, "router");
+  ++launches;
+  tm.mark("router");
+  if ((e = launch_topk(b.logits, a.T, a.E, a.k, b.topk_idx, b.topk_w, st))) return cuda_fail(e, "topk");
+  ++launches;
+  tm.mark("topk");
+  if ((e = launch_permute(b.topk_idx, a.T, a.E, a.k, b.counts, b.offsets, b.perm_token, b.perm_slot,
+                          b.inv, b.active, b.n_active, ws->err, st, &launches)))
+    return cuda_fail(e, "permute");
+  tm.mark("permute");
+  const uint16_t* act_in = a.x;
+  if (fp8) {
+    if ((e = launch_fp8_quant_as_bf16(a.x, static_cast<int64_t>(a.T) * a.H, s0, b.xq, st, ws->sms)))
+      return cuda_fail(e, "fp8 activation cast");
+    ++launches;
+    tm.mark("act_quant");
+    act_in = b.xq;
+  }
+  const int max_active = static_cast<int>(std::min<int64_t>(a.E, P));
+  if (calib_out) {
+    if ((e = cudaMemsetAsync(b.amax, 0, 2 * sizeof(unsigned), st))) return cuda_fail(e, "memset");
+    if ((e = launch_amax_bf16(a.x, static_cast<int64_t>(a.T) * a.H, b.amax, st, ws->sms))) return cuda_fail(e, "amax");
+    ++launches;
+  }
+  if ((e = launch_expert_mma(a.gu_blocks, a.gu_scales, a.gu_bias, 2 * a.I, a.H, act_in,
+                             b.perm_token, b.offsets, b.active, b.n_active, max_active, s0, 0, a.I,
+                             fp8 ? s1 : 0.0f, b.act_mid, nullptr, calib_out ? b.amax + 1 : nullptr,
+                             a.T, st)))
+    return cuda_fail(e, "gate_up");
+  ++launches;
+  tm.mark("gate_up");
+  if (calib_out) {
+    if ((e = launch_finalize_scales(b.amax, calib_out, st))) return cuda_fail(e, "finalize");
+    ++launches;
+    t_last_launches = launches;
+    return MXMOE_OK;
+  }
+  if ((e = launch_expert_mma(a.d_blocks, a.d_scales, a.d_bias, a.H, a.I, b.act_mid, nullptr,
+                             b.offsets, b.active, b.n_active, max_active, s1, 1, a.I, 0.0f, nullptr,
+                             b.y, nullptr, a.T, st)))
+    return cuda_fail(e, "down");
+  ++launches;
+  tm.mark("down");
+  if ((e = launch_combine(b.y, b.topk_idx, b.topk_w, b.inv, a.T, a.H, a.k, out, st, ws->sms)))
+    return cuda_fail(e, "combine");
+  ++launches;
+  tm.mark("combine");
+  t_last_launches = launches;
+  return MXMOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int mxfp4_quantize(const float* w, int64_t rows, int64_t K, uint8_t* blocks, uint8_t* scales,
+                   void* stream) {
+  t_last_error.clear();
+  if (rows < 0 || K < 0) return fail(MXMOE_EINVAL, "negative size rows=%lld K=%lld", (long long)rows, (long long)K);
+  if (K % 32) return fail(MXMOE_EALIGN, "K = %lld is not a multiple of 32 (MXFP4 block size)", (long long)K);
+  if (rows == 0 || K == 0) return MXMOE_OK;
+  if (!w || !blocks || !scales) return fail(MXMOE_EINVAL, "null pointer");
+  if (!aligned16(w) || !aligned16(blocks)) return fail(MXMOE_EINVAL, "w and blocks must be 16-byte aligned");
+  Workspace* ws = nullptr;
+  if (int rc = current_device_ws(&ws)) return rc;
+  cudaError_t e = mxmoe::launch_quantize(w, rows, K, blocks, scales, static_cast<cudaStream_t>(stream), ws->sms);
+  return e ? cuda_fail(e, "quantize launch") : MXMOE_OK;
+}
+
+int mxfp4_dequantize(const uint8_t* blocks, const uint8_t* scales, int64_t rows, int64_t K,
+                     void* out, int out_dtype, void* stream) {
+  t_last_error.clear();
+  if (rows < 0 || K < 0) return fail(MXMOE_EINVAL, "negative size rows=%lld K=%lld", (long long)rows, (long long)K);
+  if (K % 32) return fail(MXMOE_EALIGN, "K = %lld is not a multiple of 32 (MXFP4 block size)", (long long)K);
+  if (out_dtype != MXMOE_OUT_F32 && out_dtype != MXMOE_OUT_BF16)
+    return fail(MXMOE_EUNSUPPORTED, "out_dtype %d is neither MXMOE_OUT_F32 nor MXMOE_OUT_BF16", out_dtype);
+  if (rows == 0 || K == 0) return MXMOE_OK;
+  if (!blocks || !scales || !out) return fail(MXMOE_EINVAL, "null pointer");
+  if (!aligned16(blocks) || !aligned16(out)) return fail(MXMOE_EINVAL, "blocks and out must be 16-byte aligned");
+  Workspace* ws = nullptr;
+  if (int rc = current_device_ws(&ws)) return rc;
+  cudaError_t e = mxmoe::launch_dequantize(blocks, scales, rows, K, out, out_dtype,
+                                           static_cast<cudaStream_t>(stream), ws->sms);
+  return e ? cuda_fail(e, "dequantize launch") : MXMOE_OK;
+}
+
+int moe_route_topk(const uint16_t* x, const uint16_t* router_w, const uint16_t* router_b, int T,
+                   int H, int E, int k, float* logits_out, int32_t* topk_idx, float* topk_w,
+                   void* stream) {
+  t_last_error.clear();
+  if (int rc = check_routing_args(T, E, k)) return rc;
+  if (H <= 0) return fail(MXMOE_EINVAL, "H = %d must be positive", H);
+  if (H % 32) return fail(MXMOE_EALIGN, "H = %d is not a multiple of 32", H);
+  if (T == 0) return MXMOE_OK;
+  if (!x || !router_w || !topk_idx || !topk_w) return fail(MXMOE_EINVAL, "null pointer");
+  if (!aligned16(x) || !aligned16(router_w)) return fail(MXMOE_EINVAL, "x and router_w must be 16-byte aligned");
+  Workspace* ws = nullptr;
+  if (int rc = current_device_ws(&ws)) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* logits = logits_out;
+  if (!logits) {
+    if (int rc = ensure_capacity(ws, static_cast<size_t>(T) * E * sizeof(float))) return rc;
+    logits = reinterpret_cast<float*>(ws->base);
+  }
+  cudaError_t e = mxmoe::launch_router(x, router_w, router_b, T, H, E, logits, st);
+  if (e) return cuda_fail(e, "router launch");
+  e = mxmoe::launch_topk(logits, T, E, k, topk_idx, topk_w, st);
+  return e ? cuda_fail(e, "topk launch") : MXMOE_OK;
+}
+
+int moe_topk_from_logits(const float* logits, int T, int E, int k, int32_t* topk_idx,
+                         float* topk_w, void* stream) {
+  t_last_error.clear();
+  if (int rc = check_routing_args(T, E, k)) return rc;
+  if (T == 0) return MXMOE_OK;
+  if (!logits || !topk_idx || !topk_w) return fail(MXMOE_EINVAL, "null pointer");
+  cudaError_t e = mxmoe::launch_topk(logits, T, E, k, topk_idx, topk_w, static_cast<cudaStream_t>(stream));
+  return e ? cuda_fail(e, "topk launch") : MXMOE_OK;
+}
+
+int moe_permute(const int32_t* topk_idx, int T, int E, int k, int32_t* offsets,
+                int32_t* perm_token, int32_t* perm_slot, void* stream) {
+  t_last_error.clear();
+  if (int rc = check_routing_args(T, E, k)) return rc;
+  if (!offsets) return fail(MXMOE_EINVAL, "offsets is NULL");
+  if (T > 0 && (!topk_idx || !perm_token || !perm_slot)) return fail(MXMOE_EINVAL, "null pointer");
+  Workspace* ws = nullptr;
+  if (int rc = current_device_ws(&ws)) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t P = static_cast<int64_t>(T) * k;
+  if (T == 0) {
+    cudaError_t e = cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), st);
+    return e ? cuda_fail(e, "memset") : MXMOE_OK;
+  }
+  Carve c;
+  size_t o_counts = c.take<int32_t>(static_cast<int64_t>(mxmoe::permute_chunks(P)) * E);
+  size_t o_act = c.take<int32_t>(E), o_n = c.take<int32_t>(1);
+  if (int rc = ensure_capacity(ws, c.off)) return rc;
+  int launches = 0;
+  cudaError_t e = mxmoe::launch_permute(
+      topk_idx, T, E, k, reinterpret_cast<int32_t*>(ws->base + o_counts), offsets, perm_token,
+      perm_slot, nullptr, reinterpret_cast<int32_t*>(ws->base + o_act),
+      reinterpret_cast<int32_t*>(ws->base + o_n), ws->err, st, &launches);
+  return e ? cuda_fail(e, "permute launch") : MXMOE_OK;
+}
+
+int moe_fp8_quantize(const uint16_t* x, int64_t n, float s, uint8_t* q, void* stream) {
+  t_last_error.clear();
+  if (n < 0) return fail(MXMOE_EINVAL, "n = %lld is negative", (long long)n);
+  if (n == 0) return MXMOE_OK;
+  if (!x || !q) return fail(MXMOE_EINVAL, "null pointer");
+  if (!(s > 0.0f)) return fail(MXMOE_EINVAL, "scale must be > 0");
+  Workspace* ws = nullptr;
+  if (int rc = current_device_ws(&ws)) return rc;
+  cudaError_t e = mxmoe::launch_fp8_quant(x, n, s, q, static_cast<cudaStream_t>(stream), ws->sms);
+  return e ? cuda_fail(e, "fp8 quant launch") : MXMOE_OK;
+}
+
+int moe_mxfp4_forward(const uint16_t* x, const uint16_t* router_w, const uint16_t* router_b,
+                      const uint8_t* gu_blocks, const uint8_t* gu_scales, const float* gu_bias,
+                      const uint8_t* d_blocks, const uint8_t* d_scales, const float* d_bias,
+                      int E, int k, int T, int H, int I, const float* act_scale, uint16_t* out,
+                      void* stream) {
+  t_last_error.clear();
+  LayerArgs a{x, router_w, router_b, gu_blocks, gu_scales, gu_bias, d_blocks, d_scales, d_bias,
+              E, k, T, H, I};
+  if (T == 0) return check_routing_args(T, E, k);
+  if (int rc = check_layer_args(a)) return rc;
+  if (!out) return fail(MXMOE_EINVAL, "out is NULL");
+  if (!aligned16(out)) return fail(MXMOE_EINVAL, "out is not 16-byte aligned");
+  if (act_scale && !(act_scale[0] > 0.0f && act_scale[1] > 0.0f))
+    return fail(MXMOE_EINVAL, "act_scale values must be > 0");
+  return run_layer(a, act_scale, out, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+int moe_mxfp4_calibrate(const uint16_t* x, const uint16_t* router_w, const uint16_t* router_b,
+                        const uint8_t* gu_blocks, const uint8_t* gu_scales, const float* gu_bias,
+                        const uint8_t* d_blocks, const uint8_t* d_scales, const float* d_bias,
+                        int E, int k, int T, int H, int I, float* act_scale_out, void* stream) {
+  t_last_error.clear();
+  LayerArgs a{x, router_w, router_b, gu_blocks, gu_scales, gu_bias, d_blocks, d_scales, d_bias,
+              E, k, T, H, I};
+  if (T == 0) return fail(MXMOE_EINVAL, "calibration needs T > 0 tokens");
+  if (int rc = check_layer_args(a)) return rc;
+  if (!act_scale_out) return fail(MXMOE_EINVAL, "act_scale_out is NULL");
+  return run_layer(a, nullptr, nullptr, act_scale_out, static_cast<cudaStream_t>(stream));
+}
+
+int mxmoe_check(void* stream) {
+  t_last_error.clear();
+  Workspace* ws = nullptr;
+  if (int rc = current_device_ws(&ws)) return rc;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "stream");
+  int v = 0;
+  if ((e = cudaMemcpy(&v, ws->err, sizeof(int), cudaMemcpyDeviceToHost))) return cuda_fail(e, "read error word");
+  if (v != 0) {
+    if ((e = cudaMemset(ws->err, 0, sizeof(int)))) return cuda_fail(e, "clear error word");
+    return fail(v, "device error word = %d", v);
+  }
+  return MXMOE_OK;
+}
+
+const char* mxmoe_last_error(void) { return t_last_error.c_str(); }
+
+int mxmoe_last_launch_count(void) { return t_last_launches; }
+
+int mxmoe_profile_enable(int on) {
+  t_last_error.clear();
+  t_profile = on != 0;
+  t_marks.clear();
+  t_event_next = 0;
+  return MXMOE_OK;
+}
+
+int mxmoe_profile_read(char* names, float* total_ms, int* calls, int max_entries) {
+  t_last_error.clear();
+  if (max_entries < 0 || (max_entries > 0 && (!names || !total_ms || !calls)))
+    return fail(MXMOE_EINVAL, "bad output arrays");
+  std::vector<std::string> keys;
+  std::vector<double> ms;
+  std::vector<int> n;
+  for (const StageMark& m : t_marks) {
+    cudaError_t e = cudaEventSynchronize(m.stop);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaEventSynchronize");
+    float dt = 0.0f;
+    if ((e = cudaEventElapsedTime(&dt, m.start, m.stop)) != cudaSuccess) return cuda_fail(e, "cudaEventElapsedTime");
+    size_t i = 0;
+    while (i < keys.size() && keys[i] != m.name) ++i;
+    if (i == keys.size()) { keys.push_back(m.name); ms.push_back(0.0); n.push_back(0); }
+    ms[i] += dt;
+    n[i] += 1;
+  }
+  const int cnt = static_cast<int>(keys.size());
+  for (int i = 0; i < cnt && i < max_entries; ++i) {
+    std::snprintf(names + 32 * i, 32, "%s", keys[i].c_str());
+    total_ms[i] = static_cast<float>(ms[i]);
+    calls[i] = n[i];
+  }
+  t_marks.clear();
+  t_event_next = 0;
+  return cnt;
+}
+
+int mxmoe_release(void) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (dev >= 0 && dev < kMaxDevices && g_ws[dev].base) {
+    if ((e = cudaDeviceSynchronize()) != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+    cudaFree(g_ws[dev].base);
+    g_ws[dev].base = nullptr;
+    g_ws[dev].cap = 0;
+  }
+  return MXMOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,251 @@
+// Routed expert GEMMs with the MXFP4 weights dequantized in registers (the decode path:
+// few tokens per expert, bound by streaming the packed weight bytes from HBM).
+//
+// Page: "quantization_mxfp4" (KerasFormers), As GPT-OSS's native format -- on decode only
+// the top-k routed experts' blocks are dequantized; Primitives -- w = codebook[nibble] *
+// 2^(scale - 127).
+//
+// Shape of the work: for every active expert e and its n_e routed rows (positions
+// [off_e, off_e + n_e) of the expert-grouped order), y = s * (X_e . W_e^T) + bias.
+// Weights are the M side of mma.sync m16n8k16 (16 weight rows per warp), the routed
+// tokens the N side (8 per n-tile), so the bytes of each weight are read once whatever
+// n_e is. Per 32-value block (one e8m0 scale) a warp issues two k16 MMAs into a scratch
+// accumulator and folds it into the running sum with the block's fp32 scale, so the
+// nibbles are decoded without their scale.
+//
+// Nibble decoding: a 32-bit word holds 8 consecutive e2m1 values v0..v7 (v_i in bits
+// 4i..4i+3). The pair (v_i, v_{i+4}) sits 16 bits apart, so one shift per field places
+// the 3 magnitude bits at bf16 bits 6..8 (exponent LSBs + mantissa MSB) and the sign at
+// bit 15 of both halves at once. That bf16 equals the e2m1 value times 2^-126 (code 1
+// becomes the bf16 subnormal 2^-127); one bf16x2 multiply by 2^126 makes it exact.
+// The K order inside every group of 8 is therefore (0,4,1,5,2,6,3,7) on both operands;
+// activations get the same order with two byte permutes per register pair.
+//
+// Lane (g = lane/4, t = lane%4) owns weight rows g and g+8 and, within each 32-value
+// block, values 8t..8t+7 (bytes 4t..4t+3 of the 16-byte block).
+#include "common.cuh"
+
+namespace mxmoe {
+
+namespace {
+
+constexpr int kWarps = 4;       // warps per CTA
+constexpr int kUnroll = 8;      // 32-value blocks whose weight words are loaded ahead
+
+__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.bf16x2 %0, %1, %2;\n" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// bf16x2 (v_i, v_{i+4}) of an e2m1 word, exact (see the file comment).
+template <int i>
+__device__ __forceinline__ uint32_t e2m1_pair_bf16x2(uint32_t w) {
+  constexpr uint32_t kMag = 0x01C001C0u, kSign = 0x80008000u, k2p126 = 0x7E807E80u;
+  uint32_t mag, sgn;
+  if constexpr (i == 0) { mag = (w << 6) & kMag; sgn = (w << 12) & kSign; }
+  if constexpr (i == 1) { mag = (w << 2) & kMag; sgn = (w << 8) & kSign; }
+  if constexpr (i == 2) { mag = (w >> 2) & kMag; sgn = (w << 4) & kSign; }
+  if constexpr (i == 3) { mag = (w >> 6) & kMag; sgn = w & kSign; }
+  return bf16x2_mul(mag | sgn, k2p126);
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;\n" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+struct ExpertGemmArgs {
+  const uint8_t* blocks;   // (E, rows_total, K/2)
+  const uint8_t* scales;   // (E, rows_total, K/32)
+  const float* bias;       // (E, rows_total)
+  int rows_total;          // 2I for gate_up, H for down
+  int K;                   // H for gate_up, I for down
+  const uint16_t* act;     // activation rows (bf16 bits), K wide
+  const int32_t* act_row;  // nullptr: row = position; else row = act_row[position]
+  const int32_t* offsets;  // (E+1)
+  const int32_t* active;   // active expert ids
+  const int32_t* n_active;
+  float s_in;              // scale applied to the dot product before the bias
+  // outputs
+  int mode;                // 0: gate_up + SwiGLU -> act_out; 1: down -> y_out
+  int I;                   // gate_up: intermediate size (gate rows [0,I), up rows [I,2I))
+  float s_mid;             // fp8 path: a is quantized with this scale; 0: bf16 rounding
+  uint16_t* act_out;       // (P, I) bf16 bits (mode 0)
+  float* y_out;            // (P, rows_total) fp32 (mode 1)
+  unsigned* amax_bits;     // optional: running max |a| (fp32 bits), mode 0
+};
+
+template <int NT>
+__global__ void __launch_bounds__(kWarps * 32) expert_mma_kernel(ExpertGemmArgs p) {
+  extern __shared__ float s_scale[];  // [kWarps][16][nb]
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int slot = blockIdx.y;
+  if (slot >= *p.n_active) return;
+  const int e = p.active[slot];
+  const int pos0 = p.offsets[e], n_e = p.offsets[e + 1] - pos0;
+  const int nb = p.K / 32;
+
+  // rows of this warp: gate_up -> 8 gate rows i0.. and the matching 8 up rows; down -> 16
+  int row_lo, row_hi;
+  if (p.mode == 0) {
+    const int i0 = (blockIdx.x * kWarps + warp) * 8;
+    if (i0 >= p.I) return;
+    row_lo = i0 + g;
+    row_hi = p.I + i0 + g;
+  } else {
+    const int r0 = (blockIdx.x * kWarps + warp) * 16;
+    if (r0 >= p.rows_total) return;
+    row_lo = r0 + g;
+    row_hi = r0 + 8 + g;
+  }
+  const int64_t erow = static_cast<int64_t>(e) * p.rows_total;
+  const uint8_t* wlo = p.blocks + (erow + row_lo) * (p.K / 2) + 4 * t;
+  const uint8_t* whi = p.blocks + (erow + row_hi) * (p.K / 2) + 4 * t;
+
+  // stage this warp's 16 rows of scales as fp32 (row slot 0..7 = lo rows, 8..15 = hi rows)
+  float* sc = s_scale + static_cast<int64_t>(warp) * 16 * nb;
+  for (int i = lane; i < 16 * nb; i += 32) {
+    const int r = i / nb, b = i % nb;
+    const int row = (r < 8) ? (row_lo - g + r) : (row_hi - g + (r - 8));
+    sc[i] = e8m0_to_f32(p.scales[(erow + row) * nb + b]);
+  }
+  __syncwarp();
+  const float* sc_lo = sc + g * nb;
+  const float* sc_hi = sc + (8 + g) * nb;
+
+  for (int tp = 0; tp < n_e; tp += 8 * NT) {
+    // activation row pointers of this lane's token (column g of each n-tile)
+    const uint16_t* arow[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int j = tp + nt * 8 + g;
+      if (j < n_e) {
+        const int pos = pos0 + j;
+        const int64_t r = p.act_row ? p.act_row[pos] : pos;
+        arow[nt] = p.act + r * p.K + 8 * t;
+      } else {
+        arow[nt] = nullptr;
+      }
+    }
+    const int nt_live = min(NT, (n_e - tp + 7) / 8);
+
+    float acc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) acc[nt][r] = 0.0f;
+
+    for (int b0 = 0; b0 < nb; b0 += kUnroll) {
+      uint32_t wl[kUnroll], wh[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int b = b0 + u;
+        wl[u] = b < nb ? ld_nc_u32(wlo + 16 * b) : 0u;
+        wh[u] = b < nb ? ld_nc_u32(whi + 16 * b) : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int b = b0 + u;
+        if (b >= nb) break;
+        uint32_t a0[4], a1[4];
+        a0[0] = e2m1_pair_bf16x2<0>(wl[u]);
+        a0[1] = e2m1_pair_bf16x2<0>(wh[u]);
+        a0[2] = e2m1_pair_bf16x2<1>(wl[u]);
+        a0[3] = e2m1_pair_bf16x2<1>(wh[u]);
+        a1[0] = e2m1_pair_bf16x2<2>(wl[u]);
+        a1[1] = e2m1_pair_bf16x2<2>(wh[u]);
+        a1[2] = e2m1_pair_bf16x2<3>(wl[u]);
+        a1[3] = e2m1_pair_bf16x2<3>(wh[u]);
+        const float sl = sc_lo[b], sh = sc_hi[b];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          if (nt >= nt_live) break;
+          uint4 v = make_uint4(0u, 0u, 0u, 0u);
+          if (arow[nt]) v = ld_nc_v4(arow[nt] + 32 * b);
+          // natural (x0..x7) -> k-step 0: (x0,x4),(x1,x5); k-step 1: (x2,x6),(x3,x7)
+          const uint32_t b0r[2] = {prmt(v.x, v.z, 0x5410u), prmt(v.x, v.z, 0x7632u)};
+          const uint32_t b1r[2] = {prmt(v.y, v.w, 0x5410u), prmt(v.y, v.w, 0x7632u)};
+          float tmp[4] = {0.f, 0.f, 0.f, 0.f};
+          mma_bf16_16816(tmp, a0, b0r, tmp);
+          mma_bf16_16816(tmp, a1, b1r, tmp);
+          acc[nt][0] = fmaf(tmp[0], sl, acc[nt][0]);
+          acc[nt][1] = fmaf(tmp[1], sl, acc[nt][1]);
+          acc[nt][2] = fmaf(tmp[2], sh, acc[nt][2]);
+          acc[nt][3] = fmaf(tmp[3], sh, acc[nt][3]);
+        }
+      }
+    }
+
+    // epilogue: acc[nt][0..1] = row_lo, tokens 2t, 2t+1; acc[nt][2..3] = row_hi, same tokens
+    const float b_lo = p.bias[erow + row_lo], b_hi = p.bias[erow + row_hi];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      if (nt >= nt_live) break;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int j = tp + nt * 8 + 2 * t + c;
+        if (j >= n_e) continue;
+        const int64_t pos = pos0 + j;
+        const float lo = __fadd_rn(__fmul_rn(p.s_in, acc[nt][c]), b_lo);
+        const float hi = __fadd_rn(__fmul_rn(p.s_in, acc[nt][2 + c]), b_hi);
+        if (p.mode == 0) {
+          const float a = silu_mul(lo, hi);
+          if (p.amax_bits) atomicMax(p.amax_bits, __float_as_uint(fabsf(a)));
+          uint16_t bits;
+          if (p.s_mid > 0.0f)
+            bits = static_cast<uint16_t>(__float_as_uint(e4m3_to_f32(act_quant_e4m3(a, p.s_mid))) >> 16);
+          else
+            bits = f32_to_bf16_bits_rn(a);
+          p.act_out[pos * p.I + (row_lo)] = bits;
+        } else {
+          p.y_out[pos * p.rows_total + row_lo] = lo;
+          p.y_out[pos * p.rows_total + row_hi] = hi;
+        }
+      }
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_expert_mma(const uint8_t* blocks, const uint8_t* scales, const float* bias,
+                              int rows_total, int K, const uint16_t* act, const int32_t* act_row,
+                              const int32_t* offsets, const int32_t* active,
+                              const int32_t* n_active, int max_active, float s_in, int mode, int I,
+                              float s_mid, uint16_t* act_out, float* y_out, unsigned* amax_bits,
+                              int max_tokens_per_expert, cudaStream_t st) {
+  ExpertGemmArgs a{blocks, scales, bias, rows_total, K, act, act_row, offsets, active, n_active,
+                   s_in, mode, I, s_mid, act_out, y_out, amax_bits};
+  const int rows_per_cta = (mode == 0 ? 8 : 16) * kWarps;
+  const int out_rows = mode == 0 ? I : rows_total;
+  dim3 grid(static_cast<unsigned>(cdiv(out_rows, rows_per_cta)), static_cast<unsigned>(max_active));
+  const size_t smem = static_cast<size_t>(kWarps) * 16 * (K / 32) * sizeof(float);
+  const int nt = (max_tokens_per_expert + 7) / 8;
+  if (nt <= 1) {
+    expert_mma_kernel<1><<<grid, kWarps * 32, smem, st>>>(a);
+  } else if (nt <= 2) {
+    expert_mma_kernel<2><<<grid, kWarps * 32, smem, st>>>(a);
+  } else if (nt <= 4) {
+    expert_mma_kernel<4><<<grid, kWarps * 32, smem, st>>>(a);
+  } else {
+    expert_mma_kernel<8><<<grid, kWarps * 32, smem, st>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t expert_mma_set_smem_limits(int max_K) {
+  const int smem = kWarps * 16 * (max_K / 32) * static_cast<int>(sizeof(float));
+  cudaError_t e = cudaSuccess;
+  if (smem > 48 * 1024) {
+    if ((e = cudaFuncSetAttribute(expert_mma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
+    if ((e = cudaFuncSetAttribute(expert_mma_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
+    if ((e = cudaFuncSetAttribute(expert_mma_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
+    if ((e = cudaFuncSetAttribute(expert_mma_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
+  }
+  return e;
+}
+
+}  // namespace mxmoe

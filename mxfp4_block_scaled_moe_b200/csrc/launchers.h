@@ -1,0 +1,45 @@
+// Host-side launchers of the library's kernels (internal; the public ABI is mxfp4_moe.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace mxmoe {
+
+cudaError_t launch_quantize(const float* w, int64_t rows, int64_t K, uint8_t* blocks,
+                            uint8_t* scales, cudaStream_t st, int sms);
+cudaError_t launch_dequantize(const uint8_t* blocks, const uint8_t* scales, int64_t rows,
+                              int64_t K, void* out, int out_dtype, cudaStream_t st, int sms);
+
+cudaError_t launch_router(const uint16_t* x, const uint16_t* wr, const uint16_t* br, int T, int H,
+                          int E, float* logits, cudaStream_t st);
+cudaError_t launch_topk(const float* logits, int T, int E, int k, int32_t* idx, float* w,
+                        cudaStream_t st);
+int permute_chunks(int64_t P);
+cudaError_t launch_permute(const int32_t* idx, int T, int E, int k, int32_t* counts_ws,
+                           int32_t* offsets, int32_t* perm_token, int32_t* perm_slot,
+                           int32_t* inv, int32_t* active, int32_t* n_active, int* err,
+                           cudaStream_t st, int* launches);
+cudaError_t launch_fp8_quant(const uint16_t* x, int64_t n, float s, uint8_t* q, cudaStream_t st,
+                             int sms);
+cudaError_t launch_fp8_quant_as_bf16(const uint16_t* x, int64_t n, float s, uint16_t* xq,
+                                     cudaStream_t st, int sms);
+cudaError_t launch_gather_fp8_rows(const uint8_t* xq8, const int32_t* perm_token, int64_t P, int H,
+                                   uint8_t* a1, cudaStream_t st, int sms);
+cudaError_t launch_amax_bf16(const uint16_t* x, int64_t n, unsigned* amax_bits, cudaStream_t st,
+                             int sms);
+cudaError_t launch_finalize_scales(const unsigned* amax_bits, float* out, cudaStream_t st);
+
+cudaError_t launch_expert_mma(const uint8_t* blocks, const uint8_t* scales, const float* bias,
+                              int rows_total, int K, const uint16_t* act, const int32_t* act_row,
+                              const int32_t* offsets, const int32_t* active,
+                              const int32_t* n_active, int max_active, float s_in, int mode, int I,
+                              float s_mid, uint16_t* act_out, float* y_out, unsigned* amax_bits,
+                              int max_tokens_per_expert, cudaStream_t st);
+cudaError_t expert_mma_set_smem_limits(int max_K);
+
+cudaError_t launch_combine(const float* y, const int32_t* topk_idx, const float* topk_w,
+                           const int32_t* inv, int T, int H, int k, uint16_t* out, cudaStream_t st,
+                           int sms);
+
+}  // namespace mxmoe

@@ -1,0 +1,481 @@
+// Routing kernels: router logits (GEMV for few tokens, mma.sync GEMM for many), top-k
+// softmax, the deterministic token -> expert permutation, and the activation casts.
+//
+// Router: GPT-OSS top-k routing with the router kept in bf16 ("gpt-oss-120b-mxfp4-
+// fp8attn-v2", config.json modules_to_not_convert; "xpuenabler/gpt-oss-15.5b-23E-nf4-
+// GPU", Quantization recipe: router kept unquantized). Top-k ties go to the lower expert
+// id; the softmax runs over the k selected logits.
+// Permutation: the routed dispatch of "quantization_mxfp4", As GPT-OSS's native format:
+// pairs (token, slot) grouped by expert, ascending token inside an expert.
+#include "common.cuh"
+
+namespace mxmoe {
+
+// ------------------------------------------------------------------ router GEMV -----
+// One warp per (token, expert): 16-byte loads along H, fp32 FMA, fixed-order warp sum.
+__global__ void __launch_bounds__(256) router_gemv_kernel(const uint16_t* __restrict__ x,
+                                                           const uint16_t* __restrict__ wr,
+                                                           const uint16_t* __restrict__ br,
+                                                           int T, int H, int E,
+                                                           float* __restrict__ logits) {
+  const int lane = threadIdx.x & 31;
+  const int64_t wid = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (wid >= static_cast<int64_t>(T) * E) return;
+  const int t = static_cast<int>(wid / E), e = static_cast<int>(wid % E);
+  const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(t) * H);
+  const uint4* wrow = reinterpret_cast<const uint4*>(wr + static_cast<int64_t>(e) * H);
+  float acc = 0.0f;
+  for (int c = lane; c < H / 8; c += 32) {
+    const uint4 a = ld_nc_v4(xr + c), b = ld_nc_v4(wrow + c);
+    const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc = fmaf(__uint_as_float(av[i] << 16), __uint_as_float(bv[i] << 16), acc);
+      acc = fmaf(__uint_as_float(av[i] & 0xFFFF0000u), __uint_as_float(bv[i] & 0xFFFF0000u), acc);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) logits[wid] = br ? acc + bf16_bits_to_f32(br[e]) : acc;
+}
+
+// ------------------------------------------------------------------ router GEMM -----
+// logits (T, E) = x (T, H) . Wr (E, H)^T with mma.sync m16n8k16 (bf16 in, fp32 acc).
+// CTA tile 64 tokens x 64 experts, 4 warps as 2 x 2 (each 32 x 32), K in steps of 32
+// staged by cp.async into padded shared rows (80-byte pitch: ldmatrix conflict-free).
+namespace rg {
+constexpr int BM = 64, BN = 64, BK = 32, PITCH = 40, STAGES = 3;  // pitch in bf16 elements
+}
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool pred) {
+  const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  const int n = pred ? 16 : 0;
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem), "r"(n));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t r[4], const void* smem) {
+  const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(s));
+}
+
+__global__ void __launch_bounds__(128) router_gemm_kernel(const uint16_t* __restrict__ x,
+                                                           const uint16_t* __restrict__ wr,
+                                                           const uint16_t* __restrict__ br,
+                                                           int T, int H, int E,
+                                                           float* __restrict__ logits) {
+  using namespace rg;
+  __shared__ __align__(16) uint16_t sa[STAGES][BM * PITCH];
+  __shared__ __align__(16) uint16_t sb[STAGES][BN * PITCH];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int m0 = blockIdx.x * BM, n0 = blockIdx.y * BN;
+  const int wm = (warp >> 1) * 32, wn = (warp & 1) * 32;
+  const int nk = H / BK;
+
+  auto load_stage = [&](int stage, int kt) {
+    // 64 rows x 64 bytes per operand = 256 chunks of 16 B each; 128 threads x 2
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int c = tid + i * 128, row = c >> 2, col = (c & 3) * 8;
+      const int gm = m0 + row, gn = n0 + row;
+      const int gmc = gm < T ? gm : T - 1, gnc = gn < E ? gn : E - 1;
+      cp_async16(&sa[stage][row * PITCH + col], x + static_cast<int64_t>(gmc) * H + kt * BK + col, gm < T);
+      cp_async16(&sb[stage][row * PITCH + col], wr + static_cast<int64_t>(gnc) * H + kt * BK + col, gn < E);
+    }
+  };
+
+  float acc[2][4][4];
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) acc[i][j][r] = 0.0f;
+
+#pragma unroll
+  for (int s = 0; s < STAGES - 1; ++s) {
+    if (s < nk) load_stage(s, s);
+    cp_async_commit();
+  }
+  for (int kt = 0; kt < nk; ++kt) {
+    cp_async_wait<STAGES - 2>();
+    __syncthreads();
+    const int nxt = kt + STAGES - 1;
+    if (nxt < nk) load_stage(nxt % STAGES, nxt);
+    cp_async_commit();
+    const int st = kt % STAGES;
+#pragma unroll
+    for (int ks = 0; ks < BK; ks += 16) {
+      uint32_t af[2][4], bfr[4][2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        // x4: matrices (rows 0-7, k 0-7), (rows 8-15, k 0-7), (rows 0-7, k 8-15), (rows 8-15, k 8-15)
+        const int r = wm + i * 16 + (lane & 15), c = ks + (lane >> 4) * 8;
+        ldmatrix_x4(af[i], &sa[st][r * PITCH + c]);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; j += 2) {
+        // x4 over two n8 tiles: (n 0-7, k 0-7), (n 0-7, k 8-15), (n 8-15, k 0-7), (n 8-15, k 8-15)
+        const int r = wn + j * 8 + (lane & 7) + ((lane >> 4) << 3), c = ks + ((lane >> 3) & 1) * 8;
+        uint32_t t4[4];
+        ldmatrix_x4(t4, &sb[st][r * PITCH + c]);
+        bfr[j][0] = t4[0]; bfr[j][1] = t4[1]; bfr[j + 1][0] = t4[2]; bfr[j + 1][1] = t4[3];
+      }
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) mma_bf16_16816(acc[i][j], af[i], bfr[j], acc[i][j]);
+    }
+  }
+  cp_async_wait<0>();
+  // epilogue: c0,c1 -> (row g, cols 2t, 2t+1); c2,c3 -> (row g+8, ...)
+  const int g = lane >> 2, t4 = lane & 3;
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int row = m0 + wm + i * 16 + g + (r >> 1) * 8;
+        const int col = n0 + wn + j * 8 + 2 * t4 + (r & 1);
+        if (row < T && col < E)
+          logits[static_cast<int64_t>(row) * E + col] =
+              br ? acc[i][j][r] + bf16_bits_to_f32(br[col]) : acc[i][j][r];
+      }
+}
+
+// ----------------------------------------------------------------------- top-k -----
+// Ranking: larger logit first, NaN after every number, equal values -> lower id first.
+__device__ __forceinline__ bool ranks_before(float a, int ia, float b, int ib) {
+  const bool na = isnan(a), nb = isnan(b);
+  if (na != nb) return nb;
+  if (!na && a != b) return a > b;
+  return ia < ib;
+}
+
+// One warp per token; each lane holds up to 8 logits (E <= 256).
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E,
+                                                    int k, int32_t* __restrict__ idx,
+                                                    float* __restrict__ wts) {
+  const int lane = threadIdx.x & 31;
+  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (t >= T) return;
+  float v[8];
+  int taken = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int e = lane + 32 * i;
+    v[i] = e < E ? logits[static_cast<int64_t>(t) * E + e] : 0.0f;
+  }
+  float sel[8];
+  int sidx[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (j >= k) break;
+    float bv = 0.0f;
+    int bi = -1;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E && !((taken >> i) & 1) && (bi < 0 || ranks_before(v[i], e, bv, bi))) {
+        bv = v[i];
+        bi = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (oi >= 0 && (bi < 0 || ranks_before(ov, oi, bv, bi))) { bv = ov; bi = oi; }
+    }
+    sel[j] = bv;
+    sidx[j] = bi;
+    if ((bi & 31) == lane) taken |= 1 << (bi >> 5);
+  }
+  if (lane == 0) {
+    float p[8], z = 0.0f;
+    for (int j = 0; j < k; ++j) { p[j] = expf(sel[j] - sel[0]); z += p[j]; }
+    for (int j = 0; j < k; ++j) {
+      idx[static_cast<int64_t>(t) * k + j] = sidx[j];
+      wts[static_cast<int64_t>(t) * k + j] = __fdiv_rn(p[j], z);
+    }
+  }
+}
+
+// --------------------------------------------------------------------- permute -----
+// Stable counting sort of the P = T*k pairs by expert, in two passes over chunks of
+// kPermChunk pairs: (1) per-chunk histograms, (2) every CTA rebuilds the global offsets
+// and its own start per expert from the histograms, then places its pairs in order.
+// Within a sub-chunk of 512 pairs the rank of a pair among equal experts is its rank in
+// its warp (match_any) plus the counts of the same expert in lower warps.
+constexpr int kPermChunk = 4096;
+constexpr int kPermThreads = 512;
+
+__global__ void __launch_bounds__(kPermThreads) permute_count_kernel(
+    const int32_t* __restrict__ idx, int64_t P, int E, int32_t* __restrict__ counts) {
+  __shared__ int hist[256];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int64_t lo = static_cast<int64_t>(blockIdx.x) * kPermChunk;
+  const int64_t hi = min(P, lo + kPermChunk);
+  for (int64_t p = lo + threadIdx.x; p < hi; p += blockDim.x) {
+    const int e = idx[p];
+    if (e >= 0 && e < E) atomicAdd(&hist[e], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) counts[static_cast<int64_t>(blockIdx.x) * E + e] = hist[e];
+}
+
+// counts == nullptr: single-CTA mode (the CTA builds its own histogram first).
+__global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(
+    const int32_t* __restrict__ idx, int64_t P, int E, int k, const int32_t* __restrict__ counts,
+    int32_t* __restrict__ offsets, int32_t* __restrict__ perm_token,
+    int32_t* __restrict__ perm_slot, int32_t* __restrict__ inv, int32_t* __restrict__ active,
+    int32_t* __restrict__ n_active, int* __restrict__ err) {
+  __shared__ int base[256];
+  __shared__ int total[256];
+  __shared__ int wc[kPermThreads / 32][256];
+  __shared__ int scan_tmp[256];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nchunks = static_cast<int>(cdiv(P, kPermChunk));
+  const int64_t lo = static_cast<int64_t>(blockIdx.x) * kPermChunk;
+  const int64_t hi = min(P, lo + kPermChunk);
+
+  if (counts == nullptr) {
+    for (int e = tid; e < E; e += blockDim.x) total[e] = 0;
+    __syncthreads();
+    for (int64_t p = tid; p < P; p += blockDim.x) {
+      const int e = idx[p];
+      if (e >= 0 && e < E) atomicAdd(&total[e], 1);
+      else set_device_error(err, MXMOE_EDEVICE);
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += blockDim.x) base[e] = 0;
+  } else {
+    for (int e = tid; e < E; e += blockDim.x) {
+      int before = 0, all = 0;
+      for (int c = 0; c < nchunks; ++c) {
+        const int v = counts[static_cast<int64_t>(c) * E + e];
+        if (c < static_cast<int>(blockIdx.x)) before += v;
+        all += v;
+      }
+      total[e] = all;
+      base[e] = before;
+    }
+    if (blockIdx.x == 0)
+      for (int64_t p = tid; p < P; p += blockDim.x) {
+        const int e = idx[p];
+        if (e < 0 || e >= E) set_device_error(err, MXMOE_EDEVICE);
+      }
+  }
+  __syncthreads();
+  // exclusive scan of total[] over experts (E <= 256) by one warp, in expert order
+  if (warp == 0) {
+    int carry = 0;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+      const int e = e0 + lane;
+      const int v = e < E ? total[e] : 0;
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+      }
+      if (e < E) scan_tmp[e] = carry + incl - v;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (blockIdx.x == 0 && lane == 0) offsets[E] = carry;
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) {
+    base[e] += scan_tmp[e];
+    if (blockIdx.x == 0) offsets[e] = scan_tmp[e];
+  }
+  if (blockIdx.x == 0 && tid == 0) {
+    int n = 0;
+    for (int e = 0; e < E; ++e)
+      if (total[e] > 0) active[n++] = e;
+    *n_active = n;
+  }
+  __syncthreads();
+
+  const int64_t my_lo = counts == nullptr ? 0 : lo;
+  const int64_t my_hi = counts == nullptr ? P : hi;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int64_t sub = my_lo; sub < my_hi; sub += kPermThreads) {
+    const int64_t p = sub + tid;
+    int e = p < my_hi ? idx[p] : -1;
+    if (e >= E) e = -1;
+    for (int i = tid; i < (kPermThreads / 32) * 256; i += blockDim.x) (&wc[0][0])[i] = 0;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & lt_mask);
+    __syncthreads();
+    if (e >= 0 && rank == 0) wc[warp][e] = __popc(peers);
+    __syncthreads();
+    // exclusive prefix over warps, per expert; total of this sub-chunk into scan_tmp
+    for (int ee = tid; ee < E; ee += blockDim.x) {
+      int run = 0;
+      for (int w = 0; w < kPermThreads / 32; ++w) {
+        const int c = wc[w][ee];
+        wc[w][ee] = run;
+        run += c;
+      }
+      scan_tmp[ee] = run;
+    }
+    __syncthreads();
+    if (e >= 0) {
+      const int pos = base[e] + wc[warp][e] + rank;
+      perm_token[pos] = static_cast<int32_t>(p / k);
+      perm_slot[pos] = static_cast<int32_t>(p % k);
+      if (inv) inv[p] = pos;
+    }
+    __syncthreads();
+    for (int ee = tid; ee < E; ee += blockDim.x) base[ee] += scan_tmp[ee];
+    __syncthreads();
+  }
+}
+
+// ------------------------------------------------------------ activation casts -----
+// q = e4m3(fp32(x / s)); x bf16 (n), n % 8 == 0 not required.
+__global__ void __launch_bounds__(256) fp8_quant_kernel(const uint16_t* __restrict__ x, int64_t n,
+                                                         float s, uint8_t* __restrict__ q) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride)
+    q[i] = act_quant_e4m3(bf16_bits_to_f32(x[i]), s);
+}
+
+// The A-FP8 input of the register-dequant path: xq[i] = bf16 bits of e4m3(x[i] / s),
+// exact (every e4m3 value is a bf16 value). Vectorized by 8 (H % 32 == 0).
+__global__ void __launch_bounds__(256) fp8_quant_as_bf16_kernel(const uint4* __restrict__ x,
+                                                                 int64_t n8, float s,
+                                                                 uint4* __restrict__ xq) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8; i += stride) {
+    const uint4 v = x[i];
+    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float lo = e4m3_to_f32(act_quant_e4m3(__uint_as_float(in[j] << 16), s));
+      const float hi = e4m3_to_f32(act_quant_e4m3(__uint_as_float(in[j] & 0xFFFF0000u), s));
+      o[j] = (__float_as_uint(lo) >> 16) | (__float_as_uint(hi) & 0xFFFF0000u);
+    }
+    xq[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// Gather the e4m3 rows of the routed pairs into expert-grouped order:
+// a1[pos, :] = e4m3(x[perm_token[pos], :] / s) (one warp per row, 16 B per lane).
+__global__ void __launch_bounds__(256) gather_fp8_rows_kernel(const uint8_t* __restrict__ xq8,
+                                                               const int32_t* __restrict__ perm_token,
+                                                               int64_t P, int H,
+                                                               uint8_t* __restrict__ a1) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t pos = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; pos < P;
+       pos += nw) {
+    const int64_t t = perm_token[pos];
+    const uint4* src = reinterpret_cast<const uint4*>(xq8 + t * H);
+    uint4* dst = reinterpret_cast<uint4*>(a1 + pos * H);
+    for (int c = lane; c < H / 16; c += 32) dst[c] = src[c];
+  }
+}
+
+// amax |x| over a bf16 tensor, folded into *amax_bits (float bits; |x| >= 0 orders as int)
+__global__ void __launch_bounds__(256) amax_bf16_kernel(const uint16_t* __restrict__ x, int64_t n,
+                                                         unsigned* __restrict__ amax_bits) {
+  float m = 0.0f;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride)
+    m = fmaxf(m, fabsf(bf16_bits_to_f32(x[i])));
+  m = warp_max(m);
+  if ((threadIdx.x & 31) == 0) atomicMax(amax_bits, __float_as_uint(m));
+}
+
+__global__ void finalize_scales_kernel(const unsigned* __restrict__ amax_bits, float* __restrict__ out) {
+  if (threadIdx.x < 2) out[threadIdx.x] = __fdiv_rn(__uint_as_float(amax_bits[threadIdx.x]), 448.0f);
+}
+
+// ------------------------------------------------------------------- launchers -----
+cudaError_t launch_router(const uint16_t* x, const uint16_t* wr, const uint16_t* br, int T, int H,
+                          int E, float* logits, cudaStream_t st) {
+  if (T <= 32) {
+    const int64_t warps = static_cast<int64_t>(T) * E;
+    router_gemv_kernel<<<static_cast<unsigned>(cdiv(warps * 32, 256)), 256, 0, st>>>(x, wr, br, T, H, E, logits);
+  } else {
+    dim3 grid(static_cast<unsigned>(cdiv(T, rg::BM)), static_cast<unsigned>(cdiv(E, rg::BN)));
+    router_gemm_kernel<<<grid, 128, 0, st>>>(x, wr, br, T, H, E, logits);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_topk(const float* logits, int T, int E, int k, int32_t* idx, float* w,
+                        cudaStream_t st) {
+  topk_kernel<<<static_cast<unsigned>(cdiv(static_cast<int64_t>(T) * 32, 256)), 256, 0, st>>>(logits, T, E, k, idx, w);
+  return cudaGetLastError();
+}
+
+int permute_chunks(int64_t P) { return static_cast<int>(cdiv(P, kPermChunk)); }
+
+// counts_ws: int32 scratch of permute_chunks(P) * E entries (unused for one chunk).
+cudaError_t launch_permute(const int32_t* idx, int T, int E, int k, int32_t* counts_ws,
+                           int32_t* offsets, int32_t* perm_token, int32_t* perm_slot,
+                           int32_t* inv, int32_t* active, int32_t* n_active, int* err,
+                           cudaStream_t st, int* launches) {
+  const int64_t P = static_cast<int64_t>(T) * k;
+  const int nc = permute_chunks(P);
+  if (nc <= 1) {
+    permute_scatter_kernel<<<1, kPermThreads, 0, st>>>(idx, P, E, k, nullptr, offsets, perm_token,
+                                                       perm_slot, inv, active, n_active, err);
+    *launches += 1;
+  } else {
+    permute_count_kernel<<<nc, kPermThreads, 0, st>>>(idx, P, E, counts_ws);
+    permute_scatter_kernel<<<nc, kPermThreads, 0, st>>>(idx, P, E, k, counts_ws, offsets,
+                                                        perm_token, perm_slot, inv, active, n_active,
+                                                        err);
+    *launches += 2;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fp8_quant(const uint16_t* x, int64_t n, float s, uint8_t* q, cudaStream_t st,
+                             int sms) {
+  const int64_t g = cdiv(n, 256);
+  fp8_quant_kernel<<<static_cast<unsigned>(g < sms * 8 ? (g < 1 ? 1 : g) : sms * 8), 256, 0, st>>>(x, n, s, q);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fp8_quant_as_bf16(const uint16_t* x, int64_t n, float s, uint16_t* xq,
+                                     cudaStream_t st, int sms) {
+  const int64_t n8 = n / 8;
+  const int64_t g = cdiv(n8, 256);
+  fp8_quant_as_bf16_kernel<<<static_cast<unsigned>(g < sms * 8 ? (g < 1 ? 1 : g) : sms * 8), 256, 0, st>>>(
+      reinterpret_cast<const uint4*>(x), n8, s, reinterpret_cast<uint4*>(xq));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_fp8_rows(const uint8_t* xq8, const int32_t* perm_token, int64_t P, int H,
+                                   uint8_t* a1, cudaStream_t st, int sms) {
+  const int64_t g = cdiv(P * 32, 256);
+  gather_fp8_rows_kernel<<<static_cast<unsigned>(g < sms * 16 ? (g < 1 ? 1 : g) : sms * 16), 256, 0, st>>>(
+      xq8, perm_token, P, H, a1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_amax_bf16(const uint16_t* x, int64_t n, unsigned* amax_bits, cudaStream_t st,
+                             int sms) {
+  const int64_t g = cdiv(n, 256);
+  amax_bf16_kernel<<<static_cast<unsigned>(g < sms * 4 ? (g < 1 ? 1 : g) : sms * 4), 256, 0, st>>>(x, n, amax_bits);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_finalize_scales(const unsigned* amax_bits, float* out, cudaStream_t st) {
+  finalize_scales_kernel<<<1, 32, 0, st>>>(amax_bits, out);
+  return cudaGetLastError();
+}
+
+}  // namespace mxmoe

@@ -304,10 +304,13 @@ struct LayerArgs {
 };
 
 static void dequant_row(const uint8_t* blocks, const uint8_t* scales, int64_t K, double* out) {
-  for (int64_t k = 0; k < K; ++k) {
-    const uint8_t byte = blocks[k / 2];
-    const unsigned nib = (k % 2 == 0) ? (byte & 0x0Fu) : (byte >> 4);
-    out[k] = e2m1_value(nib) * std::ldexp(1.0, static_cast<int>(scales[k / 32]) - 127);
+  for (int64_t b = 0; b < K / 32; ++b) {
+    const double scale = std::ldexp(1.0, static_cast<int>(scales[b]) - 127);
+    for (int64_t k = 32 * b; k < 32 * b + 32; ++k) {
+      const uint8_t byte = blocks[k / 2];
+      const unsigned nib = (k % 2 == 0) ? (byte & 0x0Fu) : (byte >> 4);
+      out[k] = e2m1_value(nib) * scale;
+    }
   }
 }
 

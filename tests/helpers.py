@@ -70,3 +70,21 @@ def output_tolerance_ok(out_bits: np.ndarray, ref_acc: np.ndarray, rel: float = 
     err = np.abs(got - ref)
     excess = float(np.max(err - bound)) if ref.size else 0.0
     return bool(np.all(err <= bound)), float(np.max(err) / scale) if scale else 0.0, excess
+
+
+# ------------------------------------------------------------------ GPU helpers ----
+
+def to_device(p: Packed, device="cuda"):
+    """The packed layer as torch tensors on the GPU (bf16 bits become torch.bfloat16)."""
+    import torch
+    u8 = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+    f32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device)
+    bf = lambda a: None if a is None else inputs.from_bits(a, device)
+    return dict(x=bf(p.x), router_w=bf(p.router_w), router_b=bf(p.router_b),
+                gu_blocks=u8(p.gu_blocks), gu_scales=u8(p.gu_scales), gu_bias=f32(p.gu_bias),
+                d_blocks=u8(p.d_blocks), d_scales=u8(p.d_scales), d_bias=f32(p.d_bias))
+
+
+def gpu_bits(t) -> np.ndarray:
+    """bf16 CUDA tensor -> numpy uint16 bits."""
+    return inputs.bits(t)

@@ -1,0 +1,181 @@
+"""GPU parity of the whole MoE expert layer (moe_mxfp4_forward) against the oracle.
+
+Page "quantization_mxfp4" (KerasFormers), As GPT-OSS's native format (routed experts,
+(E, 2I, H) / (E, H, I) packed layout, full-precision biases); W-MXFP4/A-FP8 option from
+"amd/gpt-oss-20b-MoE-Quant-W-MXFP4-A-FP8-KV-FP8", Quantization schemes.
+
+Bar (stated for the layer output): |out - ref| <= 2e-3 * max|ref| + half a bf16 ulp of
+the reference element, where ref is the oracle's fp32 accumulator (the bf16 output
+carries one extra rounding the fp32 arithmetic does not). Routing indices are compared
+bit-exactly wherever the k-th and (k+1)-th router logits are not a near tie.
+
+Weights are MXFP4-packed by the oracle's quantizer; the GPU consumes the same bytes.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import Packed, output_tolerance_ok, pack, to_device
+from mxfp4_block_scaled_moe_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+_CACHE = {}
+
+
+def packed_weights(E, H, I, seed=0):
+    """Oracle-packed expert weights of a synthetic layer (cached per shape)."""
+    key = (E, H, I, seed)
+    if key not in _CACHE:
+        lay = inputs.small_layer(E=E, k=1, T=1, H=H, I=I, seed=seed, device="cuda")
+        p = pack(lay)
+        _CACHE[key] = (p, to_device(p))
+    return _CACHE[key]
+
+
+def layer_case(lay: inputs.Layer):
+    """Pair a layer's activations/router with the cached packed weights of its shape."""
+    wp, wd = packed_weights(lay.E, lay.H, lay.I, lay.seed)
+    rb = None if lay.router_b is None else inputs.bits(lay.router_b)
+    p = Packed(lay, inputs.bits(lay.x), inputs.bits(lay.router_w), rb, wp.gu_blocks,
+               wp.gu_scales, wp.gu_bias, wp.d_blocks, wp.d_scales, wp.d_bias)
+    d = dict(wd)
+    d.update(x=lay.x.contiguous(), router_w=lay.router_w.contiguous(),
+             router_b=None if lay.router_b is None else lay.router_b.contiguous())
+    return p, d
+
+
+@pytest.fixture(scope="module")
+def B():
+    from mxfp4_block_scaled_moe_b200 import binding
+    return binding
+
+
+def run_gpu(B, d, k, act_scale=None):
+    out = B.moe_mxfp4_forward(d["x"], d["router_w"], d["router_b"], d["gu_blocks"],
+                              d["gu_scales"], d["gu_bias"], d["d_blocks"], d["d_scales"],
+                              d["d_bias"], k, act_scale=act_scale)
+    B.mxmoe_check()
+    return out
+
+
+def check_rows(B, p: Packed, d, rows, act_scale=None, out=None):
+    """Compare the GPU output rows `rows` with the oracle, routing gaps respected."""
+    k = p.lay.k
+    if out is None:
+        out = run_gpu(B, d, k, act_scale)
+    got = inputs.bits(out)[rows]
+    ob, oacc, oidx, _ = p.oracle_forward(act_scale=act_scale, rows=rows)
+    # routing: the GPU's indices must equal the oracle's wherever the selection is clear
+    gi, _, gl = B.moe_route_topk(d["x"], d["router_w"], d["router_b"], k, with_logits=True)
+    gi = gi.cpu().numpy()[rows]
+    ol = oracle.router_logits(p.x[rows], p.router_w, p.router_b)
+    srt = -np.sort(-ol, axis=1)
+    clear = (srt[:, k - 1] - srt[:, k] > 1e-5 * np.abs(ol).max()) if p.lay.E > k else np.ones(len(rows), bool)
+    assert np.array_equal(gi[clear], oidx[clear])
+    ok, rel, excess = output_tolerance_ok(got[clear], oacc[clear])
+    assert ok, f"max|d|/max|ref| = {rel:.3e}, worst excess over the bound {excess:.3e}"
+    return rel
+
+
+def test_tiny_bf16_all_outputs(B):
+    p = pack(inputs.tiny_layer(seed=0))
+    d = to_device(p)
+    rel = check_rows(B, p, d, np.arange(p.lay.T))
+    assert rel < 2e-3
+
+
+def test_tiny_fp8_all_outputs(B):
+    p = pack(inputs.tiny_layer(seed=0))
+    d = to_device(p)
+    s = oracle.calibrate(p.x, p.router_w, p.router_b, *p.weights, p.lay.k)
+    check_rows(B, p, d, np.arange(p.lay.T), act_scale=s)
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_small_ragged_layer(B, fp8):
+    # H = 320 (10 blocks), I = 192 (6 blocks): neither a multiple of the 64-row tiles
+    p = pack(inputs.small_layer(E=8, k=3, T=77, H=320, I=192, seed=5, router_bias=True))
+    d = to_device(p)
+    s = oracle.calibrate(p.x, p.router_w, p.router_b, *p.weights, p.lay.k) if fp8 else None
+    check_rows(B, p, d, np.arange(p.lay.T), act_scale=s)
+
+
+@pytest.mark.parametrize("T", [1, 8, 64])
+def test_decode_20b_shape_all_outputs(B, T):
+    p, d = layer_case(inputs.decode_layer(T=T, E=32, device="cuda"))
+    check_rows(B, p, d, np.arange(T))
+
+
+def test_decode_23_experts(B):
+    p, d = layer_case(inputs.decode_layer(T=8, E=23, device="cuda"))
+    check_rows(B, p, d, np.arange(8))
+
+
+def _sample_rows(T, n, seed):
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.choice(T, size=n, replace=False))
+    rows[0], rows[-1] = 0, T - 1
+    return rows
+
+
+def test_prefill_120b_shape_fp8_sampled(B):
+    lay = inputs.prefill_layer(T=4096, E=128, device="cuda")
+    p, d = layer_case(lay)
+    xc = inputs.calibration_x(device="cuda")
+    s = oracle.calibrate(inputs.bits(xc), p.router_w, p.router_b, *p.weights, lay.k)
+    out1 = run_gpu(B, d, lay.k, act_scale=s)
+    out2 = run_gpu(B, d, lay.k, act_scale=s)
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))   # run-to-run identical
+    check_rows(B, p, d, _sample_rows(4096, 24, 1), act_scale=s, out=out1)
+
+
+def test_prefill_zipf_skew_sampled(B):
+    lay = inputs.zipf_layer(T=16384, E=128, device="cuda")
+    p, d = layer_case(lay)
+    idx, _ = B.moe_route_topk(d["x"], d["router_w"], d["router_b"], lay.k)
+    load = np.bincount(idx.cpu().numpy().reshape(-1), minlength=lay.E)
+    assert (load == 0).sum() >= 3 and load.max() > 10 * load.mean()
+    xc = inputs.calibration_x(device="cuda")
+    s = oracle.calibrate(inputs.bits(xc), p.router_w, p.router_b, *p.weights, lay.k)
+    hot = int(np.argmax(load))
+    rows = np.unique(np.concatenate([_sample_rows(16384, 12, 2),
+                                     np.nonzero((idx.cpu().numpy() == hot).any(1))[0][:4]]))
+    check_rows(B, p, d, rows, act_scale=s)
+
+
+def test_calibration_matches_oracle(B):
+    lay = inputs.decode_layer(T=1, E=32, device="cuda")
+    p, d = layer_case(lay)
+    xc = inputs.calibration_x(device="cuda")
+    g = B.moe_mxfp4_calibrate(xc, d["router_w"], d["router_b"], d["gu_blocks"], d["gu_scales"],
+                              d["gu_bias"], d["d_blocks"], d["d_scales"], d["d_bias"], lay.k).cpu().numpy()
+    o = oracle.calibrate(inputs.bits(xc), p.router_w, p.router_b, *p.weights, lay.k)
+    assert g[0] == o[0]
+    assert abs(g[1] - o[1]) <= 1e-5 * o[1]
+
+
+def test_empty_batch_and_bad_arguments(B):
+    p = pack(inputs.tiny_layer(seed=0))
+    d = to_device(p)
+    empty = dict(d, x=d["x"][:0])
+    out = B.moe_mxfp4_forward(empty["x"], d["router_w"], d["router_b"], d["gu_blocks"],
+                              d["gu_scales"], d["gu_bias"], d["d_blocks"], d["d_scales"],
+                              d["d_bias"], 2)
+    assert out.shape == (0, 256)
+    L = B.lib()
+    vp = lambda t: torch.cuda.current_stream().cuda_stream if t is None else t.data_ptr()
+    args = [d[n].data_ptr() for n in ("x", "router_w", "router_b", "gu_blocks", "gu_scales",
+                                       "gu_bias", "d_blocks", "d_scales", "d_bias")]
+    o = torch.empty(16, 256, dtype=torch.bfloat16, device="cuda")
+    import ctypes
+    c = [ctypes.c_void_p(a) for a in args]
+    assert L.moe_mxfp4_forward(*c, 4, 5, 16, 256, 256, None, ctypes.c_void_p(o.data_ptr()), None) == B.EUNSUPPORTED
+    assert L.moe_mxfp4_forward(*c, 4, 2, 16, 250, 256, None, ctypes.c_void_p(o.data_ptr()), None) == B.EALIGN
+    assert L.moe_mxfp4_forward(*c, 4, 2, 16, 256, 200, None, ctypes.c_void_p(o.data_ptr()), None) == B.EALIGN
+    assert L.moe_mxfp4_forward(*c, 300, 2, 16, 256, 256, None, ctypes.c_void_p(o.data_ptr()), None) == B.EUNSUPPORTED
+    c_bad = list(c)
+    c_bad[0] = ctypes.c_void_p(args[0] + 2)
+    assert L.moe_mxfp4_forward(*c_bad, 4, 2, 16, 256, 256, None, ctypes.c_void_p(o.data_ptr()), None) == B.EINVAL
+    assert L.moe_mxfp4_forward(*c, 4, 2, 16, 256, 256, None, None, None) == B.EINVAL
