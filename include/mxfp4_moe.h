@@ -157,8 +157,9 @@ int mxmoe_last_launch_count(void);
 /* mxmoe_profile_enable -- on != 0: from now on every moe_mxfp4_forward on this host
  * thread records a CUDA event on its stream before its first kernel and after each stage
  * (router, topk, permute, act_quant, gate_up, down, combine, ...); on == 0 stops. Either
- * call discards marks not yet read. Timing only: the results are unchanged. Returns
- * MXMOE_OK. Recording is not allowed while the stream is being captured into a graph. */
+ * call discards marks not yet read. Timing only: the results are unchanged. Inside a
+ * stream capture the records become event nodes of the graph, so a read after a replay
+ * reports that replay. Returns MXMOE_OK. */
 int mxmoe_profile_enable(int on);
 
 /* mxmoe_profile_read -- wait for the recorded events and report, per stage name, the

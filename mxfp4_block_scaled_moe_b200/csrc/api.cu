@@ -7,6 +7,7 @@
 #include <cstdio>
 #include <cstdarg>
 #include <cstring>
+#include <cstdlib>
 
 #include "common.cuh"
 #include "launchers.h"
@@ -41,14 +42,16 @@ cudaEvent_t next_event() {
 struct StageTimer {
   cudaStream_t st;
   cudaEvent_t last = nullptr;
+  // cudaEventRecordExternal: inside a stream capture the record becomes an event node of
+  // the graph (timed at every replay); outside a capture it is a plain record.
   explicit StageTimer(cudaStream_t s) : st(s) {
-    if (t_profile && (last = next_event())) cudaEventRecord(last, st);
+    if (t_profile && (last = next_event())) cudaEventRecordWithFlags(last, st, cudaEventRecordExternal);
   }
   void mark(const char* name) {
     if (!t_profile || !last) return;
     cudaEvent_t e = next_event();
     if (!e) return;
-    cudaEventRecord(e, st);
+    cudaEventRecordWithFlags(e, st, cudaEventRecordExternal);
     t_marks.push_back({name, last, e});
     last = e;
   }
@@ -77,7 +80,20 @@ struct Workspace {
   int* err = nullptr;  // device error word
   int sms = 0;
   int smem_K = 0;      // largest K the expert kernels were configured for
+  bool tc_ready = false;  // tcgen05 GEMM shared-memory limit raised
 };
+
+// Routed pairs from which the FP8 path runs on the tcgen05 grouped GEMM (fewer pairs use
+// the register-dequant kernels). MXMOE_TC_MIN_PAIRS overrides it (0 = always when the
+// shapes allow, a huge value = never).
+int64_t tc_min_pairs() {
+  static int64_t v = [] {
+    const char* s = std::getenv("MXMOE_TC_MIN_PAIRS");
+    return s ? std::atoll(s) : 1024LL;
+  }();
+  return v;
+}
+constexpr int kTcMaxNb = 144;   // K <= 4608 keeps the GEMM's shared memory within 227 KB
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
@@ -146,9 +162,12 @@ struct LayerBuffers {
   uint16_t* act_mid;   // (P, I) bf16 bits of the down-projection input
   float* y;            // (P, H) fp32 expert outputs
   unsigned* amax;      // 2 x fp32 bits (calibration)
+  uint8_t* xq8;        // tcgen05 path: e4m3 codes of x / s0, (T, H)
+  uint8_t* a1;         // tcgen05 path: gate_up input rows grouped by expert, (P, H)
+  uint8_t* a2;         // tcgen05 path: down input rows, (P, I)
 };
 
-size_t layout(int T, int E, int k, int H, int I, bool fp8, LayerBuffers* b, char* base) {
+size_t layout(int T, int E, int k, int H, int I, bool fp8, bool tc, LayerBuffers* b, char* base) {
   const int64_t P = static_cast<int64_t>(T) * k;
   Carve c;
   size_t o_logits = c.take<float>(static_cast<int64_t>(T) * E);
@@ -157,9 +176,12 @@ size_t layout(int T, int E, int k, int H, int I, bool fp8, LayerBuffers* b, char
   size_t o_off = c.take<int32_t>(E + 1), o_act = c.take<int32_t>(E), o_nact = c.take<int32_t>(1);
   size_t o_pt = c.take<int32_t>(P), o_ps = c.take<int32_t>(P), o_inv = c.take<int32_t>(P);
   size_t o_xq = c.take<uint16_t>(fp8 ? static_cast<int64_t>(T) * H : 0);
-  size_t o_mid = c.take<uint16_t>(P * I);
+  size_t o_mid = c.take<uint16_t>(tc ? 0 : P * I);
   size_t o_y = c.take<float>(P * H);
   size_t o_amax = c.take<unsigned>(2);
+  size_t o_xq8 = c.take<uint8_t>(tc ? static_cast<int64_t>(T) * H : 0);
+  size_t o_a1 = c.take<uint8_t>(tc ? P * H : 0);
+  size_t o_a2 = c.take<uint8_t>(tc ? P * I : 0);
   if (b) {
     b->logits = reinterpret_cast<float*>(base + o_logits);
     b->topk_idx = reinterpret_cast<int32_t*>(base + o_idx);
@@ -175,6 +197,9 @@ size_t layout(int T, int E, int k, int H, int I, bool fp8, LayerBuffers* b, char
     b->act_mid = reinterpret_cast<uint16_t*>(base + o_mid);
     b->y = reinterpret_cast<float*>(base + o_y);
     b->amax = reinterpret_cast<unsigned*>(base + o_amax);
+    b->xq8 = reinterpret_cast<uint8_t*>(base + o_xq8);
+    b->a1 = reinterpret_cast<uint8_t*>(base + o_a1);
+    b->a2 = reinterpret_cast<uint8_t*>(base + o_a2);
   }
   return c.off;
 }
@@ -226,16 +251,23 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
   Workspace* ws = nullptr;
   if (int rc = current_device_ws(&ws)) return rc;
   const bool fp8 = act_scale != nullptr;
-  const size_t need = layout(a.T, a.E, a.k, a.H, a.I, fp8, nullptr, nullptr);
+  const int64_t P = static_cast<int64_t>(a.T) * a.k;
+  const bool tc = fp8 && !calib_out && P >= tc_min_pairs() && std::max(a.H, a.I) / 32 <= kTcMaxNb &&
+                  tc_gemm_supported(a.H, a.I, a.gu_blocks, a.d_blocks);
+  const size_t need = layout(a.T, a.E, a.k, a.H, a.I, fp8, tc, nullptr, nullptr);
   if (int rc = ensure_capacity(ws, need)) return rc;
   if (std::max(a.H, a.I) > ws->smem_K) {
     cudaError_t e = expert_mma_set_smem_limits(std::max(a.H, a.I));
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
     ws->smem_K = std::max(a.H, a.I);
   }
+  if (tc && !ws->tc_ready) {
+    cudaError_t e = tc_gemm_prepare(kTcMaxNb, 256);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (tcgen05 GEMM)");
+    ws->tc_ready = true;
+  }
   LayerBuffers b;
-  layout(a.T, a.E, a.k, a.H, a.I, fp8, &b, ws->base);
-  const int64_t P = static_cast<int64_t>(a.T) * a.k;
+  layout(a.T, a.E, a.k, a.H, a.I, fp8, tc, &b, ws->base);
   int launches = 0;
   cudaError_t e;
   const float s0 = fp8 ? act_scale[0] : 1.0f, s1 = fp8 ? act_scale[1] : 1.0f;
@@ -251,6 +283,31 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
                           b.inv, b.active, b.n_active, ws->err, st, &launches)))
     return cuda_fail(e, "permute");
   tm.mark("permute");
+  if (tc) {
+    if ((e = launch_fp8_quant(a.x, static_cast<int64_t>(a.T) * a.H, s0, b.xq8, st, ws->sms)))
+      return cuda_fail(e, "fp8 activation cast");
+    ++launches;
+    tm.mark("act_quant");
+    if ((e = launch_gather_fp8_rows(b.xq8, b.perm_token, P, a.H, b.a1, st, ws->sms))) return cuda_fail(e, "gather");
+    ++launches;
+    tm.mark("gather");
+    if ((e = launch_tc_gemm(true, b.a1, P, a.H, a.gu_blocks, a.gu_scales, a.gu_bias, a.E, a.I, b.offsets, s0, s1,
+                            b.a2, nullptr, ws->err, ws->sms, st)))
+      return cuda_fail(e, "gate_up (tcgen05)");
+    ++launches;
+    tm.mark("gate_up");
+    if ((e = launch_tc_gemm(false, b.a2, P, a.I, a.d_blocks, a.d_scales, a.d_bias, a.E, a.H, b.offsets, s1, 0.0f,
+                            nullptr, b.y, ws->err, ws->sms, st)))
+      return cuda_fail(e, "down (tcgen05)");
+    ++launches;
+    tm.mark("down");
+    if ((e = launch_combine(b.y, b.topk_idx, b.topk_w, b.inv, a.T, a.H, a.k, out, st, ws->sms)))
+      return cuda_fail(e, "combine");
+    ++launches;
+    tm.mark("combine");
+    t_last_launches = launches;
+    return MXMOE_OK;
+  }
   const uint16_t* act_in = a.x;
   if (fp8) {
     if ((e = launch_fp8_quant_as_bf16(a.x, static_cast<int64_t>(a.T) * a.H, s0, b.xq, st, ws->sms)))

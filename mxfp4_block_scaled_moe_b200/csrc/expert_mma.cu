@@ -30,7 +30,7 @@ namespace mxmoe {
 namespace {
 
 constexpr int kWarps = 4;       // warps per CTA
-constexpr int kUnroll = 8;      // 32-value blocks whose weight words are loaded ahead
+constexpr int kUnroll = 16;     // 32-value blocks whose weight words are loaded ahead
 
 __device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
   uint32_t d;
@@ -105,12 +105,33 @@ __global__ void __launch_bounds__(kWarps * 32) expert_mma_kernel(ExpertGemmArgs 
   const uint8_t* wlo = p.blocks + (erow + row_lo) * (p.K / 2) + 4 * t;
   const uint8_t* whi = p.blocks + (erow + row_hi) * (p.K / 2) + 4 * t;
 
-  // stage this warp's 16 rows of scales as fp32 (row slot 0..7 = lo rows, 8..15 = hi rows)
+  // stage this warp's 16 rows of scales as fp32 (row slot 0..7 = lo rows, 8..15 = hi
+  // rows). The 8 lo rows (and the 8 hi rows) are 8 * nb contiguous bytes: load them with
+  // 16-byte loads when aligned so that all of them are in flight at once.
   float* sc = s_scale + static_cast<int64_t>(warp) * 16 * nb;
-  for (int i = lane; i < 16 * nb; i += 32) {
-    const int r = i / nb, b = i % nb;
-    const int row = (r < 8) ? (row_lo - g + r) : (row_hi - g + (r - 8));
-    sc[i] = e8m0_to_f32(p.scales[(erow + row) * nb + b]);
+  {
+    const uint8_t* half_src[2] = {p.scales + (erow + row_lo - g) * nb,
+                                  p.scales + (erow + row_hi - g) * nb};
+    const int half_bytes = 8 * nb;
+    const bool vec = ((reinterpret_cast<uintptr_t>(half_src[0]) | reinterpret_cast<uintptr_t>(half_src[1]) |
+                       static_cast<uintptr_t>(half_bytes)) & 15u) == 0;
+    if (vec) {
+      const int n16 = half_bytes / 16;
+      for (int c = lane; c < 2 * n16; c += 32) {
+        const int h = c >= n16 ? 1 : 0, o = (c - h * n16) * 16;
+        const uint4 v = ld_nc_v4(half_src[h] + o);
+        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+        float* dst = sc + h * half_bytes + o;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) dst[j] = e8m0_to_f32((wv[j >> 2] >> (8 * (j & 3))) & 0xFFu);
+      }
+    } else {
+#pragma unroll 8
+      for (int i = lane; i < 2 * half_bytes; i += 32) {
+        const int h = i >= half_bytes ? 1 : 0;
+        sc[i] = e8m0_to_f32(half_src[h][i - h * half_bytes]);
+      }
+    }
   }
   __syncwarp();
   const float* sc_lo = sc + g * nb;

@@ -1,0 +1,625 @@
+// Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05) with block-scaled
+// MXFP4 weights and FP8 E4M3 activations: the prefill path of the W-MXFP4 / A-FP8 layer.
+//
+// Pages: "quantization_mxfp4" (KerasFormers), As GPT-OSS's native format (gate_up_proj
+// (E, 2I, H) and down_proj (E, H, I) as e2m1 blocks + one e8m0 scale per 32 values along
+// the contracting dim, biases in full precision); "amd/gpt-oss-20b-MoE-Quant-W-MXFP4-A-
+// FP8-KV-FP8", Quantization schemes (FP8 per-tensor activations).
+//
+// One kernel, two epilogues:
+//   gate_up: acc = A1_e . Wgu_e^T on [gate rows n0.., up rows I+n0..]; a = silu(s0*acc_g
+//            + b_g) * (s0*acc_u + b_u); A2 = e4m3(a / s1)            (bytes, (P, I))
+//   down:    acc = A2_e . Wd_e^T;  y = s1 * acc + b_d                 (fp32, (P, H))
+// where A1 / A2 hold the routed rows grouped by expert (offsets[e] .. offsets[e+1]).
+//
+// MMA: tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale, M = 128, N = 240, K = 32 per
+// instruction, fp32 accumulators in tensor memory. A (e4m3) carries unit scales (e8m0
+// 127) and its per-tensor scale is applied in the epilogue; B (e2m1) carries the
+// checkpoint's e8m0 block scales. Operands arrive by TMA with 128-byte swizzle; the e2m1
+// weights use the 4-bit "16 x U4 in 16 bytes" tensor-map type, which spreads each 8 packed
+// bytes over 16 bytes of shared memory as the kind::mxf8f6f4 operand layout requires.
+// K = 2880 is 22.5 tiles of 128: the last tile reads the final 128 values through a
+// second tensor map and issues only its last two K-steps.
+//
+// Scale factors: a converter warp copies the tile's raw scale rows into shared memory
+// once per output tile and, per pipeline stage, rewrites the stage's 4 k-blocks into the
+// 512-byte atoms that tcgen05.cp (32x128b, 4 warp-quarters) moves into tensor memory:
+// row r of an atom at byte 16*(r%32) + 4*(r/32) + j for k-block j.
+//
+// Roles (256 threads, one CTA per SM, persistent over the tile list):
+//   warp 0: TMA producer          warp 1: TMEM owner + MMA issuer (one thread)
+//   warp 2: scale converter       warp 3: builds the tile schedule, then idles
+//   warps 4-7: epilogue (TMEM lane quarter = warp % 4)
+// Every mbarrier wait gives up after ~1 s (clock64): the kernel then records MXMOE_ETIMEOUT
+// in the error word, lets in-flight copies land, frees its tensor memory and returns.
+#include <cuda.h>
+
+#include "common.cuh"
+
+namespace mxmoe {
+namespace g100 {
+
+constexpr int BM = 128;             // rows of A per tile (MMA M)
+constexpr int BN = 240;             // MMA N (gate_up: 120 gate + 120 up rows)
+constexpr int BK = 128;             // K values per pipeline stage
+constexpr int kStages = 4;
+constexpr int kThreads = 256;
+constexpr int kAStage = BM * BK;            // 16 KB (e4m3, one byte per value)
+constexpr int kBStage = BN * BK;            // 30 KB (e2m1 spread to one byte per value)
+constexpr int kSfStage = 1024;              // two 512-byte scale atoms (rows 0..255)
+constexpr int kAccCols = 256;               // column stride between the two accumulators
+constexpr int kTmemCols = 512;
+constexpr int kSfaCol = 496;                // 4 columns of unit A scales
+constexpr int kSfbCol = 504;                // 8 columns of B scales (rows 0..255)
+constexpr long long kWaitCycles = 2000000000LL;  // ~1 s at the B200 clock
+
+struct Params {
+  const uint8_t* b_scales;   // raw e8m0 scales, (groups, rows_per_group, nb)
+  const float* bias;         // (E, rows_total)
+  const int32_t* offsets;    // (E+1)
+  int E;
+  int K;                     // contracting length (multiple of 64)
+  int nb;                    // K / 32
+  int rows_per_group;        // gate_up: I (one half); down: H
+  int rows_total;            // bias row length: gate_up 2I, down H
+  int n_out;                 // gate_up: I; down: H
+  int n_tiles;               // output tiles along N per m-tile
+  int nk_full;               // K / 128
+  int tail_steps;            // K-steps of 32 in the final partial tile (0 or 2)
+  float s_in;                // scale of the A operand (s0 gate_up / s1 down)
+  float s_out;               // gate_up: quantization scale s1 of a
+  uint8_t* a_out;            // gate_up output (P, I) e4m3
+  float* y_out;              // down output (P, H) fp32
+  int* err;
+};
+
+// ------------------------------------------------------------------ PTX wrappers ---
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait. Returns false (after flagging the error and the CTA abort word) on timeout.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          int* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitCycles) {
+      *abort_flag = 1;
+      set_device_error(err, MXMOE_ETIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];\n" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];\n" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;\n" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+__device__ __forceinline__ void tc_mma_mxf8f6f4(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n}\n" ::"r"(d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_ld_32x32b_x8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+
+// The registers a tcgen05.ld fills are only valid after tcgen05.wait::ld; passing them
+// through the wait as in/out operands keeps the compiler from reading them earlier.
+__device__ __forceinline__ void tc_wait_ld(uint32_t (&a)[8]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n"
+               : "+r"(a[0]), "+r"(a[1]), "+r"(a[2]), "+r"(a[3]), "+r"(a[4]), "+r"(a[5]), "+r"(a[6]), "+r"(a[7])
+               :
+               : "memory");
+}
+__device__ __forceinline__ void tc_wait_ld(uint32_t (&a)[8], uint32_t (&b)[8]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n"
+               : "+r"(a[0]), "+r"(a[1]), "+r"(a[2]), "+r"(a[3]), "+r"(a[4]), "+r"(a[5]), "+r"(a[6]), "+r"(a[7]),
+                 "+r"(b[0]), "+r"(b[1]), "+r"(b[2]), "+r"(b[3]), "+r"(b[4]), "+r"(b[5]), "+r"(b[6]), "+r"(b[7])
+               :
+               : "memory");
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(count) : "memory");
+}
+
+// Shared-memory matrix descriptor (tcgen05): start, leading/stride byte offsets (>>4),
+// version 1, layout type (0 = no swizzle, 2 = 128-byte swizzle).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= 1ull << 46;
+  d |= static_cast<uint64_t>(layout & 7u) << 61;
+  return d;
+}
+
+// Instruction descriptor, kind::mxf8f6f4 block-scaled: A = E4M3 (0), B = E2M1 (5), both
+// K-major, N/8 at bits 17..22, scale type E8M0 (bit 23), M/16 at bits 24..28, scale-factor
+// byte ids of A (bits 29..30) and B (bits 4..5).
+__host__ __device__ constexpr uint32_t idesc_mxf8f6f4(int M, int N) {
+  return (0u << 7) | (5u << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// ---------------------------------------------------------------- tile schedule ---
+struct Tile {
+  int e, mt, nt, m0, rows;  // expert, m-tile, n-tile, first grouped row, valid rows
+};
+
+__device__ __forceinline__ Tile tile_of(int t, const int* prefix, const int32_t* offsets, int E, int n_tiles) {
+  int lo = 0, hi = E;  // largest e with prefix[e] <= t
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (prefix[mid] <= t) lo = mid; else hi = mid;
+  }
+  // skip experts with no tiles (equal prefixes)
+  int e = lo;
+  while (e + 1 < E && prefix[e + 1] <= t) ++e;
+  const int rem = t - prefix[e];
+  Tile tl;
+  tl.e = e;
+  tl.mt = rem / n_tiles;
+  tl.nt = rem % n_tiles;
+  const int off = offsets[e];
+  tl.m0 = off + tl.mt * BM;
+  tl.rows = min(BM, offsets[e + 1] - tl.m0);
+  return tl;
+}
+
+// ------------------------------------------------------------------------ kernel ---
+template <bool kGateUp>
+__global__ void __launch_bounds__(kThreads, 1)
+moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                const __grid_constant__ CUtensorMap tmap_bt, Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + kStages * kAStage;
+  uint8_t* sSF = sB + kStages * kBStage;
+  uint8_t* sSFA = sSF + kStages * kSfStage;       // 512 B of unit scales
+  uint8_t* sRaw = sSFA + 512;                     // BN * nb raw scale bytes
+  const int raw_bytes = ((BN * p.nb) + 15) & ~15;
+  float* sBias = reinterpret_cast<float*>(sRaw + raw_bytes);     // BN floats
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sBias + BN);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kStages;
+  uint64_t* acc_full = bars + 2 * kStages;
+  uint64_t* acc_empty = acc_full + 2;
+  int* prefix = reinterpret_cast<int*>(acc_empty + 2);           // E + 1
+  volatile int* abort_flag = prefix + (p.E + 1);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(prefix + p.E + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bn_rows = kGateUp ? BN / 2 : BN;      // rows per B load (one half for gate_up)
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 2);     // TMA producer (expect_tx) + scale converter
+      mbar_init(&empty[s], 1);    // MMA commit
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);  // one arrive per epilogue warp
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  if (warp == 3) {
+    // tile schedule: prefix[e] = number of tiles of experts < e
+    int carry = 0;
+    for (int e0 = 0; e0 < p.E; e0 += 32) {
+      const int e = e0 + lane;
+      const int m = e < p.E ? p.offsets[e + 1] - p.offsets[e] : 0;
+      const int tiles = ((m + BM - 1) / BM) * p.n_tiles;
+      int incl = tiles;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+      }
+      if (e < p.E) prefix[e] = carry + incl - tiles;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) prefix[p.E] = carry;
+  }
+  if (warp == 1) {
+    // tensor memory: 512 columns (two 240-column accumulators + scale factors)
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(tmem_holder)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n");
+    // unit A scales (e8m0 127) in the atom layout, then into tensor memory below
+    for (int i = lane; i < 128; i += 32) reinterpret_cast<uint32_t*>(sSFA)[i] = 0x7F7F7F7Fu;
+    fence_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int total_tiles = prefix[p.E];
+  const int nkt = p.nk_full + (p.tail_steps > 0 ? 1 : 0);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer -----
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      const uint32_t tx = kAStage + (kGateUp ? 2 : 1) * bn_rows * (BK / 2);
+      for (int t = blockIdx.x; t < total_tiles && !*abort_flag; t += gridDim.x) {
+        const Tile tl = tile_of(t, prefix, p.offsets, p.E, p.n_tiles);
+        const int n0 = tl.nt * bn_rows;
+        for (int kt = 0; kt < nkt; ++kt) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err)) break;
+          mbar_arrive_expect_tx(&full[stage], tx);
+          const bool tail = kt >= p.nk_full;
+          const CUtensorMap* mb = tail ? &tmap_bt : &tmap_b;
+          const int kx = tail ? p.K - BK : kt * BK;
+          const int bx = tail ? 0 : kt * BK;
+          tma_load_2d(sA + stage * kAStage, &tmap_a, &full[stage], kx, tl.m0);
+          if (kGateUp) {
+            tma_load_3d(sB + stage * kBStage, mb, &full[stage], bx, n0, 2 * tl.e);
+            tma_load_3d(sB + stage * kBStage + bn_rows * BK, mb, &full[stage], bx, n0, 2 * tl.e + 1);
+          } else {
+            tma_load_3d(sB + stage * kBStage, mb, &full[stage], bx, n0, tl.e);
+          }
+          if (++stage == kStages) { stage = 0; phase ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issuer -----
+    if (lane == 0) {
+      tc_fence_after();
+      tc_cp_32x128b_x4(tmem + kSfaCol, smem_desc(smem_u32(sSFA), 0, 128, 0));
+    }
+    __syncwarp();
+    int stage = 0;
+    uint32_t phase = 0;
+    int it = 0;
+    const uint32_t idesc0 = idesc_mxf8f6f4(BM, BN);
+    for (int t = blockIdx.x; t < total_tiles && !*abort_flag; t += gridDim.x, ++it) {
+      const int ab = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      if (!mbar_wait(&acc_empty[ab], acc_phase ^ 1, abort_flag, p.err)) break;
+      tc_fence_after();
+      const uint32_t dacc = tmem + ab * kAccCols;
+      bool ok = true;
+      for (int kt = 0; kt < nkt; ++kt) {
+        if (!mbar_wait(&full[stage], phase, abort_flag, p.err)) { ok = false; break; }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t sf = smem_u32(sSF + stage * kSfStage);
+          tc_cp_32x128b_x4(tmem + kSfbCol, smem_desc(sf, 0, 128, 0));
+          tc_cp_32x128b_x4(tmem + kSfbCol + 4, smem_desc(sf + 512, 0, 128, 0));
+          const uint32_t a0 = smem_u32(sA + stage * kAStage), b0 = smem_u32(sB + stage * kBStage);
+          const int first = kt < p.nk_full ? 0 : 4 - p.tail_steps;
+          for (int kk = first; kk < 4; ++kk) {
+            const uint64_t ad = smem_desc(a0 + 32 * kk, 16, 1024, 2);
+            const uint64_t bd = smem_desc(b0 + 32 * kk, 16, 1024, 2);
+            const uint32_t id = idesc0 | (static_cast<uint32_t>(kk) << 4) | (static_cast<uint32_t>(kk) << 29);
+            const uint32_t sel = static_cast<uint32_t>(kk) << 30;
+            tc_mma_mxf8f6f4(dacc, ad, bd, id, (tmem + kSfaCol) | sel, (tmem + kSfbCol) | sel,
+                            (kt > 0 || kk > first) ? 1u : 0u);
+          }
+          tc_commit(&empty[stage]);
+        }
+        __syncwarp();
+        if (++stage == kStages) { stage = 0; phase ^= 1; }
+      }
+      if (!ok) break;
+      if (lane == 0) tc_commit(&acc_full[ab]);
+      __syncwarp();
+    }
+  } else if (warp == 2) {
+    // --------------------------------------------------------- scale converter -----
+    int stage = 0;
+    uint32_t phase = 0;
+    const int nb = p.nb;
+    for (int t = blockIdx.x; t < total_tiles && !*abort_flag; t += gridDim.x) {
+      const Tile tl = tile_of(t, prefix, p.offsets, p.E, p.n_tiles);
+      const int n0 = tl.nt * bn_rows;
+      // raw scale rows of this tile into shared memory (row r of the tile: r < bn_rows is
+      // the first half / whole tile, r >= bn_rows the up half of gate_up)
+      const int halves = kGateUp ? 2 : 1;
+      const int valid = min(bn_rows, p.rows_per_group - n0);
+      for (int h = 0; h < halves; ++h) {
+        const int group = kGateUp ? 2 * tl.e + h : tl.e;
+        const uint8_t* src = p.b_scales + (static_cast<int64_t>(group) * p.rows_per_group + n0) * nb;
+        uint8_t* dst = sRaw + h * bn_rows * nb;
+        const int bytes = valid * nb;
+        if (((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & 15u) == 0) {
+          for (int c = lane; c < bytes / 16; c += 32)
+            reinterpret_cast<uint4*>(dst)[c] = ld_nc_v4(src + 16 * c);
+          for (int c = (bytes / 16) * 16 + lane; c < bytes; c += 32) dst[c] = src[c];
+        } else {
+          for (int c = lane; c < bytes; c += 32) dst[c] = src[c];
+        }
+      }
+      __syncwarp();
+      for (int kt = 0; kt < nkt; ++kt) {
+        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err)) break;
+        const int kb0 = kt < p.nk_full ? 4 * kt : nb - 4;
+        uint32_t* atom = reinterpret_cast<uint32_t*>(sSF + stage * kSfStage);
+        for (int r = lane; r < 256; r += 32) {
+          uint32_t word = 0x7F7F7F7Fu;
+          const int h = r / bn_rows, rr = r - h * bn_rows;
+          if (r < BN && rr < valid) {
+            const uint8_t* s = sRaw + (h * bn_rows + rr) * nb + kb0;
+            word = static_cast<uint32_t>(s[0]) | (static_cast<uint32_t>(s[1]) << 8) |
+                   (static_cast<uint32_t>(s[2]) << 16) | (static_cast<uint32_t>(s[3]) << 24);
+          }
+          const int a = r >> 7, m = r & 127;
+          atom[(a * 512 + (m & 31) * 16 + (m >> 5) * 4) >> 2] = word;
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&full[stage]);
+        if (++stage == kStages) { stage = 0; phase ^= 1; }
+      }
+      __syncwarp();
+    }
+  } else if (warp >= 4) {
+    // --------------------------------------------------------------- epilogue -----
+    const int q = warp & 3;            // tensor-memory lane quarter of this warp
+    const int row = 32 * q + lane;     // tile row = TMEM lane
+    const int et = threadIdx.x - 128;  // 0..127
+    int it = 0;
+    for (int t = blockIdx.x; t < total_tiles && !*abort_flag; t += gridDim.x, ++it) {
+      const Tile tl = tile_of(t, prefix, p.offsets, p.E, p.n_tiles);
+      const int n0 = tl.nt * bn_rows;
+      const int ab = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      named_bar_sync(1, 128);          // previous tile's bias reads are done
+      for (int j = et; j < BN; j += 128) {
+        float b = 0.0f;
+        if (kGateUp) {
+          const int h = j / bn_rows, c = n0 + (j - h * bn_rows);
+          if (c < p.n_out) b = p.bias[static_cast<int64_t>(tl.e) * p.rows_total + h * p.n_out + c];
+        } else {
+          const int c = n0 + j;
+          if (c < p.n_out) b = p.bias[static_cast<int64_t>(tl.e) * p.rows_total + c];
+        }
+        sBias[j] = b;
+      }
+      named_bar_sync(1, 128);
+      if (!mbar_wait(&acc_full[ab], acc_phase, abort_flag, p.err)) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem + ab * kAccCols + (static_cast<uint32_t>(32 * q) << 16);
+      const bool valid = row < tl.rows;
+      const int64_t pos = tl.m0 + row;
+      if (kGateUp) {
+        for (int c0 = 0; c0 < bn_rows; c0 += 8) {
+          uint32_t g[8], u[8];
+          tc_ld_32x32b_x8(tbase + c0, g);
+          tc_ld_32x32b_x8(tbase + bn_rows + c0, u);
+          tc_wait_ld(g, u);
+          uint32_t lo = 0, hi = 0;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float gv = __fadd_rn(__fmul_rn(p.s_in, __uint_as_float(g[i])), sBias[c0 + i]);
+            const float uv = __fadd_rn(__fmul_rn(p.s_in, __uint_as_float(u[i])), sBias[bn_rows + c0 + i]);
+            const uint32_t qb = act_quant_e4m3(silu_mul(gv, uv), p.s_out);
+            if (i < 4) lo |= qb << (8 * i); else hi |= qb << (8 * (i - 4));
+          }
+          if (valid && n0 + c0 < p.n_out)
+            *reinterpret_cast<uint2*>(p.a_out + pos * p.n_out + n0 + c0) = make_uint2(lo, hi);
+        }
+      } else {
+        for (int c0 = 0; c0 < BN; c0 += 8) {
+          uint32_t v[8];
+          tc_ld_32x32b_x8(tbase + c0, v);
+          tc_wait_ld(v);
+          float o[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) o[i] = __fadd_rn(__fmul_rn(p.s_in, __uint_as_float(v[i])), sBias[c0 + i]);
+          if (valid && n0 + c0 < p.n_out) {
+            float4* dst = reinterpret_cast<float4*>(p.y_out + pos * p.n_out + n0 + c0);
+            dst[0] = make_float4(o[0], o[1], o[2], o[3]);
+            dst[1] = make_float4(o[4], o[5], o[6], o[7]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[ab]);
+    }
+  }
+
+  // --------------------------------------------------------------------- teardown ---
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) {
+    // let copies already issued land before the CTA's shared memory goes away
+    const long long t0 = clock64();
+    while (clock64() - t0 < 200000) {
+    }
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kTmemCols));
+  }
+}
+
+size_t smem_bytes(int nb, int E) {
+  size_t raw = (static_cast<size_t>(BN) * nb + 15) & ~static_cast<size_t>(15);
+  return 1024 + kStages * (kAStage + kBStage + kSfStage) + 512 + raw + BN * sizeof(float) +
+         (2 * kStages + 4) * sizeof(uint64_t) + (E + 3) * sizeof(int) + 16;
+}
+
+}  // namespace g100
+
+// ---------------------------------------------------------------- host side -------
+namespace {
+
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encoder() {
+  static EncodeTiled fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiled>(p);
+  }
+  return fn;
+}
+
+bool encode(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
+            const uint64_t* strides_bytes, const uint32_t* box) {
+  EncodeTiled fn = encoder();
+  if (!fn) return false;
+  cuuint64_t d[3], s[2];
+  cuuint32_t b[3], es[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) { d[i] = dims[i]; b[i] = box[i]; }
+  for (int i = 0; i + 1 < rank; ++i) s[i] = strides_bytes[i];
+  return fn(m, dt, rank, const_cast<void*>(base), d, s, b, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+// Whether the tcgen05 path can run these shapes/pointers (else the register-dequant path).
+bool tc_gemm_supported(int H, int I, const void* gu_blocks, const void* d_blocks) {
+  if (H % 64 || I % 64) return false;          // 16 x U4 rows: K/2 bytes a multiple of 32
+  if (H < g100::BK || I < g100::BK) return false;
+  if ((reinterpret_cast<uintptr_t>(gu_blocks) | reinterpret_cast<uintptr_t>(d_blocks)) & 31u) return false;
+  return encoder() != nullptr;
+}
+
+cudaError_t tc_gemm_prepare(int max_nb, int E) {
+  const size_t smem = g100::smem_bytes(max_nb, E);
+  cudaError_t e = cudaFuncSetAttribute(g100::moe_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e) return e;
+  return cudaFuncSetAttribute(g100::moe_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(smem));
+}
+
+size_t tc_gemm_smem_bytes(int max_nb, int E) { return g100::smem_bytes(max_nb, E); }
+
+// a: grouped activation rows (P_rows, K) e4m3; blocks/scales: (E, rows_total, K/2) and
+// (E, rows_total, K/32); gate_up: rows_total = 2I, n_out = I; down: rows_total = n_out = H.
+cudaError_t launch_tc_gemm(bool gate_up, const uint8_t* a, int64_t P_rows, int K, const uint8_t* blocks,
+                           const uint8_t* scales, const float* bias, int E, int n_out, const int32_t* offsets,
+                           float s_in, float s_out, uint8_t* a_out, float* y_out, int* err, int sms,
+                           cudaStream_t st) {
+  using namespace g100;
+  const int rows_per_group = n_out;          // one half of gate_up, or all of down
+  const int groups = gate_up ? 2 * E : E;
+  const int bn_rows = gate_up ? BN / 2 : BN;
+  CUtensorMap ma, mb, mbt;
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(P_rows > 0 ? P_rows : 1)};
+    const uint64_t strides[1] = {static_cast<uint64_t>(K)};
+    const uint32_t box[2] = {BK, BM};
+    if (!encode(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t row_bytes = static_cast<uint64_t>(K) / 2;
+    const uint64_t dims[3] = {static_cast<uint64_t>((K / BK) * BK), static_cast<uint64_t>(rows_per_group),
+                              static_cast<uint64_t>(groups)};
+    const uint64_t strides[2] = {row_bytes, row_bytes * rows_per_group};
+    const uint32_t box[3] = {BK, static_cast<uint32_t>(bn_rows), 1};
+    if (!encode(&mb, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, blocks, dims, strides, box))
+      return cudaErrorInvalidValue;
+    const uint64_t tdims[3] = {BK, static_cast<uint64_t>(rows_per_group), static_cast<uint64_t>(groups)};
+    if (!encode(&mbt, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, blocks + (K - BK) / 2, tdims, strides, box))
+      return cudaErrorInvalidValue;
+  }
+  Params prm;
+  prm.b_scales = scales;
+  prm.bias = bias;
+  prm.offsets = offsets;
+  prm.E = E;
+  prm.K = K;
+  prm.nb = K / 32;
+  prm.rows_per_group = rows_per_group;
+  prm.rows_total = gate_up ? 2 * n_out : n_out;
+  prm.n_out = n_out;
+  prm.n_tiles = (n_out + bn_rows - 1) / bn_rows;
+  prm.nk_full = K / BK;
+  prm.tail_steps = (K % BK) / 32;
+  prm.s_in = s_in;
+  prm.s_out = s_out;
+  prm.a_out = a_out;
+  prm.y_out = y_out;
+  prm.err = err;
+  const size_t smem = smem_bytes(prm.nb, E);
+  if (gate_up)
+    moe_gemm_kernel<true><<<sms, kThreads, smem, st>>>(ma, mb, mbt, prm);
+  else
+    moe_gemm_kernel<false><<<sms, kThreads, smem, st>>>(ma, mb, mbt, prm);
+  return cudaGetLastError();
+}
+
+}  // namespace mxmoe

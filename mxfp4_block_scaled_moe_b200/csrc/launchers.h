@@ -38,6 +38,14 @@ cudaError_t launch_expert_mma(const uint8_t* blocks, const uint8_t* scales, cons
                               int max_tokens_per_expert, cudaStream_t st);
 cudaError_t expert_mma_set_smem_limits(int max_K);
 
+bool tc_gemm_supported(int H, int I, const void* gu_blocks, const void* d_blocks);
+size_t tc_gemm_smem_bytes(int max_nb, int E);
+cudaError_t tc_gemm_prepare(int max_nb, int E);
+cudaError_t launch_tc_gemm(bool gate_up, const uint8_t* a, int64_t P_rows, int K, const uint8_t* blocks,
+                           const uint8_t* scales, const float* bias, int E, int n_out, const int32_t* offsets,
+                           float s_in, float s_out, uint8_t* a_out, float* y_out, int* err, int sms,
+                           cudaStream_t st);
+
 cudaError_t launch_combine(const float* y, const int32_t* topk_idx, const float* topk_w,
                            const int32_t* inv, int T, int H, int k, uint16_t* out, cudaStream_t st,
                            int sms);
