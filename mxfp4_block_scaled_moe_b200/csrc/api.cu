@@ -42,16 +42,21 @@ cudaEvent_t next_event() {
 struct StageTimer {
   cudaStream_t st;
   cudaEvent_t last = nullptr;
-  // cudaEventRecordExternal: inside a stream capture the record becomes an event node of
-  // the graph (timed at every replay); outside a capture it is a plain record.
+  unsigned flags = cudaEventRecordDefault;
+  // Inside a stream capture the records are made with cudaEventRecordExternal so that they
+  // become event nodes of the graph (timed at every replay); outside, plain records.
   explicit StageTimer(cudaStream_t s) : st(s) {
-    if (t_profile && (last = next_event())) cudaEventRecordWithFlags(last, st, cudaEventRecordExternal);
+    if (!t_profile) return;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+      flags = cudaEventRecordExternal;
+    if ((last = next_event())) cudaEventRecordWithFlags(last, st, flags);
   }
   void mark(const char* name) {
     if (!t_profile || !last) return;
     cudaEvent_t e = next_event();
     if (!e) return;
-    cudaEventRecordWithFlags(e, st, cudaEventRecordExternal);
+    cudaEventRecordWithFlags(e, st, flags);
     t_marks.push_back({name, last, e});
     last = e;
   }
