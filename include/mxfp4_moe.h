@@ -106,6 +106,27 @@ int moe_topk_from_logits(const float* logits, int T, int E, int k, int32_t* topk
 int moe_permute(const int32_t* topk_idx, int T, int E, int k, int32_t* offsets,
                 int32_t* perm_token, int32_t* perm_slot, void* stream);
 
+/* moe_permute_noalloc -- moe_permute for callers that cannot allocate device memory.
+ * The pages have no counterpart to this entry point; it exists for deployments where a
+ * library must not call cudaMalloc: a serving runtime that reserves all device memory at
+ * start-up (for example handing what is left to a KV cache) and forbids allocation on its
+ * hot path, or a latency-bound loop that cannot afford cudaMalloc's implicit device
+ * synchronization. moe_permute itself grows the library workspace with cudaMalloc on its
+ * first call at a size; this variant allocates nothing and keeps its scratch (per-chunk
+ * expert histograms, the list of active experts) in a fixed 66,816-byte array in the
+ * library's device image, which every GPU that loads the library holds until the process
+ * exits.
+ * Same arguments, outputs and ordering as moe_permute. Limits: T*k <= 262144 and
+ * E <= 256; larger sizes return MXMOE_EUNSUPPORTED with a message and launch nothing.
+ * Differences: a pair with an expert id outside [0, E) is dropped without touching the
+ * device error word. The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current), so make that first call before any
+ * stream capture begins. All calls share the one array and each call rewrites what it
+ * reads, so calls that overlap on the GPU (different streams, no ordering) race with each
+ * other: order them. */
+int moe_permute_noalloc(const int32_t* topk_idx, int T, int E, int k, int32_t* offsets,
+                        int32_t* perm_token, int32_t* perm_slot, void* stream);
+
 /* moe_fp8_quantize -- the A-FP8 activation cast ("amd/gpt-oss-20b-MoE-Quant-W-MXFP4-A-
  * FP8-KV-FP8", Quantization schemes): q[i] = e4m3(fp32(x[i] / s)), IEEE fp32 division,
  * round-to-nearest-even, saturating to +-448 (E4M3 "fn" has no infinity; NaN stays NaN).

@@ -29,6 +29,7 @@ _SIGS = {
     "moe_route_topk": [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp],
     "moe_topk_from_logits": [_vp, _i32, _i32, _i32, _vp, _vp, _vp],
     "moe_permute": [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp],
+    "moe_permute_noalloc": [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp],
     "moe_fp8_quantize": [_vp, _i64, _f32, _vp, _vp],
     "moe_mxfp4_forward": [_vp] * 9 + [_i32] * 5 + [_vp, _vp, _vp],
     "moe_mxfp4_calibrate": [_vp] * 9 + [_i32] * 5 + [_vp, _vp],
@@ -161,6 +162,16 @@ def moe_permute(topk_idx, E, stream=None):
     ps = torch.empty(T * k, dtype=torch.int32, device=dev)
     _call("moe_permute", _ptr(topk_idx), T, E, k, _ptr(offsets), _ptr(pt), _ptr(ps), _stream(stream))
     return offsets, pt, ps
+
+
+def moe_permute_noalloc(topk_idx, E, offsets, perm_token, perm_slot, stream=None):
+    """moe_permute into caller-provided outputs without any device allocation by the
+    library (its scratch is a fixed array; T*k <= 262144, E <= 256)."""
+    _dev(topk_idx, torch.int32, "topk_idx")
+    T, k = topk_idx.shape
+    _call("moe_permute_noalloc", _ptr(topk_idx), T, E, k, _ptr(offsets), _ptr(perm_token),
+          _ptr(perm_slot), _stream(stream))
+    return offsets, perm_token, perm_slot
 
 
 def moe_fp8_quantize(x, s, stream=None):

@@ -562,3 +562,68 @@ int mxmoe_release(void) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------- allocation-free permute -----
+// moe_permute_noalloc: the same grouping as moe_permute, for callers that must not
+// allocate device memory. The kernels' scratch (per-chunk expert histograms and the
+// active-expert list) lives in a fixed array of this library's device image instead of
+// the cudaMalloc'd workspace. Host code may not pass `g_noalloc_scratch` itself to a
+// kernel (in host code the name stands for a host-side shadow, not a device address),
+// so the device address is looked up with cudaGetSymbolAddress once per device.
+namespace {
+
+constexpr int64_t kNoAllocMaxPairs = 262144;   // T * k accepted by the variant
+constexpr int kNoAllocMaxExperts = 256;
+constexpr int kNoAllocMaxChunks = 64;          // permute chunks of 4096 pairs
+constexpr int kNoAllocInts = kNoAllocMaxChunks * kNoAllocMaxExperts + kNoAllocMaxExperts + 64;
+
+// 256-byte aligned, 66,816 bytes; every GPU that loads the library keeps it until exit.
+static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocInts];
+
+int32_t* g_noalloc_dev[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+}  // namespace
+
+extern "C" int moe_permute_noalloc(const int32_t* topk_idx, int T, int E, int k, int32_t* offsets,
+                                   int32_t* perm_token, int32_t* perm_slot, void* stream) {
+  t_last_error.clear();
+  if (int rc = check_routing_args(T, E, k)) return rc;
+  const int64_t P = static_cast<int64_t>(T) * k;
+  if (P > kNoAllocMaxPairs)
+    return fail(MXMOE_EUNSUPPORTED, "moe_permute_noalloc: T*k = %lld exceeds its fixed scratch limit of %lld pairs",
+                (long long)P, (long long)kNoAllocMaxPairs);
+  if (mxmoe::permute_chunks(P) > kNoAllocMaxChunks)
+    return fail(MXMOE_EUNSUPPORTED, "moe_permute_noalloc: too many chunks");
+  if (!offsets) return fail(MXMOE_EINVAL, "offsets is NULL");
+  if (T > 0 && (!topk_idx || !perm_token || !perm_slot)) return fail(MXMOE_EINVAL, "null pointer");
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(MXMOE_EUNSUPPORTED, "device %d beyond %d", dev, kMaxDevices);
+  int32_t* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_dev[dev]) {
+      void* ptr = nullptr;
+      e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);   // this device is current
+      if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+      g_noalloc_dev[dev] = static_cast<int32_t*>(ptr);
+    }
+    scratch = g_noalloc_dev[dev];
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (T == 0) {
+    e = cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), st);
+    return e ? cuda_fail(e, "memset") : MXMOE_OK;
+  }
+  // Every launch writes all the scratch it reads (each chunk's full histogram row, the
+  // active list and its count), so nothing has to be cleared between calls.
+  int32_t* counts = scratch;
+  int32_t* active = scratch + kNoAllocMaxChunks * kNoAllocMaxExperts;
+  int32_t* n_active = active + kNoAllocMaxExperts;
+  int launches = 0;
+  e = mxmoe::launch_permute(topk_idx, T, E, k, counts, offsets, perm_token, perm_slot, nullptr, active,
+                            n_active, nullptr, st, &launches);
+  return e ? cuda_fail(e, "permute launch") : MXMOE_OK;
+}
