@@ -330,7 +330,7 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
   if ((e = launch_expert_mma(a.gu_blocks, a.gu_scales, a.gu_bias, 2 * a.I, a.H, act_in,
                              b.perm_token, b.offsets, b.active, b.n_active, max_active, s0, 0, a.I,
                              fp8 ? s1 : 0.0f, b.act_mid, nullptr, calib_out ? b.amax + 1 : nullptr,
-                             a.T, st)))
+                             a.T, ws->err, st)))
     return cuda_fail(e, "gate_up");
   ++launches;
   tm.mark("gate_up");
@@ -342,7 +342,7 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
   }
   if ((e = launch_expert_mma(a.d_blocks, a.d_scales, a.d_bias, a.H, a.I, b.act_mid, nullptr,
                              b.offsets, b.active, b.n_active, max_active, s1, 1, a.I, 0.0f, nullptr,
-                             b.y, nullptr, a.T, st)))
+                             b.y, nullptr, a.T, ws->err, st)))
     return cuda_fail(e, "down");
   ++launches;
   tm.mark("down");

@@ -22,15 +22,17 @@
 // activations get the same order with two byte permutes per register pair.
 //
 // Lane (g = lane/4, t = lane%4) owns weight rows g and g+8 and, within each 32-value
-// block, values 8t..8t+7 (bytes 4t..4t+3 of the 16-byte block).
+// block, values 8t..8t+7 (bytes 4t..4t+3 of the 16-byte block). A CTA owns one 16-row
+// group; its warps split the K blocks so that many loads are in flight per SM even when
+// few experts are active, and their partial sums are added in a fixed order.
 #include "common.cuh"
 
 namespace mxmoe {
 
 namespace {
 
-constexpr int kWarps = 4;       // warps per CTA
-constexpr int kUnroll = 16;     // 32-value blocks whose weight words are loaded ahead
+constexpr int kWarps = 4;       // warps per CTA, splitting K
+constexpr int kUnroll = 8;      // 32-value blocks per load chunk (two chunks in flight)
 
 __device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
   uint32_t d;
@@ -56,6 +58,34 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return d;
 }
 
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// 1-D bulk copy global -> shared, completion counted on an mbarrier (16-byte aligned,
+// size a multiple of 16).
+__device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// Wait for phase 0 of a single-use mbarrier, giving up after ~1 s.
+__device__ __forceinline__ bool wait_phase0(uint64_t* bar) {
+  const long long t0 = clock64();
+  while (true) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], 0;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_addr(bar))
+        : "memory");
+    if (ok) return true;
+    if (clock64() - t0 > 2000000000LL) return false;
+  }
+}
+
 struct ExpertGemmArgs {
   const uint8_t* blocks;   // (E, rows_total, K/2)
   const uint8_t* scales;   // (E, rows_total, K/32)
@@ -75,11 +105,17 @@ struct ExpertGemmArgs {
   uint16_t* act_out;       // (P, I) bf16 bits (mode 0)
   float* y_out;            // (P, rows_total) fp32 (mode 1)
   unsigned* amax_bits;     // optional: running max |a| (fp32 bits), mode 0
+  int* err;                // device error word (bounded-wait timeout)
 };
 
+// One CTA = one 16-row weight group of one active expert (gate_up: 8 gate + the 8
+// matching up rows; down: 16 rows); its kWarps warps split the K blocks, then warp 0 adds
+// the partial sums of warps 1.. in a fixed order and runs the epilogue.
 template <int NT>
 __global__ void __launch_bounds__(kWarps * 32) expert_mma_kernel(ExpertGemmArgs p) {
-  extern __shared__ float s_scale[];  // [kWarps][16][nb]
+  // shared: the group's 16 weight rows [16][K/2] bytes, their scales [16][nb] fp32, the
+  // partial sums [kWarps-1][NT][4][32] fp32, one mbarrier
+  extern __shared__ __align__(16) uint8_t s_dyn[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
   const int slot = blockIdx.y;
@@ -88,36 +124,43 @@ __global__ void __launch_bounds__(kWarps * 32) expert_mma_kernel(ExpertGemmArgs 
   const int pos0 = p.offsets[e], n_e = p.offsets[e + 1] - pos0;
   const int nb = p.K / 32;
 
-  // rows of this warp: gate_up -> 8 gate rows i0.. and the matching 8 up rows; down -> 16
-  int row_lo, row_hi;
+  int lo0, hi0;   // first lo row and first hi row of the group
   if (p.mode == 0) {
-    const int i0 = (blockIdx.x * kWarps + warp) * 8;
-    if (i0 >= p.I) return;
-    row_lo = i0 + g;
-    row_hi = p.I + i0 + g;
+    lo0 = blockIdx.x * 8;
+    hi0 = p.I + lo0;
   } else {
-    const int r0 = (blockIdx.x * kWarps + warp) * 16;
-    if (r0 >= p.rows_total) return;
-    row_lo = r0 + g;
-    row_hi = r0 + 8 + g;
+    lo0 = blockIdx.x * 16;
+    hi0 = lo0 + 8;
   }
+  const int row_lo = lo0 + g, row_hi = hi0 + g;
   const int64_t erow = static_cast<int64_t>(e) * p.rows_total;
-  const uint8_t* wlo = p.blocks + (erow + row_lo) * (p.K / 2) + 4 * t;
-  const uint8_t* whi = p.blocks + (erow + row_hi) * (p.K / 2) + 4 * t;
+  const int rb = p.K / 2;   // packed bytes per row
+  uint8_t* wbuf = s_dyn;
+  float* sc = reinterpret_cast<float*>(s_dyn + 16 * rb);
+  float* red = sc + 16 * nb;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(red + (kWarps - 1) * NT * 4 * 32);
 
-  // stage this warp's 16 rows of scales as fp32 (row slot 0..7 = lo rows, 8..15 = hi
-  // rows). The 8 lo rows (and the 8 hi rows) are 8 * nb contiguous bytes: load them with
-  // 16-byte loads when aligned so that all of them are in flight at once.
-  float* sc = s_scale + static_cast<int64_t>(warp) * 16 * nb;
+  // the 8 lo rows and the 8 hi rows are each 8 * K/2 contiguous bytes: two bulk copies
+  // bring the whole group into shared memory while the scales are staged below
+  if (threadIdx.x == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(bar)));
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_addr(bar)), "r"(16 * rb)
+                 : "memory");
+    bulk_copy_g2s(wbuf, p.blocks + (erow + lo0) * rb, 8 * rb, bar);
+    bulk_copy_g2s(wbuf + 8 * rb, p.blocks + (erow + hi0) * rb, 8 * rb, bar);
+  }
+
+  // scales of the 16 rows as fp32 (slots 0..7 lo rows, 8..15 hi rows); the 8 lo rows (and
+  // the 8 hi rows) are 8 * nb contiguous bytes, loaded 16 bytes at a time when aligned
   {
-    const uint8_t* half_src[2] = {p.scales + (erow + row_lo - g) * nb,
-                                  p.scales + (erow + row_hi - g) * nb};
+    const uint8_t* half_src[2] = {p.scales + (erow + lo0) * nb, p.scales + (erow + hi0) * nb};
     const int half_bytes = 8 * nb;
     const bool vec = ((reinterpret_cast<uintptr_t>(half_src[0]) | reinterpret_cast<uintptr_t>(half_src[1]) |
                        static_cast<uintptr_t>(half_bytes)) & 15u) == 0;
     if (vec) {
       const int n16 = half_bytes / 16;
-      for (int c = lane; c < 2 * n16; c += 32) {
+      for (int c = threadIdx.x; c < 2 * n16; c += blockDim.x) {
         const int h = c >= n16 ? 1 : 0, o = (c - h * n16) * 16;
         const uint4 v = ld_nc_v4(half_src[h] + o);
         const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
@@ -126,19 +169,27 @@ __global__ void __launch_bounds__(kWarps * 32) expert_mma_kernel(ExpertGemmArgs 
         for (int j = 0; j < 16; ++j) dst[j] = e8m0_to_f32((wv[j >> 2] >> (8 * (j & 3))) & 0xFFu);
       }
     } else {
-#pragma unroll 8
-      for (int i = lane; i < 2 * half_bytes; i += 32) {
+      for (int i = threadIdx.x; i < 2 * half_bytes; i += blockDim.x) {
         const int h = i >= half_bytes ? 1 : 0;
         sc[i] = e8m0_to_f32(half_src[h][i - h * half_bytes]);
       }
     }
   }
-  __syncwarp();
+  __syncthreads();
+  if (!wait_phase0(bar)) {
+    set_device_error(p.err, MXMOE_ETIMEOUT);
+    const long long t0 = clock64();   // let the copies in flight land before leaving
+    while (clock64() - t0 < 200000) {
+    }
+    return;
+  }
   const float* sc_lo = sc + g * nb;
   const float* sc_hi = sc + (8 + g) * nb;
+  const uint8_t* wlo = wbuf + g * rb + 4 * t;
+  const uint8_t* whi = wbuf + (8 + g) * rb + 4 * t;
+  const int b_begin = (warp * nb) / kWarps, b_end = ((warp + 1) * nb) / kWarps;
 
   for (int tp = 0; tp < n_e; tp += 8 * NT) {
-    // activation row pointers of this lane's token (column g of each n-tile)
     const uint16_t* arow[NT];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -159,18 +210,22 @@ __global__ void __launch_bounds__(kWarps * 32) expert_mma_kernel(ExpertGemmArgs 
 #pragma unroll
       for (int r = 0; r < 4; ++r) acc[nt][r] = 0.0f;
 
-    for (int b0 = 0; b0 < nb; b0 += kUnroll) {
-      uint32_t wl[kUnroll], wh[kUnroll];
+    // weight words double-buffered: the loads of chunk c+1 are in flight while chunk c
+    // is decoded and multiplied (two named buffers, so every index stays static)
+    uint32_t wlA[kUnroll], whA[kUnroll], wlB[kUnroll], whB[kUnroll];
+    auto load_chunk = [&](uint32_t (&wl)[kUnroll], uint32_t (&wh)[kUnroll], int b0) {
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
         const int b = b0 + u;
-        wl[u] = b < nb ? ld_nc_u32(wlo + 16 * b) : 0u;
-        wh[u] = b < nb ? ld_nc_u32(whi + 16 * b) : 0u;
+        wl[u] = b < b_end ? *reinterpret_cast<const uint32_t*>(wlo + 16 * b) : 0u;
+        wh[u] = b < b_end ? *reinterpret_cast<const uint32_t*>(whi + 16 * b) : 0u;
       }
+    };
+    auto compute_chunk = [&](const uint32_t (&wl)[kUnroll], const uint32_t (&wh)[kUnroll], int b0) {
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
         const int b = b0 + u;
-        if (b >= nb) break;
+        if (b >= b_end) break;
         uint32_t a0[4], a1[4];
         a0[0] = e2m1_pair_bf16x2<0>(wl[u]);
         a0[1] = e2m1_pair_bf16x2<0>(wh[u]);
@@ -198,36 +253,69 @@ __global__ void __launch_bounds__(kWarps * 32) expert_mma_kernel(ExpertGemmArgs 
           acc[nt][3] = fmaf(tmp[3], sh, acc[nt][3]);
         }
       }
+    };
+    load_chunk(wlA, whA, b_begin);
+    for (int b0 = b_begin; b0 < b_end; b0 += 2 * kUnroll) {
+      if (b0 + kUnroll < b_end) load_chunk(wlB, whB, b0 + kUnroll);
+      compute_chunk(wlA, whA, b0);
+      if (b0 + kUnroll >= b_end) break;
+      if (b0 + 2 * kUnroll < b_end) load_chunk(wlA, whA, b0 + 2 * kUnroll);
+      compute_chunk(wlB, whB, b0 + kUnroll);
     }
 
-    // epilogue: acc[nt][0..1] = row_lo, tokens 2t, 2t+1; acc[nt][2..3] = row_hi, same tokens
-    const float b_lo = p.bias[erow + row_lo], b_hi = p.bias[erow + row_hi];
+    // partial sums of warps 1.. to shared memory; warp 0 adds them in warp order
+    if (warp > 0) {
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      if (nt >= nt_live) break;
+      for (int nt = 0; nt < NT; ++nt) {
+        if (nt >= nt_live) break;
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const int j = tp + nt * 8 + 2 * t + c;
-        if (j >= n_e) continue;
-        const int64_t pos = pos0 + j;
-        const float lo = __fadd_rn(__fmul_rn(p.s_in, acc[nt][c]), b_lo);
-        const float hi = __fadd_rn(__fmul_rn(p.s_in, acc[nt][2 + c]), b_hi);
-        if (p.mode == 0) {
-          const float a = silu_mul(lo, hi);
-          if (p.amax_bits) atomicMax(p.amax_bits, __float_as_uint(fabsf(a)));
-          uint16_t bits;
-          if (p.s_mid > 0.0f)
-            bits = static_cast<uint16_t>(__float_as_uint(e4m3_to_f32(act_quant_e4m3(a, p.s_mid))) >> 16);
-          else
-            bits = f32_to_bf16_bits_rn(a);
-          p.act_out[pos * p.I + (row_lo)] = bits;
-        } else {
-          p.y_out[pos * p.rows_total + row_lo] = lo;
-          p.y_out[pos * p.rows_total + row_hi] = hi;
+        for (int r = 0; r < 4; ++r) red[(((warp - 1) * NT + nt) * 4 + r) * 32 + lane] = acc[nt][r];
+      }
+    }
+    __syncthreads();
+    if (warp == 0) {
+      for (int w = 1; w < kWarps; ++w)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          if (nt >= nt_live) break;
+#pragma unroll
+          for (int r = 0; r < 4; ++r) acc[nt][r] += red[(((w - 1) * NT + nt) * 4 + r) * 32 + lane];
+        }
+      // epilogue: acc[nt][0..1] = row_lo, tokens 2t, 2t+1; acc[nt][2..3] = row_hi
+      const float b_lo = p.bias[erow + row_lo], b_hi = p.bias[erow + row_hi];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        if (nt >= nt_live) break;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int j = tp + nt * 8 + 2 * t + c;
+          if (j >= n_e) continue;
+          const int64_t pos = pos0 + j;
+          const float lo = __fadd_rn(__fmul_rn(p.s_in, acc[nt][c]), b_lo);
+          const float hi = __fadd_rn(__fmul_rn(p.s_in, acc[nt][2 + c]), b_hi);
+          if (p.mode == 0) {
+            const float a = silu_mul(lo, hi);
+            if (p.amax_bits) atomicMax(p.amax_bits, __float_as_uint(fabsf(a)));
+            uint16_t bits;
+            if (p.s_mid > 0.0f)
+              bits = static_cast<uint16_t>(__float_as_uint(e4m3_to_f32(act_quant_e4m3(a, p.s_mid))) >> 16);
+            else
+              bits = f32_to_bf16_bits_rn(a);
+            p.act_out[pos * p.I + row_lo] = bits;
+          } else {
+            p.y_out[pos * p.rows_total + row_lo] = lo;
+            p.y_out[pos * p.rows_total + row_hi] = hi;
+          }
         }
       }
     }
+    __syncthreads();
   }
+}
+
+size_t smem_bytes(int K, int nt) {
+  return static_cast<size_t>(16) * (K / 2) + static_cast<size_t>(16) * (K / 32) * sizeof(float) +
+         static_cast<size_t>(kWarps - 1) * nt * 4 * 32 * sizeof(float) + 16;
 }
 
 }  // namespace
@@ -237,34 +325,28 @@ cudaError_t launch_expert_mma(const uint8_t* blocks, const uint8_t* scales, cons
                               const int32_t* offsets, const int32_t* active,
                               const int32_t* n_active, int max_active, float s_in, int mode, int I,
                               float s_mid, uint16_t* act_out, float* y_out, unsigned* amax_bits,
-                              int max_tokens_per_expert, cudaStream_t st) {
+                              int max_tokens_per_expert, int* err, cudaStream_t st) {
   ExpertGemmArgs a{blocks, scales, bias, rows_total, K, act, act_row, offsets, active, n_active,
-                   s_in, mode, I, s_mid, act_out, y_out, amax_bits};
-  const int rows_per_cta = (mode == 0 ? 8 : 16) * kWarps;
-  const int out_rows = mode == 0 ? I : rows_total;
-  dim3 grid(static_cast<unsigned>(cdiv(out_rows, rows_per_cta)), static_cast<unsigned>(max_active));
-  const size_t smem = static_cast<size_t>(kWarps) * 16 * (K / 32) * sizeof(float);
-  const int nt = (max_tokens_per_expert + 7) / 8;
-  if (nt <= 1) {
+                   s_in, mode, I, s_mid, act_out, y_out, amax_bits, err};
+  const int groups = mode == 0 ? I / 8 : rows_total / 16;
+  dim3 grid(static_cast<unsigned>(groups), static_cast<unsigned>(max_active));
+  // one n-tile (8 tokens) per pass for up to 8 routed tokens, else two per pass; a group's
+  // weights stay in shared memory across passes
+  const int ntc = max_tokens_per_expert <= 8 ? 1 : 2;
+  const size_t smem = smem_bytes(K, ntc);
+  if (ntc == 1)
     expert_mma_kernel<1><<<grid, kWarps * 32, smem, st>>>(a);
-  } else if (nt <= 2) {
+  else
     expert_mma_kernel<2><<<grid, kWarps * 32, smem, st>>>(a);
-  } else if (nt <= 4) {
-    expert_mma_kernel<4><<<grid, kWarps * 32, smem, st>>>(a);
-  } else {
-    expert_mma_kernel<8><<<grid, kWarps * 32, smem, st>>>(a);
-  }
   return cudaGetLastError();
 }
 
 cudaError_t expert_mma_set_smem_limits(int max_K) {
-  const int smem = kWarps * 16 * (max_K / 32) * static_cast<int>(sizeof(float));
+  const int smem = static_cast<int>(smem_bytes(max_K, 2));
   cudaError_t e = cudaSuccess;
   if (smem > 48 * 1024) {
     if ((e = cudaFuncSetAttribute(expert_mma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
     if ((e = cudaFuncSetAttribute(expert_mma_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
-    if ((e = cudaFuncSetAttribute(expert_mma_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
-    if ((e = cudaFuncSetAttribute(expert_mma_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
   }
   return e;
 }

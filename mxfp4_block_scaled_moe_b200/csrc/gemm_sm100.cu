@@ -26,10 +26,11 @@
 // 512-byte atoms that tcgen05.cp (32x128b, 4 warp-quarters) moves into tensor memory:
 // row r of an atom at byte 16*(r%32) + 4*(r/32) + j for k-block j.
 //
-// Roles (256 threads, one CTA per SM, persistent over the tile list):
+// Roles (640 threads, one CTA per SM, persistent over the tile list):
 //   warp 0: TMA producer          warp 1: TMEM owner + MMA issuer (one thread)
-//   warp 2: scale converter       warp 3: builds the tile schedule, then idles
-//   warps 4-7: epilogue (TMEM lane quarter = warp % 4)
+//   warps 2-3: scale converters (rows 0..127 / 128..255); warp 3 first builds the schedule
+//   warps 4..19: epilogue; warp w reads TMEM lane quarter w % 4 and every (w-4)/4-th group
+//   of 8 accumulator columns, so each sub-partition runs 4 epilogue warps
 // Every mbarrier wait gives up after ~1 s (clock64): the kernel then records MXMOE_ETIMEOUT
 // in the error word, lets in-flight copies land, frees its tensor memory and returns.
 #include <cuda.h>
@@ -43,14 +44,17 @@ constexpr int BM = 128;             // rows of A per tile (MMA M)
 constexpr int BN = 240;             // MMA N (gate_up: 120 gate + 120 up rows)
 constexpr int BK = 128;             // K values per pipeline stage
 constexpr int kStages = 4;
-constexpr int kThreads = 256;
+constexpr int kEpiWarps = 16;                // 4 per SM sub-partition: hides the epilogue's latency
+constexpr int kThreads = 128 + 32 * kEpiWarps;  // warps 0-3 producer/MMA/scales/schedule
 constexpr int kAStage = BM * BK;            // 16 KB (e4m3, one byte per value)
 constexpr int kBStage = BN * BK;            // 30 KB (e2m1 spread to one byte per value)
 constexpr int kSfStage = 1024;              // two 512-byte scale atoms (rows 0..255)
 constexpr int kAccCols = 256;               // column stride between the two accumulators
 constexpr int kTmemCols = 512;
-constexpr int kSfaCol = 496;                // 4 columns of unit A scales
-constexpr int kSfbCol = 504;                // 8 columns of B scales (rows 0..255)
+constexpr int kSfaCol = 240;                // 4 columns of unit A scales (gap after accumulator 0)
+constexpr int kSfbCol = 496;                // two 8-column slots of B scales (rows 0..255),
+                                            // alternated per stage so the copy of stage s+1
+                                            // never overwrites scales stage s still reads
 constexpr long long kWaitCycles = 2000000000LL;  // ~1 s at the B200 clock
 
 struct Params {
@@ -133,6 +137,13 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
 }
@@ -184,9 +195,6 @@ __device__ __forceinline__ void tc_wait_ld(uint32_t (&a)[8], uint32_t (&b)[8]) {
                : "memory");
 }
 
-__device__ __forceinline__ void named_bar_sync(int id, int count) {
-  asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(count) : "memory");
-}
 
 // Shared-memory matrix descriptor (tcgen05): start, leading/stride byte offsets (>>4),
 // version 1, layout type (0 = no swizzle, 2 = 128-byte swizzle).
@@ -246,13 +254,13 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constan
   uint8_t* sSFA = sSF + kStages * kSfStage;       // 512 B of unit scales
   uint8_t* sRaw = sSFA + 512;                     // BN * nb raw scale bytes
   const int raw_bytes = ((BN * p.nb) + 15) & ~15;
-  float* sBias = reinterpret_cast<float*>(sRaw + raw_bytes);     // BN floats
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sBias + BN);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sRaw + raw_bytes);
   uint64_t* full = bars;
   uint64_t* empty = bars + kStages;
   uint64_t* acc_full = bars + 2 * kStages;
   uint64_t* acc_empty = acc_full + 2;
-  int* prefix = reinterpret_cast<int*>(acc_empty + 2);           // E + 1
+  uint64_t* raw_full = acc_empty + 2;                            // [2]: raw scales landed, per converter
+  int* prefix = reinterpret_cast<int*>(raw_full + 2);            // E + 1
   volatile int* abort_flag = prefix + (p.E + 1);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(prefix + p.E + 2);
 
@@ -261,13 +269,15 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constan
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 2);     // TMA producer (expect_tx) + scale converter
+      mbar_init(&full[s], 3);     // TMA producer (expect_tx) + the two scale-converter warps
       mbar_init(&empty[s], 1);    // MMA commit
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 4);  // one arrive per epilogue warp
+      mbar_init(&acc_empty[b], kEpiWarps);  // one arrive per epilogue warp
     }
+    mbar_init(&raw_full[0], 1);
+    mbar_init(&raw_full[1], 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
@@ -355,8 +365,9 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constan
         tc_fence_after();
         if (lane == 0) {
           const uint32_t sf = smem_u32(sSF + stage * kSfStage);
-          tc_cp_32x128b_x4(tmem + kSfbCol, smem_desc(sf, 0, 128, 0));
-          tc_cp_32x128b_x4(tmem + kSfbCol + 4, smem_desc(sf + 512, 0, 128, 0));
+          const uint32_t sfb = tmem + kSfbCol + 8 * (stage & 1);
+          tc_cp_32x128b_x4(sfb, smem_desc(sf, 0, 128, 0));
+          tc_cp_32x128b_x4(sfb + 4, smem_desc(sf + 512, 0, 128, 0));
           const uint32_t a0 = smem_u32(sA + stage * kAStage), b0 = smem_u32(sB + stage * kBStage);
           const int first = kt < p.nk_full ? 0 : 4 - p.tail_steps;
           for (int kk = first; kk < 4; ++kk) {
@@ -364,7 +375,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constan
             const uint64_t bd = smem_desc(b0 + 32 * kk, 16, 1024, 2);
             const uint32_t id = idesc0 | (static_cast<uint32_t>(kk) << 4) | (static_cast<uint32_t>(kk) << 29);
             const uint32_t sel = static_cast<uint32_t>(kk) << 30;
-            tc_mma_mxf8f6f4(dacc, ad, bd, id, (tmem + kSfaCol) | sel, (tmem + kSfbCol) | sel,
+            tc_mma_mxf8f6f4(dacc, ad, bd, id, (tmem + kSfaCol) | sel, sfb | sel,
                             (kt > 0 || kk > first) ? 1u : 0u);
           }
           tc_commit(&empty[stage]);
@@ -376,47 +387,96 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constan
       if (lane == 0) tc_commit(&acc_full[ab]);
       __syncwarp();
     }
-  } else if (warp == 2) {
-    // --------------------------------------------------------- scale converter -----
+  } else if (warp == 2 || warp == 3) {
+    // -------------------------------------------------------- scale converters -----
+    // warp 2 fills atom 0 (tile rows 0..127), warp 3 atom 1 (rows 128..255); lane l owns
+    // rows l, l+32, l+64, l+96 of its atom, whose four words sit side by side in the atom
+    // (byte 16*l + 4*i), so one 16-byte store per lane and stage writes them.
+    const int w2 = warp - 2;
     int stage = 0;
-    uint32_t phase = 0;
+    uint32_t phase = 0, raw_phase = 0;
     const int nb = p.nb;
     for (int t = blockIdx.x; t < total_tiles && !*abort_flag; t += gridDim.x) {
       const Tile tl = tile_of(t, prefix, p.offsets, p.E, p.n_tiles);
       const int n0 = tl.nt * bn_rows;
-      // raw scale rows of this tile into shared memory (row r of the tile: r < bn_rows is
-      // the first half / whole tile, r >= bn_rows the up half of gate_up)
       const int halves = kGateUp ? 2 : 1;
       const int valid = min(bn_rows, p.rows_per_group - n0);
+      // raw scale rows of this warp's tile rows [128*w2, 128*w2 + 128) into sRaw, tile row
+      // r at byte r * nb (r < bn_rows: first half or whole tile; r >= bn_rows: up half).
+      // Each half is one contiguous run in global memory: bulk copy when 16-byte aligned,
+      // else plain loads issued 8 at a time. Only this warp reads these rows.
+      fence_async_smem();   // this warp's earlier reads of its rows precede the refill
+      const uint8_t* src_h[2] = {nullptr, nullptr};
+      uint8_t* dst_h[2] = {nullptr, nullptr};
+      int bytes_h[2] = {0, 0};
+      bool bulk_h[2] = {false, false};
+      uint32_t bulk_bytes = 0;
       for (int h = 0; h < halves; ++h) {
+        const int lo = max(0, 128 * w2 - h * bn_rows);
+        const int hi = min(valid, 128 * w2 + 128 - h * bn_rows);
+        if (hi <= lo) continue;
         const int group = kGateUp ? 2 * tl.e + h : tl.e;
-        const uint8_t* src = p.b_scales + (static_cast<int64_t>(group) * p.rows_per_group + n0) * nb;
-        uint8_t* dst = sRaw + h * bn_rows * nb;
-        const int bytes = valid * nb;
-        if (((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & 15u) == 0) {
-          for (int c = lane; c < bytes / 16; c += 32)
-            reinterpret_cast<uint4*>(dst)[c] = ld_nc_v4(src + 16 * c);
-          for (int c = (bytes / 16) * 16 + lane; c < bytes; c += 32) dst[c] = src[c];
-        } else {
-          for (int c = lane; c < bytes; c += 32) dst[c] = src[c];
+        src_h[h] = p.b_scales + (static_cast<int64_t>(group) * p.rows_per_group + n0 + lo) * nb;
+        dst_h[h] = sRaw + (h * bn_rows + lo) * nb;
+        bytes_h[h] = (hi - lo) * nb;
+        bulk_h[h] = ((reinterpret_cast<uintptr_t>(src_h[h]) | reinterpret_cast<uintptr_t>(dst_h[h]) |
+                      static_cast<uintptr_t>(bytes_h[h])) & 15u) == 0;
+        if (bulk_h[h]) bulk_bytes += static_cast<uint32_t>(bytes_h[h]);
+      }
+      if (bulk_bytes > 0 && lane == 0) {
+        mbar_arrive_expect_tx(&raw_full[w2], bulk_bytes);
+        for (int h = 0; h < halves; ++h)
+          if (bulk_h[h]) bulk_g2s(dst_h[h], src_h[h], static_cast<uint32_t>(bytes_h[h]), &raw_full[w2]);
+      }
+      for (int h = 0; h < halves; ++h) {
+        if (bulk_h[h] || bytes_h[h] == 0) continue;
+        const uint8_t* src = src_h[h];
+        uint8_t* dst = dst_h[h];
+        const int bytes = bytes_h[h];
+        for (int c0 = 0; c0 < bytes; c0 += 32 * 8) {
+          uint8_t v[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int c = c0 + u * 32 + lane;
+            v[u] = c < bytes ? src[c] : 0;
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int c = c0 + u * 32 + lane;
+            if (c < bytes) dst[c] = v[u];
+          }
         }
       }
+      if (bulk_bytes > 0) {
+        if (!mbar_wait(&raw_full[w2], raw_phase, abort_flag, p.err)) break;
+        raw_phase ^= 1;
+      }
       __syncwarp();
+      // where this lane's four rows start in sRaw (-1: outside the tile -> unit scale)
+      int src_off[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = 128 * w2 + lane + 32 * i;
+        const int h = r >= bn_rows ? 1 : 0;
+        const int rr = r - h * bn_rows;
+        src_off[i] = (r < BN && rr < valid && h < halves) ? (h * bn_rows + rr) * nb : -1;
+      }
       for (int kt = 0; kt < nkt; ++kt) {
         if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err)) break;
         const int kb0 = kt < p.nk_full ? 4 * kt : nb - 4;
-        uint32_t* atom = reinterpret_cast<uint32_t*>(sSF + stage * kSfStage);
-        for (int r = lane; r < 256; r += 32) {
-          uint32_t word = 0x7F7F7F7Fu;
-          const int h = r / bn_rows, rr = r - h * bn_rows;
-          if (r < BN && rr < valid) {
-            const uint8_t* s = sRaw + (h * bn_rows + rr) * nb + kb0;
-            word = static_cast<uint32_t>(s[0]) | (static_cast<uint32_t>(s[1]) << 8) |
-                   (static_cast<uint32_t>(s[2]) << 16) | (static_cast<uint32_t>(s[3]) << 24);
+        uint32_t wv[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          if (src_off[i] < 0) {
+            wv[i] = 0x7F7F7F7Fu;
+          } else {
+            // rows are nb bytes apart and kb0 is a multiple of 4: the 4 bytes are 2-aligned
+            const uint16_t* s16 = reinterpret_cast<const uint16_t*>(sRaw + src_off[i] + kb0);
+            wv[i] = static_cast<uint32_t>(s16[0]) | (static_cast<uint32_t>(s16[1]) << 16);
           }
-          const int a = r >> 7, m = r & 127;
-          atom[(a * 512 + (m & 31) * 16 + (m >> 5) * 4) >> 2] = word;
         }
+        *reinterpret_cast<uint4*>(sSF + stage * kSfStage + 512 * w2 + 16 * lane) =
+            make_uint4(wv[0], wv[1], wv[2], wv[3]);
         fence_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&full[stage]);
@@ -426,59 +486,71 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constan
     }
   } else if (warp >= 4) {
     // --------------------------------------------------------------- epilogue -----
-    const int q = warp & 3;            // tensor-memory lane quarter of this warp
-    const int row = 32 * q + lane;     // tile row = TMEM lane
-    const int et = threadIdx.x - 128;  // 0..127
+    const int q = warp & 3;                 // tensor-memory lane quarter of this warp
+    const int slice = (warp - 4) >> 2;      // which groups of 8 columns it takes
+    constexpr int kSlices = kEpiWarps / 4;
+    const int row = 32 * q + lane;          // tile row = TMEM lane
     int it = 0;
     for (int t = blockIdx.x; t < total_tiles && !*abort_flag; t += gridDim.x, ++it) {
       const Tile tl = tile_of(t, prefix, p.offsets, p.E, p.n_tiles);
       const int n0 = tl.nt * bn_rows;
       const int ab = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
-      named_bar_sync(1, 128);          // previous tile's bias reads are done
-      for (int j = et; j < BN; j += 128) {
-        float b = 0.0f;
-        if (kGateUp) {
-          const int h = j / bn_rows, c = n0 + (j - h * bn_rows);
-          if (c < p.n_out) b = p.bias[static_cast<int64_t>(tl.e) * p.rows_total + h * p.n_out + c];
-        } else {
-          const int c = n0 + j;
-          if (c < p.n_out) b = p.bias[static_cast<int64_t>(tl.e) * p.rows_total + c];
-        }
-        sBias[j] = b;
-      }
-      named_bar_sync(1, 128);
       if (!mbar_wait(&acc_full[ab], acc_phase, abort_flag, p.err)) break;
       tc_fence_after();
       const uint32_t tbase = tmem + ab * kAccCols + (static_cast<uint32_t>(32 * q) << 16);
       const bool valid = row < tl.rows;
       const int64_t pos = tl.m0 + row;
       if (kGateUp) {
-        for (int c0 = 0; c0 < bn_rows; c0 += 8) {
+        // 15 groups of 8 gate columns (and the 8 matching up columns), round-robin over slices
+        for (int c0 = 8 * slice; c0 < bn_rows; c0 += 8 * kSlices) {
           uint32_t g[8], u[8];
           tc_ld_32x32b_x8(tbase + c0, g);
           tc_ld_32x32b_x8(tbase + bn_rows + c0, u);
+          // n_out % 8 == 0: a group of 8 columns is wholly inside or wholly past the tile
+          const bool live = n0 + c0 < p.n_out;
+          float bg[8], bu[8];
+          if (live) {
+            const float4* bp = reinterpret_cast<const float4*>(p.bias + static_cast<int64_t>(tl.e) * p.rows_total + n0 + c0);
+            const float4* bq = reinterpret_cast<const float4*>(p.bias + static_cast<int64_t>(tl.e) * p.rows_total + p.n_out + n0 + c0);
+            const float4 b0 = bp[0], b1 = bp[1], b2 = bq[0], b3 = bq[1];
+            bg[0] = b0.x; bg[1] = b0.y; bg[2] = b0.z; bg[3] = b0.w; bg[4] = b1.x; bg[5] = b1.y; bg[6] = b1.z; bg[7] = b1.w;
+            bu[0] = b2.x; bu[1] = b2.y; bu[2] = b2.z; bu[3] = b2.w; bu[4] = b3.x; bu[5] = b3.y; bu[6] = b3.z; bu[7] = b3.w;
+          } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) bg[i] = bu[i] = 0.0f;
+          }
           tc_wait_ld(g, u);
           uint32_t lo = 0, hi = 0;
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            const float gv = __fadd_rn(__fmul_rn(p.s_in, __uint_as_float(g[i])), sBias[c0 + i]);
-            const float uv = __fadd_rn(__fmul_rn(p.s_in, __uint_as_float(u[i])), sBias[bn_rows + c0 + i]);
+            const float gv = __fadd_rn(__fmul_rn(p.s_in, __uint_as_float(g[i])), bg[i]);
+            const float uv = __fadd_rn(__fmul_rn(p.s_in, __uint_as_float(u[i])), bu[i]);
             const uint32_t qb = act_quant_e4m3(silu_mul(gv, uv), p.s_out);
             if (i < 4) lo |= qb << (8 * i); else hi |= qb << (8 * (i - 4));
           }
-          if (valid && n0 + c0 < p.n_out)
+          if (valid && live)
             *reinterpret_cast<uint2*>(p.a_out + pos * p.n_out + n0 + c0) = make_uint2(lo, hi);
         }
       } else {
-        for (int c0 = 0; c0 < BN; c0 += 8) {
+        for (int c0 = 8 * slice; c0 < BN; c0 += 8 * kSlices) {
           uint32_t v[8];
           tc_ld_32x32b_x8(tbase + c0, v);
+          const bool live = n0 + c0 < p.n_out;
+          float bb[8];
+          if (live) {
+            const float4* bp = reinterpret_cast<const float4*>(p.bias + static_cast<int64_t>(tl.e) * p.rows_total + n0 + c0);
+            const float4 b0 = bp[0], b1 = bp[1];
+            bb[0] = b0.x; bb[1] = b0.y; bb[2] = b0.z; bb[3] = b0.w; bb[4] = b1.x; bb[5] = b1.y; bb[6] = b1.z; bb[7] = b1.w;
+          } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) bb[i] = 0.0f;
+          }
           tc_wait_ld(v);
           float o[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) o[i] = __fadd_rn(__fmul_rn(p.s_in, __uint_as_float(v[i])), sBias[c0 + i]);
-          if (valid && n0 + c0 < p.n_out) {
+          for (int i = 0; i < 8; ++i) o[i] = __fadd_rn(__fmul_rn(p.s_in, __uint_as_float(v[i])), bb[i]);
+          if (valid && live) {
             float4* dst = reinterpret_cast<float4*>(p.y_out + pos * p.n_out + n0 + c0);
             dst[0] = make_float4(o[0], o[1], o[2], o[3]);
             dst[1] = make_float4(o[4], o[5], o[6], o[7]);
@@ -508,8 +580,8 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constan
 
 size_t smem_bytes(int nb, int E) {
   size_t raw = (static_cast<size_t>(BN) * nb + 15) & ~static_cast<size_t>(15);
-  return 1024 + kStages * (kAStage + kBStage + kSfStage) + 512 + raw + BN * sizeof(float) +
-         (2 * kStages + 4) * sizeof(uint64_t) + (E + 3) * sizeof(int) + 16;
+  return 1024 + kStages * (kAStage + kBStage + kSfStage) + 512 + raw +
+         (2 * kStages + 6) * sizeof(uint64_t) + (E + 3) * sizeof(int) + 16;
 }
 
 }  // namespace g100

@@ -35,7 +35,7 @@ cudaError_t launch_expert_mma(const uint8_t* blocks, const uint8_t* scales, cons
                               const int32_t* offsets, const int32_t* active,
                               const int32_t* n_active, int max_active, float s_in, int mode, int I,
                               float s_mid, uint16_t* act_out, float* y_out, unsigned* amax_bits,
-                              int max_tokens_per_expert, cudaStream_t st);
+                              int max_tokens_per_expert, int* err, cudaStream_t st);
 cudaError_t expert_mma_set_smem_limits(int max_K);
 
 bool tc_gemm_supported(int H, int I, const void* gu_blocks, const void* d_blocks);
