@@ -55,6 +55,31 @@ WORKLOADS = {
 PER_EXPERT_PACKED = lambda H, I: 2 * I * H // 2 + 2 * I * H // 32 + H * I // 2 + H * I // 32
 
 
+def ncu_traffic(workload: str, kernel: str):
+    """Per-launch DRAM bytes (read + write) of `kernel` from a committed ncu summary under
+    profiles/, or None when there is none or the kernel's source changed since."""
+    import glob
+    import hashlib
+    for path in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
+        fields = {}
+        for line in open(path):
+            line = line.strip().lstrip("- ")
+            if ": " in line:
+                k, v = line.split(": ", 1)
+                fields[k.strip()] = v.strip()
+        if fields.get("workload") != workload or fields.get("kernel") != kernel:
+            continue
+        try:
+            src, _, prefix = fields["source"].partition(" sha256 prefix ")
+            digest = hashlib.sha256(open(os.path.join(ROOT, src), "rb").read()).hexdigest()
+            if not digest.startswith(prefix):
+                return None
+            return int(fields["traffic_bytes_per_launch"])
+        except (KeyError, OSError, ValueError):
+            return None
+    return None
+
+
 def peaks():
     try:
         with open(PEAKS_FILE) as f:
@@ -86,13 +111,19 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(v: float, world: int) -> float:
+def max_over_ranks(v: float, world: int, device: str = "cuda") -> float:
+    """The slowest rank's time: every rank passes its own, all get the maximum."""
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_tokens_per_s(tokens_per_rank_step: int, world: int, steps: int, max_ms: float) -> float:
+    """Whole-job throughput: the tokens every rank processed over the slowest rank's time."""
+    return tokens_per_rank_step * world * steps / (max_ms / 1e3)
 
 
 # ----------------------------------------------------------------------- setup ----
@@ -271,7 +302,7 @@ def run_ours(args, world, rank):
     total_ms = sum(a.elapsed_time(b) for a, b in ev)
     total_ms = max_over_ranks(total_ms, world)
     ms_per_step = total_ms / args.steps
-    value = T * world * args.steps / (total_ms / 1e3)
+    value = job_tokens_per_s(T, world, args.steps, total_ms)
     del graph
 
     # ---- end to end through the C ABI with host buffers
@@ -294,7 +325,7 @@ def run_ours(args, world, rank):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    e2e_value = T * world * args.steps / (e2e_ms / 1e3)
+    e2e_value = job_tokens_per_s(T, world, args.steps, e2e_ms)
 
     # ---- roofline of the dominant kernel
     dom = max((s for s in stages if s not in ("router", "topk", "permute", "act_quant", "combine")),
@@ -316,8 +347,10 @@ def run_ours(args, world, rank):
         b = work["gu_bytes"] if dom == "gate_up" else work["bytes"] - work["gu_bytes"]
         achieved = b / (dom_ms / 1e3) / 1e9
         peak_note = f"{pk_kind} hbm copy"
+    tc_path = fp8 and T * k >= 1024
+    traffic = ncu_traffic(args.workload, dom) if tc_path else None
     roofline = {"bound": bound, "kernel": dom, "achieved": round(achieved, 2), "peak": peak,
-                "unit": unit, "frac": round(achieved / peak, 4), "traffic": None,
+                "unit": unit, "frac": round(achieved / peak, 4), "traffic": traffic,
                 "peak_source": peak_note, "kernel_ms": round(dom_ms, 5)}
 
     res = {
