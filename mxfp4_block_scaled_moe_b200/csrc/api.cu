@@ -78,6 +78,10 @@ int cuda_fail(cudaError_t e, const char* what) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+constexpr size_t kTicketBytes = 4096;       // 1024 row groups of 16 rows: H <= 16384
+constexpr int kFoldCombineMaxT = 64;        // fold the combine into the down kernel up to here
+constexpr int kRouteTicket = 1023;          // ticket slot of the fused routing kernel
+
 // ------------------------------------------------------------------ workspace ------
 struct Workspace {
   char* base = nullptr;
@@ -137,11 +141,15 @@ int ensure_capacity(Workspace* w, size_t bytes) {
     cudaGetLastError();
     return fail(MXMOE_ENOMEM, "workspace of %zu bytes: %s", want, cudaGetErrorString(e));
   }
+  // the first kTicketBytes hold the down kernel's per-row-group tickets, which must read
+  // zero at the start of every call (each call leaves them at zero)
+  if ((e = cudaMemset(w->base, 0, kTicketBytes)) != cudaSuccess) return cuda_fail(e, "cudaMemset");
   w->cap = want;
   return MXMOE_OK;
 }
 
-// Bump layout over the workspace; every slice is 256-byte aligned.
+// Bump layout over the workspace; every slice is 256-byte aligned. The first slice of
+// every layout is the ticket array (kTicketBytes, see ensure_capacity).
 struct Carve {
   size_t off = 0;
   template <class T>
@@ -153,6 +161,7 @@ struct Carve {
 };
 
 struct LayerBuffers {
+  unsigned* tickets;
   float* logits;
   int32_t* topk_idx;
   float* topk_w;
@@ -175,6 +184,7 @@ struct LayerBuffers {
 size_t layout(int T, int E, int k, int H, int I, bool fp8, bool tc, LayerBuffers* b, char* base) {
   const int64_t P = static_cast<int64_t>(T) * k;
   Carve c;
+  size_t o_tickets = c.take<uint8_t>(kTicketBytes);
   size_t o_logits = c.take<float>(static_cast<int64_t>(T) * E);
   size_t o_idx = c.take<int32_t>(P), o_w = c.take<float>(P);
   size_t o_counts = c.take<int32_t>(static_cast<int64_t>(mxmoe::permute_chunks(P)) * E);
@@ -188,6 +198,7 @@ size_t layout(int T, int E, int k, int H, int I, bool fp8, bool tc, LayerBuffers
   size_t o_a1 = c.take<uint8_t>(tc ? P * H : 0);
   size_t o_a2 = c.take<uint8_t>(tc ? P * I : 0);
   if (b) {
+    b->tickets = reinterpret_cast<unsigned*>(base + o_tickets);
     b->logits = reinterpret_cast<float*>(base + o_logits);
     b->topk_idx = reinterpret_cast<int32_t*>(base + o_idx);
     b->topk_w = reinterpret_cast<float*>(base + o_w);
@@ -278,16 +289,26 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
   const float s0 = fp8 ? act_scale[0] : 1.0f, s1 = fp8 ? act_scale[1] : 1.0f;
 
   StageTimer tm(st);
-  if ((e = launch_router(a.x, a.router_w, a.router_b, a.T, a.H, a.E, b.logits, st))) return cuda_fail(e, "router");
-  ++launches;
-  tm.mark("router");
-  if ((e = launch_topk(b.logits, a.T, a.E, a.k, b.topk_idx, b.topk_w, st))) return cuda_fail(e, "topk");
-  ++launches;
-  tm.mark("topk");
-  if ((e = launch_permute(b.topk_idx, a.T, a.E, a.k, b.counts, b.offsets, b.perm_token, b.perm_slot,
-                          b.inv, b.active, b.n_active, ws->err, st, &launches)))
-    return cuda_fail(e, "permute");
-  tm.mark("permute");
+  if (route_small_supported(a.T, a.E, a.k)) {
+    // small batch: router, top-k and permutation in one CTA, one launch
+    if ((e = launch_route_small(a.x, a.router_w, a.router_b, a.T, a.H, a.E, a.k, b.logits,
+                                b.tickets + kRouteTicket, b.topk_idx, b.topk_w, b.offsets, b.perm_token,
+                                b.perm_slot, b.inv, b.active, b.n_active, ws->err, st)))
+      return cuda_fail(e, "route");
+    ++launches;
+    tm.mark("route");
+  } else {
+    if ((e = launch_router(a.x, a.router_w, a.router_b, a.T, a.H, a.E, b.logits, st))) return cuda_fail(e, "router");
+    ++launches;
+    tm.mark("router");
+    if ((e = launch_topk(b.logits, a.T, a.E, a.k, b.topk_idx, b.topk_w, st))) return cuda_fail(e, "topk");
+    ++launches;
+    tm.mark("topk");
+    if ((e = launch_permute(b.topk_idx, a.T, a.E, a.k, b.counts, b.offsets, b.perm_token, b.perm_slot,
+                            b.inv, b.active, b.n_active, ws->err, st, &launches)))
+      return cuda_fail(e, "permute");
+    tm.mark("permute");
+  }
   if (tc) {
     if ((e = launch_fp8_quant(a.x, static_cast<int64_t>(a.T) * a.H, s0, b.xq8, st, ws->sms)))
       return cuda_fail(e, "fp8 activation cast");
@@ -330,7 +351,7 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
   if ((e = launch_expert_mma(a.gu_blocks, a.gu_scales, a.gu_bias, 2 * a.I, a.H, act_in,
                              b.perm_token, b.offsets, b.active, b.n_active, max_active, s0, 0, a.I,
                              fp8 ? s1 : 0.0f, b.act_mid, nullptr, calib_out ? b.amax + 1 : nullptr,
-                             a.T, ws->err, st)))
+                             a.T, ws->err, nullptr, st)))
     return cuda_fail(e, "gate_up");
   ++launches;
   tm.mark("gate_up");
@@ -340,16 +361,20 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
     t_last_launches = launches;
     return MXMOE_OK;
   }
+  const bool fold = a.T <= kFoldCombineMaxT && a.H / 16 <= kRouteTicket;
+  const CombineArgs cmb{out, b.topk_idx, b.topk_w, b.inv, b.tickets, a.T, a.k};
   if ((e = launch_expert_mma(a.d_blocks, a.d_scales, a.d_bias, a.H, a.I, b.act_mid, nullptr,
                              b.offsets, b.active, b.n_active, max_active, s1, 1, a.I, 0.0f, nullptr,
-                             b.y, nullptr, a.T, ws->err, st)))
+                             b.y, nullptr, a.T, ws->err, fold ? &cmb : nullptr, st)))
     return cuda_fail(e, "down");
   ++launches;
-  tm.mark("down");
-  if ((e = launch_combine(b.y, b.topk_idx, b.topk_w, b.inv, a.T, a.H, a.k, out, st, ws->sms)))
-    return cuda_fail(e, "combine");
-  ++launches;
-  tm.mark("combine");
+  tm.mark(fold ? "down+combine" : "down");
+  if (!fold) {
+    if ((e = launch_combine(b.y, b.topk_idx, b.topk_w, b.inv, a.T, a.H, a.k, out, st, ws->sms)))
+      return cuda_fail(e, "combine");
+    ++launches;
+    tm.mark("combine");
+  }
   t_last_launches = launches;
   return MXMOE_OK;
 }
@@ -404,8 +429,8 @@ int moe_route_topk(const uint16_t* x, const uint16_t* router_w, const uint16_t* 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float* logits = logits_out;
   if (!logits) {
-    if (int rc = ensure_capacity(ws, static_cast<size_t>(T) * E * sizeof(float))) return rc;
-    logits = reinterpret_cast<float*>(ws->base);
+    if (int rc = ensure_capacity(ws, kTicketBytes + static_cast<size_t>(T) * E * sizeof(float))) return rc;
+    logits = reinterpret_cast<float*>(ws->base + kTicketBytes);
   }
   cudaError_t e = mxmoe::launch_router(x, router_w, router_b, T, H, E, logits, st);
   if (e) return cuda_fail(e, "router launch");
@@ -438,6 +463,7 @@ int moe_permute(const int32_t* topk_idx, int T, int E, int k, int32_t* offsets,
     return e ? cuda_fail(e, "memset") : MXMOE_OK;
   }
   Carve c;
+  c.take<uint8_t>(kTicketBytes);
   size_t o_counts = c.take<int32_t>(static_cast<int64_t>(mxmoe::permute_chunks(P)) * E);
   size_t o_act = c.take<int32_t>(E), o_n = c.take<int32_t>(1);
   if (int rc = ensure_capacity(ws, c.off)) return rc;

@@ -26,6 +26,7 @@
 // group; its warps split the K blocks so that many loads are in flight per SM even when
 // few experts are active, and their partial sums are added in a fixed order.
 #include "common.cuh"
+#include "launchers.h"
 
 namespace mxmoe {
 
@@ -106,6 +107,14 @@ struct ExpertGemmArgs {
   float* y_out;            // (P, rows_total) fp32 (mode 1)
   unsigned* amax_bits;     // optional: running max |a| (fp32 bits), mode 0
   int* err;                // device error word (bounded-wait timeout)
+  // mode 1 with the combine folded in (combine_out != nullptr): the last CTA of each
+  // 16-row group writes out[t, rows] = bf16(sum_j w[t,j] * y[inv[t,j], rows])
+  uint16_t* combine_out;   // (T, rows_total) bf16
+  const int32_t* topk_idx; // (T, k)
+  const float* topk_w;     // (T, k)
+  const int32_t* inv;      // (T*k) pair -> position
+  unsigned* tickets;       // one per 16-row group, zero between calls
+  int T, k;
 };
 
 // One CTA = one 16-row weight group of one active expert (gate_up: 8 gate + the 8
@@ -311,6 +320,39 @@ __global__ void __launch_bounds__(kWarps * 32) expert_mma_kernel(ExpertGemmArgs 
     }
     __syncthreads();
   }
+
+  if (p.mode == 1 && p.combine_out != nullptr) {
+    // every CTA of this row group (one per active expert) stores its y rows and takes a
+    // ticket; the last one adds the group's rows for all tokens in ascending expert id
+    __shared__ unsigned s_last;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(&p.tickets[blockIdx.x], 1u) == static_cast<unsigned>(*p.n_active) - 1u;
+    __syncthreads();
+    if (s_last) {
+      __threadfence();
+      for (int i = threadIdx.x; i < p.T * 16; i += blockDim.x) {
+        const int t = i >> 4, r = lo0 + (i & 15);
+        int ord[8], eid[8];
+        for (int j = 0; j < p.k; ++j) {
+          const int ex = p.topk_idx[static_cast<int64_t>(t) * p.k + j];
+          int q = j;
+          while (q > 0 && eid[q - 1] > ex) { eid[q] = eid[q - 1]; ord[q] = ord[q - 1]; --q; }
+          eid[q] = ex;
+          ord[q] = j;
+        }
+        float acc = 0.0f;
+        for (int q = 0; q < p.k; ++q) {
+          const int j = ord[q];
+          const int64_t pos = p.inv[static_cast<int64_t>(t) * p.k + j];
+          acc = __fadd_rn(acc, __fmul_rn(p.topk_w[static_cast<int64_t>(t) * p.k + j],
+                                         __ldcg(p.y_out + pos * p.rows_total + r)));
+        }
+        p.combine_out[static_cast<int64_t>(t) * p.rows_total + r] = f32_to_bf16_bits_rn(acc);
+      }
+      if (threadIdx.x == 0) p.tickets[blockIdx.x] = 0u;
+    }
+  }
 }
 
 size_t smem_bytes(int K, int nt) {
@@ -325,9 +367,13 @@ cudaError_t launch_expert_mma(const uint8_t* blocks, const uint8_t* scales, cons
                               const int32_t* offsets, const int32_t* active,
                               const int32_t* n_active, int max_active, float s_in, int mode, int I,
                               float s_mid, uint16_t* act_out, float* y_out, unsigned* amax_bits,
-                              int max_tokens_per_expert, int* err, cudaStream_t st) {
+                              int max_tokens_per_expert, int* err, const CombineArgs* combine,
+                              cudaStream_t st) {
   ExpertGemmArgs a{blocks, scales, bias, rows_total, K, act, act_row, offsets, active, n_active,
-                   s_in, mode, I, s_mid, act_out, y_out, amax_bits, err};
+                   s_in, mode, I, s_mid, act_out, y_out, amax_bits, err,
+                   combine ? combine->out : nullptr, combine ? combine->topk_idx : nullptr,
+                   combine ? combine->topk_w : nullptr, combine ? combine->inv : nullptr,
+                   combine ? combine->tickets : nullptr, combine ? combine->T : 0, combine ? combine->k : 0};
   const int groups = mode == 0 ? I / 8 : rows_total / 16;
   dim3 grid(static_cast<unsigned>(groups), static_cast<unsigned>(max_active));
   // one n-tile (8 tokens) per pass for up to 8 routed tokens, else two per pass; a group's

@@ -20,6 +20,11 @@ cudaError_t launch_permute(const int32_t* idx, int T, int E, int k, int32_t* cou
                            int32_t* offsets, int32_t* perm_token, int32_t* perm_slot,
                            int32_t* inv, int32_t* active, int32_t* n_active, int* err,
                            cudaStream_t st, int* launches);
+bool route_small_supported(int T, int E, int k);
+cudaError_t launch_route_small(const uint16_t* x, const uint16_t* wr, const uint16_t* br, int T, int H, int E,
+                               int k, float* logits, unsigned* ticket, int32_t* topk_idx, float* topk_w,
+                               int32_t* offsets, int32_t* perm_token, int32_t* perm_slot, int32_t* inv,
+                               int32_t* active, int32_t* n_active, int* err, cudaStream_t st);
 cudaError_t launch_fp8_quant(const uint16_t* x, int64_t n, float s, uint8_t* q, cudaStream_t st,
                              int sms);
 cudaError_t launch_fp8_quant_as_bf16(const uint16_t* x, int64_t n, float s, uint16_t* xq,
@@ -30,12 +35,21 @@ cudaError_t launch_amax_bf16(const uint16_t* x, int64_t n, unsigned* amax_bits, 
                              int sms);
 cudaError_t launch_finalize_scales(const unsigned* amax_bits, float* out, cudaStream_t st);
 
+struct CombineArgs {      // the combine folded into the down kernel (small batches)
+  uint16_t* out;
+  const int32_t* topk_idx;
+  const float* topk_w;
+  const int32_t* inv;
+  unsigned* tickets;      // rows_total / 16 counters, zero between calls
+  int T, k;
+};
 cudaError_t launch_expert_mma(const uint8_t* blocks, const uint8_t* scales, const float* bias,
                               int rows_total, int K, const uint16_t* act, const int32_t* act_row,
                               const int32_t* offsets, const int32_t* active,
                               const int32_t* n_active, int max_active, float s_in, int mode, int I,
                               float s_mid, uint16_t* act_out, float* y_out, unsigned* amax_bits,
-                              int max_tokens_per_expert, int* err, cudaStream_t st);
+                              int max_tokens_per_expert, int* err, const CombineArgs* combine,
+                              cudaStream_t st);
 cudaError_t expert_mma_set_smem_limits(int max_K);
 
 bool tc_gemm_supported(int H, int I, const void* gu_blocks, const void* d_blocks);

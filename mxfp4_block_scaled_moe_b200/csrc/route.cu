@@ -157,19 +157,17 @@ __device__ __forceinline__ bool ranks_before(float a, int ia, float b, int ib) {
   return ia < ib;
 }
 
-// One warp per token; each lane holds up to 8 logits (E <= 256).
-__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E,
-                                                    int k, int32_t* __restrict__ idx,
-                                                    float* __restrict__ wts) {
+// One warp selects the k largest of a token's E logits (E <= 256, each lane holds up to 8)
+// and writes the indices and the softmax over them.
+__device__ __forceinline__ void topk_warp(const float* __restrict__ l, int E, int k,
+                                          int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
   const int lane = threadIdx.x & 31;
-  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (t >= T) return;
   float v[8];
   int taken = 0;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int e = lane + 32 * i;
-    v[i] = e < E ? logits[static_cast<int64_t>(t) * E + e] : 0.0f;
+    v[i] = e < E ? l[e] : 0.0f;
   }
   float sel[8];
   int sidx[8];
@@ -200,10 +198,19 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
     float p[8], z = 0.0f;
     for (int j = 0; j < k; ++j) { p[j] = expf(sel[j] - sel[0]); z += p[j]; }
     for (int j = 0; j < k; ++j) {
-      idx[static_cast<int64_t>(t) * k + j] = sidx[j];
-      wts[static_cast<int64_t>(t) * k + j] = __fdiv_rn(p[j], z);
+      idx_out[j] = sidx[j];
+      w_out[j] = __fdiv_rn(p[j], z);
     }
   }
+}
+
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E,
+                                                    int k, int32_t* __restrict__ idx,
+                                                    float* __restrict__ wts) {
+  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (t >= T) return;
+  topk_warp(logits + static_cast<int64_t>(t) * E, E, k, idx + static_cast<int64_t>(t) * k,
+            wts + static_cast<int64_t>(t) * k);
 }
 
 // --------------------------------------------------------------------- permute -----
@@ -230,19 +237,27 @@ __global__ void __launch_bounds__(kPermThreads) permute_count_kernel(
   for (int e = threadIdx.x; e < E; e += blockDim.x) counts[static_cast<int64_t>(blockIdx.x) * E + e] = hist[e];
 }
 
-// counts == nullptr: single-CTA mode (the CTA builds its own histogram first).
-__global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(
-    const int32_t* __restrict__ idx, int64_t P, int E, int k, const int32_t* __restrict__ counts,
-    int32_t* __restrict__ offsets, int32_t* __restrict__ perm_token,
+struct PermuteSmem {
+  int base[256];
+  int total[256];
+  int wc[kPermThreads / 32][256];
+  int scan_tmp[256];
+};
+
+// The scatter pass, run by one CTA of kPermThreads threads for chunk `cta` (counts ==
+// nullptr: single-CTA mode, the CTA builds its own histogram of all P pairs first).
+__device__ void permute_scatter_body(
+    PermuteSmem& sm, int cta, const int32_t* __restrict__ idx, int64_t P, int E, int k,
+    const int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ perm_token,
     int32_t* __restrict__ perm_slot, int32_t* __restrict__ inv, int32_t* __restrict__ active,
     int32_t* __restrict__ n_active, int* __restrict__ err) {
-  __shared__ int base[256];
-  __shared__ int total[256];
-  __shared__ int wc[kPermThreads / 32][256];
-  __shared__ int scan_tmp[256];
+  int* base = sm.base;
+  int* total = sm.total;
+  int (*wc)[256] = sm.wc;
+  int* scan_tmp = sm.scan_tmp;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nchunks = static_cast<int>(cdiv(P, kPermChunk));
-  const int64_t lo = static_cast<int64_t>(blockIdx.x) * kPermChunk;
+  const int64_t lo = static_cast<int64_t>(cta) * kPermChunk;
   const int64_t hi = min(P, lo + kPermChunk);
 
   if (counts == nullptr) {
@@ -260,13 +275,13 @@ __global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(
       int before = 0, all = 0;
       for (int c = 0; c < nchunks; ++c) {
         const int v = counts[static_cast<int64_t>(c) * E + e];
-        if (c < static_cast<int>(blockIdx.x)) before += v;
+        if (c < cta) before += v;
         all += v;
       }
       total[e] = all;
       base[e] = before;
     }
-    if (blockIdx.x == 0)
+    if (cta == 0)
       for (int64_t p = tid; p < P; p += blockDim.x) {
         const int e = idx[p];
         if (e < 0 || e >= E) set_device_error(err, MXMOE_EDEVICE);
@@ -288,14 +303,14 @@ __global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(
       if (e < E) scan_tmp[e] = carry + incl - v;
       carry += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (blockIdx.x == 0 && lane == 0) offsets[E] = carry;
+    if (cta == 0 && lane == 0) offsets[E] = carry;
   }
   __syncthreads();
   for (int e = tid; e < E; e += blockDim.x) {
     base[e] += scan_tmp[e];
-    if (blockIdx.x == 0) offsets[e] = scan_tmp[e];
+    if (cta == 0) offsets[e] = scan_tmp[e];
   }
-  if (blockIdx.x == 0 && tid == 0) {
+  if (cta == 0 && tid == 0) {
     int n = 0;
     for (int e = 0; e < E; ++e)
       if (total[e] > 0) active[n++] = e;
@@ -306,11 +321,11 @@ __global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(
   const int64_t my_lo = counts == nullptr ? 0 : lo;
   const int64_t my_hi = counts == nullptr ? P : hi;
   const unsigned lt_mask = (1u << lane) - 1u;
-  for (int64_t sub = my_lo; sub < my_hi; sub += kPermThreads) {
+  for (int64_t sub = my_lo; sub < my_hi; sub += blockDim.x) {
     const int64_t p = sub + tid;
     int e = p < my_hi ? idx[p] : -1;
     if (e >= E) e = -1;
-    for (int i = tid; i < (kPermThreads / 32) * 256; i += blockDim.x) (&wc[0][0])[i] = 0;
+    for (int i = tid; i < (kPermThreads / 32) * 256; i += blockDim.x) (&wc[0][0])[i] = 0;  // all slots
     const unsigned peers = __match_any_sync(0xffffffffu, e);
     const int rank = __popc(peers & lt_mask);
     __syncthreads();
@@ -337,6 +352,97 @@ __global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(
     for (int ee = tid; ee < E; ee += blockDim.x) base[ee] += scan_tmp[ee];
     __syncthreads();
   }
+}
+
+__global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(
+    const int32_t* __restrict__ idx, int64_t P, int E, int k, const int32_t* __restrict__ counts,
+    int32_t* __restrict__ offsets, int32_t* __restrict__ perm_token,
+    int32_t* __restrict__ perm_slot, int32_t* __restrict__ inv, int32_t* __restrict__ active,
+    int32_t* __restrict__ n_active, int* __restrict__ err) {
+  __shared__ PermuteSmem sm;
+  permute_scatter_body(sm, blockIdx.x, idx, P, E, k, counts, offsets, perm_token, perm_slot, inv, active,
+                       n_active, err);
+}
+
+// ----------------------------------------------------------- fused small-batch routing -
+// One launch for the routing of a small batch: every warp computes one (token, expert)
+// logit (the router GEMV's arithmetic), and the CTA that finishes last (an atomic ticket,
+// reset for the next call) runs the top-k softmax (one warp per token) and the single-CTA
+// permutation. Saves two launches on the latency-bound decode path.
+constexpr int kSmallT = 64, kSmallE = 256;
+
+__global__ void __launch_bounds__(kPermThreads) route_small_kernel(
+    const uint16_t* __restrict__ x, const uint16_t* __restrict__ wr, const uint16_t* __restrict__ br,
+    int T, int H, int E, int k, float* __restrict__ logits, unsigned* __restrict__ ticket,
+    int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+    int32_t* __restrict__ offsets, int32_t* __restrict__ perm_token, int32_t* __restrict__ perm_slot,
+    int32_t* __restrict__ inv, int32_t* __restrict__ active, int32_t* __restrict__ n_active,
+    int* __restrict__ err) {
+  __shared__ PermuteSmem sm;
+  __shared__ unsigned s_last;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int64_t wid = static_cast<int64_t>(blockIdx.x) * nwarps + warp;
+  if (wid < static_cast<int64_t>(T) * E) {
+    const int t = static_cast<int>(wid / E), e = static_cast<int>(wid % E);
+    const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(t) * H);
+    const uint4* wrow = reinterpret_cast<const uint4*>(wr + static_cast<int64_t>(e) * H);
+    float acc = 0.0f;
+    for (int c = lane; c < H / 8; c += 32) {
+      const uint4 a = ld_nc_v4(xr + c), b = ld_nc_v4(wrow + c);
+      const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc = fmaf(__uint_as_float(av[i] << 16), __uint_as_float(bv[i] << 16), acc);
+        acc = fmaf(__uint_as_float(av[i] & 0xFFFF0000u), __uint_as_float(bv[i] & 0xFFFF0000u), acc);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) logits[wid] = br ? acc + bf16_bits_to_f32(br[e]) : acc;
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = atomicAdd(ticket, 1u) == gridDim.x - 1u;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  for (int t = warp; t < T; t += nwarps) {
+    // the other CTAs' logits: read through L2
+    float lv[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane + 32 * i;
+      lv[i] = e < E ? __ldcg(logits + static_cast<int64_t>(t) * E + e) : 0.0f;
+    }
+    __shared__ float s_row[kPermThreads / 32][256];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E) s_row[warp][e] = lv[i];
+    }
+    __syncwarp();
+    topk_warp(s_row[warp], E, k, topk_idx + static_cast<int64_t>(t) * k, topk_w + static_cast<int64_t>(t) * k);
+    __syncwarp();
+  }
+  __syncthreads();   // the CTA's global writes of topk_idx are visible to all its threads
+  permute_scatter_body(sm, 0, topk_idx, static_cast<int64_t>(T) * k, E, k, nullptr, offsets, perm_token,
+                       perm_slot, inv, active, n_active, err);
+  if (threadIdx.x == 0) *ticket = 0u;
+}
+
+bool route_small_supported(int T, int E, int k) {
+  return T <= kSmallT && E <= kSmallE && static_cast<int64_t>(T) * k <= kPermChunk;
+}
+
+cudaError_t launch_route_small(const uint16_t* x, const uint16_t* wr, const uint16_t* br, int T, int H, int E,
+                               int k, float* logits, unsigned* ticket, int32_t* topk_idx, float* topk_w,
+                               int32_t* offsets, int32_t* perm_token, int32_t* perm_slot, int32_t* inv,
+                               int32_t* active, int32_t* n_active, int* err, cudaStream_t st) {
+  const int64_t warps = static_cast<int64_t>(T) * E;
+  const unsigned grid = static_cast<unsigned>(cdiv(warps, kPermThreads / 32));
+  route_small_kernel<<<grid, kPermThreads, 0, st>>>(x, wr, br, T, H, E, k, logits, ticket, topk_idx, topk_w,
+                                                    offsets, perm_token, perm_slot, inv, active, n_active, err);
+  return cudaGetLastError();
 }
 
 // ------------------------------------------------------------ activation casts -----
