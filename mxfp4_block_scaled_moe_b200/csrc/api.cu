@@ -90,6 +90,7 @@ struct Workspace {
   int sms = 0;
   int smem_K = 0;      // largest K the expert kernels were configured for
   bool tc_ready = false;  // tcgen05 GEMM shared-memory limit raised
+  bool dtc_ready = false; // tensor-core decode kernels' shared-memory limit raised
 };
 
 // Routed pairs from which the FP8 path runs on the tcgen05 grouped GEMM (fewer pairs use
@@ -179,9 +180,13 @@ struct LayerBuffers {
   uint8_t* xq8;        // tcgen05 path: e4m3 codes of x / s0, (T, H)
   uint8_t* a1;         // tcgen05 path: gate_up input rows grouped by expert, (P, H)
   uint8_t* a2;         // tcgen05 path: down input rows, (P, I)
+  uint8_t* xs;         // tensor-core decode: gate_up B rows (P*np, H) e4m3 parts
+  uint8_t* sfb;        // their scale records
+  uint8_t* xs_mid;     // down B rows (P*np, I)
+  uint8_t* sfb_mid;
 };
 
-size_t layout(int T, int E, int k, int H, int I, bool fp8, bool tc, LayerBuffers* b, char* base) {
+size_t layout(int T, int E, int k, int H, int I, bool fp8, bool tc, bool dtc, LayerBuffers* b, char* base) {
   const int64_t P = static_cast<int64_t>(T) * k;
   Carve c;
   size_t o_tickets = c.take<uint8_t>(kTicketBytes);
@@ -197,6 +202,11 @@ size_t layout(int T, int E, int k, int H, int I, bool fp8, bool tc, LayerBuffers
   size_t o_xq8 = c.take<uint8_t>(tc ? static_cast<int64_t>(T) * H : 0);
   size_t o_a1 = c.take<uint8_t>(tc ? P * H : 0);
   size_t o_a2 = c.take<uint8_t>(tc ? P * I : 0);
+  const int np = fp8 ? 1 : 3;
+  size_t o_xs = c.take<uint8_t>(dtc ? P * np * H : 0);
+  size_t o_sfb = c.take<uint8_t>(dtc ? static_cast<int64_t>(mxmoe::decode_tc_sfb_bytes(E, H)) : 0);
+  size_t o_xsm = c.take<uint8_t>(dtc ? P * np * I : 0);
+  size_t o_sfbm = c.take<uint8_t>(dtc ? static_cast<int64_t>(mxmoe::decode_tc_sfb_bytes(E, I)) : 0);
   if (b) {
     b->tickets = reinterpret_cast<unsigned*>(base + o_tickets);
     b->logits = reinterpret_cast<float*>(base + o_logits);
@@ -216,6 +226,10 @@ size_t layout(int T, int E, int k, int H, int I, bool fp8, bool tc, LayerBuffers
     b->xq8 = reinterpret_cast<uint8_t*>(base + o_xq8);
     b->a1 = reinterpret_cast<uint8_t*>(base + o_a1);
     b->a2 = reinterpret_cast<uint8_t*>(base + o_a2);
+    b->xs = reinterpret_cast<uint8_t*>(base + o_xs);
+    b->sfb = reinterpret_cast<uint8_t*>(base + o_sfb);
+    b->xs_mid = reinterpret_cast<uint8_t*>(base + o_xsm);
+    b->sfb_mid = reinterpret_cast<uint8_t*>(base + o_sfbm);
   }
   return c.off;
 }
@@ -270,7 +284,10 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
   const int64_t P = static_cast<int64_t>(a.T) * a.k;
   const bool tc = fp8 && !calib_out && P >= tc_min_pairs() && std::max(a.H, a.I) / 32 <= kTcMaxNb &&
                   tc_gemm_supported(a.H, a.I, a.gu_blocks, a.d_blocks);
-  const size_t need = layout(a.T, a.E, a.k, a.H, a.I, fp8, tc, nullptr, nullptr);
+  const int np = fp8 ? 1 : 3;
+  const bool dtc = !tc && !calib_out && a.T <= kFoldCombineMaxT && a.H / 128 < kRouteTicket &&
+                   decode_tc_supported(a.H, a.I, np, a.T, a.gu_blocks, a.d_blocks);
+  const size_t need = layout(a.T, a.E, a.k, a.H, a.I, fp8, tc, dtc, nullptr, nullptr);
   if (int rc = ensure_capacity(ws, need)) return rc;
   if (std::max(a.H, a.I) > ws->smem_K) {
     cudaError_t e = expert_mma_set_smem_limits(std::max(a.H, a.I));
@@ -282,8 +299,13 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (tcgen05 GEMM)");
     ws->tc_ready = true;
   }
+  if (dtc && !ws->dtc_ready) {
+    cudaError_t e = decode_tc_prepare();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (tensor-core decode)");
+    ws->dtc_ready = true;
+  }
   LayerBuffers b;
-  layout(a.T, a.E, a.k, a.H, a.I, fp8, tc, &b, ws->base);
+  layout(a.T, a.E, a.k, a.H, a.I, fp8, tc, dtc, &b, ws->base);
   int launches = 0;
   cudaError_t e;
   const float s0 = fp8 ? act_scale[0] : 1.0f, s1 = fp8 ? act_scale[1] : 1.0f;
@@ -331,6 +353,34 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
       return cuda_fail(e, "combine");
     ++launches;
     tm.mark("combine");
+    t_last_launches = launches;
+    return MXMOE_OK;
+  }
+  if (dtc) {
+    // small batch on the tensor cores: tokens as MX-FP8 parts, weights as the A operand
+    if ((e = launch_split_tokens(np, a.x, b.perm_token, b.perm_slot, b.topk_idx, b.offsets, P, a.H, a.k, s0,
+                                 b.xs, b.sfb, st)))
+      return cuda_fail(e, "split");
+    ++launches;
+    tm.mark("act_split");
+    DecodeGemmArgs d{};
+    d.gu_blocks = a.gu_blocks; d.gu_scales = a.gu_scales; d.gu_bias = a.gu_bias;
+    d.d_blocks = a.d_blocks; d.d_scales = a.d_scales; d.d_bias = a.d_bias;
+    d.E = a.E; d.H = a.H; d.I = a.I; d.T = a.T; d.k = a.k; d.P = P;
+    d.np = np; d.np_mid = np;
+    d.max_tokens_per_expert = a.T;
+    d.max_active = static_cast<int>(std::min<int64_t>(a.E, P));
+    d.offsets = b.offsets; d.active = b.active; d.n_active = b.n_active;
+    d.topk_idx = b.topk_idx; d.topk_w = b.topk_w; d.inv = b.inv;
+    d.xs = b.xs; d.sfb = b.sfb; d.xs_mid = b.xs_mid; d.sfb_mid = b.sfb_mid;
+    d.s0 = s0; d.s1_quant = fp8 ? s1 : 0.0f; d.s1_in = s1;
+    d.amax_bits = nullptr; d.y = b.y; d.out = out; d.tickets = b.tickets; d.err = ws->err;
+    if ((e = launch_decode_gemm(true, d, st))) return cuda_fail(e, "gate_up (tensor-core decode)");
+    ++launches;
+    tm.mark("gate_up");
+    if ((e = launch_decode_gemm(false, d, st))) return cuda_fail(e, "down+combine (tensor-core decode)");
+    ++launches;
+    tm.mark("down+combine");
     t_last_launches = launches;
     return MXMOE_OK;
   }

@@ -25,13 +25,22 @@ __global__ void __launch_bounds__(256) router_gemv_kernel(const uint16_t* __rest
   const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(t) * H);
   const uint4* wrow = reinterpret_cast<const uint4*>(wr + static_cast<int64_t>(e) * H);
   float acc = 0.0f;
-  for (int c = lane; c < H / 8; c += 32) {
-    const uint4 a = ld_nc_v4(xr + c), b = ld_nc_v4(wrow + c);
-    const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+  for (int c0 = lane; c0 < H / 8; c0 += 4 * 32) {
+    uint4 a[4], b[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      acc = fmaf(__uint_as_float(av[i] << 16), __uint_as_float(bv[i] << 16), acc);
-      acc = fmaf(__uint_as_float(av[i] & 0xFFFF0000u), __uint_as_float(bv[i] & 0xFFFF0000u), acc);
+    for (int u = 0; u < 4; ++u) {
+      const int c = c0 + 32 * u;
+      if (c < H / 8) { a[u] = ld_nc_v4(xr + c); b[u] = ld_nc_v4(wrow + c); }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (c0 + 32 * u >= H / 8) break;
+      const uint32_t av[4] = {a[u].x, a[u].y, a[u].z, a[u].w}, bv[4] = {b[u].x, b[u].y, b[u].z, b[u].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc = fmaf(__uint_as_float(av[i] << 16), __uint_as_float(bv[i] << 16), acc);
+        acc = fmaf(__uint_as_float(av[i] & 0xFFFF0000u), __uint_as_float(bv[i] & 0xFFFF0000u), acc);
+      }
     }
   }
 #pragma unroll
@@ -387,13 +396,24 @@ __global__ void __launch_bounds__(kPermThreads) route_small_kernel(
     const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(t) * H);
     const uint4* wrow = reinterpret_cast<const uint4*>(wr + static_cast<int64_t>(e) * H);
     float acc = 0.0f;
-    for (int c = lane; c < H / 8; c += 32) {
-      const uint4 a = ld_nc_v4(xr + c), b = ld_nc_v4(wrow + c);
-      const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+    // four 16-byte chunks of each operand in flight per lane, then their FMAs in chunk
+    // order (the same order as one chunk at a time)
+    for (int c0 = lane; c0 < H / 8; c0 += 4 * 32) {
+      uint4 a[4], b[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        acc = fmaf(__uint_as_float(av[i] << 16), __uint_as_float(bv[i] << 16), acc);
-        acc = fmaf(__uint_as_float(av[i] & 0xFFFF0000u), __uint_as_float(bv[i] & 0xFFFF0000u), acc);
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + 32 * u;
+        if (c < H / 8) { a[u] = ld_nc_v4(xr + c); b[u] = ld_nc_v4(wrow + c); }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (c0 + 32 * u >= H / 8) break;
+        const uint32_t av[4] = {a[u].x, a[u].y, a[u].z, a[u].w}, bv[4] = {b[u].x, b[u].y, b[u].z, b[u].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          acc = fmaf(__uint_as_float(av[i] << 16), __uint_as_float(bv[i] << 16), acc);
+          acc = fmaf(__uint_as_float(av[i] & 0xFFFF0000u), __uint_as_float(bv[i] & 0xFFFF0000u), acc);
+        }
       }
     }
 #pragma unroll

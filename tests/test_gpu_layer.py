@@ -107,6 +107,15 @@ def test_decode_20b_shape_all_outputs(B, T):
     check_rows(B, p, d, np.arange(T))
 
 
+def test_decode_20b_shape_fp8(B):
+    """FP8 activations on a decode batch: one MX-FP8 part per token on the tensor-core
+    decode path (static scales from the calibration batch)."""
+    p, d = layer_case(inputs.decode_layer(T=8, E=32, device="cuda"))
+    xc = inputs.calibration_x(device="cuda")
+    s = oracle.calibrate(inputs.bits(xc), p.router_w, p.router_b, *p.weights, p.lay.k)
+    check_rows(B, p, d, np.arange(8), act_scale=s)
+
+
 def test_decode_23_experts(B):
     p, d = layer_case(inputs.decode_layer(T=8, E=23, device="cuda"))
     check_rows(B, p, d, np.arange(8))
