@@ -91,6 +91,7 @@ struct Workspace {
   int smem_K = 0;      // largest K the expert kernels were configured for
   bool tc_ready = false;  // tcgen05 GEMM shared-memory limit raised
   bool dtc_ready = false; // tensor-core decode kernels' shared-memory limit raised
+  size_t tickets_zeroed = 0;  // bytes at the start of the workspace known to be zero
 };
 
 // Routed pairs from which the FP8 path runs on the tcgen05 grouped GEMM (fewer pairs use
@@ -145,6 +146,7 @@ int ensure_capacity(Workspace* w, size_t bytes) {
   // the first kTicketBytes hold the down kernel's per-row-group tickets, which must read
   // zero at the start of every call (each call leaves them at zero)
   if ((e = cudaMemset(w->base, 0, kTicketBytes)) != cudaSuccess) return cuda_fail(e, "cudaMemset");
+  w->tickets_zeroed = kTicketBytes;
   w->cap = want;
   return MXMOE_OK;
 }
@@ -180,16 +182,21 @@ struct LayerBuffers {
   uint8_t* xq8;        // tcgen05 path: e4m3 codes of x / s0, (T, H)
   uint8_t* a1;         // tcgen05 path: gate_up input rows grouped by expert, (P, H)
   uint8_t* a2;         // tcgen05 path: down input rows, (P, I)
-  uint8_t* xs;         // tensor-core decode: gate_up B rows (P*np, H) e4m3 parts
+  uint8_t* xs;         // tensor-core decode: gate_up B rows (P*4, H/2) packed e2m1 parts
   uint8_t* sfb;        // their scale records
-  uint8_t* xs_mid;     // down B rows (P*np, I)
+  uint8_t* xs_mid;     // down B rows (P*4, I/2)
   uint8_t* sfb_mid;
+  unsigned* dtickets;  // tensor-core decode: split-K and combine tickets (zero between calls)
+  size_t tickets_end;  // bytes from the workspace start that hold tickets
+  float* part;         // tensor-core decode: split-K partial accumulators
 };
 
 size_t layout(int T, int E, int k, int H, int I, bool fp8, bool tc, bool dtc, LayerBuffers* b, char* base) {
   const int64_t P = static_cast<int64_t>(T) * k;
   Carve c;
   size_t o_tickets = c.take<uint8_t>(kTicketBytes);
+  size_t o_dtick = c.take<unsigned>(dtc ? static_cast<int64_t>(mxmoe::decode_tc_ticket_count(H, I)) : 0);
+  const size_t tickets_end = c.off;
   size_t o_logits = c.take<float>(static_cast<int64_t>(T) * E);
   size_t o_idx = c.take<int32_t>(P), o_w = c.take<float>(P);
   size_t o_counts = c.take<int32_t>(static_cast<int64_t>(mxmoe::permute_chunks(P)) * E);
@@ -202,12 +209,15 @@ size_t layout(int T, int E, int k, int H, int I, bool fp8, bool tc, bool dtc, La
   size_t o_xq8 = c.take<uint8_t>(tc ? static_cast<int64_t>(T) * H : 0);
   size_t o_a1 = c.take<uint8_t>(tc ? P * H : 0);
   size_t o_a2 = c.take<uint8_t>(tc ? P * I : 0);
-  const int np = fp8 ? 1 : 3;
-  size_t o_xs = c.take<uint8_t>(dtc ? P * np * H : 0);
-  size_t o_sfb = c.take<uint8_t>(dtc ? static_cast<int64_t>(mxmoe::decode_tc_sfb_bytes(E, H)) : 0);
-  size_t o_xsm = c.take<uint8_t>(dtc ? P * np * I : 0);
-  size_t o_sfbm = c.take<uint8_t>(dtc ? static_cast<int64_t>(mxmoe::decode_tc_sfb_bytes(E, I)) : 0);
+  size_t o_xs = c.take<uint8_t>(dtc ? static_cast<int64_t>(mxmoe::decode_tc_xs_bytes(P, H)) : 0);
+  size_t o_sfb = c.take<uint8_t>(dtc ? static_cast<int64_t>(mxmoe::decode_tc_sfb_bytes(E, H, T)) : 0);
+  size_t o_xsm = c.take<uint8_t>(dtc ? static_cast<int64_t>(mxmoe::decode_tc_xs_bytes(P, I)) : 0);
+  size_t o_sfbm = c.take<uint8_t>(dtc ? static_cast<int64_t>(mxmoe::decode_tc_sfb_bytes(E, I, T)) : 0);
+  size_t o_part = c.take<uint8_t>(dtc ? static_cast<int64_t>(mxmoe::decode_tc_part_bytes(P, H, I)) : 0);
   if (b) {
+    b->dtickets = reinterpret_cast<unsigned*>(base + o_dtick);
+    b->tickets_end = tickets_end;
+    b->part = reinterpret_cast<float*>(base + o_part);
     b->tickets = reinterpret_cast<unsigned*>(base + o_tickets);
     b->logits = reinterpret_cast<float*>(base + o_logits);
     b->topk_idx = reinterpret_cast<int32_t*>(base + o_idx);
@@ -284,9 +294,7 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
   const int64_t P = static_cast<int64_t>(a.T) * a.k;
   const bool tc = fp8 && !calib_out && P >= tc_min_pairs() && std::max(a.H, a.I) / 32 <= kTcMaxNb &&
                   tc_gemm_supported(a.H, a.I, a.gu_blocks, a.d_blocks);
-  const int np = fp8 ? 1 : 3;
-  const bool dtc = !tc && !calib_out && a.T <= kFoldCombineMaxT && a.H / 128 < kRouteTicket &&
-                   decode_tc_supported(a.H, a.I, np, a.T, a.gu_blocks, a.d_blocks);
+  const bool dtc = !tc && !calib_out && decode_tc_supported(a.H, a.I, a.T, a.gu_blocks, a.d_blocks);
   const size_t need = layout(a.T, a.E, a.k, a.H, a.I, fp8, tc, dtc, nullptr, nullptr);
   if (int rc = ensure_capacity(ws, need)) return rc;
   if (std::max(a.H, a.I) > ws->smem_K) {
@@ -306,6 +314,13 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
   }
   LayerBuffers b;
   layout(a.T, a.E, a.k, a.H, a.I, fp8, tc, dtc, &b, ws->base);
+  if (b.tickets_end > ws->tickets_zeroed) {
+    // the decode path's tickets reach past what is known to be zero: clear them once
+    // (every call leaves them at zero again)
+    cudaError_t e = cudaMemsetAsync(ws->base, 0, b.tickets_end, st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync (tickets)");
+    ws->tickets_zeroed = b.tickets_end;
+  }
   int launches = 0;
   cudaError_t e;
   const float s0 = fp8 ? act_scale[0] : 1.0f, s1 = fp8 ? act_scale[1] : 1.0f;
@@ -358,7 +373,7 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
   }
   if (dtc) {
     // small batch on the tensor cores: tokens as MX-FP8 parts, weights as the A operand
-    if ((e = launch_split_tokens(np, a.x, b.perm_token, b.perm_slot, b.topk_idx, b.offsets, P, a.H, a.k, s0,
+    if ((e = launch_split_tokens(fp8, a.x, b.perm_token, b.perm_slot, b.topk_idx, b.offsets, P, a.H, a.k, s0, a.T,
                                  b.xs, b.sfb, st)))
       return cuda_fail(e, "split");
     ++launches;
@@ -367,19 +382,34 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
     d.gu_blocks = a.gu_blocks; d.gu_scales = a.gu_scales; d.gu_bias = a.gu_bias;
     d.d_blocks = a.d_blocks; d.d_scales = a.d_scales; d.d_bias = a.d_bias;
     d.E = a.E; d.H = a.H; d.I = a.I; d.T = a.T; d.k = a.k; d.P = P;
-    d.np = np; d.np_mid = np;
-    d.max_tokens_per_expert = a.T;
     d.max_active = static_cast<int>(std::min<int64_t>(a.E, P));
+    d.sms = ws->sms;
     d.offsets = b.offsets; d.active = b.active; d.n_active = b.n_active;
     d.topk_idx = b.topk_idx; d.topk_w = b.topk_w; d.inv = b.inv;
     d.xs = b.xs; d.sfb = b.sfb; d.xs_mid = b.xs_mid; d.sfb_mid = b.sfb_mid;
     d.s0 = s0; d.s1_quant = fp8 ? s1 : 0.0f; d.s1_in = s1;
-    d.amax_bits = nullptr; d.y = b.y; d.out = out; d.tickets = b.tickets; d.err = ws->err;
+    d.y = b.y;
+    const bool fold = a.T <= kDecodeFoldMaxT;
+    d.out = fold ? out : nullptr;
+    d.part = b.part;
+    d.split_tickets_gu = b.dtickets;
+    d.split_tickets_d = b.dtickets + decode_tc_tickets_d(a.I);
+    d.comb_tickets = b.dtickets + decode_tc_tickets_comb(a.H, a.I);
+    d.err = ws->err;
     if ((e = launch_decode_gemm(true, d, st))) return cuda_fail(e, "gate_up (tensor-core decode)");
     ++launches;
     tm.mark("gate_up");
-    if ((e = launch_decode_gemm(false, d, st))) return cuda_fail(e, "down+combine (tensor-core decode)");
+    if ((e = launch_decode_gemm(false, d, st))) return cuda_fail(e, "down (tensor-core decode)");
     ++launches;
+    if (!fold) {
+      tm.mark("down");
+      if ((e = launch_combine(b.y, b.topk_idx, b.topk_w, b.inv, a.T, a.H, a.k, out, st, ws->sms)))
+        return cuda_fail(e, "combine");
+      ++launches;
+      tm.mark("combine");
+      t_last_launches = launches;
+      return MXMOE_OK;
+    }
     tm.mark("down+combine");
     t_last_launches = launches;
     return MXMOE_OK;

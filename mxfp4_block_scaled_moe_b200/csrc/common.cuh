@@ -72,6 +72,7 @@ __device__ __forceinline__ float warp_max(float v) {
 
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 
+
 // -------------------------------------------------------------- legacy MMA (mma.sync)
 // m16n8k16, bf16 x bf16 -> fp32. a: 4 regs, b: 2 regs, c/d: 4 fp32.
 __device__ __forceinline__ void mma_bf16_16816(float d[4], const uint32_t a[4], const uint32_t b[2],

@@ -1,30 +1,45 @@
-// Routed expert GEMMs for small batches on the tensor cores, with the MXFP4 weights as
-// the MMA's A operand: the tensor core decodes the e2m1 nibbles and applies their e8m0
-// block scales (tcgen05.mma kind::mxf8f6f4 block_scale), TMA streams the packed weight
-// bytes, and no instruction of the SM touches a nibble. This is the decode path of
-// "quantization_mxfp4" (KerasFormers), As GPT-OSS's native format: only the routed
-// experts' blocks are read, once per layer.
+// Routed expert GEMMs for small batches on the tensor cores (tcgen05.mma kind::mxf4
+// block_scale): both operands are packed e2m1 with e8m0 block scales, so TMA copies the
+// checkpoint's MXFP4 bytes into shared memory as they are and the tensor core decodes the
+// nibbles and applies the scales. This is the decode path of "quantization_mxfp4"
+// (KerasFormers), As GPT-OSS's native format: only the routed experts' blocks are read,
+// once per layer.
 //
-// Operands of one expert e with n_e routed rows:
+// Operands of one expert e (or one group of at most 56 of its routed rows):
 //   A = 128 weight rows (gate_up: 128 gate rows and, in a second MMA, the 128 matching up
-//       rows; down: 128 rows of down_proj), e2m1 with the checkpoint's e8m0 scales;
-//   B = the expert's token rows as FP8 E4M3 "parts" with their own e8m0 block scales
-//       (MX-FP8). With FP8 activations a token is one part (its static-scale e4m3 code,
-//       unit block scales; the per-tensor scale multiplies in the epilogue). With bf16
-//       activations a token is np = 3 parts: p1 = e4m3(x / 2^s1), p2 = e4m3((x - p1)/2^s2),
-//       p3 the same on the next residual, each s from its block's amax, so that
-//       p1 + p2 + p3 reproduces x to about 2^-12 of the block's largest value.
-//   D = 128 x N fp32 in tensor memory, N = np * n_e rounded up to 16; the epilogue adds a
-//       token's np columns.
-// The gate_up epilogue applies bias + SwiGLU and writes a directly as the down GEMM's B
-// operand (its 32-row warp is exactly one 32-value block of the down contraction, so the
-// block amax is a warp reduction); the down epilogue writes y and, in the last CTA of
-// each 128-row tile (an atomic ticket reset for the next call), the weighted combine.
+//       rows; down: 128 rows of down_proj) with the checkpoint's e8m0 scales;
+//   B = the routed token rows as four MXFP4 "parts" each: p1 = e2m1(x / 2^s1), p2 the same
+//       on the residual x - p1, and so on, each s chosen from its 32-value block's largest
+//       residual so that nothing saturates. Every part keeps about two more bits of the
+//       block, and four parts reproduce a bf16 row to about 1e-5 of a dot product's size
+//       (the per-tensor FP8 path splits the e4m3 value of x / s0 the same way).
+//   D = 128 x N fp32 in tensor memory, N = 4 * rows rounded up to 16; the epilogue adds a
+//       token's four columns.
+// Why not FP8 tokens against FP4 weights (kind::mxf8f6f4): a block-scaled MMA costs the
+// tensor pipe about 100 cycles whatever N is, and kind::mxf4 covers K = 64 per
+// instruction instead of 32, so it moves twice the weight bytes per instruction; with
+// K = 32 the pipe, not HBM, bounded decode. The packed operands also halve the shared
+// memory per weight byte (no 8-bit containers), which doubles the bytes in flight.
 //
-// Scale-factor records of the B operand ("SFB"): for expert e and k-tile kt, 1024 bytes
-// = two 512-byte tcgen05.cp atoms (rows 0..127, 128..255), row r of an atom at byte
-// 16*(r%32) + 4*((r/32)%4) + j for the tile's k-block j. The final (tail) k-tile of a
-// K = 22.5 x 128 contraction holds k-blocks nb-4 .. nb-1, consumed by k-steps 2 and 3.
+// Persistent schedule. One CTA per SM walks the work units u = blockIdx.x, +gridDim.x, ...
+// of the list (row group, 128-row tile, K split), so the TMA ring stays full across unit
+// boundaries and two TMEM accumulator slots let the epilogue of one unit overlap the MMAs
+// of the next. Few units (one token) are split along K so that every SM streams: each
+// split writes its fp32 partial accumulator, and the last split of a 32-row slice (an
+// atomic ticket) adds the partials in split order, so results do not depend on which CTA
+// finishes last.
+//
+// The gate_up epilogue applies bias + SwiGLU and writes a directly as the down GEMM's B
+// operand (its 32-row warp is exactly one 32-value block of the down contraction, so a
+// part's block amax is a warp reduction); the down epilogue writes y and, for a few
+// tokens, the weighted combine of each 32-row slice, by the last of the slice's row
+// groups to finish.
+//
+// Scale-factor records of the B operand ("SFB"): for row group g and 128-wide k-tile kt,
+// 1024 bytes = two 512-byte tcgen05.cp atoms (B rows 0..127, 128..255), row r at byte
+// 512*(r/128) + 16*(r%32) + 4*((r/32)%4) + j for the tile's k-block j.
+#include <climits>
+
 #include <cuda.h>
 
 #include "common.cuh"
@@ -37,73 +52,97 @@ namespace dec {
 using namespace tc;
 
 constexpr int BM = 128;
-constexpr int BK = 128;
-constexpr int kBoxRows = 32;       // token-part rows per TMA box of B
-constexpr int kMaxN = 192;         // largest B width (np * n_e rounded up) this path takes
+constexpr int BKS = 256;           // K per pipeline stage (128 packed bytes per row)
+constexpr int kRowBytes = 128;     // packed bytes of a row per stage
+constexpr int kParts = 4;          // e2m1 parts per token row
+constexpr int kGroupRows = 56;     // routed rows per row group: N = 4 * 56 = 224 at most
+constexpr int kMaxN = kParts * kGroupRows;
 constexpr int kThreads = 256;      // warp 0 TMA, 1 MMA, 2-3 A-scale converters, 4-7 epilogue
-constexpr int kMaxStages = 8;
+constexpr int kEpiWarps = 4;
+constexpr int kMaxStages = 10;
 constexpr int kTmemCols = 512;
-constexpr int kAccUpCol = 256;     // second accumulator (up rows)
-constexpr int kSfaCol0 = 192;      // A scales: gate (or down) at 192..195, up at 196..199
-constexpr int kSfbCol = 200;       // B scales: 200..207 (two atoms)
-constexpr int kSfRecord = 1024;
+constexpr int kSlot1 = 240;        // accumulator slot 1 starts here (slot 0 at column 0)
+constexpr int kBigCols = 112;      // gate_up units wider than this take both slots
+constexpr int kSfaCol = 480;       // A scales: tile h, atom a at 480 + 8h + 4a
+constexpr int kSfbCol = 496;       // B scales: k-tile t, atom b at 496 + 8t + 4b
+constexpr int kSfRecord = 1024;    // B scale record per (row group, 128-wide k-tile)
+constexpr int kSfStage = 4096;     // per stage: A atoms (2 tiles x 2) + B records (2)
+constexpr int kMaxE = 256;
+constexpr int kMaxGrp = kDecodeMaxGroups;
+constexpr int kMaxSplit = 8;
+constexpr int kMaxTopK = 8;
+constexpr int kSmemBytes = 227 * 1024;
 
-// instruction descriptor, kind::mxf8f6f4 block-scaled: A = E2M1 (5), B = E4M3 (0)
-__host__ __device__ constexpr uint32_t idesc_w_by_x(int M, int N) {
-  return (5u << 7) | (0u << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
+// instruction descriptor, kind::mxf4 block-scaled (scale_vec::2X): A = B = E2M1 (1),
+// e8m0 scales; sf_id (0 or 2) selects the scale-byte pair of a K = 64 step.
+__host__ __device__ constexpr uint32_t idesc_mxf4(int M, int N) {
+  return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-// Where the scale of k-block kb lives: k-tile and byte within the tile's 4 blocks. The
-// tail tile (K % 128 == 64) holds blocks nb-4 .. nb-1.
-__device__ __forceinline__ void sf_slot(int kb, int nb, int nk_full, int& kt, int& j) {
-  if (kb < 4 * nk_full) {
-    kt = kb >> 2;
-    j = kb & 3;
-  } else {
-    kt = nk_full;
-    j = kb - (nb - 4);
-  }
-}
-
-__device__ __forceinline__ int sf_atom_byte(int r, int j) {
+__host__ __device__ __forceinline__ int sf_atom_byte(int r, int j) {   // r < 256
   return (r >> 7) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + j;
-}
-
-// e8m0 exponent s for a block whose largest magnitude is amax: amax / 2^s in [128, 256),
-// inside e4m3's range. amax == 0 gives 0.
-__device__ __forceinline__ int part_exponent(float amax) {
-  if (!(amax > 0.0f)) return 0;
-  const uint32_t u = __float_as_uint(amax);
-  int ex = static_cast<int>(u >> 23);
-  int fl = ex > 0 ? ex - 127 : (31 - __clz(u)) - 149;
-  return max(-127, min(127, fl - 7));
 }
 
 __device__ __forceinline__ float pow2f(int s) {   // exact 2^s for s in [-126, 127]
   return __uint_as_float(static_cast<uint32_t>(s + 127) << 23);
 }
 
-// Split v (this lane's element of a 32-value block held by the warp) into np e4m3 parts.
-// Writes part bytes and scale exponents (same in every lane). Lanes outside the data pass
-// v = 0.
-template <int NP>
-__device__ __forceinline__ void split_parts(float v, uint8_t (&q)[NP], int (&s)[NP]) {
-  float r = v;
+// Scale exponent of an e2m1 part: the smallest s with amax / 2^s <= 6 (the e2m1 maximum),
+// clamped to [-126, 125]. amax == 0 gives 0.
+__device__ __forceinline__ int e2m1_part_exponent(float amax) {
+  if (!(amax > 0.0f)) return 0;
+  const uint32_t u = __float_as_uint(amax);
+  const int ex = static_cast<int>(u >> 23);
+  const int fl = ex > 0 ? ex - 127 : (31 - __clz(u)) - 149;   // floor(log2(amax))
+  int s = max(-126, min(125, fl - 2));                       // amax / 2^s in [4, 8)
+  if (amax > 6.0f * pow2f(s)) s = min(125, s + 1);
+  return s;
+}
+
+// e2m1 code (sign in bit 3) of v, |v| <= 6, rounded to nearest with ties to the even
+// code, as a count of the rounding thresholds that |v| passes (no branches: the lanes of
+// a warp hold different values).
+__device__ __forceinline__ uint32_t e2m1_code(float v) {
+  const float a = fabsf(v);
+  const uint32_t c = static_cast<uint32_t>(a > 0.25f) + static_cast<uint32_t>(a >= 0.75f) +
+                     static_cast<uint32_t>(a > 1.25f) + static_cast<uint32_t>(a >= 1.75f) +
+                     static_cast<uint32_t>(a > 2.5f) + static_cast<uint32_t>(a >= 3.5f) +
+                     static_cast<uint32_t>(a > 5.0f);
+  return c | (v < 0.0f && c != 0u ? 8u : 0u);
+}
+
+// Twice the magnitude of e2m1 code c & 7 (0, 1, 2, 3, 4, 6, 8, 12), from a nibble table.
+__device__ __forceinline__ uint32_t e2m1_twice(uint32_t c) { return (0xC8643210u >> (4u * (c & 7u))) & 15u; }
+
+// One e2m1 part of 8 rows' values r[j] (this lane's element of a 32-value block held by
+// the warp): the part codes q[j] and scale exponents sc[j] (the same in every lane), and
+// r[j] becomes the residual. The eight chains are independent, so their shuffles overlap.
+// Lanes outside the data pass 0. The residual update is exact: a part value has two
+// significant bits and a power-of-two scale.
+__device__ __forceinline__ void e2m1_part8(float (&r)[8], uint32_t (&q)[8], int (&sc)[8]) {
+  float a[8];
 #pragma unroll
-  for (int p = 0; p < NP; ++p) {
-    const float amax = warp_max(fabsf(r));
-    s[p] = part_exponent(amax);
-    const int sc = max(s[p], -126);
-    q[p] = f32_to_e4m3_satfinite(r * pow2f(-sc));   // power-of-two scaling: exact
-    r = r - e4m3_to_f32(q[p]) * pow2f(sc);         // exact residual
+  for (int j = 0; j < 8; ++j) a[j] = fabsf(r[j]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) a[j] = fmaxf(a[j], __shfl_xor_sync(0xffffffffu, a[j], o));
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    sc[j] = e2m1_part_exponent(a[j]);
+    q[j] = e2m1_code(r[j] * pow2f(-sc[j]));
+    const float qv = static_cast<float>(e2m1_twice(q[j])) * 0.5f * pow2f(sc[j]);   // exact
+    r[j] = r[j] - ((q[j] & 8u) ? -qv : qv);
   }
 }
 
-// Bytes of one pipeline stage: A tiles, B tile, A scale atoms, B scale record, rounded up
-// to 1024 so that every stage's tiles keep the 1024-byte alignment of 128-byte swizzle.
-__host__ __device__ constexpr int stage_size(int kA, int b_stage_bytes) {
-  return ((kA * BM * BK + b_stage_bytes + kA * 512 + kSfRecord) + 1023) & ~1023;
+// Two lanes' codes into one byte (element 2i in the low nibble, as the weights pack);
+// meaningful in even lanes.
+__device__ __forceinline__ uint32_t pack_pair(uint32_t code) {
+  const uint32_t hi = __shfl_down_sync(0xffffffffu, code, 1);
+  return (code & 15u) | ((hi & 15u) << 4);
 }
 
 struct Params {
@@ -114,74 +153,222 @@ struct Params {
   int rows_total;            // 2I or H
   int n_out;                 // I or H
   // shapes
-  int E, K, nb, nk_full, tail_steps, np;
+  int E, K, nb, nst, n_m, box_rows, split_cap, max_chunks;
+  int smem_bytes;            // dynamic shared memory of the launch
+  int64_t P;
   const int32_t* offsets;
   const int32_t* active;
   const int32_t* n_active;
-  const uint8_t* sfb;        // B scale records [E][nkt][1024]
+  const uint8_t* sfb;        // B scale records [E][max_chunks][2*nst][1024]
   float s_in;                // per-tensor scale of the B operand (FP8) or 1
   // gate_up outputs (the down GEMM's B operand)
-  uint8_t* xs_out;           // (P * np_out, I) e4m3
-  uint8_t* sfb_out;          // [E][nkt_out][1024]
-  int np_out, nb_out, nk_full_out, nkt_out;
-  float s_out;               // FP8: static scale of a; 0: bf16 split
-  unsigned* amax_bits;       // calibration: running max |a|
+  uint8_t* xs_out;           // (P * 4, I / 2) packed e2m1 parts
+  uint8_t* sfb_out;          // [E][max_chunks][2*nst_out][1024]
+  int nst_out;
+  float s_out;               // FP8: static scale of a; 0: bf16 intermediate
   // down outputs
   float* y_out;              // (P, H) fp32
-  uint16_t* out;             // (T, H) bf16, combine
+  uint16_t* out;             // (T, H) bf16, combine (nullable: no fold)
   const int32_t* topk_idx;
   const float* topk_w;
   const int32_t* inv;
-  unsigned* tickets;         // per 128-row tile
   int T, k;
+  // split-K
+  float* part;               // [split][kA][P * 4][n_out] fp32 partial accumulators
+  unsigned* split_tickets;   // [kMaxGrp][n_m][4], zero between calls
+  unsigned* comb_tickets;    // [n_m][4], zero between calls
   int* err;
-  int stages, b_stage_bytes;
 };
 
-template <bool kGateUp, int NP>
-__global__ void __launch_bounds__(kThreads, 1)
-decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_wt,
-                   const __grid_constant__ CUtensorMap map_x, Params p) {
-  const int slot = blockIdx.y;
-  if (slot >= *p.n_active) return;   // the whole CTA, before any barrier or allocation
-  const int e = p.active[slot];
-  const int off = p.offsets[e], n_e = p.offsets[e + 1] - off;
-  const int ncols = ((p.np * n_e + 15) / 16) * 16;
-  const int nboxes = (p.np * n_e + kBoxRows - 1) / kBoxRows;
-  const int row0 = blockIdx.x * BM;
-  const int nkt = p.nk_full + (p.tail_steps > 0 ? 1 : 0);
-  const int S = p.stages;
-  constexpr int kA = kGateUp ? 2 : 1;   // A tiles per stage
+// Per-CTA schedule, in shared memory, identical in every CTA: the row groups (an expert's
+// routed rows in chunks of at most kGroupRows) and the derived unit count.
+struct Sched {
+  int n_active, n_grp, nsplit, units, stages, stage_bytes;
+  int act[kMaxE];
+  int off[kMaxE + 1];
+  int g_e[kMaxGrp];          // expert of the group
+  int g_c[kMaxGrp];          // chunk index within the expert
+  int g_off[kMaxGrp];        // first routed row (expert-grouped order)
+  int g_n[kMaxGrp];          // rows in the group
+};
 
+struct Unit {
+  int g, e, c, m, s, k0, k1, off, j0, n, cols, ncols, nbox;
+};
+
+__device__ __forceinline__ Unit unit_at(const Sched& sc, const Params& p, int u) {
+  Unit w;
+  w.s = u % sc.nsplit;
+  const int t = u / sc.nsplit;
+  w.m = t % p.n_m;
+  w.g = t / p.n_m;
+  w.e = sc.g_e[w.g];
+  w.c = sc.g_c[w.g];
+  w.off = sc.g_off[w.g];
+  w.j0 = w.c * kGroupRows;   // first row of the group within its expert
+  w.n = sc.g_n[w.g];
+  w.k0 = w.s * p.nst / sc.nsplit;
+  w.k1 = (w.s + 1) * p.nst / sc.nsplit;
+  w.cols = kParts * w.n;
+  w.ncols = max(16, (w.cols + 15) & ~15);
+  w.nbox = (w.cols + p.box_rows - 1) / p.box_rows;
+  return w;
+}
+
+// Byte offsets of the fixed part of the shared-memory layout (host and device agree).
+__host__ __device__ constexpr int sched_bytes() { return (static_cast<int>(sizeof(Sched)) + 127) & ~127; }
+__host__ __device__ constexpr int bar_bytes() { return 256; }
+__host__ __device__ constexpr int ring_offset() { return (sched_bytes() + bar_bytes() + 1023) & ~1023; }
+__host__ __device__ inline int stage_bytes_for(int kA, int b_rows) {
+  return ((kA * BM * kRowBytes + b_rows * kRowBytes) + 1023) & ~1023;
+}
+
+// ------------------------------------------------------------------- epilogue pieces --
+// Accumulator columns of 8 rows (kParts per row, row-major) for this warp's 32 lanes.
+// Every index is static, so the tcgen05.ld destinations stay in registers until the wait
+// that makes them valid.
+template <bool kGateUp>
+__device__ __forceinline__ void read_tmem8(uint32_t tg, uint32_t tu, int j0, float (&vg)[8 * kParts],
+                                           float (&vu)[8 * kParts]) {
+  uint32_t g[kParts][8], u[kParts][8];
+#pragma unroll
+  for (int c = 0; c < kParts; ++c) {
+    tc_ld_32x32b_x8(tg + kParts * j0 + 8 * c, g[c]);
+    if (kGateUp) tc_ld_32x32b_x8(tu + kParts * j0 + 8 * c, u[c]);
+  }
+#pragma unroll
+  for (int c = 0; c < kParts; ++c) {
+    tc_wait_ld(g[c]);
+    if (kGateUp) tc_wait_ld(u[c]);
+  }
+#pragma unroll
+  for (int f = 0; f < 8 * kParts; ++f) {
+    vg[f] = __uint_as_float(g[f >> 3][f & 7]);
+    vu[f] = kGateUp ? __uint_as_float(u[f >> 3][f & 7]) : 0.0f;
+  }
+}
+
+// Address of the fp32 partial of (split s, accumulator h, global column c, row).
+__device__ __forceinline__ float* part_at(const Params& p, int kA, int s, int h, int64_t c, int row) {
+  return p.part + ((static_cast<int64_t>(s) * kA + h) * (p.P * kParts) + c) * p.n_out + row;
+}
+
+// Sum a row's kParts part columns (in part order) for the 8 rows of a group.
+__device__ __forceinline__ void sum_parts(const float (&v)[8 * kParts], float (&s)[8]) {
+#pragma unroll
+  for (int jj = 0; jj < 8; ++jj) {
+    float a = 0.0f;
+#pragma unroll
+    for (int pp = 0; pp < kParts; ++pp) a += v[kParts * jj + pp];
+    s[jj] = a;
+  }
+}
+
+// gate_up: bias, SwiGLU and the down GEMM's B operand for rows j0 .. j0+7 of the unit's
+// group. gs / us: the accumulators summed over a row's parts (before the per-tensor scale).
+__device__ __forceinline__ void finish_gate_up(const Params& p, const Unit& w, int j0, const float (&gs)[8],
+                                               const float (&us)[8], float bg, float bu, int row, int lane) {
+  const int kb = row >> 5;   // the warp's 32 rows: one 32-value block of the down contraction
+  uint8_t* rec = p.sfb_out + ((static_cast<int64_t>(w.e) * p.max_chunks + w.c) * 2 * p.nst_out + (kb >> 2)) * kSfRecord;
+  float a[8];
+#pragma unroll
+  for (int jj = 0; jj < 8; ++jj) {
+    const float gv = __fadd_rn(__fmul_rn(p.s_in, gs[jj]), bg);
+    const float uv = __fadd_rn(__fmul_rn(p.s_in, us[jj]), bu);
+    float v = j0 + jj < w.n ? silu_mul(gv, uv) : 0.0f;
+    // the layer's intermediate: e4m3(a / s1) with FP8 activations, else bf16(a)
+    v = p.s_out > 0.0f ? e4m3_to_f32(act_quant_e4m3(v, p.s_out)) : bf16_bits_to_f32(f32_to_bf16_bits_rn(v));
+    a[jj] = v;
+  }
+  const int64_t row_bytes = p.n_out / 2;
+  // one part at a time, stored as it is made: a rolled loop keeps this code small, which
+  // matters because it runs once per unit and its instructions are fetched cold
+#pragma unroll 1
+  for (int pp = 0; pp < kParts; ++pp) {
+    uint32_t q[8];
+    int sv[8];
+    e2m1_part8(a, q, sv);
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      const uint32_t byte = pack_pair(q[jj]);
+      if (j0 + jj < w.n) {
+        if ((lane & 1) == 0)
+          p.xs_out[(static_cast<int64_t>(w.off + j0 + jj) * kParts + pp) * row_bytes + (row >> 1)] = static_cast<uint8_t>(byte);
+        if (lane == 0) rec[sf_atom_byte(kParts * (j0 + jj) + pp, kb & 3)] = static_cast<uint8_t>(sv[jj] + 127);
+      }
+    }
+  }
+}
+
+// down: y = s_in * acc + bias for rows j0 .. j0+7 of the unit's group.
+__device__ __forceinline__ void finish_down(const Params& p, const Unit& w, int j0, const float (&ys)[8], float bd,
+                                            int row) {
+#pragma unroll
+  for (int jj = 0; jj < 8; ++jj)
+    if (j0 + jj < w.n)
+      p.y_out[static_cast<int64_t>(w.off + j0 + jj) * p.n_out + row] = __fadd_rn(__fmul_rn(p.s_in, ys[jj]), bd);
+}
+
+// Weighted combine of one 32-row slice of the output (lane = row) for every token: the
+// token's k expert outputs in ascending expert id, which is ascending position in the
+// expert-grouped order.
+__device__ __forceinline__ void combine_slice(const Params& p, int row) {
+  for (int t = 0; t < p.T; ++t) {
+    int pos[kMaxTopK];
+    float wt[kMaxTopK];
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+      const bool v = j < p.k;
+      pos[j] = v ? p.inv[static_cast<int64_t>(t) * p.k + j] : INT_MAX;
+      wt[j] = v ? p.topk_w[static_cast<int64_t>(t) * p.k + j] : 0.0f;
+    }
+#pragma unroll
+    for (int r = 0; r < kMaxTopK; ++r) {
+#pragma unroll
+      for (int j = (r & 1); j + 1 < kMaxTopK; j += 2) {
+        if (pos[j] > pos[j + 1]) {
+          const int tp = pos[j]; pos[j] = pos[j + 1]; pos[j + 1] = tp;
+          const float tw = wt[j]; wt[j] = wt[j + 1]; wt[j + 1] = tw;
+        }
+      }
+    }
+    float acc = 0.0f;
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j)
+      if (j < p.k) acc = __fadd_rn(acc, __fmul_rn(wt[j], __ldcg(p.y_out + static_cast<int64_t>(pos[j]) * p.n_out + row)));
+    p.out[static_cast<int64_t>(t) * p.n_out + row] = f32_to_bf16_bits_rn(acc);
+  }
+}
+
+// ---------------------------------------------------------------------- the kernel --
+template <bool kGateUp>
+__global__ void __launch_bounds__(kThreads, 1)
+decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x, Params p) {
+  constexpr int kA = kGateUp ? 2 : 1;   // A tiles (accumulators) per unit
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int a_bytes = kA * BM * BK;                       // unpacked e2m1, one byte per value
-  const int stage_bytes = stage_size(kA, p.b_stage_bytes);  // a multiple of 1024
-  uint8_t* sRaw = smem + S * stage_bytes;                 // kA * 128 rows * nb raw scale bytes
-  const int raw_bytes = ((kA * BM * p.nb) + 15) & ~15;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sRaw + raw_bytes);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + kMaxStages;
-  uint64_t* acc_full = bars + 2 * kMaxStages;
-  uint64_t* raw_full = acc_full + 1;                      // [2]
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(raw_full + 2);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(raw_full + 2) + 1;
-  unsigned* last_flag = tmem_holder + 1;
-
-  auto sA = [&](int s, int h) { return smem + s * stage_bytes + h * BM * BK; };
-  auto sB = [&](int s) { return smem + s * stage_bytes + a_bytes; };
-  auto sSFA = [&](int s, int h) { return smem + s * stage_bytes + a_bytes + p.b_stage_bytes + h * 512; };
-  auto sSFB = [&](int s) { return smem + s * stage_bytes + a_bytes + p.b_stage_bytes + kA * 512; };
+  Sched& sc = *reinterpret_cast<Sched*>(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + sched_bytes());
+  uint64_t* full = bars;                       // [kMaxStages]
+  uint64_t* empty = bars + kMaxStages;         // [kMaxStages]
+  uint64_t* acc_full = bars + 2 * kMaxStages;  // [2]
+  uint64_t* acc_empty = acc_full + 2;          // [2]
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(acc_empty + 2);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_empty + 2) + 1;
+  uint8_t* ring = smem + ring_offset();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
+    asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&map_w)) : "memory");
+    asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&map_x)) : "memory");
+    for (int s = 0; s < kMaxStages; ++s) {
       mbar_init(&full[s], 1 + kA);   // TMA producer (expect_tx) + one scale converter per A tile
       mbar_init(&empty[s], 1);
     }
-    mbar_init(acc_full, 1);
-    mbar_init(&raw_full[0], 1);
-    mbar_init(&raw_full[1], 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], kEpiWarps);
+    }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
@@ -190,220 +377,334 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
                  "r"(kTmemCols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n");
   }
+  for (int i = threadIdx.x; i <= p.E; i += blockDim.x) sc.off[i] = p.offsets[i];
+  for (int i = threadIdx.x; i < p.E; i += blockDim.x) sc.act[i] = p.active[i];
+  if (threadIdx.x == 0) sc.n_active = *p.n_active;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (warp == 0) {
+    // row groups: an exclusive scan of the active experts' chunk counts, 32 at a time
+    const int na = min(max(sc.n_active, 0), p.E);
+    int base = 0, maxcols = 0;
+    bool fits = true;
+    for (int i0 = 0; i0 < na; i0 += 32) {
+      const int i = i0 + lane;
+      int e = 0, off = 0, n_e = 0, nch = 0;
+      if (i < na) {
+        e = sc.act[i];
+        off = sc.off[e];
+        n_e = sc.off[e + 1] - off;
+        nch = (n_e + kGroupRows - 1) / kGroupRows;
+      }
+      int incl = nch;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      if (nch > p.max_chunks) fits = false;
+      for (int c = 0, g = base + incl - nch; c < nch; ++c, ++g) {
+        const int n = min(kGroupRows, n_e - c * kGroupRows);
+        if (g < kMaxGrp) {
+          sc.g_e[g] = e;
+          sc.g_c[g] = c;
+          sc.g_off[g] = off + c * kGroupRows;
+          sc.g_n[g] = n;
+        }
+        maxcols = max(maxcols, kParts * n);
+      }
+      base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) maxcols = max(maxcols, __shfl_xor_sync(0xffffffffu, maxcols, o));
+    fits = __all_sync(0xffffffffu, fits) && base <= kMaxGrp;
+    if (lane == 0) {
+      const int ng = base;
+      sc.n_grp = ng;
+      const int ncols_max = max(16, (maxcols + 15) & ~15);
+      const int nbox_max = (maxcols + p.box_rows - 1) / p.box_rows;
+      const int b_rows = max(ncols_max, nbox_max * p.box_rows);
+      sc.stage_bytes = stage_bytes_for(kA, b_rows);
+      const int avail = static_cast<int>((smem_raw + p.smem_bytes) - ring);
+      sc.stages = min(kMaxStages, avail / (sc.stage_bytes + kSfStage));
+      // K split: fewest stages on the busiest CTA, counting half a stage per partial
+      const int tiles = ng * p.n_m, G = gridDim.x;
+      int best = 1, best_cost = INT_MAX;
+      for (int s = 1; s <= min(p.split_cap, p.nst); ++s) {
+        const int per = (tiles * s + G - 1) / G;
+        const int cost = 2 * per * ((p.nst + s - 1) / s) + (s > 1 ? per : 0);
+        if (cost < best_cost) { best_cost = cost; best = s; }
+      }
+      sc.nsplit = best;
+      sc.units = tiles * best;
+      if (!fits || sc.stages < 2) {   // the host's checks exclude both; never expected
+        set_device_error(p.err, MXMOE_EUNSUPPORTED);
+        sc.units = 0;
+      }
+    }
+  }
+  __syncthreads();
   const uint32_t tmem = *tmem_holder;
+  const int S = sc.stages;
+  auto sA = [&](int s, int h) { return ring + s * sc.stage_bytes + h * BM * kRowBytes; };
+  auto sB = [&](int s) { return ring + s * sc.stage_bytes + kA * BM * kRowBytes; };
+  uint8_t* sf_base = ring + S * sc.stage_bytes;
+  auto sSFA = [&](int s, int h) { return sf_base + s * kSfStage + h * 1024; };
+  auto sSFB = [&](int s) { return sf_base + s * kSfStage + 2048; };
+  auto n_ksteps = [&](int kst) { return min(4, (p.K - BKS * kst + 63) / 64); };
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer -----
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      const uint32_t tx = kA * BM * (BK / 2) + nboxes * kBoxRows * BK + kSfRecord;
-      for (int kt = 0; kt < nkt; ++kt) {
-        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err)) break;
-        mbar_arrive_expect_tx(&full[stage], tx);
-        const bool tail = kt >= p.nk_full;
-        const CUtensorMap* mw = tail ? &map_wt : &map_w;
-        const int wx = tail ? 0 : kt * BK;
-        const int kx = tail ? p.K - BK : kt * BK;
-        if (kGateUp) {
-          tma_load_3d(sA(stage, 0), mw, &full[stage], wx, row0, 2 * e);
-          tma_load_3d(sA(stage, 1), mw, &full[stage], wx, row0, 2 * e + 1);
-        } else {
-          tma_load_3d(sA(stage, 0), mw, &full[stage], wx, row0, e);
+      bool ok = true;
+      for (int u = blockIdx.x; u < sc.units && ok; u += gridDim.x) {
+        const Unit w = unit_at(sc, p, u);
+        const uint32_t tx = kA * BM * kRowBytes + w.nbox * p.box_rows * kRowBytes + 2 * kSfRecord;
+        const uint8_t* rec = p.sfb + (static_cast<int64_t>(w.e) * p.max_chunks + w.c) * 2 * p.nst * kSfRecord;
+        for (int kst = w.k0; kst < w.k1; ++kst) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[stage], tx);
+          tma_load_3d(sA(stage, 0), &map_w, &full[stage], kRowBytes * kst, w.m * BM, kA * w.e);
+          for (int b = 0; b < w.nbox; ++b)
+            tma_load_2d(sB(stage) + b * p.box_rows * kRowBytes, &map_x, &full[stage], kRowBytes * kst,
+                        kParts * w.off + b * p.box_rows);
+          bulk_g2s(sSFB(stage), rec + 2 * kst * kSfRecord, 2 * kSfRecord, &full[stage]);
+          if (++stage == S) { stage = 0; phase ^= 1; }
         }
-        for (int b = 0; b < nboxes; ++b)
-          tma_load_2d(sB(stage) + b * kBoxRows * BK, &map_x, &full[stage], kx, p.np * off + b * kBoxRows);
-        bulk_g2s(sSFB(stage), p.sfb + (static_cast<int64_t>(e) * nkt + kt) * kSfRecord, kSfRecord, &full[stage]);
-        if (++stage == S) { stage = 0; phase ^= 1; }
       }
     }
   } else if (warp == 1) {
     // --------------------------------------------------------------------- MMA -----
     int stage = 0;
     uint32_t phase = 0;
-    const uint32_t id0 = idesc_w_by_x(BM, ncols);
+    uint32_t use0 = 0u, use1 = 0u;   // completed uses of each accumulator slot
+    int nxt = 0;
     bool ok = true;
-    for (int kt = 0; kt < nkt; ++kt) {
-      if (!mbar_wait(&full[stage], phase, abort_flag, p.err)) { ok = false; break; }
+    for (int u = blockIdx.x; u < sc.units && ok; u += gridDim.x) {
+      const Unit w = unit_at(sc, p, u);
+      const bool big = kGateUp && w.ncols > kBigCols;
+      const int slot = big ? 0 : nxt;
+      if (big) {
+        ok = mbar_wait(&acc_empty[0], (use0 & 1u) ^ 1u, abort_flag, p.err) &&
+             mbar_wait(&acc_empty[1], (use1 & 1u) ^ 1u, abort_flag, p.err);
+      } else {
+        ok = mbar_wait(&acc_empty[slot], ((slot ? use1 : use0) & 1u) ^ 1u, abort_flag, p.err);
+      }
+      if (!ok) break;
       tc_fence_after();
-      if (lane == 0) {
-        for (int h = 0; h < kA; ++h)
-          tc_cp_32x128b_x4(tmem + kSfaCol0 + 4 * h, smem_desc(smem_u32(sSFA(stage, h)), 0, 128, 0));
-        const uint32_t sfb = smem_u32(sSFB(stage));
-        tc_cp_32x128b_x4(tmem + kSfbCol, smem_desc(sfb, 0, 128, 0));
-        tc_cp_32x128b_x4(tmem + kSfbCol + 4, smem_desc(sfb + 512, 0, 128, 0));
-        const uint32_t b0 = smem_u32(sB(stage));
-        const int first = kt < p.nk_full ? 0 : 4 - p.tail_steps;
-        for (int kk = first; kk < 4; ++kk) {
-          const uint64_t bd = smem_desc(b0 + 32 * kk, 16, 1024, 2);
-          const uint32_t id = id0 | (static_cast<uint32_t>(kk) << 4) | (static_cast<uint32_t>(kk) << 29);
-          const uint32_t sel = static_cast<uint32_t>(kk) << 30;
-          const uint32_t acc = (kt > 0 || kk > first) ? 1u : 0u;
-          for (int h = 0; h < kA; ++h) {
-            const uint64_t ad = smem_desc(smem_u32(sA(stage, h)) + 32 * kk, 16, 1024, 2);
-            tc_mma_mxf8f6f4(tmem + h * kAccUpCol, ad, bd, id, (tmem + kSfaCol0 + 4 * h) | sel,
-                            (tmem + kSfbCol) | sel, acc);
+      const uint32_t dg = big ? 0u : static_cast<uint32_t>(slot * kSlot1);
+      const uint32_t du = big ? static_cast<uint32_t>(kSlot1) : dg + static_cast<uint32_t>(w.ncols);
+      const uint32_t id0 = idesc_mxf4(BM, w.ncols);
+      const int nat = w.ncols > 128 ? 2 : 1;   // B scale atoms per k-tile
+      for (int kst = w.k0; kst < w.k1; ++kst) {
+        if (!mbar_wait(&full[stage], phase, abort_flag, p.err)) { ok = false; break; }
+        tc_fence_after();
+        if (lane == 0) {
+          const int nks = n_ksteps(kst);
+          const int nkt = (nks + 1) >> 1;   // 128-wide k-tiles this stage uses
+          for (int t = 0; t < nkt; ++t) {
+#pragma unroll
+            for (int h = 0; h < kA; ++h)
+              tc_cp_32x128b_x4(tmem + kSfaCol + 8 * h + 4 * t, smem_desc(smem_u32(sSFA(stage, h) + 512 * t), 0, 128, 0));
+            for (int b = 0; b < nat; ++b)
+              tc_cp_32x128b_x4(tmem + kSfbCol + 8 * t + 4 * b,
+                               smem_desc(smem_u32(sSFB(stage) + kSfRecord * t + 512 * b), 0, 128, 0));
           }
+          const uint32_t b0 = smem_u32(sB(stage));
+          for (int sk = 0; sk < nks; ++sk) {
+            const int t = sk >> 1;
+            const uint32_t sfid = static_cast<uint32_t>(sk & 1) * 2u;
+            const uint32_t id = id0 | (sfid << 4) | (sfid << 29);
+            const uint32_t sel = sfid << 30;
+            const uint64_t bd = smem_desc(b0 + 32 * sk, 16, 1024, 2);
+            const uint32_t acc = (kst > w.k0 || sk > 0) ? 1u : 0u;
+#pragma unroll
+            for (int h = 0; h < kA; ++h) {
+              const uint64_t ad = smem_desc(smem_u32(sA(stage, h)) + 32 * sk, 16, 1024, 2);
+              tc_mma_mxf4(tmem + (h ? du : dg), ad, bd, id, (tmem + kSfaCol + 8 * h + 4 * t) | sel,
+                          (tmem + kSfbCol + 8 * t) | sel, acc);
+            }
+          }
+          tc_commit(&empty[stage]);
         }
-        tc_commit(&empty[stage]);
+        __syncwarp();
+        if (++stage == S) { stage = 0; phase ^= 1; }
+      }
+      if (!ok) break;
+      if (lane == 0) {
+        tc_commit(&acc_full[slot]);
+        if (big) tc_commit(&acc_full[1]);
       }
       __syncwarp();
-      if (++stage == S) { stage = 0; phase ^= 1; }
+      if (big) {
+        ++use0;
+        ++use1;
+        nxt = 0;
+      } else {
+        if (slot) ++use1; else ++use0;
+        nxt ^= 1;
+      }
     }
-    if (ok && lane == 0) tc_commit(acc_full);
-    __syncwarp();
   } else if (warp == 2 || warp == 3) {
     // ------------------------------------------------ A (weight) scale converters -----
     const int h = warp - 2;   // 0: gate / down rows, 1: up rows
     if (h < kA) {
-      const int group = kGateUp ? 2 * e + h : e;
-      const int valid = min(BM, p.rows_per_group - row0);
-      const int bytes = valid * p.nb;
-      const uint8_t* src = p.w_scales + (static_cast<int64_t>(group) * p.rows_per_group + row0) * p.nb;
-      uint8_t* dst = sRaw + h * BM * p.nb;
-      const bool bulk = ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst) |
-                          static_cast<uintptr_t>(bytes)) & 15u) == 0;
+      int stage = 0;
+      uint32_t phase = 0;
       bool ok = true;
-      if (bulk) {
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&raw_full[h], static_cast<uint32_t>(bytes));
-          bulk_g2s(dst, src, static_cast<uint32_t>(bytes), &raw_full[h]);
-        }
-        ok = mbar_wait(&raw_full[h], 0, abort_flag, p.err);
-      } else {
-        for (int c0 = 0; c0 < bytes; c0 += 32 * 8) {
-          uint8_t v[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const int c = c0 + u * 32 + lane;
-            v[u] = c < bytes ? src[c] : 0;
-          }
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const int c = c0 + u * 32 + lane;
-            if (c < bytes) dst[c] = v[u];
-          }
-        }
-      }
-      __syncwarp();
-      if (ok) {
-        // lane l owns atom rows l, l+32, l+64, l+96: bytes 16*l .. 16*l+15 of the atom
-        int src_off[4];
+      for (int u = blockIdx.x; u < sc.units && ok; u += gridDim.x) {
+        const Unit w = unit_at(sc, p, u);
+        const int valid = min(BM, p.rows_per_group - w.m * BM);
+        const int group = kGateUp ? 2 * w.e + h : w.e;
+        const uint8_t* blk = p.w_scales + (static_cast<int64_t>(group) * p.rows_per_group + w.m * BM) * p.nb;
+        // lane l owns atom rows l, l+32, l+64, l+96 (bytes 16*l .. 16*l+15 of an atom); a
+        // stage's 8 scale bytes of a row are four aligned 16-bit words (nb is even)
+        const uint16_t* rp[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int r = lane + 32 * i;
-          src_off[i] = r < valid ? (h * BM + r) * p.nb : -1;
+          rp[i] = r < valid ? reinterpret_cast<const uint16_t*>(blk + static_cast<int64_t>(r) * p.nb) : nullptr;
         }
-        int stage = 0;
-        uint32_t phase = 0;
-        for (int kt = 0; kt < nkt; ++kt) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err)) break;
-          const int kb0 = kt < p.nk_full ? 4 * kt : p.nb - 4;
-          uint32_t wv[4];
+        auto load = [&](int kst, uint32_t (&a0)[4], uint32_t (&a1)[4]) {
+          const int b0 = 8 * kst;
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            if (src_off[i] < 0) {
-              wv[i] = 0x7F7F7F7Fu;
-            } else {
-              const uint8_t* s8 = sRaw + src_off[i] + kb0;
-              wv[i] = static_cast<uint32_t>(s8[0]) | (static_cast<uint32_t>(s8[1]) << 8) |
-                      (static_cast<uint32_t>(s8[2]) << 16) | (static_cast<uint32_t>(s8[3]) << 24);
-            }
+            uint32_t wd[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              wd[q] = (rp[i] && b0 + 2 * q < p.nb) ? static_cast<uint32_t>(__ldg(rp[i] + b0 / 2 + q)) : 0x7F7Fu;
+            a0[i] = wd[0] | (wd[1] << 16);
+            a1[i] = wd[2] | (wd[3] << 16);
           }
-          *reinterpret_cast<uint4*>(sSFA(stage, h) + 16 * lane) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        };
+        uint32_t c0[4], c1[4];
+        load(w.k0, c0, c1);
+        for (int kst = w.k0; kst < w.k1; ++kst) {
+          uint32_t n0[4] = {0u, 0u, 0u, 0u}, n1[4] = {0u, 0u, 0u, 0u};
+          if (kst + 1 < w.k1) load(kst + 1, n0, n1);   // one stage ahead
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err)) { ok = false; break; }
+          *reinterpret_cast<uint4*>(sSFA(stage, h) + 16 * lane) = make_uint4(c0[0], c0[1], c0[2], c0[3]);
+          *reinterpret_cast<uint4*>(sSFA(stage, h) + 512 + 16 * lane) = make_uint4(c1[0], c1[1], c1[2], c1[3]);
           fence_async_smem();
           __syncwarp();
           if (lane == 0) mbar_arrive(&full[stage]);
           if (++stage == S) { stage = 0; phase ^= 1; }
+#pragma unroll
+          for (int i = 0; i < 4; ++i) { c0[i] = n0[i]; c1[i] = n1[i]; }
         }
       }
     }
   } else {
     // ----------------------------------------------------------------- epilogue -----
     const int q = warp & 3;
-    const int m = 32 * q + lane;           // accumulator row = TMEM lane
-    const int row = row0 + m;              // weight row within the half / down_proj
-    const bool live = row < p.n_out;
-    if (mbar_wait(acc_full, 0, abort_flag, p.err)) {
+    uint32_t use0 = 0u, use1 = 0u;
+    int nxt = 0;
+    for (int u = blockIdx.x; u < sc.units; u += gridDim.x) {
+      const Unit w = unit_at(sc, p, u);
+      const bool big = kGateUp && w.ncols > kBigCols;
+      const int slot = big ? 0 : nxt;
+      // this warp's biases, loaded before the wait so that their latency overlaps the MMAs
+      const int brow = min(w.m * BM + 32 * q + lane, p.n_out - 1);
+      const float* bias_e = p.bias + static_cast<int64_t>(w.e) * p.rows_total;
+      const float bias0 = __ldg(bias_e + brow);
+      const float bias1 = kGateUp ? __ldg(bias_e + p.n_out + brow) : 0.0f;
+      bool ok = mbar_wait(&acc_full[slot], (slot ? use1 : use0) & 1u, abort_flag, p.err);
+      if (ok && big) ok = mbar_wait(&acc_full[1], use1 & 1u, abort_flag, p.err);
+      if (!ok) break;
       tc_fence_after();
-      const uint32_t tb = tmem + (static_cast<uint32_t>(32 * q) << 16);
-      // NP (parts per token) is a template parameter and every loop over accumulator
-      // columns is unrolled, so the tcgen05.ld destinations stay in registers until the
-      // wait that makes them valid
-      const float* bias_e = p.bias + static_cast<int64_t>(e) * p.rows_total;
-      if (kGateUp) {
-        const float bg = live ? bias_e[row] : 0.0f;
-        const float bu = live ? bias_e[p.n_out + row] : 0.0f;
-        const int kb = row >> 5;           // k-block of the down contraction (warp-uniform)
-        int okt, oj;
-        sf_slot(kb, p.nb_out, p.nk_full_out, okt, oj);
-        uint8_t* rec = p.sfb_out + (static_cast<int64_t>(e) * p.nkt_out + okt) * kSfRecord;
-        const bool warp_live = (row0 + 32 * q) < p.n_out;
-        for (int j0 = 0; j0 < n_e; j0 += 8) {
-          uint32_t g[NP][8], u[NP][8];
+      const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * q) << 16);
+      const uint32_t tg = lane_base + (big ? 0u : static_cast<uint32_t>(slot * kSlot1));
+      const uint32_t tu = lane_base + (big ? static_cast<uint32_t>(kSlot1)
+                                           : static_cast<uint32_t>(slot * kSlot1 + w.ncols));
+      const int row = w.m * BM + 32 * q + lane;
+      const bool live = (w.m * BM + 32 * q) < p.n_out;   // n_out % 64 == 0: whole warps
+      const bool split = sc.nsplit > 1;
+      const int64_t col0 = static_cast<int64_t>(w.off) * kParts;
+      if (live && split) {
+        // this split's partials
+        for (int j0 = 0; j0 < w.n; j0 += 8) {
+          float vg[8 * kParts], vu[8 * kParts];
+          read_tmem8<kGateUp>(tg, tu, j0, vg, vu);
 #pragma unroll
-          for (int c = 0; c < NP; ++c) {
-            tc_ld_32x32b_x8(tb + NP * j0 + 8 * c, g[c]);
-            tc_ld_32x32b_x8(tb + kAccUpCol + NP * j0 + 8 * c, u[c]);
-            tc_wait_ld(g[c], u[c]);
+          for (int f = 0; f < 8 * kParts; ++f) {
+            if (j0 + f / kParts < w.n) {
+              *part_at(p, kA, w.s, 0, col0 + kParts * j0 + f, row) = vg[f];
+              if (kGateUp) *part_at(p, kA, w.s, 1, col0 + kParts * j0 + f, row) = vu[f];
+            }
           }
+        }
+      }
+      bool finished = live && !split;
+      unsigned* stk = p.split_tickets + (static_cast<int64_t>(w.g) * p.n_m + w.m) * 4 + q;
+      if (live && split) {
+        // the last split of this 32-row slice adds the partials in split order
+        __threadfence();
+        __syncwarp();
+        unsigned t = 0;
+        if (lane == 0) t = atomicAdd(stk, 1u);
+        t = __shfl_sync(0xffffffffu, t, 0);
+        finished = t == static_cast<unsigned>(sc.nsplit - 1);
+        if (finished) __threadfence();
+      }
+      if (finished) {
+        for (int j0 = 0; j0 < w.n; j0 += 8) {
+          float vg[8 * kParts], vu[8 * kParts];
+          if (!split) {
+            read_tmem8<kGateUp>(tg, tu, j0, vg, vu);
+          } else {
 #pragma unroll
-          for (int jj = 0; jj < 8; ++jj) {
-            if (j0 + jj < n_e) {
-              float gs = 0.0f, us = 0.0f;
+            for (int f = 0; f < 8 * kParts; ++f) { vg[f] = 0.0f; vu[f] = 0.0f; }
+            for (int s = 0; s < sc.nsplit; ++s) {
 #pragma unroll
-              for (int pp = 0; pp < NP; ++pp) {
-                gs += __uint_as_float(g[(NP * jj + pp) >> 3][(NP * jj + pp) & 7]);
-                us += __uint_as_float(u[(NP * jj + pp) >> 3][(NP * jj + pp) & 7]);
-              }
-              const float gv = __fadd_rn(__fmul_rn(p.s_in, gs), bg);
-              const float uv = __fadd_rn(__fmul_rn(p.s_in, us), bu);
-              const float a = live ? silu_mul(gv, uv) : 0.0f;
-              if (p.amax_bits && live) atomicMax(p.amax_bits, __float_as_uint(fabsf(a)));
-              const int64_t pos = off + j0 + jj;
-              if (p.s_out > 0.0f) {
-                // FP8 intermediate: one part, unit block scale
-                if (live) p.xs_out[pos * p.n_out + row] = act_quant_e4m3(a, p.s_out);
-                if (warp_live && lane == 0) rec[sf_atom_byte(j0 + jj, oj)] = 127;
-              } else {
-                // bf16 intermediate, split into 3 MX-FP8 parts over this warp's 32 rows
-                const float ar = bf16_bits_to_f32(f32_to_bf16_bits_rn(a));
-                uint8_t qv[3];
-                int sv[3];
-                split_parts<3>(live ? ar : 0.0f, qv, sv);
-                if (warp_live) {
-#pragma unroll
-                  for (int pp = 0; pp < 3; ++pp) {
-                    if (live) p.xs_out[(pos * 3 + pp) * p.n_out + row] = qv[pp];
-                    if (lane == 0) rec[sf_atom_byte(3 * (j0 + jj) + pp, oj)] = static_cast<uint8_t>(sv[pp] + 127);
-                  }
+              for (int f = 0; f < 8 * kParts; ++f) {
+                if (j0 + f / kParts < w.n) {
+                  vg[f] += __ldcg(part_at(p, kA, s, 0, col0 + kParts * j0 + f, row));
+                  if (kGateUp) vu[f] += __ldcg(part_at(p, kA, s, 1, col0 + kParts * j0 + f, row));
                 }
               }
             }
           }
+          float gs[8], us[8];
+          sum_parts(vg, gs);
+          if (kGateUp) {
+            sum_parts(vu, us);
+            finish_gate_up(p, w, j0, gs, us, bias0, bias1, row, lane);
+          } else {
+            finish_down(p, w, j0, gs, bias0, row);
+          }
         }
+        if (split && lane == 0) *stk = 0u;   // ready for the next call
+      }
+      // the accumulator slot is free for the unit after next
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&acc_empty[slot]);
+        if (big) mbar_arrive(&acc_empty[1]);
+      }
+      if (big) {
+        ++use0;
+        ++use1;
+        nxt = 0;
       } else {
-        const float bd = live ? bias_e[row] : 0.0f;
-        for (int j0 = 0; j0 < n_e; j0 += 8) {
-          uint32_t v[NP][8];
-#pragma unroll
-          for (int c = 0; c < NP; ++c) {
-            tc_ld_32x32b_x8(tb + NP * j0 + 8 * c, v[c]);
-            tc_wait_ld(v[c]);
-          }
-#pragma unroll
-          for (int jj = 0; jj < 8; ++jj) {
-            if (j0 + jj < n_e) {
-              float ys = 0.0f;
-#pragma unroll
-              for (int pp = 0; pp < NP; ++pp) ys += __uint_as_float(v[(NP * jj + pp) >> 3][(NP * jj + pp) & 7]);
-              if (live)
-                p.y_out[static_cast<int64_t>(off + j0 + jj) * p.n_out + row] = __fadd_rn(__fmul_rn(p.s_in, ys), bd);
-            }
-          }
+        if (slot) ++use1; else ++use0;
+        nxt ^= 1;
+      }
+      if (!kGateUp && finished && p.out != nullptr) {
+        // the last row group to finish this 32-row slice combines it for every token
+        __threadfence();
+        __syncwarp();
+        unsigned* tk = p.comb_tickets + w.m * 4 + q;
+        unsigned t = 0;
+        if (lane == 0) t = atomicAdd(tk, 1u);
+        t = __shfl_sync(0xffffffffu, t, 0);
+        if (t == static_cast<unsigned>(sc.n_grp - 1)) {
+          __threadfence();
+          combine_slice(p, row);
+          if (lane == 0) *tk = 0u;
         }
       }
     }
@@ -412,7 +713,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
   // ---------------------------------------------------------------------- teardown ---
   tc_fence_before();
   __syncthreads();
-  if (*abort_flag) {
+  if (*abort_flag) {   // let copies still in flight land before the CTA's memory goes
     const long long t0 = clock64();
     while (clock64() - t0 < 200000) {
     }
@@ -421,80 +722,51 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kTmemCols));
   }
-  if (!kGateUp && p.out != nullptr && !*abort_flag) {
-    // weighted combine of this 128-row tile, by the last of the tile's CTAs
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0)
-      *last_flag = atomicAdd(&p.tickets[blockIdx.x], 1u) == static_cast<unsigned>(*p.n_active) - 1u;
-    __syncthreads();
-    if (*last_flag) {
-      __threadfence();
-      for (int i = threadIdx.x; i < p.T * BM; i += blockDim.x) {
-        const int t = i / BM, r = row0 + (i % BM);
-        if (r >= p.n_out) continue;
-        int ord[8], eid[8];
-        for (int j = 0; j < p.k; ++j) {
-          const int ex = p.topk_idx[static_cast<int64_t>(t) * p.k + j];
-          int qq = j;
-          while (qq > 0 && eid[qq - 1] > ex) { eid[qq] = eid[qq - 1]; ord[qq] = ord[qq - 1]; --qq; }
-          eid[qq] = ex;
-          ord[qq] = j;
-        }
-        float acc = 0.0f;
-        for (int qq = 0; qq < p.k; ++qq) {
-          const int j = ord[qq];
-          const int64_t pos = p.inv[static_cast<int64_t>(t) * p.k + j];
-          acc = __fadd_rn(acc, __fmul_rn(p.topk_w[static_cast<int64_t>(t) * p.k + j],
-                                         __ldcg(p.y_out + pos * p.n_out + r)));
-        }
-        p.out[static_cast<int64_t>(t) * p.n_out + r] = f32_to_bf16_bits_rn(acc);
-      }
-      if (threadIdx.x == 0) p.tickets[blockIdx.x] = 0u;
-    }
-  }
 }
 
 // ------------------------------------------------ token operand of the gate_up GEMM --
-// One warp per (routed pair, 32-value block): x's block as np MX-FP8 parts (bf16 path) or
-// its static-scale e4m3 code with a unit block scale (FP8 path), written in expert-grouped
-// row order with the block scales into the expert's scale records.
-template <int NP>
+// One warp per (routed pair, 8 consecutive 32-value blocks): the pair's x (or, with FP8
+// activations, the e4m3 value of x / s0) as four e2m1 parts per block, packed in
+// expert-grouped row order, with the block scales in the row group's scale records.
 __global__ void __launch_bounds__(256) split_tokens_kernel(
     const uint16_t* __restrict__ x, const int32_t* __restrict__ perm_token, const int32_t* __restrict__ perm_slot,
-    const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ offsets, int64_t P, int H, int k,
-    float s0, uint8_t* __restrict__ xs, uint8_t* __restrict__ sfb, int nb, int nk_full, int nkt) {
+    const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ offsets, int64_t P, int H, int k, float s0,
+    int fp8, uint8_t* __restrict__ xs, uint8_t* __restrict__ sfb, int nst, int max_chunks) {
   const int lane = threadIdx.x & 31;
+  const int nb = H / 32, nb8 = (nb + 7) / 8;
   const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  if (w >= P * nb) return;
-  const int64_t pos = w / nb;
-  const int kb = static_cast<int>(w % nb);
+  if (w >= P * nb8) return;
+  const int64_t pos = w / nb8;
+  const int kb0 = static_cast<int>(w % nb8) * 8;
   const int t = perm_token[pos];
   const int e = topk_idx[static_cast<int64_t>(t) * k + perm_slot[pos]];
-  const int j = static_cast<int>(pos - offsets[e]);
-  const float v = bf16_bits_to_f32(x[static_cast<int64_t>(t) * H + 32 * kb + lane]);
-  int kt, jb;
-  sf_slot(kb, nb, nk_full, kt, jb);
-  uint8_t* rec = sfb + (static_cast<int64_t>(e) * nkt + kt) * kSfRecord;
-  if (NP == 1) {
-    xs[pos * H + 32 * kb + lane] = act_quant_e4m3(v, s0);
-    if (lane == 0) rec[sf_atom_byte(j, jb)] = 127;
-  } else {
-    uint8_t qv[NP];
-    int sv[NP];
-    split_parts<NP>(v, qv, sv);
+  const int je = static_cast<int>(pos - offsets[e]);   // row within the expert
+  const int c = je / kGroupRows, jr = je % kGroupRows;
+  float r[8];
 #pragma unroll
-    for (int pp = 0; pp < NP; ++pp) {
-      xs[(pos * NP + pp) * H + 32 * kb + lane] = qv[pp];
-      if (lane == 0) rec[sf_atom_byte(NP * j + pp, jb)] = static_cast<uint8_t>(sv[pp] + 127);
+  for (int j = 0; j < 8; ++j) {
+    float v = 0.0f;
+    if (kb0 + j < nb) v = bf16_bits_to_f32(x[static_cast<int64_t>(t) * H + 32 * (kb0 + j) + lane]);
+    r[j] = fp8 ? e4m3_to_f32(act_quant_e4m3(v, s0)) : v;
+  }
+  const int64_t row_bytes = H / 2;
+  uint8_t* rec = sfb + (static_cast<int64_t>(e) * max_chunks + c) * 2 * nst * kSfRecord;
+#pragma unroll 1
+  for (int pp = 0; pp < kParts; ++pp) {
+    uint32_t q[8];
+    int sv[8];
+    e2m1_part8(r, q, sv);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t byte = pack_pair(q[j]);
+      const int kb = kb0 + j;
+      if (kb < nb) {
+        if ((lane & 1) == 0) xs[(pos * kParts + pp) * row_bytes + 16 * kb + (lane >> 1)] = static_cast<uint8_t>(byte);
+        if (lane == 0)
+          rec[(kb >> 2) * kSfRecord + sf_atom_byte(kParts * jr + pp, kb & 3)] = static_cast<uint8_t>(sv[j] + 127);
+      }
     }
   }
-}
-
-size_t smem_bytes(bool gate_up, int stages, int b_stage_bytes, int nb) {
-  const int kA = gate_up ? 2 : 1;
-  const size_t stage = static_cast<size_t>(stage_size(kA, b_stage_bytes));
-  return 1024 + stages * stage + ((kA * BM * nb + 15) & ~15) + (2 * kMaxStages + 3) * sizeof(uint64_t) + 32;
 }
 
 }  // namespace dec
@@ -517,100 +789,110 @@ EncodeTiled encoder() {
   return fn;
 }
 
-bool encode(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
-            const uint64_t* strides_bytes, const uint32_t* box) {
+bool encode(CUtensorMap* m, int rank, const void* base, const uint64_t* dims, const uint64_t* strides_bytes,
+            const uint32_t* box) {
   EncodeTiled fn = encoder();
   if (!fn) return false;
   cuuint64_t d[3], s[2];
   cuuint32_t b[3], es[3] = {1, 1, 1};
   for (int i = 0; i < rank; ++i) { d[i] = dims[i]; b[i] = box[i]; }
   for (int i = 0; i + 1 < rank; ++i) s[i] = strides_bytes[i];
-  return fn(m, dt, rank, const_cast<void*>(base), d, s, b, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, const_cast<void*>(base), d, s, b, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int stages_for(bool gate_up, int b_stage_bytes, int nb) {
-  for (int s = dec::kMaxStages; s >= 2; --s)
-    if (dec::smem_bytes(gate_up, s, b_stage_bytes, nb) <= 227 * 1024) return s;
-  return 0;
+constexpr size_t kPartBudget = 16u << 20;   // split-K partials, bytes
+
+int split_cap(int kA, int64_t P, int n_out) {
+  const double per = static_cast<double>(kA) * P * dec::kParts * n_out * 4.0;
+  const int64_t c = per > 0 ? static_cast<int64_t>(kPartBudget / per) : dec::kMaxSplit;
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(dec::kMaxSplit, c)));
 }
+
+int box_rows_for(int T) {
+  const int n = dec::kParts * T;
+  return n <= 8 ? 8 : (n <= 64 ? 16 : 32);
+}
+
+int max_chunks_for(int T) { return std::max(1, (T + dec::kGroupRows - 1) / dec::kGroupRows); }
+int nst_for(int K) { return (K + dec::BKS - 1) / dec::BKS; }
 
 }  // namespace
 
-bool decode_tc_supported(int H, int I, int np, int max_tokens_per_expert, const void* gu_blocks,
-                         const void* d_blocks) {
-  if (H % 64 || I % 64 || H < dec::BK || I < dec::BK) return false;
-  if (np * max_tokens_per_expert > dec::kMaxN) return false;
-  if ((reinterpret_cast<uintptr_t>(gu_blocks) | reinterpret_cast<uintptr_t>(d_blocks)) & 31u) return false;
-  const int bst = ((np * max_tokens_per_expert + dec::kBoxRows - 1) / dec::kBoxRows) * dec::kBoxRows * dec::BK;
-  if (stages_for(true, bst, std::max(H, I) / 32) < 2) return false;
+bool decode_tc_supported(int H, int I, int T, const void* gu_blocks, const void* d_blocks) {
+  if (H % 64 || I % 64 || H < 64 || I < 64 || T < 1 || T > kDecodeMaxT) return false;
+  if ((reinterpret_cast<uintptr_t>(gu_blocks) | reinterpret_cast<uintptr_t>(d_blocks)) & 15u) return false;
+  // the widest B tile must still leave two pipeline stages
+  const int worst = dec::ring_offset() + 2 * (dec::stage_bytes_for(2, dec::kMaxN) + dec::kSfStage);
+  if (worst + 1024 > dec::kSmemBytes) return false;
   return encoder() != nullptr;
 }
 
 cudaError_t decode_tc_prepare() {
-  const int smem = 227 * 1024;
+  const int smem = dec::kSmemBytes;
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(dec::decode_gemm_kernel<true, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
-  if ((e = cudaFuncSetAttribute(dec::decode_gemm_kernel<true, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
-  if ((e = cudaFuncSetAttribute(dec::decode_gemm_kernel<false, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
-  return cudaFuncSetAttribute(dec::decode_gemm_kernel<false, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if ((e = cudaFuncSetAttribute(dec::decode_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) return e;
+  return cudaFuncSetAttribute(dec::decode_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
 }
 
-size_t decode_tc_sfb_bytes(int E, int K) {
-  const int nkt = K / dec::BK + (K % dec::BK ? 1 : 0);
-  return static_cast<size_t>(E) * nkt * dec::kSfRecord;
+size_t decode_tc_xs_bytes(int64_t P, int K) { return static_cast<size_t>(P) * dec::kParts * (K / 2); }
+
+size_t decode_tc_sfb_bytes(int E, int K, int T) {
+  return static_cast<size_t>(E) * max_chunks_for(T) * 2 * nst_for(K) * dec::kSfRecord;
 }
 
-cudaError_t launch_split_tokens(int np, const uint16_t* x, const int32_t* perm_token, const int32_t* perm_slot,
+size_t decode_tc_part_bytes(int64_t P, int H, int I) {
+  const size_t gu = static_cast<size_t>(split_cap(2, P, I)) * 2 * P * dec::kParts * I * 4;
+  const size_t d = static_cast<size_t>(split_cap(1, P, H)) * 1 * P * dec::kParts * H * 4;
+  return std::max(gu, d);
+}
+
+size_t decode_tc_ticket_count(int H, int I) {
+  const size_t m_gu = (I + dec::BM - 1) / dec::BM, m_d = (H + dec::BM - 1) / dec::BM;
+  return static_cast<size_t>(dec::kMaxGrp) * (m_gu + m_d) * 4 + m_d * 4;
+}
+
+cudaError_t launch_split_tokens(bool fp8, const uint16_t* x, const int32_t* perm_token, const int32_t* perm_slot,
                                 const int32_t* topk_idx, const int32_t* offsets, int64_t P, int H, int k, float s0,
-                                uint8_t* xs, uint8_t* sfb, cudaStream_t st) {
-  const int nb = H / 32, nk_full = H / dec::BK, nkt = nk_full + (H % dec::BK ? 1 : 0);
-  const int64_t warps = P * nb;
-  const unsigned grid = static_cast<unsigned>(cdiv(warps * 32, 256));
-  if (np == 1)
-    dec::split_tokens_kernel<1><<<grid, 256, 0, st>>>(x, perm_token, perm_slot, topk_idx, offsets, P, H, k, s0,
-                                                      xs, sfb, nb, nk_full, nkt);
-  else
-    dec::split_tokens_kernel<3><<<grid, 256, 0, st>>>(x, perm_token, perm_slot, topk_idx, offsets, P, H, k, s0,
-                                                      xs, sfb, nb, nk_full, nkt);
-  return cudaGetLastError();
+                                int T, uint8_t* xs, uint8_t* sfb, cudaStream_t st) {
+  const int nb8 = (H / 32 + 7) / 8;
+  const int64_t warps = P * nb8;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(std::max<int64_t>(1, cdiv(warps * 32, 256))));
+  cfg.blockDim = dim3(256);
+  cfg.stream = st;
+  return cudaLaunchKernelEx(&cfg, dec::split_tokens_kernel, x, perm_token, perm_slot, topk_idx, offsets, P, H, k, s0,
+                            fp8 ? 1 : 0, xs, sfb, nst_for(H), max_chunks_for(T));
 }
 
-// gate_up (gate_up = true): A = gu weights, B = xs (np parts per row), writes xs_out /
-// sfb_out for the down GEMM. down: A = d weights, B = xs_out, writes y and the combine.
+// gate_up (gate_up = true): A = gu weights, B = xs (4 parts per routed row), writes xs_mid
+// / sfb_mid for the down GEMM. down: A = d weights, B = xs_mid, writes y and (a.out) the
+// combine of a few tokens.
 cudaError_t launch_decode_gemm(bool gate_up, const DecodeGemmArgs& a, cudaStream_t st) {
   using namespace dec;
+  const int kA = gate_up ? 2 : 1;
   const int K = gate_up ? a.H : a.I;
   const int n_out = gate_up ? a.I : a.H;
   const int groups = gate_up ? 2 * a.E : a.E;
-  const int np = gate_up ? a.np : a.np_mid;
-  const int64_t b_rows = a.P * np;
-  const int nb = K / 32, nk_full = K / BK, tail = (K % BK) / 32;
-  const int nkt = nk_full + (tail ? 1 : 0);
-  const int n_max = np * a.max_tokens_per_expert;
-  const int bst = ((n_max + kBoxRows - 1) / kBoxRows) * kBoxRows * BK;
-  const int S = stages_for(gate_up, bst, std::max(a.H, a.I) / 32);
-  if (S < 2) return cudaErrorInvalidValue;
-  CUtensorMap mw, mwt, mx;
+  const int64_t b_rows = a.P * kParts;
+  const int n_m = (n_out + BM - 1) / BM;
+  const int box_rows = box_rows_for(a.T);
+  if (a.E > kMaxE || a.k > kMaxTopK || a.T > kDecodeMaxT || (!gate_up && a.out && a.T > kDecodeFoldMaxT))
+    return cudaErrorInvalidValue;
+  CUtensorMap mw, mx;
   {
     const uint64_t row_bytes = static_cast<uint64_t>(K) / 2;
-    const uint64_t dims[3] = {static_cast<uint64_t>(nk_full * BK), static_cast<uint64_t>(n_out),
-                              static_cast<uint64_t>(groups)};
+    const uint64_t dims[3] = {row_bytes, static_cast<uint64_t>(n_out), static_cast<uint64_t>(groups)};
     const uint64_t strides[2] = {row_bytes, row_bytes * n_out};
-    const uint32_t box[3] = {BK, BM, 1};
-    const uint8_t* blocks = gate_up ? a.gu_blocks : a.d_blocks;
-    if (!encode(&mw, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, blocks, dims, strides, box)) return cudaErrorInvalidValue;
-    const uint64_t tdims[3] = {BK, static_cast<uint64_t>(n_out), static_cast<uint64_t>(groups)};
-    if (!encode(&mwt, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, blocks + (K - BK) / 2, tdims, strides, box))
-      return cudaErrorInvalidValue;
+    const uint32_t box[3] = {static_cast<uint32_t>(kRowBytes), BM, static_cast<uint32_t>(kA)};
+    if (!encode(&mw, 3, gate_up ? a.gu_blocks : a.d_blocks, dims, strides, box)) return cudaErrorInvalidValue;
   }
   {
-    const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(b_rows > 0 ? b_rows : 1)};
-    const uint64_t strides[1] = {static_cast<uint64_t>(K)};
-    const uint32_t box[2] = {BK, kBoxRows};
-    if (!encode(&mx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, gate_up ? a.xs : a.xs_mid, dims, strides, box))
-      return cudaErrorInvalidValue;
+    const uint64_t dims[2] = {static_cast<uint64_t>(K) / 2, static_cast<uint64_t>(b_rows > 0 ? b_rows : 1)};
+    const uint64_t strides[1] = {static_cast<uint64_t>(K) / 2};
+    const uint32_t box[2] = {static_cast<uint32_t>(kRowBytes), static_cast<uint32_t>(box_rows)};
+    if (!encode(&mx, 2, gate_up ? a.xs : a.xs_mid, dims, strides, box)) return cudaErrorInvalidValue;
   }
   Params prm{};
   prm.w_scales = gate_up ? a.gu_scales : a.d_scales;
@@ -620,10 +902,14 @@ cudaError_t launch_decode_gemm(bool gate_up, const DecodeGemmArgs& a, cudaStream
   prm.n_out = n_out;
   prm.E = a.E;
   prm.K = K;
-  prm.nb = nb;
-  prm.nk_full = nk_full;
-  prm.tail_steps = tail;
-  prm.np = np;
+  prm.nb = K / 32;
+  prm.nst = nst_for(K);
+  prm.n_m = n_m;
+  prm.box_rows = box_rows;
+  prm.split_cap = split_cap(kA, a.P, n_out);
+  prm.max_chunks = max_chunks_for(a.T);
+  prm.smem_bytes = kSmemBytes;
+  prm.P = a.P;
   prm.offsets = a.offsets;
   prm.active = a.active;
   prm.n_active = a.n_active;
@@ -631,35 +917,29 @@ cudaError_t launch_decode_gemm(bool gate_up, const DecodeGemmArgs& a, cudaStream
   prm.s_in = gate_up ? a.s0 : a.s1_in;
   prm.xs_out = a.xs_mid;
   prm.sfb_out = a.sfb_mid;
-  prm.np_out = a.np_mid;
-  prm.nb_out = a.I / 32;
-  prm.nk_full_out = a.I / BK;
-  prm.nkt_out = a.I / BK + (a.I % BK ? 1 : 0);
+  prm.nst_out = nst_for(a.I);
   prm.s_out = a.s1_quant;
-  prm.amax_bits = a.amax_bits;
   prm.y_out = a.y;
-  prm.out = a.out;
+  prm.out = gate_up ? nullptr : a.out;
   prm.topk_idx = a.topk_idx;
   prm.topk_w = a.topk_w;
   prm.inv = a.inv;
-  prm.tickets = a.tickets;
   prm.T = a.T;
   prm.k = a.k;
+  prm.part = a.part;
+  prm.split_tickets = gate_up ? a.split_tickets_gu : a.split_tickets_d;
+  prm.comb_tickets = a.comb_tickets;
   prm.err = a.err;
-  prm.stages = S;
-  prm.b_stage_bytes = bst;
-  dim3 grid(static_cast<unsigned>((n_out + BM - 1) / BM), static_cast<unsigned>(a.max_active));
-  const size_t smem = smem_bytes(gate_up, S, bst, std::max(a.H, a.I) / 32);
-  if (np != 1 && np != 3) return cudaErrorInvalidValue;
-  if (gate_up && np == 1)
-    decode_gemm_kernel<true, 1><<<grid, kThreads, smem, st>>>(mw, mwt, mx, prm);
-  else if (gate_up)
-    decode_gemm_kernel<true, 3><<<grid, kThreads, smem, st>>>(mw, mwt, mx, prm);
-  else if (np == 1)
-    decode_gemm_kernel<false, 1><<<grid, kThreads, smem, st>>>(mw, mwt, mx, prm);
-  else
-    decode_gemm_kernel<false, 3><<<grid, kThreads, smem, st>>>(mw, mwt, mx, prm);
-  return cudaGetLastError();
+  const int64_t max_grp = std::min<int64_t>(kMaxGrp, static_cast<int64_t>(a.max_active) + a.P / kGroupRows + 1);
+  const int64_t max_units = max_grp * n_m * prm.split_cap;
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(a.sms, max_units)));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = st;
+  if (gate_up) return cudaLaunchKernelEx(&cfg, decode_gemm_kernel<true>, mw, mx, prm);
+  return cudaLaunchKernelEx(&cfg, decode_gemm_kernel<false>, mw, mx, prm);
 }
 
 }  // namespace mxmoe

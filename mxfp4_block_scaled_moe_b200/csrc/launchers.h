@@ -60,7 +60,7 @@ cudaError_t launch_tc_gemm(bool gate_up, const uint8_t* a, int64_t P_rows, int K
                            float s_in, float s_out, uint8_t* a_out, float* y_out, int* err, int sms,
                            cudaStream_t st);
 
-struct DecodeGemmArgs {   // tensor-core decode path (weights as the MMA's A operand)
+struct DecodeGemmArgs {   // tensor-core decode path (kind::mxf4: packed e2m1 weights x e2m1 token parts)
   const uint8_t* gu_blocks;
   const uint8_t* gu_scales;
   const float* gu_bias;
@@ -69,38 +69,51 @@ struct DecodeGemmArgs {   // tensor-core decode path (weights as the MMA's A ope
   const float* d_bias;
   int E, H, I, T, k;
   int64_t P;
-  int np, np_mid;               // parts per token row of the two B operands (1 or 3)
-  int max_tokens_per_expert, max_active;
+  int max_active;               // bound on the active experts (min(E, P))
+  int sms;
   const int32_t* offsets;
   const int32_t* active;
   const int32_t* n_active;
   const int32_t* topk_idx;
   const float* topk_w;
   const int32_t* inv;
-  const uint8_t* xs;            // gate_up B operand rows (P*np, H) e4m3
-  const uint8_t* sfb;           // its scale records [E][nkt(H)][1024]
-  uint8_t* xs_mid;              // down B operand rows (P*np_mid, I)
-  uint8_t* sfb_mid;             // [E][nkt(I)][1024]
+  const uint8_t* xs;            // gate_up B operand: (P*4, H/2) packed e2m1 parts
+  const uint8_t* sfb;           // its scale records (decode_tc_sfb_bytes(E, H, T))
+  uint8_t* xs_mid;              // down B operand: (P*4, I/2)
+  uint8_t* sfb_mid;             // (decode_tc_sfb_bytes(E, I, T))
   float s0;                     // B scale of gate_up (FP8 s0, else 1)
-  float s1_quant;               // FP8: scale of a's e4m3 cast; 0: bf16 3-part split
+  float s1_quant;               // FP8: scale of a's e4m3 cast; 0: bf16 intermediate
   float s1_in;                  // B scale of down (FP8 s1, else 1)
-  unsigned* amax_bits;          // calibration: max |a| (nullable)
   float* y;                     // (P, H) fp32
-  uint16_t* out;                // (T, H) bf16 (combine; nullable = no combine)
-  unsigned* tickets;
+  uint16_t* out;                // (T, H) bf16: combine folded into the down kernel (nullable)
+  float* part;                  // split-K partials (decode_tc_part_bytes)
+  unsigned* split_tickets_gu;   // zero between calls (decode_tc_ticket_count covers all three)
+  unsigned* split_tickets_d;
+  unsigned* comb_tickets;
   int* err;
 };
-bool decode_tc_supported(int H, int I, int np, int max_tokens_per_expert, const void* gu_blocks,
-                         const void* d_blocks);
+constexpr int kDecodeMaxT = 64;      // tokens the tensor-core decode path takes
+constexpr int kDecodeMaxGroups = 320;  // row groups (an expert's routed rows, 56 at a time)
+constexpr int kDecodeFoldMaxT = 8;   // the down kernel folds the combine up to this many tokens
+bool decode_tc_supported(int H, int I, int T, const void* gu_blocks, const void* d_blocks);
 cudaError_t decode_tc_prepare();
-size_t decode_tc_sfb_bytes(int E, int K);
-cudaError_t launch_split_tokens(int np, const uint16_t* x, const int32_t* perm_token, const int32_t* perm_slot,
+size_t decode_tc_xs_bytes(int64_t P, int K);
+size_t decode_tc_sfb_bytes(int E, int K, int T);
+size_t decode_tc_part_bytes(int64_t P, int H, int I);
+size_t decode_tc_ticket_count(int H, int I);
+// offsets of the three ticket arrays inside the decode_tc_ticket_count block
+inline size_t decode_tc_tickets_d(int I) { return static_cast<size_t>(kDecodeMaxGroups) * ((I + 127) / 128) * 4; }
+inline size_t decode_tc_tickets_comb(int H, int I) {
+  return decode_tc_tickets_d(I) + static_cast<size_t>(kDecodeMaxGroups) * ((H + 127) / 128) * 4;
+}
+cudaError_t launch_split_tokens(bool fp8, const uint16_t* x, const int32_t* perm_token, const int32_t* perm_slot,
                                 const int32_t* topk_idx, const int32_t* offsets, int64_t P, int H, int k, float s0,
-                                uint8_t* xs, uint8_t* sfb, cudaStream_t st);
+                                int T, uint8_t* xs, uint8_t* sfb, cudaStream_t st);
 cudaError_t launch_decode_gemm(bool gate_up, const DecodeGemmArgs& a, cudaStream_t st);
 
 cudaError_t launch_combine(const float* y, const int32_t* topk_idx, const float* topk_w,
                            const int32_t* inv, int T, int H, int k, uint16_t* out, cudaStream_t st,
                            int sms);
+
 
 }  // namespace mxmoe
