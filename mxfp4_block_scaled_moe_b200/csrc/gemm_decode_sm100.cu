@@ -41,6 +41,7 @@
 #include <climits>
 
 #include <cuda.h>
+#include <cuda_fp4.h>
 
 #include "common.cuh"
 #include "launchers.h"
@@ -100,49 +101,27 @@ __device__ __forceinline__ int e2m1_part_exponent(float amax) {
   return s;
 }
 
-// e2m1 code (sign in bit 3) of v, |v| <= 6, rounded to nearest with ties to the even
-// code, as a count of the rounding thresholds that |v| passes (no branches: the lanes of
-// a warp hold different values).
-__device__ __forceinline__ uint32_t e2m1_code(float v) {
-  const float a = fabsf(v);
-  const uint32_t c = static_cast<uint32_t>(a > 0.25f) + static_cast<uint32_t>(a >= 0.75f) +
-                     static_cast<uint32_t>(a > 1.25f) + static_cast<uint32_t>(a >= 1.75f) +
-                     static_cast<uint32_t>(a > 2.5f) + static_cast<uint32_t>(a >= 3.5f) +
-                     static_cast<uint32_t>(a > 5.0f);
-  return c | (v < 0.0f && c != 0u ? 8u : 0u);
-}
-
-// Twice the magnitude of e2m1 code c & 7 (0, 1, 2, 3, 4, 6, 8, 12), from a nibble table.
-__device__ __forceinline__ uint32_t e2m1_twice(uint32_t c) { return (0xC8643210u >> (4u * (c & 7u))) & 15u; }
-
 // One e2m1 part of 8 rows' values r[j] (this lane's element of a 32-value block held by
-// the warp): the part codes q[j] and scale exponents sc[j] (the same in every lane), and
-// r[j] becomes the residual. The eight chains are independent, so their shuffles overlap.
-// Lanes outside the data pass 0. The residual update is exact: a part value has two
-// significant bits and a power-of-two scale.
-__device__ __forceinline__ void e2m1_part8(float (&r)[8], uint32_t (&q)[8], int (&sc)[8]) {
-  float a[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) a[j] = fabsf(r[j]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) a[j] = fmaxf(a[j], __shfl_xor_sync(0xffffffffu, a[j], o));
-  }
+// the warp). The block's largest magnitude is one warp max-reduction of the bit patterns
+// (non-negative floats order like their bits); the value is scaled by 2^-s and rounded
+// to e2m1 (nearest, ties to even) by the hardware conversion, which also packs this
+// lane's value with the next lane's into bytes[j] (even element in the low nibble;
+// meaningful in even lanes). sc[j] is the scale exponent (the same in every lane) and
+// r[j] becomes the residual; the update is exact (a part value has two significant bits
+// and a power-of-two scale). The eight chains are independent, so their latencies
+// overlap. Lanes outside the data pass 0.
+__device__ __forceinline__ void e2m1_part8(float (&r)[8], uint32_t (&bytes)[8], int (&sc)[8]) {
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
-    sc[j] = e2m1_part_exponent(a[j]);
-    q[j] = e2m1_code(r[j] * pow2f(-sc[j]));
-    const float qv = static_cast<float>(e2m1_twice(q[j])) * 0.5f * pow2f(sc[j]);   // exact
-    r[j] = r[j] - ((q[j] & 8u) ? -qv : qv);
+    const float amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(r[j]))));
+    sc[j] = e2m1_part_exponent(amax);
+    const float v = r[j] * pow2f(-sc[j]);
+    const float vn = __shfl_down_sync(0xffffffffu, v, 1);
+    bytes[j] = __nv_cvt_float2_to_fp4x2(make_float2(v, vn), __NV_E2M1, cudaRoundNearest);
+    const __nv_fp4x2_storage_t own = __nv_cvt_float2_to_fp4x2(make_float2(v, v), __NV_E2M1, cudaRoundNearest);
+    const __half2_raw h = __nv_cvt_fp4x2_to_halfraw2(own, __NV_E2M1);
+    r[j] = r[j] - __half2float(__half(__half_raw{h.x})) * pow2f(sc[j]);
   }
-}
-
-// Two lanes' codes into one byte (element 2i in the low nibble, as the weights pack);
-// meaningful in even lanes.
-__device__ __forceinline__ uint32_t pack_pair(uint32_t code) {
-  const uint32_t hi = __shfl_down_sync(0xffffffffu, code, 1);
-  return (code & 15u) | ((hi & 15u) << 4);
 }
 
 struct Params {
@@ -266,8 +245,10 @@ __device__ __forceinline__ void sum_parts(const float (&v)[8 * kParts], float (&
 
 // gate_up: bias, SwiGLU and the down GEMM's B operand for rows j0 .. j0+7 of the unit's
 // group. gs / us: the accumulators summed over a row's parts (before the per-tensor scale).
+// dry: the same instructions with every store masked off (warms the instruction cache).
 __device__ __forceinline__ void finish_gate_up(const Params& p, const Unit& w, int j0, const float (&gs)[8],
-                                               const float (&us)[8], float bg, float bu, int row, int lane) {
+                                               const float (&us)[8], float bg, float bu, int row, int lane,
+                                               bool dry) {
   const int kb = row >> 5;   // the warp's 32 rows: one 32-value block of the down contraction
   uint8_t* rec = p.sfb_out + ((static_cast<int64_t>(w.e) * p.max_chunks + w.c) * 2 * p.nst_out + (kb >> 2)) * kSfRecord;
   float a[8];
@@ -285,13 +266,13 @@ __device__ __forceinline__ void finish_gate_up(const Params& p, const Unit& w, i
   // matters because it runs once per unit and its instructions are fetched cold
 #pragma unroll 1
   for (int pp = 0; pp < kParts; ++pp) {
-    uint32_t q[8];
+    uint32_t bytes[8];
     int sv[8];
-    e2m1_part8(a, q, sv);
+    e2m1_part8(a, bytes, sv);
 #pragma unroll
     for (int jj = 0; jj < 8; ++jj) {
-      const uint32_t byte = pack_pair(q[jj]);
-      if (j0 + jj < w.n) {
+      const uint32_t byte = bytes[jj];
+      if (j0 + jj < w.n && !dry) {
         if ((lane & 1) == 0)
           p.xs_out[(static_cast<int64_t>(w.off + j0 + jj) * kParts + pp) * row_bytes + (row >> 1)] = static_cast<uint8_t>(byte);
         if (lane == 0) rec[sf_atom_byte(kParts * (j0 + jj) + pp, kb & 3)] = static_cast<uint8_t>(sv[jj] + 127);
@@ -428,12 +409,13 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
       sc.stage_bytes = stage_bytes_for(kA, b_rows);
       const int avail = static_cast<int>((smem_raw + p.smem_bytes) - ring);
       sc.stages = min(kMaxStages, avail / (sc.stage_bytes + kSfStage));
-      // K split: fewest stages on the busiest CTA, counting half a stage per partial
+      // K split: fewest stages on the busiest CTA, counting about four stages for each
+      // split unit's partial write, ticket and the finisher's reduction
       const int tiles = ng * p.n_m, G = gridDim.x;
       int best = 1, best_cost = INT_MAX;
       for (int s = 1; s <= min(p.split_cap, p.nst); ++s) {
         const int per = (tiles * s + G - 1) / G;
-        const int cost = 2 * per * ((p.nst + s - 1) / s) + (s > 1 ? per : 0);
+        const int cost = per * ((p.nst + s - 1) / s) + (s > 1 ? 4 * per : 0);
         if (cost < best_cost) { best_cost = cost; best = s; }
       }
       sc.nsplit = best;
@@ -600,6 +582,15 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
   } else {
     // ----------------------------------------------------------------- epilogue -----
     const int q = warp & 3;
+    if (kGateUp && blockIdx.x < sc.units) {
+      // The part-splitting epilogue runs once per unit, long after the kernel starts, and
+      // its instructions would come cold from memory that the weight stream saturates:
+      // run it once now, stores masked off, while the first stages load.
+      Unit dw{};
+      dw.n = 8;
+      float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      finish_gate_up(p, dw, 0, z, z, 0.0f, 0.0f, lane, lane, true);
+    }
     uint32_t use0 = 0u, use1 = 0u;
     int nxt = 0;
     for (int u = blockIdx.x; u < sc.units; u += gridDim.x) {
@@ -671,7 +662,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
           sum_parts(vg, gs);
           if (kGateUp) {
             sum_parts(vu, us);
-            finish_gate_up(p, w, j0, gs, us, bias0, bias1, row, lane);
+            finish_gate_up(p, w, j0, gs, us, bias0, bias1, row, lane, false);
           } else {
             finish_down(p, w, j0, gs, bias0, row);
           }
@@ -753,12 +744,12 @@ __global__ void __launch_bounds__(256) split_tokens_kernel(
   uint8_t* rec = sfb + (static_cast<int64_t>(e) * max_chunks + c) * 2 * nst * kSfRecord;
 #pragma unroll 1
   for (int pp = 0; pp < kParts; ++pp) {
-    uint32_t q[8];
+    uint32_t bytes[8];
     int sv[8];
-    e2m1_part8(r, q, sv);
+    e2m1_part8(r, bytes, sv);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      const uint32_t byte = pack_pair(q[j]);
+      const uint32_t byte = bytes[j];
       const int kb = kb0 + j;
       if (kb < nb) {
         if ((lane & 1) == 0) xs[(pos * kParts + pp) * row_bytes + 16 * kb + (lane >> 1)] = static_cast<uint8_t>(byte);
