@@ -314,13 +314,14 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
   }
   LayerBuffers b;
   layout(a.T, a.E, a.k, a.H, a.I, fp8, tc, dtc, &b, ws->base);
-  if (b.tickets_end > ws->tickets_zeroed) {
-    // the decode path's tickets reach past what is known to be zero: clear them once
-    // (every call leaves them at zero again)
+  // The decode path's tickets follow the fixed ticket block, where other layouts keep
+  // ordinary buffers: they are known to be zero only after a decode-path call, which
+  // leaves them at zero. Clear them when that is not known.
+  if (dtc && b.tickets_end > ws->tickets_zeroed) {
     cudaError_t e = cudaMemsetAsync(ws->base, 0, b.tickets_end, st);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync (tickets)");
-    ws->tickets_zeroed = b.tickets_end;
   }
+  ws->tickets_zeroed = dtc ? b.tickets_end : kTicketBytes;
   int launches = 0;
   cudaError_t e;
   const float s0 = fp8 ? act_scale[0] : 1.0f, s1 = fp8 ? act_scale[1] : 1.0f;
@@ -511,6 +512,7 @@ int moe_route_topk(const uint16_t* x, const uint16_t* router_w, const uint16_t* 
   if (!logits) {
     if (int rc = ensure_capacity(ws, kTicketBytes + static_cast<size_t>(T) * E * sizeof(float))) return rc;
     logits = reinterpret_cast<float*>(ws->base + kTicketBytes);
+    ws->tickets_zeroed = kTicketBytes;   // the decode path's tickets may lie here
   }
   cudaError_t e = mxmoe::launch_router(x, router_w, router_b, T, H, E, logits, st);
   if (e) return cuda_fail(e, "router launch");
@@ -547,6 +549,7 @@ int moe_permute(const int32_t* topk_idx, int T, int E, int k, int32_t* offsets,
   size_t o_counts = c.take<int32_t>(static_cast<int64_t>(mxmoe::permute_chunks(P)) * E);
   size_t o_act = c.take<int32_t>(E), o_n = c.take<int32_t>(1);
   if (int rc = ensure_capacity(ws, c.off)) return rc;
+  ws->tickets_zeroed = kTicketBytes;   // the decode path's tickets may lie here
   int launches = 0;
   cudaError_t e = mxmoe::launch_permute(
       topk_idx, T, E, k, reinterpret_cast<int32_t*>(ws->base + o_counts), offsets, perm_token,

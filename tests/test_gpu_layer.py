@@ -107,13 +107,40 @@ def test_decode_20b_shape_all_outputs(B, T):
     check_rows(B, p, d, np.arange(T))
 
 
-def test_decode_20b_shape_fp8(B):
-    """FP8 activations on a decode batch: one MX-FP8 part per token on the tensor-core
-    decode path (static scales from the calibration batch)."""
-    p, d = layer_case(inputs.decode_layer(T=8, E=32, device="cuda"))
+@pytest.mark.parametrize("T", [1, 8])
+def test_decode_20b_shape_fp8(B, T):
+    """FP8 activations on a decode batch (static scales from the calibration batch): the
+    e4m3 values are what the tensor-core decode path splits into e2m1 parts; T = 1 also
+    takes the split-K reduction."""
+    p, d = layer_case(inputs.decode_layer(T=T, E=32, device="cuda"))
     xc = inputs.calibration_x(device="cuda")
     s = oracle.calibrate(inputs.bits(xc), p.router_w, p.router_b, *p.weights, p.lay.k)
-    check_rows(B, p, d, np.arange(8), act_scale=s)
+    check_rows(B, p, d, np.arange(T), act_scale=s)
+
+
+@pytest.mark.parametrize("T,fp8", [(64, False), (57, True), (56, False), (29, False)])
+def test_decode_row_groups(B, T, fp8):
+    """Top-4 of 4 experts: every expert takes all T tokens. Above 56 routed rows an
+    expert splits into row groups (56 + the rest), and groups wider than 28 rows take
+    both accumulator slots of the decode GEMM."""
+    p, d = layer_case(inputs.small_layer(E=4, k=4, T=T, H=512, I=512, seed=3, device="cuda"))
+    s = None
+    if fp8:
+        xc = inputs.calibration_x(H=512, device="cuda")
+        s = oracle.calibrate(inputs.bits(xc), p.router_w, p.router_b, *p.weights, p.lay.k)
+    check_rows(B, p, d, np.arange(T), act_scale=s)
+
+
+def test_decode_after_other_workspace_users(B):
+    """The decode path's split-K and combine tickets share workspace bytes with other
+    calls' buffers (here the router's logits): a call that overwrites them between two
+    decode calls must not disturb the second."""
+    p, d = layer_case(inputs.decode_layer(T=8, E=32, device="cuda"))
+    check_rows(B, p, d, np.arange(8))
+    big = inputs.small_layer(E=64, k=4, T=2000, H=320, I=192, seed=9, device="cuda")
+    B.moe_route_topk(big.x, big.router_w, None, 4)   # logits land in the workspace
+    torch.cuda.synchronize()
+    check_rows(B, p, d, np.arange(8))
 
 
 def test_decode_23_experts(B):
