@@ -194,6 +194,16 @@ int mxmoe_profile_read(char* names, float* total_ms, int* calls, int max_entries
  * Returns MXMOE_OK or MXMOE_ECUDA. */
 int mxmoe_release(void);
 
+/* mxmoe_selftest_wait_timeout -- exercise the failure path of the library's bounded
+ * device waits. The pages have no counterpart: every mbarrier wait in the tensor-core
+ * kernels gives up after about a second (about 2e9 SM cycles), sets MXMOE_ETIMEOUT in the
+ * device error word and lets its kernel return instead of hanging. This call launches
+ * one CTA on `stream` whose thread waits, through that same bounded wait, on an mbarrier
+ * that nothing completes; the wait expires and the next mxmoe_check on the stream
+ * returns MXMOE_ETIMEOUT. Nothing faults or traps and the context stays usable.
+ * Returns MXMOE_OK (launched) or MXMOE_ECUDA. */
+int mxmoe_selftest_wait_timeout(void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -37,6 +37,7 @@ _SIGS = {
     "mxmoe_last_error": [],
     "mxmoe_last_launch_count": [],
     "mxmoe_release": [],
+    "mxmoe_selftest_wait_timeout": [_vp],
     "mxmoe_profile_enable": [_i32],
     "mxmoe_profile_read": [_vp, _vp, _vp, _i32],
 }
@@ -239,6 +240,12 @@ def mxmoe_last_launch_count() -> int:
 
 def mxmoe_release():
     _call("mxmoe_release")
+
+
+def mxmoe_selftest_wait_timeout(stream=None):
+    """Launch a bounded device wait that expires (about a second); the next
+    mxmoe_check raises MxmoeError with MXMOE_ETIMEOUT."""
+    _call("mxmoe_selftest_wait_timeout", _stream(stream))
 
 
 def mxmoe_profile_enable(on: bool = True):

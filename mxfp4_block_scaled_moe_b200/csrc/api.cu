@@ -615,6 +615,14 @@ int mxmoe_check(void* stream) {
   return MXMOE_OK;
 }
 
+int mxmoe_selftest_wait_timeout(void* stream) {
+  t_last_error.clear();
+  Workspace* ws = nullptr;
+  if (int rc = current_device_ws(&ws)) return rc;
+  cudaError_t e = mxmoe::launch_wait_selftest(ws->err, static_cast<cudaStream_t>(stream));
+  return e ? cuda_fail(e, "wait self-test launch") : MXMOE_OK;
+}
+
 const char* mxmoe_last_error(void) { return t_last_error.c_str(); }
 
 int mxmoe_last_launch_count(void) { return t_last_launches; }

@@ -116,4 +116,7 @@ cudaError_t launch_combine(const float* y, const int32_t* topk_idx, const float*
                            int sms);
 
 
+// mxmoe_selftest_wait_timeout: a bounded wait that expires (ETIMEOUT in *err)
+cudaError_t launch_wait_selftest(int* err, cudaStream_t st);
+
 }  // namespace mxmoe
