@@ -210,7 +210,7 @@ size_t layout(int T, int E, int k, int H, int I, bool fp8, bool tc, bool dtc, La
   size_t o_a1 = c.take<uint8_t>(tc ? P * H : 0);
   size_t o_a2 = c.take<uint8_t>(tc ? P * I : 0);
   size_t o_xs = c.take<uint8_t>(dtc ? static_cast<int64_t>(mxmoe::decode_tc_xs_bytes(P, H)) : 0);
-  size_t o_sfb = c.take<uint8_t>(dtc ? static_cast<int64_t>(mxmoe::decode_tc_sfb_bytes(E, H, T)) : 0);
+  size_t o_sfb = c.take<uint8_t>(dtc ? static_cast<int64_t>(mxmoe::decode_tc_sfb_row_bytes(E, T)) : 0);
   size_t o_xsm = c.take<uint8_t>(dtc ? static_cast<int64_t>(mxmoe::decode_tc_xs_bytes(P, I)) : 0);
   size_t o_sfbm = c.take<uint8_t>(dtc ? static_cast<int64_t>(mxmoe::decode_tc_sfb_bytes(E, I, T)) : 0);
   size_t o_part = c.take<uint8_t>(dtc ? static_cast<int64_t>(mxmoe::decode_tc_part_bytes(P, H, I)) : 0);

@@ -444,8 +444,12 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
       bool ok = true;
       for (int u = blockIdx.x; u < sc.units && ok; u += gridDim.x) {
         const Unit w = unit_at(sc, p, u);
-        const uint32_t tx = kA * BM * kRowBytes + w.nbox * p.box_rows * kRowBytes + 2 * kSfRecord;
-        const uint8_t* rec = p.sfb + (static_cast<int64_t>(w.e) * p.max_chunks + w.c) * 2 * p.nst * kSfRecord;
+        // B scales: gate_up has one record per row group (the same for every k-tile); down
+        // one per 128-wide k-tile
+        const uint32_t sfb_bytes = kGateUp ? kSfRecord : 2 * kSfRecord;
+        const uint32_t tx = kA * BM * kRowBytes + w.nbox * p.box_rows * kRowBytes + sfb_bytes;
+        const uint8_t* rec = kGateUp ? p.sfb + (static_cast<int64_t>(w.e) * p.max_chunks + w.c) * kSfRecord
+                                     : p.sfb + (static_cast<int64_t>(w.e) * p.max_chunks + w.c) * 2 * p.nst * kSfRecord;
         for (int kst = w.k0; kst < w.k1; ++kst) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[stage], tx);
@@ -453,7 +457,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
           for (int b = 0; b < w.nbox; ++b)
             tma_load_2d(sB(stage) + b * p.box_rows * kRowBytes, &map_x, &full[stage], kRowBytes * kst,
                         kParts * w.off + b * p.box_rows);
-          bulk_g2s(sSFB(stage), rec + 2 * kst * kSfRecord, 2 * kSfRecord, &full[stage]);
+          bulk_g2s(sSFB(stage), kGateUp ? rec : rec + 2 * kst * kSfRecord, sfb_bytes, &full[stage]);
           if (++stage == S) { stage = 0; phase ^= 1; }
         }
       }
@@ -465,7 +469,8 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
     uint32_t use0 = 0u, use1 = 0u;   // completed uses of each accumulator slot
     int nxt = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < sc.units && ok; u += gridDim.x) {
+    int uj = 0;   // units issued by this CTA
+    for (int u = blockIdx.x; u < sc.units && ok; u += gridDim.x, ++uj) {
       const Unit w = unit_at(sc, p, u);
       const bool big = kGateUp && w.ncols > kBigCols;
       const int slot = big ? 0 : nxt;
@@ -481,6 +486,9 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
       const uint32_t du = big ? static_cast<uint32_t>(kSlot1) : dg + static_cast<uint32_t>(w.ncols);
       const uint32_t id0 = idesc_mxf4(BM, w.ncols);
       const int nat = w.ncols > 128 ? 2 : 1;   // B scale atoms per k-tile
+      // gate_up: the unit's B scale atoms, copied once at its first stage into the slot of
+      // this unit's parity (the previous unit may still be reading the other slot)
+      const uint32_t sfb_unit = tmem + kSfbCol + 8 * static_cast<uint32_t>(uj & 1);
       for (int kst = w.k0; kst < w.k1; ++kst) {
         if (!mbar_wait(&full[stage], phase, abort_flag, p.err)) { ok = false; break; }
         tc_fence_after();
@@ -491,10 +499,14 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
 #pragma unroll
             for (int h = 0; h < kA; ++h)
               tc_cp_32x128b_x4(tmem + kSfaCol + 8 * h + 4 * t, smem_desc(smem_u32(sSFA(stage, h) + 512 * t), 0, 128, 0));
-            for (int b = 0; b < nat; ++b)
-              tc_cp_32x128b_x4(tmem + kSfbCol + 8 * t + 4 * b,
-                               smem_desc(smem_u32(sSFB(stage) + kSfRecord * t + 512 * b), 0, 128, 0));
+            if (!kGateUp)
+              for (int b = 0; b < nat; ++b)
+                tc_cp_32x128b_x4(tmem + kSfbCol + 8 * t + 4 * b,
+                                 smem_desc(smem_u32(sSFB(stage) + kSfRecord * t + 512 * b), 0, 128, 0));
           }
+          if (kGateUp && kst == w.k0)
+            for (int b = 0; b < nat; ++b)
+              tc_cp_32x128b_x4(sfb_unit + 4 * b, smem_desc(smem_u32(sSFB(stage) + 512 * b), 0, 128, 0));
           const uint32_t b0 = smem_u32(sB(stage));
           for (int sk = 0; sk < nks; ++sk) {
             const int t = sk >> 1;
@@ -507,7 +519,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
             for (int h = 0; h < kA; ++h) {
               const uint64_t ad = smem_desc(smem_u32(sA(stage, h)) + 32 * sk, 16, 1024, 2);
               tc_mma_mxf4(tmem + (h ? du : dg), ad, bd, id, (tmem + kSfaCol + 8 * h + 4 * t) | sel,
-                          (tmem + kSfbCol + 8 * t) | sel, acc);
+                          (kGateUp ? sfb_unit : tmem + kSfbCol + 8 * t) | sel, acc);
             }
           }
           tc_commit(&empty[stage]);
@@ -716,47 +728,64 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
 }
 
 // ------------------------------------------------ token operand of the gate_up GEMM --
-// One warp per (routed pair, 8 consecutive 32-value blocks): the pair's x (or, with FP8
-// activations, the e4m3 value of x / s0) as four e2m1 parts per block, packed in
-// expert-grouped row order, with the block scales in the row group's scale records.
-__global__ void __launch_bounds__(256) split_tokens_kernel(
+// One CTA per routed pair: the pair's x (or, with FP8 activations, the e4m3 value of
+// x / s0) as four e2m1 parts, each with ONE e8m0 scale for the whole row (the smallest s
+// with the row's largest residual / 2^s <= 6), packed in expert-grouped row order. A
+// row-wide scale costs a little accuracy against per-block scales (a simulation of the
+// 2880-long dot products: 1.2e-4 of the largest output instead of 4e-5, against a 2e-3
+// bar) and makes the gate_up GEMM's B scale atom the same for every k-tile, so the GEMM
+// copies it into tensor memory once per unit instead of twice per stage. Its record:
+// [expert][row group][two 512-byte atoms], the four k-block bytes of a row all equal.
+constexpr int kSplitThreads = 256;
+constexpr int kSplitVals = 16;   // values per thread: H <= 4096
+__global__ void __launch_bounds__(kSplitThreads) split_tokens_kernel(
     const uint16_t* __restrict__ x, const int32_t* __restrict__ perm_token, const int32_t* __restrict__ perm_slot,
     const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ offsets, int64_t P, int H, int k, float s0,
-    int fp8, uint8_t* __restrict__ xs, uint8_t* __restrict__ sfb, int nst, int max_chunks) {
-  const int lane = threadIdx.x & 31;
-  const int nb = H / 32, nb8 = (nb + 7) / 8;
-  const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  if (w >= P * nb8) return;
-  const int64_t pos = w / nb8;
-  const int kb0 = static_cast<int>(w % nb8) * 8;
+    int fp8, uint8_t* __restrict__ xs, uint8_t* __restrict__ sfb, int max_chunks) {
+  __shared__ float s_max[kSplitThreads / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t pos = blockIdx.x;
+  if (pos >= P) return;
   const int t = perm_token[pos];
   const int e = topk_idx[static_cast<int64_t>(t) * k + perm_slot[pos]];
   const int je = static_cast<int>(pos - offsets[e]);   // row within the expert
   const int c = je / kGroupRows, jr = je % kGroupRows;
-  float r[8];
+  // thread i holds elements i + 256 v: neighbouring lanes hold neighbouring elements
+  float r[kSplitVals];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    float v = 0.0f;
-    if (kb0 + j < nb) v = bf16_bits_to_f32(x[static_cast<int64_t>(t) * H + 32 * (kb0 + j) + lane]);
-    r[j] = fp8 ? e4m3_to_f32(act_quant_e4m3(v, s0)) : v;
+  for (int v = 0; v < kSplitVals; ++v) {
+    const int kk = static_cast<int>(threadIdx.x) + kSplitThreads * v;
+    float val = 0.0f;
+    if (kk < H) val = bf16_bits_to_f32(x[static_cast<int64_t>(t) * H + kk]);
+    r[v] = fp8 ? e4m3_to_f32(act_quant_e4m3(val, s0)) : val;
   }
   const int64_t row_bytes = H / 2;
-  uint8_t* rec = sfb + (static_cast<int64_t>(e) * max_chunks + c) * 2 * nst * kSfRecord;
+  uint8_t* rec = sfb + (static_cast<int64_t>(e) * max_chunks + c) * kSfRecord;
 #pragma unroll 1
   for (int pp = 0; pp < kParts; ++pp) {
-    uint32_t bytes[8];
-    int sv[8];
-    e2m1_part8(r, bytes, sv);
+    float m = 0.0f;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const uint32_t byte = bytes[j];
-      const int kb = kb0 + j;
-      if (kb < nb) {
-        if ((lane & 1) == 0) xs[(pos * kParts + pp) * row_bytes + 16 * kb + (lane >> 1)] = static_cast<uint8_t>(byte);
-        if (lane == 0)
-          rec[(kb >> 2) * kSfRecord + sf_atom_byte(kParts * jr + pp, kb & 3)] = static_cast<uint8_t>(sv[j] + 127);
-      }
+    for (int v = 0; v < kSplitVals; ++v) m = fmaxf(m, fabsf(r[v]));
+    m = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(m)));
+    __syncthreads();   // the previous part's maxima have been read
+    if (lane == 0) s_max[warp] = m;
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < kSplitThreads / 32; ++w) m = fmaxf(m, s_max[w]);
+    const int sc = e2m1_part_exponent(m);
+#pragma unroll
+    for (int v = 0; v < kSplitVals; ++v) {
+      const float q = r[v] * pow2f(-sc);
+      const float qn = __shfl_down_sync(0xffffffffu, q, 1);
+      const uint32_t byte = __nv_cvt_float2_to_fp4x2(make_float2(q, qn), __NV_E2M1, cudaRoundNearest);
+      const __nv_fp4x2_storage_t own = __nv_cvt_float2_to_fp4x2(make_float2(q, q), __NV_E2M1, cudaRoundNearest);
+      const __half2_raw h = __nv_cvt_fp4x2_to_halfraw2(own, __NV_E2M1);
+      r[v] = r[v] - __half2float(__half(__half_raw{h.x})) * pow2f(sc);   // exact
+      const int kk = static_cast<int>(threadIdx.x) + kSplitThreads * v;
+      if (kk < H && (lane & 1) == 0) xs[(pos * kParts + pp) * row_bytes + (kk >> 1)] = static_cast<uint8_t>(byte);
     }
+    if (threadIdx.x == 0)   // the row's scale for all four k-blocks of the atom word
+      *reinterpret_cast<uint32_t*>(rec + sf_atom_byte(kParts * jr + pp, 0)) = 0x01010101u * static_cast<uint32_t>(sc + 127);
   }
 }
 
@@ -813,6 +842,7 @@ int nst_for(int K) { return (K + dec::BKS - 1) / dec::BKS; }
 
 bool decode_tc_supported(int H, int I, int T, const void* gu_blocks, const void* d_blocks) {
   if (H % 64 || I % 64 || H < 64 || I < 64 || T < 1 || T > kDecodeMaxT) return false;
+  if (H > dec::kSplitThreads * dec::kSplitVals) return false;   // the token split holds a row
   if ((reinterpret_cast<uintptr_t>(gu_blocks) | reinterpret_cast<uintptr_t>(d_blocks)) & 15u) return false;
   // the widest B tile must still leave two pipeline stages
   const int worst = dec::ring_offset() + 2 * (dec::stage_bytes_for(2, dec::kMaxN) + dec::kSfStage);
@@ -833,6 +863,8 @@ size_t decode_tc_sfb_bytes(int E, int K, int T) {
   return static_cast<size_t>(E) * max_chunks_for(T) * 2 * nst_for(K) * dec::kSfRecord;
 }
 
+size_t decode_tc_sfb_row_bytes(int E, int T) { return static_cast<size_t>(E) * max_chunks_for(T) * dec::kSfRecord; }
+
 size_t decode_tc_part_bytes(int64_t P, int H, int I) {
   const size_t gu = static_cast<size_t>(split_cap(2, P, I)) * 2 * P * dec::kParts * I * 4;
   const size_t d = static_cast<size_t>(split_cap(1, P, H)) * 1 * P * dec::kParts * H * 4;
@@ -847,14 +879,10 @@ size_t decode_tc_ticket_count(int H, int I) {
 cudaError_t launch_split_tokens(bool fp8, const uint16_t* x, const int32_t* perm_token, const int32_t* perm_slot,
                                 const int32_t* topk_idx, const int32_t* offsets, int64_t P, int H, int k, float s0,
                                 int T, uint8_t* xs, uint8_t* sfb, cudaStream_t st) {
-  const int nb8 = (H / 32 + 7) / 8;
-  const int64_t warps = P * nb8;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(std::max<int64_t>(1, cdiv(warps * 32, 256))));
-  cfg.blockDim = dim3(256);
-  cfg.stream = st;
-  return cudaLaunchKernelEx(&cfg, dec::split_tokens_kernel, x, perm_token, perm_slot, topk_idx, offsets, P, H, k, s0,
-                            fp8 ? 1 : 0, xs, sfb, nst_for(H), max_chunks_for(T));
+  if (P <= 0) return cudaSuccess;
+  dec::split_tokens_kernel<<<static_cast<unsigned>(P), dec::kSplitThreads, 0, st>>>(
+      x, perm_token, perm_slot, topk_idx, offsets, P, H, k, s0, fp8 ? 1 : 0, xs, sfb, max_chunks_for(T));
+  return cudaGetLastError();
 }
 
 // gate_up (gate_up = true): A = gu weights, B = xs (4 parts per routed row), writes xs_mid

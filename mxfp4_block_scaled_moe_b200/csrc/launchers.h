@@ -78,7 +78,7 @@ struct DecodeGemmArgs {   // tensor-core decode path (kind::mxf4: packed e2m1 we
   const float* topk_w;
   const int32_t* inv;
   const uint8_t* xs;            // gate_up B operand: (P*4, H/2) packed e2m1 parts
-  const uint8_t* sfb;           // its scale records (decode_tc_sfb_bytes(E, H, T))
+  const uint8_t* sfb;           // its scale records, one per row group (decode_tc_sfb_row_bytes)
   uint8_t* xs_mid;              // down B operand: (P*4, I/2)
   uint8_t* sfb_mid;             // (decode_tc_sfb_bytes(E, I, T))
   float s0;                     // B scale of gate_up (FP8 s0, else 1)
@@ -98,7 +98,8 @@ constexpr int kDecodeFoldMaxT = 8;   // the down kernel folds the combine up to 
 bool decode_tc_supported(int H, int I, int T, const void* gu_blocks, const void* d_blocks);
 cudaError_t decode_tc_prepare();
 size_t decode_tc_xs_bytes(int64_t P, int K);
-size_t decode_tc_sfb_bytes(int E, int K, int T);
+size_t decode_tc_sfb_bytes(int E, int K, int T);       // per 128-wide k-tile records (down's B)
+size_t decode_tc_sfb_row_bytes(int E, int T);          // one record per row group (gate_up's B)
 size_t decode_tc_part_bytes(int64_t P, int H, int I);
 size_t decode_tc_ticket_count(int H, int I);
 // offsets of the three ticket arrays inside the decode_tc_ticket_count block
