@@ -246,22 +246,24 @@ __device__ __forceinline__ void sum_parts(const float (&v)[8 * kParts], float (&
 // gate_up: bias, SwiGLU and the down GEMM's B operand for rows j0 .. j0+7 of the unit's
 // group. gs / us: the accumulators summed over a row's parts (before the per-tensor scale).
 // dry: the same instructions with every store masked off (warms the instruction cache).
-__device__ __forceinline__ void finish_gate_up(const Params& p, const Unit& w, int j0, const float (&gs)[8],
-                                               const float (&us)[8], float bg, float bu, int row, int lane,
-                                               bool dry) {
+// Not inlined, so that the warm-up call and the real ones run the same code.
+__device__ __noinline__ void finish_gate_up(uint8_t* xs_out, uint8_t* sfb_out, int n_out, int nst_out,
+                                            int max_chunks, float s_in, float s_out, int e, int c, int off, int n,
+                                            int j0, const float (&gs)[8], const float (&us)[8], float bg, float bu,
+                                            int row, int lane, bool dry) {
   const int kb = row >> 5;   // the warp's 32 rows: one 32-value block of the down contraction
-  uint8_t* rec = p.sfb_out + ((static_cast<int64_t>(w.e) * p.max_chunks + w.c) * 2 * p.nst_out + (kb >> 2)) * kSfRecord;
+  uint8_t* rec = sfb_out + ((static_cast<int64_t>(e) * max_chunks + c) * 2 * nst_out + (kb >> 2)) * kSfRecord;
   float a[8];
 #pragma unroll
   for (int jj = 0; jj < 8; ++jj) {
-    const float gv = __fadd_rn(__fmul_rn(p.s_in, gs[jj]), bg);
-    const float uv = __fadd_rn(__fmul_rn(p.s_in, us[jj]), bu);
-    float v = j0 + jj < w.n ? silu_mul(gv, uv) : 0.0f;
+    const float gv = __fadd_rn(__fmul_rn(s_in, gs[jj]), bg);
+    const float uv = __fadd_rn(__fmul_rn(s_in, us[jj]), bu);
+    float v = j0 + jj < n ? silu_mul(gv, uv) : 0.0f;
     // the layer's intermediate: e4m3(a / s1) with FP8 activations, else bf16(a)
-    v = p.s_out > 0.0f ? e4m3_to_f32(act_quant_e4m3(v, p.s_out)) : bf16_bits_to_f32(f32_to_bf16_bits_rn(v));
+    v = s_out > 0.0f ? e4m3_to_f32(act_quant_e4m3(v, s_out)) : bf16_bits_to_f32(f32_to_bf16_bits_rn(v));
     a[jj] = v;
   }
-  const int64_t row_bytes = p.n_out / 2;
+  const int64_t row_bytes = n_out / 2;
   // one part at a time, stored as it is made: a rolled loop keeps this code small, which
   // matters because it runs once per unit and its instructions are fetched cold
 #pragma unroll 1
@@ -272,9 +274,9 @@ __device__ __forceinline__ void finish_gate_up(const Params& p, const Unit& w, i
 #pragma unroll
     for (int jj = 0; jj < 8; ++jj) {
       const uint32_t byte = bytes[jj];
-      if (j0 + jj < w.n && !dry) {
+      if (j0 + jj < n && !dry) {
         if ((lane & 1) == 0)
-          p.xs_out[(static_cast<int64_t>(w.off + j0 + jj) * kParts + pp) * row_bytes + (row >> 1)] = static_cast<uint8_t>(byte);
+          xs_out[(static_cast<int64_t>(off + j0 + jj) * kParts + pp) * row_bytes + (row >> 1)] = static_cast<uint8_t>(byte);
         if (lane == 0) rec[sf_atom_byte(kParts * (j0 + jj) + pp, kb & 3)] = static_cast<uint8_t>(sv[jj] + 127);
       }
     }
@@ -598,10 +600,9 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
       // The part-splitting epilogue runs once per unit, long after the kernel starts, and
       // its instructions would come cold from memory that the weight stream saturates:
       // run it once now, stores masked off, while the first stages load.
-      Unit dw{};
-      dw.n = 8;
       float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      finish_gate_up(p, dw, 0, z, z, 0.0f, 0.0f, lane, lane, true);
+      finish_gate_up(p.xs_out, p.sfb_out, p.n_out, p.nst_out, p.max_chunks, p.s_in, p.s_out, 0, 0, 0, 8, 0, z, z,
+                     0.0f, 0.0f, lane, lane, true);
     }
     uint32_t use0 = 0u, use1 = 0u;
     int nxt = 0;
@@ -674,7 +675,8 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
           sum_parts(vg, gs);
           if (kGateUp) {
             sum_parts(vu, us);
-            finish_gate_up(p, w, j0, gs, us, bias0, bias1, row, lane, false);
+            finish_gate_up(p.xs_out, p.sfb_out, p.n_out, p.nst_out, p.max_chunks, p.s_in, p.s_out, w.e, w.c, w.off,
+                           w.n, j0, gs, us, bias0, bias1, row, lane, false);
           } else {
             finish_down(p, w, j0, gs, bias0, row);
           }
