@@ -113,7 +113,7 @@ int moe_permute(const int32_t* topk_idx, int T, int E, int k, int32_t* offsets,
  * hot path, or a latency-bound loop that cannot afford cudaMalloc's implicit device
  * synchronization. moe_permute itself grows the library workspace with cudaMalloc on its
  * first call at a size; this variant allocates nothing and keeps its scratch (per-chunk
- * expert histograms, the list of active experts) in a fixed 66,816-byte array in the
+ * expert histograms, the list of active experts) in a fixed 132,352-byte array in the
  * library's device image, which every GPU that loads the library holds until the process
  * exits.
  * Same arguments, outputs and ordering as moe_permute. Limits: T*k <= 262144 and

@@ -179,7 +179,6 @@ struct LayerBuffers {
   uint16_t* act_mid;   // (P, I) bf16 bits of the down-projection input
   float* y;            // (P, H) fp32 expert outputs
   unsigned* amax;      // 2 x fp32 bits (calibration)
-  uint8_t* xq8;        // tcgen05 path: e4m3 codes of x / s0, (T, H)
   uint8_t* a1;         // tcgen05 path: gate_up input rows grouped by expert, (P, H)
   uint8_t* a2;         // tcgen05 path: down input rows, (P, I)
   uint8_t* xs;         // tensor-core decode: gate_up B rows (P*4, H/2) packed e2m1 parts
@@ -206,7 +205,6 @@ size_t layout(int T, int E, int k, int H, int I, bool fp8, bool tc, bool dtc, La
   size_t o_mid = c.take<uint16_t>(tc ? 0 : P * I);
   size_t o_y = c.take<float>(P * H);
   size_t o_amax = c.take<unsigned>(2);
-  size_t o_xq8 = c.take<uint8_t>(tc ? static_cast<int64_t>(T) * H : 0);
   size_t o_a1 = c.take<uint8_t>(tc ? P * H : 0);
   size_t o_a2 = c.take<uint8_t>(tc ? P * I : 0);
   size_t o_xs = c.take<uint8_t>(dtc ? static_cast<int64_t>(mxmoe::decode_tc_xs_bytes(P, H)) : 0);
@@ -233,7 +231,6 @@ size_t layout(int T, int E, int k, int H, int I, bool fp8, bool tc, bool dtc, La
     b->act_mid = reinterpret_cast<uint16_t*>(base + o_mid);
     b->y = reinterpret_cast<float*>(base + o_y);
     b->amax = reinterpret_cast<unsigned*>(base + o_amax);
-    b->xq8 = reinterpret_cast<uint8_t*>(base + o_xq8);
     b->a1 = reinterpret_cast<uint8_t*>(base + o_a1);
     b->a2 = reinterpret_cast<uint8_t*>(base + o_a2);
     b->xs = reinterpret_cast<uint8_t*>(base + o_xs);
@@ -348,13 +345,11 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
     tm.mark("permute");
   }
   if (tc) {
-    if ((e = launch_fp8_quant(a.x, static_cast<int64_t>(a.T) * a.H, s0, b.xq8, st, ws->sms)))
-      return cuda_fail(e, "fp8 activation cast");
+    // the A-FP8 cast and the scatter into expert-grouped rows: one pass over x, one cast per token
+    if ((e = launch_quant_scatter_fp8(a.x, b.topk_idx, b.inv, a.T, a.k, a.E, P, a.H, s0, b.a1, st, ws->sms)))
+      return cuda_fail(e, "fp8 activation cast + scatter");
     ++launches;
-    tm.mark("act_quant");
-    if ((e = launch_gather_fp8_rows(b.xq8, b.perm_token, P, a.H, b.a1, st, ws->sms))) return cuda_fail(e, "gather");
-    ++launches;
-    tm.mark("gather");
+    tm.mark("act_quant+scatter");
     if ((e = launch_tc_gemm(true, b.a1, P, a.H, a.gu_blocks, a.gu_scales, a.gu_bias, a.E, a.I, b.offsets, s0, s1,
                             b.a2, nullptr, ws->err, ws->sms, st)))
       return cuda_fail(e, "gate_up (tcgen05)");
@@ -691,10 +686,10 @@ namespace {
 
 constexpr int64_t kNoAllocMaxPairs = 262144;   // T * k accepted by the variant
 constexpr int kNoAllocMaxExperts = 256;
-constexpr int kNoAllocMaxChunks = 64;          // permute chunks of 4096 pairs
+constexpr int kNoAllocMaxChunks = 128;         // the permute never uses more chunks
 constexpr int kNoAllocInts = kNoAllocMaxChunks * kNoAllocMaxExperts + kNoAllocMaxExperts + 64;
 
-// 256-byte aligned, 66,816 bytes; every GPU that loads the library keeps it until exit.
+// 256-byte aligned, 132,352 bytes; every GPU that loads the library keeps it until exit.
 static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocInts];
 
 int32_t* g_noalloc_dev[kMaxDevices] = {};

@@ -29,8 +29,9 @@ cudaError_t launch_fp8_quant(const uint16_t* x, int64_t n, float s, uint8_t* q, 
                              int sms);
 cudaError_t launch_fp8_quant_as_bf16(const uint16_t* x, int64_t n, float s, uint16_t* xq,
                                      cudaStream_t st, int sms);
-cudaError_t launch_gather_fp8_rows(const uint8_t* xq8, const int32_t* perm_token, int64_t P, int H,
-                                   uint8_t* a1, cudaStream_t st, int sms);
+cudaError_t launch_quant_scatter_fp8(const uint16_t* x, const int32_t* topk_idx, const int32_t* inv, int T,
+                                    int k, int E, int64_t P, int H, float s, uint8_t* a1, cudaStream_t st,
+                                    int sms);
 cudaError_t launch_amax_bf16(const uint16_t* x, int64_t n, unsigned* amax_bits, cudaStream_t st,
                              int sms);
 cudaError_t launch_finalize_scales(const unsigned* amax_bits, float* out, cudaStream_t st);

@@ -7,6 +7,8 @@
 // id; the softmax runs over the k selected logits.
 // Permutation: the routed dispatch of "quantization_mxfp4", As GPT-OSS's native format:
 // pairs (token, slot) grouped by expert, ascending token inside an expert.
+#include <atomic>
+
 #include "common.cuh"
 
 namespace mxmoe {
@@ -50,10 +52,13 @@ __global__ void __launch_bounds__(256) router_gemv_kernel(const uint16_t* __rest
 
 // ------------------------------------------------------------------ router GEMM -----
 // logits (T, E) = x (T, H) . Wr (E, H)^T with mma.sync m16n8k16 (bf16 in, fp32 acc).
-// CTA tile 64 tokens x 64 experts, 4 warps as 2 x 2 (each 32 x 32), K in steps of 32
-// staged by cp.async into padded shared rows (80-byte pitch: ldmatrix conflict-free).
+// CTA tile 64 tokens x 64 experts, 4 warps as 2 x 2 (each 32 x 32), K in steps of 128
+// staged by cp.async into padded shared rows (272-byte pitch: ldmatrix conflict-free).
+// The work is small (2*T*H*E FLOP) and each K step ends in a CTA barrier, so the steps are
+// wide: 23 of them at H = 2880 rather than 90.
 namespace rg {
-constexpr int BM = 64, BN = 64, BK = 32, PITCH = 40, STAGES = 3;  // pitch in bf16 elements
+constexpr int BM = 64, BN = 64, BK = 128, PITCH = 136, STAGES = 3;  // pitch in bf16 elements
+constexpr int kSmemBytes = STAGES * (BM + BN) * PITCH * 2;
 }
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool pred) {
@@ -78,22 +83,25 @@ __global__ void __launch_bounds__(128) router_gemm_kernel(const uint16_t* __rest
                                                            int T, int H, int E,
                                                            float* __restrict__ logits) {
   using namespace rg;
-  __shared__ __align__(16) uint16_t sa[STAGES][BM * PITCH];
-  __shared__ __align__(16) uint16_t sb[STAGES][BN * PITCH];
+  extern __shared__ __align__(16) uint16_t rg_smem[];
+  uint16_t (*sa)[BM * PITCH] = reinterpret_cast<uint16_t (*)[BM * PITCH]>(rg_smem);
+  uint16_t (*sb)[BN * PITCH] = reinterpret_cast<uint16_t (*)[BN * PITCH]>(rg_smem + STAGES * BM * PITCH);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int m0 = blockIdx.x * BM, n0 = blockIdx.y * BN;
   const int wm = (warp >> 1) * 32, wn = (warp & 1) * 32;
-  const int nk = H / BK;
+  const int nk = (H + BK - 1) / BK;   // the last K step may be partial (H % 32 == 0)
 
   auto load_stage = [&](int stage, int kt) {
-    // 64 rows x 64 bytes per operand = 256 chunks of 16 B each; 128 threads x 2
+    // 64 rows x 256 bytes per operand = 1024 chunks of 16 B each; 128 threads x 8
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int c = tid + i * 128, row = c >> 2, col = (c & 3) * 8;
+    for (int i = 0; i < 8; ++i) {
+      const int c = tid + i * 128, row = c >> 4, col = (c & 15) * 8;
       const int gm = m0 + row, gn = n0 + row;
       const int gmc = gm < T ? gm : T - 1, gnc = gn < E ? gn : E - 1;
-      cp_async16(&sa[stage][row * PITCH + col], x + static_cast<int64_t>(gmc) * H + kt * BK + col, gm < T);
-      cp_async16(&sb[stage][row * PITCH + col], wr + static_cast<int64_t>(gnc) * H + kt * BK + col, gn < E);
+      const int kc = kt * BK + col;
+      const bool kin = kc < H;   // columns past H read as zeros
+      cp_async16(&sa[stage][row * PITCH + col], x + static_cast<int64_t>(gmc) * H + (kin ? kc : 0), gm < T && kin);
+      cp_async16(&sb[stage][row * PITCH + col], wr + static_cast<int64_t>(gnc) * H + (kin ? kc : 0), gn < E && kin);
     }
   };
 
@@ -224,23 +232,32 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
 
 // --------------------------------------------------------------------- permute -----
 // Stable counting sort of the P = T*k pairs by expert, in two passes over chunks of
-// kPermChunk pairs: (1) per-chunk histograms, (2) every CTA rebuilds the global offsets
-// and its own start per expert from the histograms, then places its pairs in order.
-// Within a sub-chunk of 512 pairs the rank of a pair among equal experts is its rank in
-// its warp (match_any) plus the counts of the same expert in lower warps.
-constexpr int kPermChunk = 4096;
+// `chunk` pairs (a multiple of kPermThreads, at most kPermMaxChunks chunks): (1) per-chunk
+// histograms, (2) every CTA rebuilds the global offsets and its own start per expert from
+// the histograms, then places its pairs in order. Within a sub-chunk of kPermThreads pairs
+// the rank of a pair among equal experts is its rank in its warp (match_any) plus the
+// counts of the same expert in lower warps. Small chunks keep many CTAs busy: at 16K
+// pairs there are 32 CTAs and each places its pairs in one round.
 constexpr int kPermThreads = 512;
+constexpr int kPermMaxChunks = 128;
+
+__host__ __device__ __forceinline__ int64_t permute_chunk_size(int64_t P) {
+  const int64_t subs = cdiv(P, kPermThreads);
+  return kPermThreads * (subs < kPermMaxChunks ? 1 : cdiv(subs, kPermMaxChunks));
+}
 
 __global__ void __launch_bounds__(kPermThreads) permute_count_kernel(
-    const int32_t* __restrict__ idx, int64_t P, int E, int32_t* __restrict__ counts) {
+    const int32_t* __restrict__ idx, int64_t P, int E, int32_t* __restrict__ counts, int* __restrict__ err) {
   __shared__ int hist[256];
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
-  const int64_t lo = static_cast<int64_t>(blockIdx.x) * kPermChunk;
-  const int64_t hi = min(P, lo + kPermChunk);
+  const int64_t chunk = permute_chunk_size(P);
+  const int64_t lo = static_cast<int64_t>(blockIdx.x) * chunk;
+  const int64_t hi = min(P, lo + chunk);
   for (int64_t p = lo + threadIdx.x; p < hi; p += blockDim.x) {
     const int e = idx[p];
     if (e >= 0 && e < E) atomicAdd(&hist[e], 1);
+    else set_device_error(err, MXMOE_EDEVICE);
   }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) counts[static_cast<int64_t>(blockIdx.x) * E + e] = hist[e];
@@ -265,9 +282,10 @@ __device__ void permute_scatter_body(
   int (*wc)[256] = sm.wc;
   int* scan_tmp = sm.scan_tmp;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nchunks = static_cast<int>(cdiv(P, kPermChunk));
-  const int64_t lo = static_cast<int64_t>(cta) * kPermChunk;
-  const int64_t hi = min(P, lo + kPermChunk);
+  const int64_t chunk = permute_chunk_size(P);
+  const int nchunks = static_cast<int>(cdiv(P, chunk));
+  const int64_t lo = static_cast<int64_t>(cta) * chunk;
+  const int64_t hi = min(P, lo + chunk);
 
   if (counts == nullptr) {
     for (int e = tid; e < E; e += blockDim.x) total[e] = 0;
@@ -290,11 +308,6 @@ __device__ void permute_scatter_body(
       total[e] = all;
       base[e] = before;
     }
-    if (cta == 0)
-      for (int64_t p = tid; p < P; p += blockDim.x) {
-        const int e = idx[p];
-        if (e < 0 || e >= E) set_device_error(err, MXMOE_EDEVICE);
-      }
   }
   __syncthreads();
   // exclusive scan of total[] over experts (E <= 256) by one warp, in expert order
@@ -451,7 +464,7 @@ __global__ void __launch_bounds__(kPermThreads) route_small_kernel(
 }
 
 bool route_small_supported(int T, int E, int k) {
-  return T <= kSmallT && E <= kSmallE && static_cast<int64_t>(T) * k <= kPermChunk;
+  return T <= kSmallT && E <= kSmallE && static_cast<int64_t>(T) * k <= 4096;   // one CTA places at most 4096 pairs
 }
 
 cudaError_t launch_route_small(const uint16_t* x, const uint16_t* wr, const uint16_t* br, int T, int H, int E,
@@ -494,20 +507,51 @@ __global__ void __launch_bounds__(256) fp8_quant_as_bf16_kernel(const uint4* __r
   }
 }
 
-// Gather the e4m3 rows of the routed pairs into expert-grouped order:
-// a1[pos, :] = e4m3(x[perm_token[pos], :] / s) (one warp per row, 16 B per lane).
-__global__ void __launch_bounds__(256) gather_fp8_rows_kernel(const uint8_t* __restrict__ xq8,
-                                                               const int32_t* __restrict__ perm_token,
-                                                               int64_t P, int H,
-                                                               uint8_t* __restrict__ a1) {
+// The A-FP8 cast fused with the scatter into expert-grouped order (one pass over x, one cast
+// per token): a1[inv[t*k + j], :] = e4m3(fp32(x[t, :] / s)) for each of token t's k routed
+// slots. One warp per token, eight values per lane and chunk, four chunks in flight; a slot
+// whose expert id or position is out of range is skipped (the permute has flagged it).
+__global__ void __launch_bounds__(256) quant_scatter_fp8_kernel(const uint16_t* __restrict__ x,
+                                                                 const int32_t* __restrict__ topk_idx,
+                                                                 const int32_t* __restrict__ inv, int T,
+                                                                 int k, int E, int64_t P, int H, float s,
+                                                                 uint8_t* __restrict__ a1) {
   const int lane = threadIdx.x & 31;
-  const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  for (int64_t pos = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; pos < P;
-       pos += nw) {
-    const int64_t t = perm_token[pos];
-    const uint4* src = reinterpret_cast<const uint4*>(xq8 + t * H);
-    uint4* dst = reinterpret_cast<uint4*>(a1 + pos * H);
-    for (int c = lane; c < H / 16; c += 32) dst[c] = src[c];
+  const int nw = static_cast<int>((static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5);
+  const int n8 = H / 8;
+  for (int t = static_cast<int>((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5); t < T;
+       t += nw) {
+    int my_pos = -1;
+    if (lane < k) {
+      const int64_t p = static_cast<int64_t>(t) * k + lane;
+      const int e = topk_idx[p];
+      const int pos = inv[p];
+      if (e >= 0 && e < E && pos >= 0 && pos < P) my_pos = pos;
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(t) * H);
+    for (int c0 = lane; c0 < n8; c0 += 4 * 32) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (c0 + 32 * u < n8) v[u] = ld_nc_v4(src + c0 + 32 * u);   // four chunks in flight
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (c0 + 32 * u >= n8) break;
+        const uint32_t in[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+        uint32_t q[2] = {0u, 0u};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t lo = act_quant_e4m3(__uint_as_float(in[j] << 16), s);
+          const uint32_t hi = act_quant_e4m3(__uint_as_float(in[j] & 0xFFFF0000u), s);
+          q[j >> 1] |= (lo | (hi << 8)) << (16 * (j & 1));
+        }
+        const uint2 qv = make_uint2(q[0], q[1]);
+        for (int j = 0; j < k; ++j) {
+          const int pos = __shfl_sync(0xffffffffu, my_pos, j);
+          if (pos >= 0) reinterpret_cast<uint2*>(a1 + static_cast<int64_t>(pos) * H)[c0 + 32 * u] = qv;
+        }
+      }
+    }
   }
 }
 
@@ -533,8 +577,18 @@ cudaError_t launch_router(const uint16_t* x, const uint16_t* wr, const uint16_t*
     const int64_t warps = static_cast<int64_t>(T) * E;
     router_gemv_kernel<<<static_cast<unsigned>(cdiv(warps * 32, 256)), 256, 0, st>>>(x, wr, br, T, H, E, logits);
   } else {
+    static std::atomic<uint64_t> smem_set{0};   // one bit per device
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(smem_set.load() & bit)) {
+      e = cudaFuncSetAttribute(router_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, rg::kSmemBytes);
+      if (e != cudaSuccess) return e;
+      smem_set.fetch_or(bit);
+    }
     dim3 grid(static_cast<unsigned>(cdiv(T, rg::BM)), static_cast<unsigned>(cdiv(E, rg::BN)));
-    router_gemm_kernel<<<grid, 128, 0, st>>>(x, wr, br, T, H, E, logits);
+    router_gemm_kernel<<<grid, 128, rg::kSmemBytes, st>>>(x, wr, br, T, H, E, logits);
   }
   return cudaGetLastError();
 }
@@ -545,7 +599,7 @@ cudaError_t launch_topk(const float* logits, int T, int E, int k, int32_t* idx, 
   return cudaGetLastError();
 }
 
-int permute_chunks(int64_t P) { return static_cast<int>(cdiv(P, kPermChunk)); }
+int permute_chunks(int64_t P) { return static_cast<int>(cdiv(P, permute_chunk_size(P))); }
 
 // counts_ws: int32 scratch of permute_chunks(P) * E entries (unused for one chunk).
 cudaError_t launch_permute(const int32_t* idx, int T, int E, int k, int32_t* counts_ws,
@@ -559,7 +613,7 @@ cudaError_t launch_permute(const int32_t* idx, int T, int E, int k, int32_t* cou
                                                        perm_slot, inv, active, n_active, err);
     *launches += 1;
   } else {
-    permute_count_kernel<<<nc, kPermThreads, 0, st>>>(idx, P, E, counts_ws);
+    permute_count_kernel<<<nc, kPermThreads, 0, st>>>(idx, P, E, counts_ws, err);
     permute_scatter_kernel<<<nc, kPermThreads, 0, st>>>(idx, P, E, k, counts_ws, offsets,
                                                         perm_token, perm_slot, inv, active, n_active,
                                                         err);
@@ -584,11 +638,13 @@ cudaError_t launch_fp8_quant_as_bf16(const uint16_t* x, int64_t n, float s, uint
   return cudaGetLastError();
 }
 
-cudaError_t launch_gather_fp8_rows(const uint8_t* xq8, const int32_t* perm_token, int64_t P, int H,
-                                   uint8_t* a1, cudaStream_t st, int sms) {
-  const int64_t g = cdiv(P * 32, 256);
-  gather_fp8_rows_kernel<<<static_cast<unsigned>(g < sms * 16 ? (g < 1 ? 1 : g) : sms * 16), 256, 0, st>>>(
-      xq8, perm_token, P, H, a1);
+cudaError_t launch_quant_scatter_fp8(const uint16_t* x, const int32_t* topk_idx, const int32_t* inv, int T,
+                                    int k, int E, int64_t P, int H, float s, uint8_t* a1, cudaStream_t st,
+                                    int sms) {
+  if (k > 32) return cudaErrorInvalidValue;
+  const int64_t g = cdiv(static_cast<int64_t>(T) * 32, 256);
+  quant_scatter_fp8_kernel<<<static_cast<unsigned>(g < sms * 16 ? (g < 1 ? 1 : g) : sms * 16), 256, 0, st>>>(
+      x, topk_idx, inv, T, k, E, P, H, s, a1);
   return cudaGetLastError();
 }
 

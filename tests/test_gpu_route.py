@@ -70,7 +70,8 @@ def test_router_logits_and_indices(B, T, E, H, bias):
 @pytest.mark.parametrize("T,E,k,skew", [(1, 32, 4, 0.0), (8, 32, 4, 0.0), (64, 32, 4, 0.0),
                                         (1000, 128, 4, 0.0), (1025, 128, 4, 0.0),
                                         (4096, 128, 4, 0.0), (16384, 128, 4, 1.1),
-                                        (3, 256, 8, 0.0), (513, 23, 4, 2.0)])
+                                        (3, 256, 8, 0.0), (513, 23, 4, 2.0), (129, 32, 4, 0.0),
+                                        (40000, 128, 4, 0.0), (65536, 256, 4, 0.5)])
 def test_permute_bit_exact(B, T, E, k, skew):
     idx = inputs.random_topk_idx(T, E, k, seed=T + E, skew=skew) if T <= 4096 else None
     if idx is None:   # large case: draw on the host with numpy, vectorised
@@ -89,6 +90,17 @@ def test_permute_bit_exact(B, T, E, k, skew):
 def test_permute_flags_bad_expert_id(B):
     idx = torch.tensor([[0, 1], [2, 9]], dtype=torch.int32, device="cuda")
     B.moe_permute(idx, 4)
+    with pytest.raises(B.MxmoeError) as e:
+        B.mxmoe_check()
+    assert e.value.rc == B.EDEVICE
+    B.mxmoe_check()   # cleared
+
+
+def test_permute_flags_bad_expert_id_in_a_late_chunk(B):
+    # 3000 tokens x 4 = 12000 pairs span many chunks; only the last pair is bad
+    idx = torch.from_numpy(inputs.random_topk_idx(3000, 64, 4, seed=5)).cuda()
+    idx[-1, -1] = 64
+    B.moe_permute(idx, 64)
     with pytest.raises(B.MxmoeError) as e:
         B.mxmoe_check()
     assert e.value.rc == B.EDEVICE
