@@ -104,7 +104,7 @@ int64_t tc_min_pairs() {
   }();
   return v;
 }
-constexpr int kTcMaxNb = 144;   // K <= 4608 keeps the GEMM's shared memory within 227 KB
+constexpr int kTcMaxNb = 144;   // K <= 4608: the range the tcgen05 GEMM is tested on
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
@@ -290,8 +290,9 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
   const bool fp8 = act_scale != nullptr;
   const int64_t P = static_cast<int64_t>(a.T) * a.k;
   const bool tc = fp8 && !calib_out && P >= tc_min_pairs() && std::max(a.H, a.I) / 32 <= kTcMaxNb &&
-                  tc_gemm_supported(a.H, a.I, a.gu_blocks, a.d_blocks);
-  const bool dtc = !tc && !calib_out && decode_tc_supported(a.H, a.I, a.T, a.gu_blocks, a.d_blocks);
+                  tc_gemm_supported(a.H, a.I, a.gu_blocks, a.d_blocks, a.gu_scales, a.d_scales);
+  const bool dtc = !tc && !calib_out && decode_tc_supported(a.H, a.I, a.T, a.gu_blocks, a.d_blocks, a.gu_scales,
+                                                             a.d_scales);
   const size_t need = layout(a.T, a.E, a.k, a.H, a.I, fp8, tc, dtc, nullptr, nullptr);
   if (int rc = ensure_capacity(ws, need)) return rc;
   if (std::max(a.H, a.I) > ws->smem_K) {
@@ -300,7 +301,7 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
     ws->smem_K = std::max(a.H, a.I);
   }
   if (tc && !ws->tc_ready) {
-    cudaError_t e = tc_gemm_prepare(kTcMaxNb, 256);
+    cudaError_t e = tc_gemm_prepare(256);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (tcgen05 GEMM)");
     ws->tc_ready = true;
   }

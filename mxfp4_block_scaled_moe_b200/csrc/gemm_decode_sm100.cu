@@ -842,10 +842,13 @@ int nst_for(int K) { return (K + dec::BKS - 1) / dec::BKS; }
 
 }  // namespace
 
-bool decode_tc_supported(int H, int I, int T, const void* gu_blocks, const void* d_blocks) {
+bool decode_tc_supported(int H, int I, int T, const void* gu_blocks, const void* d_blocks, const void* gu_scales,
+                         const void* d_scales) {
   if (H % 64 || I % 64 || H < 64 || I < 64 || T < 1 || T > kDecodeMaxT) return false;
   if (H > dec::kSplitThreads * dec::kSplitVals) return false;   // the token split holds a row
   if ((reinterpret_cast<uintptr_t>(gu_blocks) | reinterpret_cast<uintptr_t>(d_blocks)) & 15u) return false;
+  // the weight-scale converters read the e8m0 bytes as 16-bit words
+  if ((reinterpret_cast<uintptr_t>(gu_scales) | reinterpret_cast<uintptr_t>(d_scales)) & 1u) return false;
   // the widest B tile must still leave two pipeline stages
   const int worst = dec::ring_offset() + 2 * (dec::stage_bytes_for(2, dec::kMaxN) + dec::kSfStage);
   if (worst + 1024 > dec::kSmemBytes) return false;

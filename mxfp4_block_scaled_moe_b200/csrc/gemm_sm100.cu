@@ -23,8 +23,11 @@
 //
 // Scale factors: a converter warp copies the tile's raw scale rows into shared memory
 // once per output tile and, per pipeline stage, rewrites the stage's 4 k-blocks into the
-// 512-byte atoms that tcgen05.cp (32x128b, 4 warp-quarters) moves into tensor memory:
-// row r of an atom at byte 16*(r%32) + 4*(r/32) + j for k-block j.
+// layout the MMA reads from tensor memory: weight row n at column n/32, lane n%32 of every
+// 32-lane quarter, byte j for k-block j. The stage's 8 columns go in with ONE tcgen05.cp
+// 128x256b from a 4 KB source that repeats the 32 lanes for each quarter: in the tensor
+// pipe a scale copy costs about as much as an MMA whatever its size (measured: 4 MMAs of
+// N = 240 take ~550 cycles; adding two 32x128b.warpx4 copies ~880, one 128x256b ~730).
 //
 // Roles (640 threads, one CTA per SM, persistent over the tile list):
 //   warp 0: TMA producer          warp 1: TMEM owner + MMA issuer (one thread)
@@ -51,7 +54,7 @@ constexpr int kEpiWarps = 16;                // 4 per SM sub-partition: hides th
 constexpr int kThreads = 128 + 32 * kEpiWarps;  // warps 0-3 producer/MMA/scales/schedule
 constexpr int kAStage = BM * BK;            // 16 KB (e4m3, one byte per value)
 constexpr int kBStage = BN * BK;            // 30 KB (e2m1 spread to one byte per value)
-constexpr int kSfStage = 1024;              // two 512-byte scale atoms (rows 0..255)
+constexpr int kSfStage = 4096;              // 128 lanes x 32 bytes: columns 0-3 at 0, 4-7 at 2048
 constexpr int kAccCols = 256;               // column stride between the two accumulators
 constexpr int kTmemCols = 512;
 constexpr int kSfaCol = 240;                // 4 columns of unit A scales (gap after accumulator 0)
@@ -115,15 +118,12 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constan
   uint8_t* sB = sA + kStages * kAStage;
   uint8_t* sSF = sB + kStages * kBStage;
   uint8_t* sSFA = sSF + kStages * kSfStage;       // 512 B of unit scales
-  uint8_t* sRaw = sSFA + 512;                     // BN * nb raw scale bytes
-  const int raw_bytes = ((BN * p.nb) + 15) & ~15;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sRaw + raw_bytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sSFA + 512);
   uint64_t* full = bars;
   uint64_t* empty = bars + kStages;
   uint64_t* acc_full = bars + 2 * kStages;
   uint64_t* acc_empty = acc_full + 2;
-  uint64_t* raw_full = acc_empty + 2;                            // [2]: raw scales landed, per converter
-  int* prefix = reinterpret_cast<int*>(raw_full + 2);            // E + 1
+  int* prefix = reinterpret_cast<int*>(acc_empty + 2);           // E + 1
   volatile int* abort_flag = prefix + (p.E + 1);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(prefix + p.E + 2);
 
@@ -139,8 +139,6 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constan
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], kEpiWarps);  // one arrive per epilogue warp
     }
-    mbar_init(&raw_full[0], 1);
-    mbar_init(&raw_full[1], 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
@@ -229,8 +227,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constan
         if (lane == 0) {
           const uint32_t sf = smem_u32(sSF + stage * kSfStage);
           const uint32_t sfb = tmem + kSfbCol + 8 * (stage & 1);
-          tc_cp_32x128b_x4(sfb, smem_desc(sf, 0, 128, 0));
-          tc_cp_32x128b_x4(sfb + 4, smem_desc(sf + 512, 0, 128, 0));
+          tc_cp_128x256b(sfb, smem_desc(sf, 2048, 128, 0));
           const uint32_t a0 = smem_u32(sA + stage * kAStage), b0 = smem_u32(sB + stage * kBStage);
           const int first = kt < p.nk_full ? 0 : 4 - p.tail_steps;
           for (int kk = first; kk < 4; ++kk) {
@@ -252,100 +249,77 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constan
     }
   } else if (warp == 2 || warp == 3) {
     // -------------------------------------------------------- scale converters -----
-    // warp 2 fills atom 0 (tile rows 0..127), warp 3 atom 1 (rows 128..255); lane l owns
-    // rows l, l+32, l+64, l+96 of its atom, whose four words sit side by side in the atom
-    // (byte 16*l + 4*i), so one 16-byte store per lane and stage writes them.
+    // warp 2 fills columns 0-3 (tile rows 0..127), warp 3 columns 4-7 (rows 128..255);
+    // lane l owns rows l, l+32, l+64, l+96 of its half, whose four words sit side by side
+    // (byte 16*L + 4*i for tensor-memory lane L = 32*q + l), stored once per quarter q.
+    // The scale bytes come straight from the checkpoint's (groups, rows, nb) array through
+    // the L1 cache, loaded kStages stages ahead (also across tile boundaries): a stage's 4 bytes
+    // of a row are two aligned 16-bit words (nb is even, k-blocks start at multiples of 4).
     const int w2 = warp - 2;
-    int stage = 0;
-    uint32_t phase = 0, raw_phase = 0;
-    const int nb = p.nb;
-    for (int t = blockIdx.x; t < total_tiles && !*abort_flag; t += gridDim.x) {
+    const int halves = kGateUp ? 2 : 1;
+    uint32_t phase = 0;
+    // rows of tile t this lane converts (nullptr: outside the tile -> unit scale)
+    auto rows_of = [&](int t, const uint16_t* (&rp)[4]) {
       const Tile tl = tile_of(t, prefix, p.offsets, p.E, p.n_tiles);
       const int n0 = tl.nt * bn_rows;
-      const int halves = kGateUp ? 2 : 1;
       const int valid = min(bn_rows, p.rows_per_group - n0);
-      // raw scale rows of this warp's tile rows [128*w2, 128*w2 + 128) into sRaw, tile row
-      // r at byte r * nb (r < bn_rows: first half or whole tile; r >= bn_rows: up half).
-      // Each half is one contiguous run in global memory: bulk copy when 16-byte aligned,
-      // else plain loads issued 8 at a time. Only this warp reads these rows.
-      fence_async_smem();   // this warp's earlier reads of its rows precede the refill
-      const uint8_t* src_h[2] = {nullptr, nullptr};
-      uint8_t* dst_h[2] = {nullptr, nullptr};
-      int bytes_h[2] = {0, 0};
-      bool bulk_h[2] = {false, false};
-      uint32_t bulk_bytes = 0;
-      for (int h = 0; h < halves; ++h) {
-        const int lo = max(0, 128 * w2 - h * bn_rows);
-        const int hi = min(valid, 128 * w2 + 128 - h * bn_rows);
-        if (hi <= lo) continue;
-        const int group = kGateUp ? 2 * tl.e + h : tl.e;
-        src_h[h] = p.b_scales + (static_cast<int64_t>(group) * p.rows_per_group + n0 + lo) * nb;
-        dst_h[h] = sRaw + (h * bn_rows + lo) * nb;
-        bytes_h[h] = (hi - lo) * nb;
-        bulk_h[h] = ((reinterpret_cast<uintptr_t>(src_h[h]) | reinterpret_cast<uintptr_t>(dst_h[h]) |
-                      static_cast<uintptr_t>(bytes_h[h])) & 15u) == 0;
-        if (bulk_h[h]) bulk_bytes += static_cast<uint32_t>(bytes_h[h]);
-      }
-      if (bulk_bytes > 0 && lane == 0) {
-        mbar_arrive_expect_tx(&raw_full[w2], bulk_bytes);
-        for (int h = 0; h < halves; ++h)
-          if (bulk_h[h]) bulk_g2s(dst_h[h], src_h[h], static_cast<uint32_t>(bytes_h[h]), &raw_full[w2]);
-      }
-      for (int h = 0; h < halves; ++h) {
-        if (bulk_h[h] || bytes_h[h] == 0) continue;
-        const uint8_t* src = src_h[h];
-        uint8_t* dst = dst_h[h];
-        const int bytes = bytes_h[h];
-        for (int c0 = 0; c0 < bytes; c0 += 32 * 8) {
-          uint8_t v[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const int c = c0 + u * 32 + lane;
-            v[u] = c < bytes ? src[c] : 0;
-          }
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const int c = c0 + u * 32 + lane;
-            if (c < bytes) dst[c] = v[u];
-          }
-        }
-      }
-      if (bulk_bytes > 0) {
-        if (!mbar_wait(&raw_full[w2], raw_phase, abort_flag, p.err)) break;
-        raw_phase ^= 1;
-      }
-      __syncwarp();
-      // where this lane's four rows start in sRaw (-1: outside the tile -> unit scale)
-      int src_off[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int r = 128 * w2 + lane + 32 * i;
         const int h = r >= bn_rows ? 1 : 0;
         const int rr = r - h * bn_rows;
-        src_off[i] = (r < BN && rr < valid && h < halves) ? (h * bn_rows + rr) * nb : -1;
+        const int group = kGateUp ? 2 * tl.e + h : tl.e;
+        rp[i] = (r < BN && rr < valid && h < halves)
+                    ? reinterpret_cast<const uint16_t*>(p.b_scales +
+                                                        (static_cast<int64_t>(group) * p.rows_per_group + n0 + rr) * p.nb)
+                    : nullptr;
       }
-      for (int kt = 0; kt < nkt; ++kt) {
-        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err)) break;
-        const int kb0 = kt < p.nk_full ? 4 * kt : nb - 4;
-        uint32_t wv[4];
+    };
+    // the stage's two 16-bit words of each row, kept apart until the store (combining
+    // them here would wait for the loads)
+    auto load = [&](const uint16_t* const (&rp)[4], int kt, uint32_t (&wv)[8]) {
+      const int kw = (kt < p.nk_full ? 4 * kt : p.nb - 4) >> 1;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          if (src_off[i] < 0) {
-            wv[i] = 0x7F7F7F7Fu;
-          } else {
-            // rows are nb bytes apart and kb0 is a multiple of 4: the 4 bytes are 2-aligned
-            const uint16_t* s16 = reinterpret_cast<const uint16_t*>(sRaw + src_off[i] + kb0);
-            wv[i] = static_cast<uint32_t>(s16[0]) | (static_cast<uint32_t>(s16[1]) << 16);
-          }
+      for (int i = 0; i < 4; ++i) {
+        wv[2 * i] = rp[i] ? static_cast<uint32_t>(__ldg(rp[i] + kw)) : 0x7F7Fu;
+        wv[2 * i + 1] = rp[i] ? static_cast<uint32_t>(__ldg(rp[i] + kw + 1)) : 0x7F7Fu;
+      }
+    };
+    // A ring of kStages register sets, unrolled so that no set is ever moved: the loads of
+    // a stage are issued kStages stages before its store (a register move would wait for
+    // them at once).
+    int lt = blockIdx.x, lkt = 0;   // next stage to load
+    int st = blockIdx.x, skt = 0;   // next stage to store
+    const uint16_t* rp[4] = {nullptr, nullptr, nullptr, nullptr};
+    uint32_t buf[kStages][8] = {};
+    auto load_next = [&](uint32_t (&wv)[8]) {
+      if (lt >= total_tiles) return;
+      if (lkt == 0) rows_of(lt, rp);
+      load(rp, lkt, wv);
+      if (++lkt == nkt) { lkt = 0; lt += gridDim.x; }
+    };
+#pragma unroll
+    for (int j = 0; j < kStages; ++j) load_next(buf[j]);
+    bool run = true;
+    while (run) {
+#pragma unroll
+      for (int j = 0; j < kStages; ++j) {
+        if (st >= total_tiles || *abort_flag || !mbar_wait(&empty[j], phase ^ 1, abort_flag, p.err)) {
+          run = false;
+          break;
         }
-        *reinterpret_cast<uint4*>(sSF + stage * kSfStage + 512 * w2 + 16 * lane) =
-            make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        const uint4 wq = make_uint4(buf[j][0] | (buf[j][1] << 16), buf[j][2] | (buf[j][3] << 16),
+                                    buf[j][4] | (buf[j][5] << 16), buf[j][6] | (buf[j][7] << 16));
+        uint8_t* dst = sSF + j * kSfStage + 2048 * w2 + 16 * lane;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(dst + 512 * q) = wq;
         fence_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&full[stage]);
-        if (++stage == kStages) { stage = 0; phase ^= 1; }
+        if (lane == 0) mbar_arrive(&full[j]);
+        if (++skt == nkt) { skt = 0; st += gridDim.x; }
+        load_next(buf[j]);
       }
-      __syncwarp();
+      phase ^= 1;
     }
   } else if (warp >= 4) {
     // --------------------------------------------------------------- epilogue -----
@@ -441,10 +415,9 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constan
   }
 }
 
-size_t smem_bytes(int nb, int E) {
-  size_t raw = (static_cast<size_t>(BN) * nb + 15) & ~static_cast<size_t>(15);
-  return 1024 + kStages * (kAStage + kBStage + kSfStage) + 512 + raw +
-         (2 * kStages + 6) * sizeof(uint64_t) + (E + 3) * sizeof(int) + 16;
+size_t smem_bytes(int E) {
+  return 1024 + kStages * (kAStage + kBStage + kSfStage) + 512 + (2 * kStages + 4) * sizeof(uint64_t) +
+         (E + 3) * sizeof(int) + 16;
 }
 
 }  // namespace g100
@@ -484,15 +457,18 @@ bool encode(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, 
 }  // namespace
 
 // Whether the tcgen05 path can run these shapes/pointers (else the register-dequant path).
-bool tc_gemm_supported(int H, int I, const void* gu_blocks, const void* d_blocks) {
+bool tc_gemm_supported(int H, int I, const void* gu_blocks, const void* d_blocks, const void* gu_scales,
+                       const void* d_scales) {
   if (H % 64 || I % 64) return false;          // 16 x U4 rows: K/2 bytes a multiple of 32
   if (H < g100::BK || I < g100::BK) return false;
   if ((reinterpret_cast<uintptr_t>(gu_blocks) | reinterpret_cast<uintptr_t>(d_blocks)) & 31u) return false;
+  // the scale converters read the e8m0 bytes as 16-bit words
+  if ((reinterpret_cast<uintptr_t>(gu_scales) | reinterpret_cast<uintptr_t>(d_scales)) & 1u) return false;
   return encoder() != nullptr;
 }
 
-cudaError_t tc_gemm_prepare(int max_nb, int E) {
-  const size_t smem = g100::smem_bytes(max_nb, E);
+cudaError_t tc_gemm_prepare(int E) {
+  const size_t smem = g100::smem_bytes(E);
   cudaError_t e = cudaFuncSetAttribute(g100::moe_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e) return e;
@@ -500,7 +476,6 @@ cudaError_t tc_gemm_prepare(int max_nb, int E) {
                               static_cast<int>(smem));
 }
 
-size_t tc_gemm_smem_bytes(int max_nb, int E) { return g100::smem_bytes(max_nb, E); }
 
 // a: grouped activation rows (P_rows, K) e4m3; blocks/scales: (E, rows_total, K/2) and
 // (E, rows_total, K/32); gate_up: rows_total = 2I, n_out = I; down: rows_total = n_out = H.
@@ -549,7 +524,7 @@ cudaError_t launch_tc_gemm(bool gate_up, const uint8_t* a, int64_t P_rows, int K
   prm.a_out = a_out;
   prm.y_out = y_out;
   prm.err = err;
-  const size_t smem = smem_bytes(prm.nb, E);
+  const size_t smem = smem_bytes(E);
   if (gate_up)
     moe_gemm_kernel<true><<<sms, kThreads, smem, st>>>(ma, mb, mbt, prm);
   else

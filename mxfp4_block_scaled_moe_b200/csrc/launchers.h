@@ -53,9 +53,9 @@ cudaError_t launch_expert_mma(const uint8_t* blocks, const uint8_t* scales, cons
                               cudaStream_t st);
 cudaError_t expert_mma_set_smem_limits(int max_K);
 
-bool tc_gemm_supported(int H, int I, const void* gu_blocks, const void* d_blocks);
-size_t tc_gemm_smem_bytes(int max_nb, int E);
-cudaError_t tc_gemm_prepare(int max_nb, int E);
+bool tc_gemm_supported(int H, int I, const void* gu_blocks, const void* d_blocks, const void* gu_scales,
+                       const void* d_scales);
+cudaError_t tc_gemm_prepare(int E);
 cudaError_t launch_tc_gemm(bool gate_up, const uint8_t* a, int64_t P_rows, int K, const uint8_t* blocks,
                            const uint8_t* scales, const float* bias, int E, int n_out, const int32_t* offsets,
                            float s_in, float s_out, uint8_t* a_out, float* y_out, int* err, int sms,
@@ -96,7 +96,8 @@ struct DecodeGemmArgs {   // tensor-core decode path (kind::mxf4: packed e2m1 we
 constexpr int kDecodeMaxT = 64;      // tokens the tensor-core decode path takes
 constexpr int kDecodeMaxGroups = 320;  // row groups (an expert's routed rows, 56 at a time)
 constexpr int kDecodeFoldMaxT = 8;   // the down kernel folds the combine up to this many tokens
-bool decode_tc_supported(int H, int I, int T, const void* gu_blocks, const void* d_blocks);
+bool decode_tc_supported(int H, int I, int T, const void* gu_blocks, const void* d_blocks, const void* gu_scales,
+                         const void* d_scales);
 cudaError_t decode_tc_prepare();
 size_t decode_tc_xs_bytes(int64_t P, int K);
 size_t decode_tc_sfb_bytes(int E, int K, int T);       // per 128-wide k-tile records (down's B)
