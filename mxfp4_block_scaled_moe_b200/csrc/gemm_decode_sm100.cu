@@ -67,7 +67,11 @@ constexpr int kBigCols = 112;      // gate_up units wider than this take both sl
 constexpr int kSfaCol = 480;       // A scales: tile h, atom a at 480 + 8h + 4a
 constexpr int kSfbCol = 496;       // B scales: k-tile t, atom b at 496 + 8t + 4b
 constexpr int kSfRecord = 1024;    // B scale record per (row group, 128-wide k-tile)
-constexpr int kSfStage = 4096;     // per stage: A atoms (2 tiles x 2) + B records (2)
+// Per stage: the A (weight) scales of each tile as one 128x256b tcgen05.cp source (4 KB:
+// the two 128-wide k-tiles' atoms, repeated for the four 32-lane quarters), then the B
+// scale record(s): gate_up one 1 KB record per unit (copied once), down two per stage.
+__host__ __device__ constexpr int sf_stage_bytes(int kA) { return kA * 4096 + (kA == 2 ? 1024 : 2048); }
+constexpr int kSfStageMax = sf_stage_bytes(2);
 constexpr int kMaxE = 256;
 constexpr int kMaxGrp = kDecodeMaxGroups;
 constexpr int kMaxSplit = 8;
@@ -410,7 +414,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
       const int b_rows = max(ncols_max, nbox_max * p.box_rows);
       sc.stage_bytes = stage_bytes_for(kA, b_rows);
       const int avail = static_cast<int>((smem_raw + p.smem_bytes) - ring);
-      sc.stages = min(kMaxStages, avail / (sc.stage_bytes + kSfStage));
+      sc.stages = min(kMaxStages, avail / (sc.stage_bytes + sf_stage_bytes(kA)));
       // K split: fewest stages on the busiest CTA, counting about four stages for each
       // split unit's partial write, ticket and the finisher's reduction
       const int tiles = ng * p.n_m, G = gridDim.x;
@@ -434,8 +438,9 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
   auto sA = [&](int s, int h) { return ring + s * sc.stage_bytes + h * BM * kRowBytes; };
   auto sB = [&](int s) { return ring + s * sc.stage_bytes + kA * BM * kRowBytes; };
   uint8_t* sf_base = ring + S * sc.stage_bytes;
-  auto sSFA = [&](int s, int h) { return sf_base + s * kSfStage + h * 1024; };
-  auto sSFB = [&](int s) { return sf_base + s * kSfStage + 2048; };
+  constexpr int kSfStage = sf_stage_bytes(kA);
+  auto sSFA = [&](int s, int h) { return sf_base + s * kSfStage + h * 4096; };
+  auto sSFB = [&](int s) { return sf_base + s * kSfStage + kA * 4096; };
   auto n_ksteps = [&](int kst) { return min(4, (p.K - BKS * kst + 63) / 64); };
 
   if (warp == 0) {
@@ -497,10 +502,12 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
         if (lane == 0) {
           const int nks = n_ksteps(kst);
           const int nkt = (nks + 1) >> 1;   // 128-wide k-tiles this stage uses
-          for (int t = 0; t < nkt; ++t) {
+          // each tile's weight scales for both k-tiles: 8 columns in one copy (a scale copy
+          // costs the tensor pipe about as much as an MMA whatever its size)
 #pragma unroll
-            for (int h = 0; h < kA; ++h)
-              tc_cp_32x128b_x4(tmem + kSfaCol + 8 * h + 4 * t, smem_desc(smem_u32(sSFA(stage, h) + 512 * t), 0, 128, 0));
+          for (int h = 0; h < kA; ++h)
+            tc_cp_128x256b(tmem + kSfaCol + 8 * h, smem_desc(smem_u32(sSFA(stage, h)), 2048, 128, 0));
+          for (int t = 0; t < nkt; ++t) {
             if (!kGateUp)
               for (int b = 0; b < nat; ++b)
                 tc_cp_32x128b_x4(tmem + kSfbCol + 8 * t + 4 * b,
@@ -548,48 +555,80 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
     // ------------------------------------------------ A (weight) scale converters -----
     const int h = warp - 2;   // 0: gate / down rows, 1: up rows
     if (h < kA) {
+      // lane l owns rows l, l+32, l+64, l+96 of the tile; a stage's 8 scale bytes of a row
+      // are four aligned 16-bit words (nb is even). They are loaded kRing stages ahead
+      // into an unrolled ring of register sets (never moved, and combined only at the
+      // store, so no instruction waits for them early) and stored as the 128x256b copy
+      // source: k-tile 0's word of row 32i + l at 16*L + 4*i, k-tile 1's at 2048 + 16*L + 4*i,
+      // for each tensor-memory lane L = 32*q + l.
+      constexpr int kRing = 3;
       int stage = 0;
       uint32_t phase = 0;
-      bool ok = true;
-      for (int u = blockIdx.x; u < sc.units && ok; u += gridDim.x) {
+      const uint16_t* rp[4] = {nullptr, nullptr, nullptr, nullptr};
+      int lu = blockIdx.x, lk = 0, lk1 = 0;   // load cursor: unit, stage, end stage
+      auto start_unit = [&](int u) {
         const Unit w = unit_at(sc, p, u);
         const int valid = min(BM, p.rows_per_group - w.m * BM);
         const int group = kGateUp ? 2 * w.e + h : w.e;
         const uint8_t* blk = p.w_scales + (static_cast<int64_t>(group) * p.rows_per_group + w.m * BM) * p.nb;
-        // lane l owns atom rows l, l+32, l+64, l+96 (bytes 16*l .. 16*l+15 of an atom); a
-        // stage's 8 scale bytes of a row are four aligned 16-bit words (nb is even)
-        const uint16_t* rp[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int r = lane + 32 * i;
           rp[i] = r < valid ? reinterpret_cast<const uint16_t*>(blk + static_cast<int64_t>(r) * p.nb) : nullptr;
         }
-        auto load = [&](int kst, uint32_t (&a0)[4], uint32_t (&a1)[4]) {
-          const int b0 = 8 * kst;
+        lk = w.k0;
+        lk1 = w.k1;
+      };
+      auto load_next = [&](uint32_t (&wd)[16]) {
+        if (lu >= sc.units) return;
+        const int b0 = 8 * lk;
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            uint32_t wd[4];
+        for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-              wd[q] = (rp[i] && b0 + 2 * q < p.nb) ? static_cast<uint32_t>(__ldg(rp[i] + b0 / 2 + q)) : 0x7F7Fu;
-            a0[i] = wd[0] | (wd[1] << 16);
-            a1[i] = wd[2] | (wd[3] << 16);
+          for (int q = 0; q < 4; ++q)
+            wd[4 * i + q] = (rp[i] && b0 + 2 * q < p.nb) ? static_cast<uint32_t>(__ldg(rp[i] + b0 / 2 + q)) : 0x7F7Fu;
+        if (++lk == lk1) {
+          lu += gridDim.x;
+          if (lu < sc.units) start_unit(lu);
+        }
+      };
+      if (lu < sc.units) start_unit(lu);
+      int su = blockIdx.x, sk = 0, sk1 = 0;    // store cursor
+      if (su < sc.units) {
+        const Unit w = unit_at(sc, p, su);
+        sk = w.k0;
+        sk1 = w.k1;
+      }
+      uint32_t ring[kRing][16] = {};
+#pragma unroll
+      for (int j = 0; j < kRing; ++j) load_next(ring[j]);
+      bool run = su < sc.units;
+      while (run) {
+#pragma unroll
+        for (int j = 0; j < kRing; ++j) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err)) { run = false; break; }
+          const uint4 c0 = make_uint4(ring[j][0] | (ring[j][1] << 16), ring[j][4] | (ring[j][5] << 16),
+                                      ring[j][8] | (ring[j][9] << 16), ring[j][12] | (ring[j][13] << 16));
+          const uint4 c1 = make_uint4(ring[j][2] | (ring[j][3] << 16), ring[j][6] | (ring[j][7] << 16),
+                                      ring[j][10] | (ring[j][11] << 16), ring[j][14] | (ring[j][15] << 16));
+          uint8_t* dst = sSFA(stage, h) + 16 * lane;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            *reinterpret_cast<uint4*>(dst + 512 * q) = c0;
+            *reinterpret_cast<uint4*>(dst + 2048 + 512 * q) = c1;
           }
-        };
-        uint32_t c0[4], c1[4];
-        load(w.k0, c0, c1);
-        for (int kst = w.k0; kst < w.k1; ++kst) {
-          uint32_t n0[4] = {0u, 0u, 0u, 0u}, n1[4] = {0u, 0u, 0u, 0u};
-          if (kst + 1 < w.k1) load(kst + 1, n0, n1);   // one stage ahead
-          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err)) { ok = false; break; }
-          *reinterpret_cast<uint4*>(sSFA(stage, h) + 16 * lane) = make_uint4(c0[0], c0[1], c0[2], c0[3]);
-          *reinterpret_cast<uint4*>(sSFA(stage, h) + 512 + 16 * lane) = make_uint4(c1[0], c1[1], c1[2], c1[3]);
           fence_async_smem();
           __syncwarp();
           if (lane == 0) mbar_arrive(&full[stage]);
           if (++stage == S) { stage = 0; phase ^= 1; }
-#pragma unroll
-          for (int i = 0; i < 4; ++i) { c0[i] = n0[i]; c1[i] = n1[i]; }
+          if (++sk == sk1) {
+            su += gridDim.x;
+            if (su >= sc.units) { run = false; break; }
+            const Unit w = unit_at(sc, p, su);
+            sk = w.k0;
+            sk1 = w.k1;
+          }
+          load_next(ring[j]);
         }
       }
     }
@@ -850,7 +889,7 @@ bool decode_tc_supported(int H, int I, int T, const void* gu_blocks, const void*
   // the weight-scale converters read the e8m0 bytes as 16-bit words
   if ((reinterpret_cast<uintptr_t>(gu_scales) | reinterpret_cast<uintptr_t>(d_scales)) & 1u) return false;
   // the widest B tile must still leave two pipeline stages
-  const int worst = dec::ring_offset() + 2 * (dec::stage_bytes_for(2, dec::kMaxN) + dec::kSfStage);
+  const int worst = dec::ring_offset() + 2 * (dec::stage_bytes_for(2, dec::kMaxN) + dec::kSfStageMax);
   if (worst + 1024 > dec::kSmemBytes) return false;
   return encoder() != nullptr;
 }
