@@ -94,19 +94,17 @@ __device__ __forceinline__ float pow2f(int s) {   // exact 2^s for s in [-126, 1
 }
 
 // Scale exponent of an e2m1 part: the smallest s with amax / 2^s <= 6 (the e2m1 maximum),
-// clamped to [-126, 125]. amax == 0 gives 0.
+// clamped to [-126, 125]; amax == 0 gives 0. Branch-free: a subnormal amax reads as
+// floor(log2) = -127, which the clamp maps to -126 exactly as its true exponent would.
 __device__ __forceinline__ int e2m1_part_exponent(float amax) {
-  if (!(amax > 0.0f)) return 0;
-  const uint32_t u = __float_as_uint(amax);
-  const int ex = static_cast<int>(u >> 23);
-  const int fl = ex > 0 ? ex - 127 : (31 - __clz(u)) - 149;   // floor(log2(amax))
-  int s = max(-126, min(125, fl - 2));                       // amax / 2^s in [4, 8)
-  if (amax > 6.0f * pow2f(s)) s = min(125, s + 1);
-  return s;
+  const int fl = static_cast<int>(__float_as_uint(amax) >> 23) - 127;   // amax >= 0
+  int s = max(-126, min(125, fl - 2));                                   // amax / 2^s in [4, 8)
+  s = (amax > 6.0f * pow2f(s)) ? min(125, s + 1) : s;
+  return amax > 0.0f ? s : 0;
 }
 
-// One e2m1 part of 8 rows' values r[j] (this lane's element of a 32-value block held by
-// the warp). The block's largest magnitude is one warp max-reduction of the bit patterns
+// One e2m1 part of the first nv (warp-uniform) of 8 rows' values r[j] (this lane's
+// element of a 32-value block held by the warp). The block's largest magnitude is one warp max-reduction of the bit patterns
 // (non-negative floats order like their bits); the value is scaled by 2^-s and rounded
 // to e2m1 (nearest, ties to even) by the hardware conversion, which also packs this
 // lane's value with the next lane's into bytes[j] (even element in the low nibble;
@@ -114,9 +112,12 @@ __device__ __forceinline__ int e2m1_part_exponent(float amax) {
 // r[j] becomes the residual; the update is exact (a part value has two significant bits
 // and a power-of-two scale). The eight chains are independent, so their latencies
 // overlap. Lanes outside the data pass 0.
-__device__ __forceinline__ void e2m1_part8(float (&r)[8], uint32_t (&bytes)[8], int (&sc)[8]) {
+__device__ __forceinline__ void e2m1_part8(float (&r)[8], uint32_t (&bytes)[8], int (&sc)[8], int nv) {
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
+    bytes[j] = 0u;
+    sc[j] = 0;
+    if (j >= nv) continue;
     const float amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(r[j]))));
     sc[j] = e2m1_part_exponent(amax);
     const float v = r[j] * pow2f(-sc[j]);
@@ -201,7 +202,11 @@ __device__ __forceinline__ Unit unit_at(const Sched& sc, const Params& p, int u)
 // Byte offsets of the fixed part of the shared-memory layout (host and device agree).
 __host__ __device__ constexpr int sched_bytes() { return (static_cast<int>(sizeof(Sched)) + 127) & ~127; }
 __host__ __device__ constexpr int bar_bytes() { return 256; }
-__host__ __device__ constexpr int ring_offset() { return (sched_bytes() + bar_bytes() + 1023) & ~1023; }
+constexpr int kEpiStageBytes = 512;   // per epilogue warp: 8 rows x 4 parts x 16 bytes
+__host__ __device__ constexpr int epi_stage_offset() { return sched_bytes() + bar_bytes(); }
+__host__ __device__ constexpr int ring_offset() {
+  return (epi_stage_offset() + kEpiWarps * kEpiStageBytes + 1023) & ~1023;
+}
 __host__ __device__ inline int stage_bytes_for(int kA, int b_rows) {
   return ((kA * BM * kRowBytes + b_rows * kRowBytes) + 1023) & ~1023;
 }
@@ -248,43 +253,53 @@ __device__ __forceinline__ void sum_parts(const float (&v)[8 * kParts], float (&
 }
 
 // gate_up: bias, SwiGLU and the down GEMM's B operand for rows j0 .. j0+7 of the unit's
-// group. gs / us: the accumulators summed over a row's parts (before the per-tensor scale).
-// dry: the same instructions with every store masked off (warms the instruction cache).
-// Not inlined, so that the warm-up call and the real ones run the same code.
-__device__ __noinline__ void finish_gate_up(uint8_t* xs_out, uint8_t* sfb_out, int n_out, int nst_out,
+// group (only the first nv = min(8, n - j0) are computed). gs / us: the accumulators
+// summed over a row's parts (before the per-tensor scale). The warp's 16 bytes of each
+// (row, part) are gathered in its 512-byte shared staging area and leave as one 16-byte
+// store per (row, part) lane, the part scales as one byte store per lane.
+// dry: the same instructions with every global store masked off (warms the instruction
+// cache). Not inlined, so that the warm-up call and the real ones run the same code.
+__device__ __noinline__ void finish_gate_up(uint8_t* xs_out, uint8_t* sfb_out, uint8_t* stage, int n_out, int nst_out,
                                             int max_chunks, float s_in, float s_out, int e, int c, int off, int n,
                                             int j0, const float (&gs)[8], const float (&us)[8], float bg, float bu,
                                             int row, int lane, bool dry) {
   const int kb = row >> 5;   // the warp's 32 rows: one 32-value block of the down contraction
+  const int nv = min(8, n - j0);
   uint8_t* rec = sfb_out + ((static_cast<int64_t>(e) * max_chunks + c) * 2 * nst_out + (kb >> 2)) * kSfRecord;
   float a[8];
 #pragma unroll
   for (int jj = 0; jj < 8; ++jj) {
+    a[jj] = 0.0f;
+    if (jj >= nv) continue;
     const float gv = __fadd_rn(__fmul_rn(s_in, gs[jj]), bg);
     const float uv = __fadd_rn(__fmul_rn(s_in, us[jj]), bu);
-    float v = j0 + jj < n ? silu_mul(gv, uv) : 0.0f;
+    const float v = silu_mul(gv, uv);
     // the layer's intermediate: e4m3(a / s1) with FP8 activations, else bf16(a)
-    v = s_out > 0.0f ? e4m3_to_f32(act_quant_e4m3(v, s_out)) : bf16_bits_to_f32(f32_to_bf16_bits_rn(v));
-    a[jj] = v;
+    a[jj] = s_out > 0.0f ? e4m3_to_f32(act_quant_e4m3(v, s_out)) : bf16_bits_to_f32(f32_to_bf16_bits_rn(v));
   }
-  const int64_t row_bytes = n_out / 2;
-  // one part at a time, stored as it is made: a rolled loop keeps this code small, which
-  // matters because it runs once per unit and its instructions are fetched cold
+  int my_sc = 0;   // lane 4*jj + pp keeps the scale of (row jj, part pp)
+  // one part at a time: a rolled loop keeps this code small, which matters because it
+  // runs once per unit and its instructions are fetched cold
 #pragma unroll 1
   for (int pp = 0; pp < kParts; ++pp) {
     uint32_t bytes[8];
     int sv[8];
-    e2m1_part8(a, bytes, sv);
+    e2m1_part8(a, bytes, sv, nv);
 #pragma unroll
     for (int jj = 0; jj < 8; ++jj) {
-      const uint32_t byte = bytes[jj];
-      if (j0 + jj < n && !dry) {
-        if ((lane & 1) == 0)
-          xs_out[(static_cast<int64_t>(off + j0 + jj) * kParts + pp) * row_bytes + (row >> 1)] = static_cast<uint8_t>(byte);
-        if (lane == 0) rec[sf_atom_byte(kParts * (j0 + jj) + pp, kb & 3)] = static_cast<uint8_t>(sv[jj] + 127);
-      }
+      if (jj < nv && (lane & 1) == 0) stage[(kParts * jj + pp) * 16 + (lane >> 1)] = static_cast<uint8_t>(bytes[jj]);
+      if (lane == kParts * jj + pp) my_sc = sv[jj];
     }
   }
+  __syncwarp();
+  if (!dry && lane < kParts * nv) {
+    const int jj = lane / kParts, pp = lane % kParts;
+    const uint4 v = *reinterpret_cast<const uint4*>(stage + 16 * lane);
+    const int64_t row_bytes = n_out / 2;
+    *reinterpret_cast<uint4*>(xs_out + (static_cast<int64_t>(off + j0 + jj) * kParts + pp) * row_bytes + 16 * kb) = v;
+    rec[sf_atom_byte(kParts * (j0 + jj) + pp, kb & 3)] = static_cast<uint8_t>(my_sc + 127);
+  }
+  __syncwarp();   // the staging area is reused by the next call
 }
 
 // down: y = s_in * acc + bias for rows j0 .. j0+7 of the unit's group.
@@ -635,12 +650,13 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
   } else {
     // ----------------------------------------------------------------- epilogue -----
     const int q = warp & 3;
+    uint8_t* epi_stage = smem + epi_stage_offset() + (warp - 4) * kEpiStageBytes;
     if (kGateUp && blockIdx.x < sc.units) {
       // The part-splitting epilogue runs once per unit, long after the kernel starts, and
       // its instructions would come cold from memory that the weight stream saturates:
       // run it once now, stores masked off, while the first stages load.
       float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      finish_gate_up(p.xs_out, p.sfb_out, p.n_out, p.nst_out, p.max_chunks, p.s_in, p.s_out, 0, 0, 0, 8, 0, z, z,
+      finish_gate_up(p.xs_out, p.sfb_out, epi_stage, p.n_out, p.nst_out, p.max_chunks, p.s_in, p.s_out, 0, 0, 0, 8, 0, z, z,
                      0.0f, 0.0f, lane, lane, true);
     }
     uint32_t use0 = 0u, use1 = 0u;
@@ -714,7 +730,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
           sum_parts(vg, gs);
           if (kGateUp) {
             sum_parts(vu, us);
-            finish_gate_up(p.xs_out, p.sfb_out, p.n_out, p.nst_out, p.max_chunks, p.s_in, p.s_out, w.e, w.c, w.off,
+            finish_gate_up(p.xs_out, p.sfb_out, epi_stage, p.n_out, p.nst_out, p.max_chunks, p.s_in, p.s_out, w.e, w.c, w.off,
                            w.n, j0, gs, us, bias0, bias1, row, lane, false);
           } else {
             finish_down(p, w, j0, gs, bias0, row);
