@@ -103,32 +103,6 @@ __device__ __forceinline__ int e2m1_part_exponent(float amax) {
   return amax > 0.0f ? s : 0;
 }
 
-// One e2m1 part of the first nv (warp-uniform) of 8 rows' values r[j] (this lane's
-// element of a 32-value block held by the warp). The block's largest magnitude is one warp max-reduction of the bit patterns
-// (non-negative floats order like their bits); the value is scaled by 2^-s and rounded
-// to e2m1 (nearest, ties to even) by the hardware conversion, which also packs this
-// lane's value with the next lane's into bytes[j] (even element in the low nibble;
-// meaningful in even lanes). sc[j] is the scale exponent (the same in every lane) and
-// r[j] becomes the residual; the update is exact (a part value has two significant bits
-// and a power-of-two scale). The eight chains are independent, so their latencies
-// overlap. Lanes outside the data pass 0.
-__device__ __forceinline__ void e2m1_part8(float (&r)[8], uint32_t (&bytes)[8], int (&sc)[8], int nv) {
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    bytes[j] = 0u;
-    sc[j] = 0;
-    if (j >= nv) continue;
-    const float amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(r[j]))));
-    sc[j] = e2m1_part_exponent(amax);
-    const float v = r[j] * pow2f(-sc[j]);
-    const float vn = __shfl_down_sync(0xffffffffu, v, 1);
-    bytes[j] = __nv_cvt_float2_to_fp4x2(make_float2(v, vn), __NV_E2M1, cudaRoundNearest);
-    const __nv_fp4x2_storage_t own = __nv_cvt_float2_to_fp4x2(make_float2(v, v), __NV_E2M1, cudaRoundNearest);
-    const __half2_raw h = __nv_cvt_fp4x2_to_halfraw2(own, __NV_E2M1);
-    r[j] = r[j] - __half2float(__half(__half_raw{h.x})) * pow2f(sc[j]);
-  }
-}
-
 struct Params {
   // A: weights
   const uint8_t* w_scales;   // (groups, rows_per_group, nb) e8m0
@@ -202,7 +176,7 @@ __device__ __forceinline__ Unit unit_at(const Sched& sc, const Params& p, int u)
 // Byte offsets of the fixed part of the shared-memory layout (host and device agree).
 __host__ __device__ constexpr int sched_bytes() { return (static_cast<int>(sizeof(Sched)) + 127) & ~127; }
 __host__ __device__ constexpr int bar_bytes() { return 256; }
-constexpr int kEpiStageBytes = 512;   // per epilogue warp: 8 rows x 4 parts x 16 bytes
+constexpr int kEpiStageBytes = 512;   // per epilogue warp: 4 rows x 32 fp32 values
 __host__ __device__ constexpr int epi_stage_offset() { return sched_bytes() + bar_bytes(); }
 __host__ __device__ constexpr int ring_offset() {
   return (epi_stage_offset() + kEpiWarps * kEpiStageBytes + 1023) & ~1023;
@@ -253,51 +227,69 @@ __device__ __forceinline__ void sum_parts(const float (&v)[8 * kParts], float (&
 }
 
 // gate_up: bias, SwiGLU and the down GEMM's B operand for rows j0 .. j0+7 of the unit's
-// group (only the first nv = min(8, n - j0) are computed). gs / us: the accumulators
-// summed over a row's parts (before the per-tensor scale). The warp's 16 bytes of each
-// (row, part) are gathered in its 512-byte shared staging area and leave as one 16-byte
-// store per (row, part) lane, the part scales as one byte store per lane.
+// group (gs / us: the accumulators summed over a row's parts, before the per-tensor
+// scale; lane = intermediate index within the warp's 32-value block of the down
+// contraction). The intermediate a = silu(g) * u is rounded as the layer defines it
+// (e4m3(a / s1) with FP8 activations, else bf16); silu uses the fast exponential and
+// division (a few ulp, far inside the layer tolerance; branch-free, so the eight rows'
+// chains overlap). It is then written as kParts e2m1 parts, part p the residual of the
+// parts before it rounded to nearest-even at the scale 2^s (s: the smallest with
+// max|residual| / 2^s <= 6 over the 32-value block). The warp first transposes four
+// rows at a time through its 512-byte shared staging area so that each lane holds four
+// consecutive values of one row: a block maximum is then three shuffles, and a lane's
+// four codes leave as one 16-bit store (even value in the low nibble).
 // dry: the same instructions with every global store masked off (warms the instruction
 // cache). Not inlined, so that the warm-up call and the real ones run the same code.
-__device__ __noinline__ void finish_gate_up(uint8_t* xs_out, uint8_t* sfb_out, uint8_t* stage, int n_out, int nst_out,
+__device__ __noinline__ void finish_gate_up(uint8_t* xs_out, uint8_t* sfb_out, float* stage, int n_out, int nst_out,
                                             int max_chunks, float s_in, float s_out, int e, int c, int off, int n,
                                             int j0, const float (&gs)[8], const float (&us)[8], float bg, float bu,
                                             int row, int lane, bool dry) {
   const int kb = row >> 5;   // the warp's 32 rows: one 32-value block of the down contraction
   const int nv = min(8, n - j0);
   uint8_t* rec = sfb_out + ((static_cast<int64_t>(e) * max_chunks + c) * 2 * nst_out + (kb >> 2)) * kSfRecord;
+  const int64_t row_bytes = n_out / 2;
   float a[8];
 #pragma unroll
   for (int jj = 0; jj < 8; ++jj) {
-    a[jj] = 0.0f;
-    if (jj >= nv) continue;
     const float gv = __fadd_rn(__fmul_rn(s_in, gs[jj]), bg);
     const float uv = __fadd_rn(__fmul_rn(s_in, us[jj]), bu);
-    const float v = silu_mul(gv, uv);
-    // the layer's intermediate: e4m3(a / s1) with FP8 activations, else bf16(a)
+    const float v = __fmul_rn(__fdividef(gv, 1.0f + __expf(-gv)), uv);
     a[jj] = s_out > 0.0f ? e4m3_to_f32(act_quant_e4m3(v, s_out)) : bf16_bits_to_f32(f32_to_bf16_bits_rn(v));
   }
-  int my_sc = 0;   // lane 4*jj + pp keeps the scale of (row jj, part pp)
-  // one part at a time: a rolled loop keeps this code small, which matters because it
-  // runs once per unit and its instructions are fetched cold
-#pragma unroll 1
-  for (int pp = 0; pp < kParts; ++pp) {
-    uint32_t bytes[8];
-    int sv[8];
-    e2m1_part8(a, bytes, sv, nv);
+  const int j = lane >> 3, sub = lane & 7;   // after the transpose: row p0 + j, values 4 sub .. 4 sub + 3
 #pragma unroll
-    for (int jj = 0; jj < 8; ++jj) {
-      if (jj < nv && (lane & 1) == 0) stage[(kParts * jj + pp) * 16 + (lane >> 1)] = static_cast<uint8_t>(bytes[jj]);
-      if (lane == kParts * jj + pp) my_sc = sv[jj];
+  for (int p0 = 0; p0 < 8; p0 += 4) {
+    if (p0 >= nv) break;
+    __syncwarp();   // the previous pass has read the staging area
+#pragma unroll
+    for (int t = 0; t < 4; ++t) stage[32 * t + lane] = a[p0 + t];
+    __syncwarp();
+    const float4 v4 = *reinterpret_cast<const float4*>(stage + 32 * j + 4 * sub);
+    float v[4] = {v4.x, v4.y, v4.z, v4.w};
+    const bool mine = p0 + j < nv && !dry;
+    uint8_t* dst = xs_out + (static_cast<int64_t>(off + j0 + p0 + j) * kParts) * row_bytes + 16 * kb + 2 * sub;
+#pragma unroll 1
+    for (int pp = 0; pp < kParts; ++pp) {
+      float m = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+      const int sc = e2m1_part_exponent(m);
+      const float down = pow2f(-sc), up = pow2f(sc);
+      const uint32_t b0 = __nv_cvt_float2_to_fp4x2(make_float2(v[0] * down, v[1] * down), __NV_E2M1, cudaRoundNearest);
+      const uint32_t b1 = __nv_cvt_float2_to_fp4x2(make_float2(v[2] * down, v[3] * down), __NV_E2M1, cudaRoundNearest);
+      const __half2_raw h0 = __nv_cvt_fp4x2_to_halfraw2(static_cast<__nv_fp4x2_storage_t>(b0), __NV_E2M1);
+      const __half2_raw h1 = __nv_cvt_fp4x2_to_halfraw2(static_cast<__nv_fp4x2_storage_t>(b1), __NV_E2M1);
+      // the residual update is exact: a part value has two significant bits, its scale is a power of two
+      v[0] -= __half2float(__half(__half_raw{h0.x})) * up;
+      v[1] -= __half2float(__half(__half_raw{h0.y})) * up;
+      v[2] -= __half2float(__half(__half_raw{h1.x})) * up;
+      v[3] -= __half2float(__half(__half_raw{h1.y})) * up;
+      if (mine) {
+        *reinterpret_cast<uint16_t*>(dst + pp * row_bytes) = static_cast<uint16_t>(b0 | (b1 << 8));
+        if (sub == 0) rec[sf_atom_byte(kParts * (j0 + p0 + j) + pp, kb & 3)] = static_cast<uint8_t>(sc + 127);
+      }
     }
-  }
-  __syncwarp();
-  if (!dry && lane < kParts * nv) {
-    const int jj = lane / kParts, pp = lane % kParts;
-    const uint4 v = *reinterpret_cast<const uint4*>(stage + 16 * lane);
-    const int64_t row_bytes = n_out / 2;
-    *reinterpret_cast<uint4*>(xs_out + (static_cast<int64_t>(off + j0 + jj) * kParts + pp) * row_bytes + 16 * kb) = v;
-    rec[sf_atom_byte(kParts * (j0 + jj) + pp, kb & 3)] = static_cast<uint8_t>(my_sc + 127);
   }
   __syncwarp();   // the staging area is reused by the next call
 }
@@ -650,7 +642,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
   } else {
     // ----------------------------------------------------------------- epilogue -----
     const int q = warp & 3;
-    uint8_t* epi_stage = smem + epi_stage_offset() + (warp - 4) * kEpiStageBytes;
+    float* epi_stage = reinterpret_cast<float*>(smem + epi_stage_offset() + (warp - 4) * kEpiStageBytes);
     if (kGateUp && blockIdx.x < sc.units) {
       // The part-splitting epilogue runs once per unit, long after the kernel starts, and
       // its instructions would come cold from memory that the weight stream saturates:
