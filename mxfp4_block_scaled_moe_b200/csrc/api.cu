@@ -81,6 +81,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 constexpr size_t kTicketBytes = 4096;       // 1024 row groups of 16 rows: H <= 16384
 constexpr int kFoldCombineMaxT = 64;        // fold the combine into the down kernel up to here
 constexpr int kRouteTicket = 1023;          // ticket slot of the fused routing kernel
+constexpr int kRouteTokTickets = 959;       // its per-token counters: slots 959 .. 1022 (T <= 64)
 
 // ------------------------------------------------------------------ workspace ------
 struct Workspace {
@@ -328,8 +329,8 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
   if (route_small_supported(a.T, a.E, a.k)) {
     // small batch: router, top-k and permutation in one CTA, one launch
     if ((e = launch_route_small(a.x, a.router_w, a.router_b, a.T, a.H, a.E, a.k, b.logits,
-                                b.tickets + kRouteTicket, b.topk_idx, b.topk_w, b.offsets, b.perm_token,
-                                b.perm_slot, b.inv, b.active, b.n_active, ws->err, st)))
+                                b.tickets + kRouteTicket, b.tickets + kRouteTokTickets, b.topk_idx, b.topk_w,
+                                b.offsets, b.perm_token, b.perm_slot, b.inv, b.active, b.n_active, ws->err, st)))
       return cuda_fail(e, "route");
     ++launches;
     tm.mark("route");
@@ -438,7 +439,7 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
     t_last_launches = launches;
     return MXMOE_OK;
   }
-  const bool fold = a.T <= kFoldCombineMaxT && a.H / 16 <= kRouteTicket;
+  const bool fold = a.T <= kFoldCombineMaxT && a.H / 16 <= kRouteTokTickets;
   const CombineArgs cmb{out, b.topk_idx, b.topk_w, b.inv, b.tickets, a.T, a.k};
   if ((e = launch_expert_mma(a.d_blocks, a.d_scales, a.d_bias, a.H, a.I, b.act_mid, nullptr,
                              b.offsets, b.active, b.n_active, max_active, s1, 1, a.I, 0.0f, nullptr,

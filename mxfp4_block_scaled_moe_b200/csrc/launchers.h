@@ -22,8 +22,8 @@ cudaError_t launch_permute(const int32_t* idx, int T, int E, int k, int32_t* cou
                            cudaStream_t st, int* launches);
 bool route_small_supported(int T, int E, int k);
 cudaError_t launch_route_small(const uint16_t* x, const uint16_t* wr, const uint16_t* br, int T, int H, int E,
-                               int k, float* logits, unsigned* ticket, int32_t* topk_idx, float* topk_w,
-                               int32_t* offsets, int32_t* perm_token, int32_t* perm_slot, int32_t* inv,
+                               int k, float* logits, unsigned* ticket, unsigned* tok_tickets, int32_t* topk_idx,
+                               float* topk_w, int32_t* offsets, int32_t* perm_token, int32_t* perm_slot, int32_t* inv,
                                int32_t* active, int32_t* n_active, int* err, cudaStream_t st);
 cudaError_t launch_fp8_quant(const uint16_t* x, int64_t n, float s, uint8_t* q, cudaStream_t st,
                              int sms);

@@ -211,13 +211,19 @@ __device__ __forceinline__ void topk_warp(const float* __restrict__ l, int E, in
     sidx[j] = bi;
     if ((bi & 31) == lane) taken |= 1 << (bi >> 5);
   }
-  if (lane == 0) {
-    float p[8], z = 0.0f;
-    for (int j = 0; j < k; ++j) { p[j] = expf(sel[j] - sel[0]); z += p[j]; }
-    for (int j = 0; j < k; ++j) {
-      idx_out[j] = sidx[j];
-      w_out[j] = __fdiv_rn(p[j], z);
-    }
+  // softmax over the k selected logits: lane j < k takes term j; every lane adds the terms
+  // in order j = 0 .. k-1 (the same sum as a sequential loop)
+  float my_sel = sel[0];
+  int my_idx = sidx[0];
+#pragma unroll
+  for (int j = 1; j < 8; ++j)
+    if (j < k && lane == j) { my_sel = sel[j]; my_idx = sidx[j]; }
+  const float pj = lane < k ? expf(my_sel - sel[0]) : 0.0f;
+  float z = 0.0f;
+  for (int j = 0; j < k; ++j) z += __shfl_sync(0xffffffffu, pj, j);
+  if (lane < k) {
+    idx_out[lane] = my_idx;
+    w_out[lane] = __fdiv_rn(pj, z);
   }
 }
 
@@ -291,7 +297,7 @@ __device__ void permute_scatter_body(
     for (int e = tid; e < E; e += blockDim.x) total[e] = 0;
     __syncthreads();
     for (int64_t p = tid; p < P; p += blockDim.x) {
-      const int e = idx[p];
+      const int e = __ldcg(idx + p);   // may have been written by other CTAs of this launch
       if (e >= 0 && e < E) atomicAdd(&total[e], 1);
       else set_device_error(err, MXMOE_EDEVICE);
     }
@@ -345,7 +351,7 @@ __device__ void permute_scatter_body(
   const unsigned lt_mask = (1u << lane) - 1u;
   for (int64_t sub = my_lo; sub < my_hi; sub += blockDim.x) {
     const int64_t p = sub + tid;
-    int e = p < my_hi ? idx[p] : -1;
+    int e = p < my_hi ? __ldcg(idx + p) : -1;
     if (e >= E) e = -1;
     for (int i = tid; i < (kPermThreads / 32) * 256; i += blockDim.x) (&wc[0][0])[i] = 0;  // all slots
     const unsigned peers = __match_any_sync(0xffffffffu, e);
@@ -388,20 +394,23 @@ __global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(
 
 // ----------------------------------------------------------- fused small-batch routing -
 // One launch for the routing of a small batch: every warp computes one (token, expert)
-// logit (the router GEMV's arithmetic), and the CTA that finishes last (an atomic ticket,
-// reset for the next call) runs the top-k softmax (one warp per token) and the single-CTA
-// permutation. Saves two launches on the latency-bound decode path.
+// logit (the router GEMV's arithmetic). The CTA that completes a token's logits last (a
+// per-token arrival counter) runs that token's top-k softmax, so the tokens' top-k run in
+// parallel across CTAs; the CTA that finishes last overall (a second counter) runs the
+// single-CTA permutation. Every counter is reset by the CTA that consumed it. Saves two
+// launches on the latency-bound decode path.
 constexpr int kSmallT = 64, kSmallE = 256;
 
 __global__ void __launch_bounds__(kPermThreads) route_small_kernel(
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ wr, const uint16_t* __restrict__ br,
     int T, int H, int E, int k, float* __restrict__ logits, unsigned* __restrict__ ticket,
-    int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+    unsigned* __restrict__ tok_tickets, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
     int32_t* __restrict__ offsets, int32_t* __restrict__ perm_token, int32_t* __restrict__ perm_slot,
     int32_t* __restrict__ inv, int32_t* __restrict__ active, int32_t* __restrict__ n_active,
     int* __restrict__ err) {
   __shared__ PermuteSmem sm;
   __shared__ unsigned s_last;
+  __shared__ int s_tok[kPermThreads / 32], s_ntok;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   const int64_t wid = static_cast<int64_t>(blockIdx.x) * nwarps + warp;
   if (wid < static_cast<int64_t>(T) * E) {
@@ -433,30 +442,52 @@ __global__ void __launch_bounds__(kPermThreads) route_small_kernel(
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     if (lane == 0) logits[wid] = br ? acc + bf16_bits_to_f32(br[e]) : acc;
   }
+  // tokens whose logits this CTA helped compute: the last of a token's CTAs runs its top-k
+  __threadfence();
+  if (threadIdx.x == 0) s_ntok = 0;
+  __syncthreads();
+  {
+    const int64_t w_lo = static_cast<int64_t>(blockIdx.x) * nwarps;
+    const int64_t w_hi = min(static_cast<int64_t>(T) * E, w_lo + nwarps);   // > w_lo: the grid covers T*E warps
+    const int t_lo = static_cast<int>(w_lo / E), t_hi = static_cast<int>((w_hi - 1) / E);
+    if (static_cast<int>(threadIdx.x) <= t_hi - t_lo) {
+      const int t = t_lo + static_cast<int>(threadIdx.x);
+      const int64_t c_first = static_cast<int64_t>(t) * E / nwarps;
+      const int64_t c_last = (static_cast<int64_t>(t) * E + E - 1) / nwarps;
+      const unsigned need = static_cast<unsigned>(c_last - c_first + 1);
+      if (atomicAdd(&tok_tickets[t], 1u) == need - 1u) {
+        tok_tickets[t] = 0u;   // every CTA of the token has arrived
+        s_tok[atomicAdd(&s_ntok, 1)] = t;
+      }
+    }
+  }
+  __syncthreads();
+  __threadfence();
+  for (int i = warp; i < s_ntok; i += nwarps) {
+    const int t = s_tok[i];
+    // the other CTAs' logits: read through L2
+    float lv[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = lane + 32 * j;
+      lv[j] = e < E ? __ldcg(logits + static_cast<int64_t>(t) * E + e) : 0.0f;
+    }
+    __shared__ float s_row[kPermThreads / 32][256];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = lane + 32 * j;
+      if (e < E) s_row[warp][e] = lv[j];
+    }
+    __syncwarp();
+    topk_warp(s_row[warp], E, k, topk_idx + static_cast<int64_t>(t) * k, topk_w + static_cast<int64_t>(t) * k);
+    __syncwarp();
+  }
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) s_last = atomicAdd(ticket, 1u) == gridDim.x - 1u;
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  for (int t = warp; t < T; t += nwarps) {
-    // the other CTAs' logits: read through L2
-    float lv[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int e = lane + 32 * i;
-      lv[i] = e < E ? __ldcg(logits + static_cast<int64_t>(t) * E + e) : 0.0f;
-    }
-    __shared__ float s_row[kPermThreads / 32][256];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E) s_row[warp][e] = lv[i];
-    }
-    __syncwarp();
-    topk_warp(s_row[warp], E, k, topk_idx + static_cast<int64_t>(t) * k, topk_w + static_cast<int64_t>(t) * k);
-    __syncwarp();
-  }
   __syncthreads();   // the CTA's global writes of topk_idx are visible to all its threads
   permute_scatter_body(sm, 0, topk_idx, static_cast<int64_t>(T) * k, E, k, nullptr, offsets, perm_token,
                        perm_slot, inv, active, n_active, err);
@@ -468,12 +499,12 @@ bool route_small_supported(int T, int E, int k) {
 }
 
 cudaError_t launch_route_small(const uint16_t* x, const uint16_t* wr, const uint16_t* br, int T, int H, int E,
-                               int k, float* logits, unsigned* ticket, int32_t* topk_idx, float* topk_w,
-                               int32_t* offsets, int32_t* perm_token, int32_t* perm_slot, int32_t* inv,
+                               int k, float* logits, unsigned* ticket, unsigned* tok_tickets, int32_t* topk_idx,
+                               float* topk_w, int32_t* offsets, int32_t* perm_token, int32_t* perm_slot, int32_t* inv,
                                int32_t* active, int32_t* n_active, int* err, cudaStream_t st) {
   const int64_t warps = static_cast<int64_t>(T) * E;
   const unsigned grid = static_cast<unsigned>(cdiv(warps, kPermThreads / 32));
-  route_small_kernel<<<grid, kPermThreads, 0, st>>>(x, wr, br, T, H, E, k, logits, ticket, topk_idx, topk_w,
+  route_small_kernel<<<grid, kPermThreads, 0, st>>>(x, wr, br, T, H, E, k, logits, ticket, tok_tickets, topk_idx, topk_w,
                                                     offsets, perm_token, perm_slot, inv, active, n_active, err);
   return cudaGetLastError();
 }
