@@ -371,8 +371,7 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
   }
   if (dtc) {
     // small batch on the tensor cores: tokens as MX-FP8 parts, weights as the A operand
-    if ((e = launch_split_tokens(fp8, a.x, b.perm_token, b.perm_slot, b.topk_idx, b.offsets, P, a.H, a.k, s0, a.T,
-                                 b.xs, b.sfb, st)))
+    if ((e = launch_split_tokens(fp8, a.x, b.topk_idx, b.inv, b.offsets, a.T, a.E, a.H, a.k, s0, b.xs, b.sfb, st)))
       return cuda_fail(e, "split");
     ++launches;
     tm.mark("act_split");

@@ -777,63 +777,95 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
 }
 
 // ------------------------------------------------ token operand of the gate_up GEMM --
-// One CTA per routed pair: the pair's x (or, with FP8 activations, the e4m3 value of
-// x / s0) as four e2m1 parts, each with ONE e8m0 scale for the whole row (the smallest s
-// with the row's largest residual / 2^s <= 6), packed in expert-grouped row order. A
-// row-wide scale costs a little accuracy against per-block scales (a simulation of the
-// 2880-long dot products: 1.2e-4 of the largest output instead of 4e-5, against a 2e-3
-// bar) and makes the gate_up GEMM's B scale atom the same for every k-tile, so the GEMM
-// copies it into tensor memory once per unit instead of twice per stage. Its record:
-// [expert][row group][two 512-byte atoms], the four k-block bytes of a row all equal.
+// One CTA per token: the token's x (or, with FP8 activations, the e4m3 value of x / s0)
+// as four e2m1 parts, each with ONE e8m0 scale for the whole row (the smallest s with the
+// row's largest residual / 2^s <= 6), written to each of the token's k routed rows in
+// expert-grouped order (its position inv[t*k + j]). A row-wide scale costs a little
+// accuracy against per-block scales (a simulation of the 2880-long dot products: 1.2e-4
+// of the largest output instead of 4e-5, against a 2e-3 bar) and makes the gate_up GEMM's
+// B scale atom the same for every k-tile, so the GEMM copies it into tensor memory once
+// per unit instead of twice per stage. Its record: [expert][row group][two 512-byte
+// atoms], the four k-block bytes of a row all equal. The row's loads are issued first
+// (they depend on nothing), the routing lookups beside them; each thread holds 16
+// consecutive values, so a part leaves as one 8-byte store per routed row.
 constexpr int kSplitThreads = 256;
 constexpr int kSplitVals = 16;   // values per thread: H <= 4096
 __global__ void __launch_bounds__(kSplitThreads) split_tokens_kernel(
-    const uint16_t* __restrict__ x, const int32_t* __restrict__ perm_token, const int32_t* __restrict__ perm_slot,
-    const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ offsets, int64_t P, int H, int k, float s0,
-    int fp8, uint8_t* __restrict__ xs, uint8_t* __restrict__ sfb, int max_chunks) {
+    const uint16_t* __restrict__ x, const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ inv,
+    const int32_t* __restrict__ offsets, int E, int64_t P, int H, int k, float s0, int fp8,
+    uint8_t* __restrict__ xs, uint8_t* __restrict__ sfb, int max_chunks) {
   __shared__ float s_max[kSplitThreads / 32];
+  __shared__ int s_pos[kMaxTopK];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t pos = blockIdx.x;
-  if (pos >= P) return;
-  const int t = perm_token[pos];
-  const int e = topk_idx[static_cast<int64_t>(t) * k + perm_slot[pos]];
-  const int je = static_cast<int>(pos - offsets[e]);   // row within the expert
-  const int c = je / kGroupRows, jr = je % kGroupRows;
-  // thread i holds elements i + 256 v: neighbouring lanes hold neighbouring elements
+  const int t = blockIdx.x;
+  const int i0 = kSplitVals * static_cast<int>(threadIdx.x);
+  const bool act = i0 < H;   // H % 64 == 0: a thread's 16 values are all in or all out
+  uint4 raw[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+  if (act) {
+    const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(t) * H + i0);
+    raw[0] = ld_nc_v4(src);
+    raw[1] = ld_nc_v4(src + 1);
+  }
+  // thread j < k: the token's routed row j (its scale record is written by this thread)
+  uint8_t* rec = nullptr;
+  int jr = 0;
+  if (static_cast<int>(threadIdx.x) < k) {
+    const int64_t pr = static_cast<int64_t>(t) * k + threadIdx.x;
+    const int e = topk_idx[pr];
+    const int pos = inv[pr];
+    int ps = -1;
+    if (e >= 0 && e < E && pos >= 0 && pos < P) {   // else the permutation has flagged it
+      const int je = pos - offsets[e];   // row within the expert
+      rec = sfb + (static_cast<int64_t>(e) * max_chunks + je / kGroupRows) * kSfRecord;
+      jr = je % kGroupRows;
+      ps = pos;
+    }
+    s_pos[threadIdx.x] = ps;
+  }
   float r[kSplitVals];
 #pragma unroll
-  for (int v = 0; v < kSplitVals; ++v) {
-    const int kk = static_cast<int>(threadIdx.x) + kSplitThreads * v;
-    float val = 0.0f;
-    if (kk < H) val = bf16_bits_to_f32(x[static_cast<int64_t>(t) * H + kk]);
-    r[v] = fp8 ? e4m3_to_f32(act_quant_e4m3(val, s0)) : val;
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t w4[4] = {raw[h].x, raw[h].y, raw[h].z, raw[h].w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float lo = __uint_as_float(w4[q] << 16), hi = __uint_as_float(w4[q] & 0xFFFF0000u);
+      r[8 * h + 2 * q] = fp8 ? e4m3_to_f32(act_quant_e4m3(lo, s0)) : lo;
+      r[8 * h + 2 * q + 1] = fp8 ? e4m3_to_f32(act_quant_e4m3(hi, s0)) : hi;
+    }
   }
   const int64_t row_bytes = H / 2;
-  uint8_t* rec = sfb + (static_cast<int64_t>(e) * max_chunks + c) * kSfRecord;
+  __syncthreads();   // s_pos
 #pragma unroll 1
   for (int pp = 0; pp < kParts; ++pp) {
     float m = 0.0f;
 #pragma unroll
     for (int v = 0; v < kSplitVals; ++v) m = fmaxf(m, fabsf(r[v]));
     m = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(m)));
-    __syncthreads();   // the previous part's maxima have been read
     if (lane == 0) s_max[warp] = m;
     __syncthreads();
 #pragma unroll
     for (int w = 0; w < kSplitThreads / 32; ++w) m = fmaxf(m, s_max[w]);
+    __syncthreads();   // every thread has read s_max before the next part writes it
     const int sc = e2m1_part_exponent(m);
+    const float down = pow2f(-sc), up = pow2f(sc);
+    uint32_t packed[2] = {0u, 0u};
 #pragma unroll
-    for (int v = 0; v < kSplitVals; ++v) {
-      const float q = r[v] * pow2f(-sc);
-      const float qn = __shfl_down_sync(0xffffffffu, q, 1);
-      const uint32_t byte = __nv_cvt_float2_to_fp4x2(make_float2(q, qn), __NV_E2M1, cudaRoundNearest);
-      const __nv_fp4x2_storage_t own = __nv_cvt_float2_to_fp4x2(make_float2(q, q), __NV_E2M1, cudaRoundNearest);
-      const __half2_raw h = __nv_cvt_fp4x2_to_halfraw2(own, __NV_E2M1);
-      r[v] = r[v] - __half2float(__half(__half_raw{h.x})) * pow2f(sc);   // exact
-      const int kk = static_cast<int>(threadIdx.x) + kSplitThreads * v;
-      if (kk < H && (lane & 1) == 0) xs[(pos * kParts + pp) * row_bytes + (kk >> 1)] = static_cast<uint8_t>(byte);
+    for (int j = 0; j < kSplitVals / 2; ++j) {
+      const uint32_t byte =
+          __nv_cvt_float2_to_fp4x2(make_float2(r[2 * j] * down, r[2 * j + 1] * down), __NV_E2M1, cudaRoundNearest);
+      const __half2_raw hv = __nv_cvt_fp4x2_to_halfraw2(static_cast<__nv_fp4x2_storage_t>(byte), __NV_E2M1);
+      r[2 * j] -= __half2float(__half(__half_raw{hv.x})) * up;       // exact
+      r[2 * j + 1] -= __half2float(__half(__half_raw{hv.y})) * up;
+      packed[j >> 2] |= byte << (8 * (j & 3));
     }
-    if (threadIdx.x == 0)   // the row's scale for all four k-blocks of the atom word
+    if (act)
+      for (int j = 0; j < k; ++j) {
+        const int pos = s_pos[j];
+        if (pos >= 0)
+          *reinterpret_cast<uint2*>(xs + (static_cast<int64_t>(pos) * kParts + pp) * row_bytes + i0 / 2) =
+              make_uint2(packed[0], packed[1]);
+      }
+    if (rec)   // the row's scale for all four k-blocks of the atom word
       *reinterpret_cast<uint32_t*>(rec + sf_atom_byte(kParts * jr + pp, 0)) = 0x01010101u * static_cast<uint32_t>(sc + 127);
   }
 }
@@ -928,12 +960,13 @@ size_t decode_tc_ticket_count(int H, int I) {
   return static_cast<size_t>(dec::kMaxGrp) * (m_gu + m_d) * 4 + m_d * 4;
 }
 
-cudaError_t launch_split_tokens(bool fp8, const uint16_t* x, const int32_t* perm_token, const int32_t* perm_slot,
-                                const int32_t* topk_idx, const int32_t* offsets, int64_t P, int H, int k, float s0,
-                                int T, uint8_t* xs, uint8_t* sfb, cudaStream_t st) {
-  if (P <= 0) return cudaSuccess;
-  dec::split_tokens_kernel<<<static_cast<unsigned>(P), dec::kSplitThreads, 0, st>>>(
-      x, perm_token, perm_slot, topk_idx, offsets, P, H, k, s0, fp8 ? 1 : 0, xs, sfb, max_chunks_for(T));
+cudaError_t launch_split_tokens(bool fp8, const uint16_t* x, const int32_t* topk_idx, const int32_t* inv,
+                                const int32_t* offsets, int T, int E, int H, int k, float s0, uint8_t* xs, uint8_t* sfb,
+                                cudaStream_t st) {
+  if (T <= 0) return cudaSuccess;
+  if (k > dec::kMaxTopK || H > dec::kSplitThreads * dec::kSplitVals || H % 64) return cudaErrorInvalidValue;
+  dec::split_tokens_kernel<<<static_cast<unsigned>(T), dec::kSplitThreads, 0, st>>>(
+      x, topk_idx, inv, offsets, E, static_cast<int64_t>(T) * k, H, k, s0, fp8 ? 1 : 0, xs, sfb, max_chunks_for(T));
   return cudaGetLastError();
 }
 

@@ -109,9 +109,9 @@ inline size_t decode_tc_tickets_d(int I) { return static_cast<size_t>(kDecodeMax
 inline size_t decode_tc_tickets_comb(int H, int I) {
   return decode_tc_tickets_d(I) + static_cast<size_t>(kDecodeMaxGroups) * ((H + 127) / 128) * 4;
 }
-cudaError_t launch_split_tokens(bool fp8, const uint16_t* x, const int32_t* perm_token, const int32_t* perm_slot,
-                                const int32_t* topk_idx, const int32_t* offsets, int64_t P, int H, int k, float s0,
-                                int T, uint8_t* xs, uint8_t* sfb, cudaStream_t st);
+cudaError_t launch_split_tokens(bool fp8, const uint16_t* x, const int32_t* topk_idx, const int32_t* inv,
+                                const int32_t* offsets, int T, int E, int H, int k, float s0, uint8_t* xs, uint8_t* sfb,
+                                cudaStream_t st);
 cudaError_t launch_decode_gemm(bool gate_up, const DecodeGemmArgs& a, cudaStream_t st);
 
 cudaError_t launch_combine(const float* y, const int32_t* topk_idx, const float* topk_w,
