@@ -352,6 +352,9 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
   uint8_t* ring = smem + ring_offset();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // The next kernel (down after gate_up) may launch now: its CTAs take the SMs this grid
+  // leaves free or frees, and wait for this grid's results only where they read them.
+  griddep_launch_dependents();
   if (threadIdx.x == 0) {
     asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&map_w)) : "memory");
     asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&map_x)) : "memory");
@@ -456,6 +459,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      bool dep_ready = false;
       for (int u = blockIdx.x; u < sc.units && ok; u += gridDim.x) {
         const Unit w = unit_at(sc, p, u);
         // B scales: gate_up has one record per row group (the same for every k-tile); down
@@ -468,6 +472,13 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[stage], tx);
           tma_load_3d(sA(stage, 0), &map_w, &full[stage], kRowBytes * kst, w.m * BM, kA * w.e);
+          if (!dep_ready) {
+            // the token operand and its scales are the previous kernel's output: everything
+            // before this point (setup, the first weight stage, the scale converters' start)
+            // overlaps that kernel's tail
+            griddep_wait();
+            dep_ready = true;
+          }
           for (int b = 0; b < w.nbox; ++b)
             tma_load_2d(sB(stage) + b * p.box_rows * kRowBytes, &map_x, &full[stage], kRowBytes * kst,
                         kParts * w.off + b * p.box_rows);
@@ -564,40 +575,49 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
     if (h < kA) {
       // lane l owns rows l, l+32, l+64, l+96 of the tile; a stage's 8 scale bytes of a row
       // are four aligned 16-bit words (nb is even). They are loaded kRing stages ahead
-      // into an unrolled ring of register sets (never moved, and combined only at the
-      // store, so no instruction waits for them early) and stored as the 128x256b copy
+      // into an unrolled ring of register sets (never moved, always from a valid address,
+      // with a mask of the words that exist beside them, and combined only at the store,
+      // so no instruction waits for them early) and stored as the 128x256b copy
       // source: k-tile 0's word of row 32i + l at 16*L + 4*i, k-tile 1's at 2048 + 16*L + 4*i,
       // for each tensor-memory lane L = 32*q + l.
       constexpr int kRing = 3;
       int stage = 0;
       uint32_t phase = 0;
       const uint16_t* rp[4] = {nullptr, nullptr, nullptr, nullptr};
+      uint32_t rows_ok = 0u;                  // bit i: row lane + 32 i is in the tile
       int lu = blockIdx.x, lk = 0, lk1 = 0;   // load cursor: unit, stage, end stage
       auto start_unit = [&](int u) {
         const Unit w = unit_at(sc, p, u);
         const int valid = min(BM, p.rows_per_group - w.m * BM);
         const int group = kGateUp ? 2 * w.e + h : w.e;
         const uint8_t* blk = p.w_scales + (static_cast<int64_t>(group) * p.rows_per_group + w.m * BM) * p.nb;
+        rows_ok = 0u;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int r = lane + 32 * i;
-          rp[i] = r < valid ? reinterpret_cast<const uint16_t*>(blk + static_cast<int64_t>(r) * p.nb) : nullptr;
+          rp[i] = reinterpret_cast<const uint16_t*>(blk + static_cast<int64_t>(r < valid ? r : 0) * p.nb);
+          rows_ok |= (r < valid ? 1u : 0u) << i;
         }
         lk = w.k0;
         lk1 = w.k1;
       };
-      auto load_next = [&](uint32_t (&wd)[16]) {
-        if (lu >= sc.units) return;
+      // wd: the raw words; returns the mask of those that exist (bit 4 i + q)
+      auto load_next = [&](uint32_t (&wd)[16]) -> uint32_t {
+        if (lu >= sc.units) return 0u;
         const int b0 = 8 * lk;
+        uint32_t ok = 0u;
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            wd[4 * i + q] = (rp[i] && b0 + 2 * q < p.nb) ? static_cast<uint32_t>(__ldg(rp[i] + b0 / 2 + q)) : 0x7F7Fu;
+          for (int q = 0; q < 4; ++q) {
+            wd[4 * i + q] = __ldg(rp[i] + min(b0 / 2 + q, p.nb / 2 - 1));
+            ok |= (((rows_ok >> i) & 1u) && b0 + 2 * q < p.nb ? 1u : 0u) << (4 * i + q);
+          }
         if (++lk == lk1) {
           lu += gridDim.x;
           if (lu < sc.units) start_unit(lu);
         }
+        return ok;
       };
       if (lu < sc.units) start_unit(lu);
       int su = blockIdx.x, sk = 0, sk1 = 0;    // store cursor
@@ -607,17 +627,21 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
         sk1 = w.k1;
       }
       uint32_t ring[kRing][16] = {};
+      uint32_t ring_ok[kRing] = {};
 #pragma unroll
-      for (int j = 0; j < kRing; ++j) load_next(ring[j]);
+      for (int j = 0; j < kRing; ++j) ring_ok[j] = load_next(ring[j]);
       bool run = su < sc.units;
       while (run) {
 #pragma unroll
         for (int j = 0; j < kRing; ++j) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err)) { run = false; break; }
-          const uint4 c0 = make_uint4(ring[j][0] | (ring[j][1] << 16), ring[j][4] | (ring[j][5] << 16),
-                                      ring[j][8] | (ring[j][9] << 16), ring[j][12] | (ring[j][13] << 16));
-          const uint4 c1 = make_uint4(ring[j][2] | (ring[j][3] << 16), ring[j][6] | (ring[j][7] << 16),
-                                      ring[j][10] | (ring[j][11] << 16), ring[j][14] | (ring[j][15] << 16));
+          uint32_t wv[16];
+#pragma unroll
+          for (int f = 0; f < 16; ++f) wv[f] = ((ring_ok[j] >> f) & 1u) ? (ring[j][f] & 0xFFFFu) : 0x7F7Fu;
+          const uint4 c0 = make_uint4(wv[0] | (wv[1] << 16), wv[4] | (wv[5] << 16), wv[8] | (wv[9] << 16),
+                                      wv[12] | (wv[13] << 16));
+          const uint4 c1 = make_uint4(wv[2] | (wv[3] << 16), wv[6] | (wv[7] << 16), wv[10] | (wv[11] << 16),
+                                      wv[14] | (wv[15] << 16));
           uint8_t* dst = sSFA(stage, h) + 16 * lane;
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -635,7 +659,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
             sk = w.k0;
             sk1 = w.k1;
           }
-          load_next(ring[j]);
+          ring_ok[j] = load_next(ring[j]);
         }
       }
     }
@@ -796,6 +820,7 @@ __global__ void __launch_bounds__(kSplitThreads) split_tokens_kernel(
     uint8_t* __restrict__ xs, uint8_t* __restrict__ sfb, int max_chunks) {
   __shared__ float s_max[kSplitThreads / 32];
   __shared__ int s_pos[kMaxTopK];
+  griddep_launch_dependents();   // the gate_up GEMM may start its setup and weight stream
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int t = blockIdx.x;
   const int i0 = kSplitVals * static_cast<int>(threadIdx.x);
@@ -1042,6 +1067,13 @@ cudaError_t launch_decode_gemm(bool gate_up, const DecodeGemmArgs& a, cudaStream
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = st;
+  // programmatic dependent launch: the kernel starts during its predecessor (the token
+  // split, or gate_up for down) and waits for it only before reading its output
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (gate_up) return cudaLaunchKernelEx(&cfg, decode_gemm_kernel<true>, mw, mx, prm);
   return cudaLaunchKernelEx(&cfg, decode_gemm_kernel<false>, mw, mx, prm);
 }

@@ -258,8 +258,9 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constan
     const int w2 = warp - 2;
     const int halves = kGateUp ? 2 : 1;
     uint32_t phase = 0;
-    // rows of tile t this lane converts (nullptr: outside the tile -> unit scale)
-    auto rows_of = [&](int t, const uint16_t* (&rp)[4]) {
+    // rows of tile t this lane converts; a row outside the tile reads the array's first
+    // row and its bit in ok is clear (its words become unit scales at the store)
+    auto rows_of = [&](int t, const uint16_t* (&rp)[4], uint32_t& ok) {
       const Tile tl = tile_of(t, prefix, p.offsets, p.E, p.n_tiles);
       const int n0 = tl.nt * bn_rows;
       const int valid = min(bn_rows, p.rows_per_group - n0);
@@ -269,10 +270,10 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constan
         const int h = r >= bn_rows ? 1 : 0;
         const int rr = r - h * bn_rows;
         const int group = kGateUp ? 2 * tl.e + h : tl.e;
-        rp[i] = (r < BN && rr < valid && h < halves)
-                    ? reinterpret_cast<const uint16_t*>(p.b_scales +
-                                                        (static_cast<int64_t>(group) * p.rows_per_group + n0 + rr) * p.nb)
-                    : nullptr;
+        const bool in = r < BN && rr < valid && h < halves;
+        rp[i] = reinterpret_cast<const uint16_t*>(
+            p.b_scales + (in ? (static_cast<int64_t>(group) * p.rows_per_group + n0 + rr) * p.nb : 0));
+        ok = (ok & ~(1u << i)) | ((in ? 1u : 0u) << i);
       }
     };
     // the stage's two 16-bit words of each row, kept apart until the store (combining
@@ -281,8 +282,8 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constan
       const int kw = (kt < p.nk_full ? 4 * kt : p.nb - 4) >> 1;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        wv[2 * i] = rp[i] ? static_cast<uint32_t>(__ldg(rp[i] + kw)) : 0x7F7Fu;
-        wv[2 * i + 1] = rp[i] ? static_cast<uint32_t>(__ldg(rp[i] + kw + 1)) : 0x7F7Fu;
+        wv[2 * i] = __ldg(rp[i] + kw);
+        wv[2 * i + 1] = __ldg(rp[i] + kw + 1);
       }
     };
     // A ring of kStages register sets, unrolled so that no set is ever moved: the loads of
@@ -291,15 +292,18 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constan
     int lt = blockIdx.x, lkt = 0;   // next stage to load
     int st = blockIdx.x, skt = 0;   // next stage to store
     const uint16_t* rp[4] = {nullptr, nullptr, nullptr, nullptr};
+    uint32_t rows_ok = 0u;
     uint32_t buf[kStages][8] = {};
-    auto load_next = [&](uint32_t (&wv)[8]) {
-      if (lt >= total_tiles) return;
-      if (lkt == 0) rows_of(lt, rp);
+    uint32_t buf_ok[kStages] = {};   // the rows_ok of each set's tile
+    auto load_next = [&](uint32_t (&wv)[8]) -> uint32_t {
+      if (lt >= total_tiles) return 0u;
+      if (lkt == 0) rows_of(lt, rp, rows_ok);
       load(rp, lkt, wv);
       if (++lkt == nkt) { lkt = 0; lt += gridDim.x; }
+      return rows_ok;
     };
 #pragma unroll
-    for (int j = 0; j < kStages; ++j) load_next(buf[j]);
+    for (int j = 0; j < kStages; ++j) buf_ok[j] = load_next(buf[j]);
     bool run = true;
     while (run) {
 #pragma unroll
@@ -308,8 +312,11 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constan
           run = false;
           break;
         }
-        const uint4 wq = make_uint4(buf[j][0] | (buf[j][1] << 16), buf[j][2] | (buf[j][3] << 16),
-                                    buf[j][4] | (buf[j][5] << 16), buf[j][6] | (buf[j][7] << 16));
+        uint32_t wq4[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          wq4[i] = ((buf_ok[j] >> i) & 1u) ? ((buf[j][2 * i] & 0xFFFFu) | (buf[j][2 * i + 1] << 16)) : 0x7F7F7F7Fu;
+        const uint4 wq = make_uint4(wq4[0], wq4[1], wq4[2], wq4[3]);
         uint8_t* dst = sSF + j * kSfStage + 2048 * w2 + 16 * lane;
 #pragma unroll
         for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(dst + 512 * q) = wq;
@@ -317,7 +324,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constan
         __syncwarp();
         if (lane == 0) mbar_arrive(&full[j]);
         if (++skt == nkt) { skt = 0; st += gridDim.x; }
-        load_next(buf[j]);
+        buf_ok[j] = load_next(buf[j]);
       }
       phase ^= 1;
     }
