@@ -63,6 +63,15 @@ __device__ __forceinline__ float silu_mul(float gate, float up) {
   return __fdiv_rn(gate, 1.0f + expf(-gate)) * up;
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream serialization
+// may start once every CTA of the previous kernel in the stream has called
+// griddep_launch_dependents() (or exited); griddep_wait() returns once that kernel has
+// completed and its memory operations are visible. Both are no-ops without the attribute.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
 // ------------------------------------------------------------------ warp utilities
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll

@@ -129,6 +129,9 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constan
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bn_rows = kGateUp ? BN / 2 : BN;      // rows per B load (one half for gate_up)
+  // The next kernel (down after gate_up) may launch now: its CTAs take the SMs this grid
+  // frees and wait for this grid's results only where they read them.
+  griddep_launch_dependents();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -181,6 +184,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constan
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
+      bool dep_ready = false;
       const uint32_t tx = kAStage + (kGateUp ? 2 : 1) * bn_rows * (BK / 2);
       for (int t = blockIdx.x; t < total_tiles && !*abort_flag; t += gridDim.x) {
         const Tile tl = tile_of(t, prefix, p.offsets, p.E, p.n_tiles);
@@ -192,13 +196,19 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constan
           const CUtensorMap* mb = tail ? &tmap_bt : &tmap_b;
           const int kx = tail ? p.K - BK : kt * BK;
           const int bx = tail ? 0 : kt * BK;
-          tma_load_2d(sA + stage * kAStage, &tmap_a, &full[stage], kx, tl.m0);
           if (kGateUp) {
             tma_load_3d(sB + stage * kBStage, mb, &full[stage], bx, n0, 2 * tl.e);
             tma_load_3d(sB + stage * kBStage + bn_rows * BK, mb, &full[stage], bx, n0, 2 * tl.e + 1);
           } else {
             tma_load_3d(sB + stage * kBStage, mb, &full[stage], bx, n0, tl.e);
           }
+          if (!dep_ready) {
+            // the activation rows are the previous kernel's output: setup and the first
+            // weight stage overlap that kernel's tail
+            griddep_wait();
+            dep_ready = true;
+          }
+          tma_load_2d(sA + stage * kAStage, &tmap_a, &full[stage], kx, tl.m0);
           if (++stage == kStages) { stage = 0; phase ^= 1; }
         }
       }
@@ -531,12 +541,20 @@ cudaError_t launch_tc_gemm(bool gate_up, const uint8_t* a, int64_t P_rows, int K
   prm.a_out = a_out;
   prm.y_out = y_out;
   prm.err = err;
-  const size_t smem = smem_bytes(E);
-  if (gate_up)
-    moe_gemm_kernel<true><<<sms, kThreads, smem, st>>>(ma, mb, mbt, prm);
-  else
-    moe_gemm_kernel<false><<<sms, kThreads, smem, st>>>(ma, mb, mbt, prm);
-  return cudaGetLastError();
+  // programmatic dependent launch: the kernel starts during its predecessor (the FP8 cast
+  // and scatter, or gate_up for down) and waits for it only before reading its output
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(sms));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem_bytes(E);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (gate_up) return cudaLaunchKernelEx(&cfg, moe_gemm_kernel<true>, ma, mb, mbt, prm);
+  return cudaLaunchKernelEx(&cfg, moe_gemm_kernel<false>, ma, mb, mbt, prm);
 }
 
 }  // namespace mxmoe

@@ -547,6 +547,7 @@ __global__ void __launch_bounds__(256) quant_scatter_fp8_kernel(const uint16_t* 
                                                                  const int32_t* __restrict__ inv, int T,
                                                                  int k, int E, int64_t P, int H, float s,
                                                                  uint8_t* __restrict__ a1) {
+  griddep_launch_dependents();   // the gate_up GEMM may start its setup and weight stream
   const int lane = threadIdx.x & 31;
   const int nw = static_cast<int>((static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5);
   const int n8 = H / 8;

@@ -96,25 +96,6 @@ __device__ __forceinline__ void tc_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc)
   asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;\n" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
-// Programmatic dependent launch: a kernel launched with programmatic stream serialization
-// may start once every CTA of the previous kernel in the stream has called
-// griddep_launch_dependents() (or exited); griddep_wait() returns once that kernel has
-// completed and its memory operations are visible. Both are no-ops without the attribute.
-__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
-__device__ __forceinline__ void griddep_launch_dependents() {
-  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
-}
-
-// L2 prefetch of the 16-byte-aligned interior of [p, p + bytes): a hint, nothing is
-// written, the bytes outside the interior are simply not prefetched.
-__device__ __forceinline__ void l2_prefetch_range(const void* p, uint64_t bytes) {
-  const uint64_t b = reinterpret_cast<uint64_t>(p);
-  const uint64_t lo = (b + 15) & ~uint64_t(15), hi = (b + bytes) & ~uint64_t(15);
-  if (hi > lo)
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(lo), "r"(static_cast<uint32_t>(hi - lo))
-                 : "memory");
-}
-
 // 128 lanes x 32 bytes (8 columns) from a no-swizzle K-major source: lane L's bytes 0-15
 // at 16*L and bytes 16-31 at LBO + 16*L (core matrices of 8 rows x 16 bytes, SBO = 128).
 __device__ __forceinline__ void tc_cp_128x256b(uint32_t taddr, uint64_t sdesc) {
