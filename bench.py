@@ -57,26 +57,33 @@ PER_EXPERT_PACKED = lambda H, I: 2 * I * H // 2 + 2 * I * H // 32 + H * I // 2 +
 
 def ncu_traffic(workload: str, kernel: str):
     """Per-launch DRAM bytes (read + write) of `kernel` from a committed ncu summary under
-    profiles/, or None when there is none or the kernel's source changed since."""
+    profiles/ (a block of "- key: value" lines starting at "- workload:"), or None when
+    there is none or the kernel's source changed since."""
     import glob
     import hashlib
-    for path in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
-        fields = {}
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        records, cur = [], None
         for line in open(path):
-            line = line.strip().lstrip("- ")
-            if ": " in line:
-                k, v = line.split(": ", 1)
-                fields[k.strip()] = v.strip()
-        if fields.get("workload") != workload or fields.get("kernel") != kernel:
-            continue
-        try:
-            src, _, prefix = fields["source"].partition(" sha256 prefix ")
-            digest = hashlib.sha256(open(os.path.join(ROOT, src), "rb").read()).hexdigest()
-            if not digest.startswith(prefix):
+            line = line.strip()
+            if not line.startswith("- ") or ": " not in line:
+                continue
+            k, v = line[2:].split(": ", 1)
+            if k.strip() == "workload":
+                cur = {}
+                records.append(cur)
+            if cur is not None:
+                cur[k.strip()] = v.strip()
+        for fields in records:
+            if fields.get("workload") != workload or fields.get("kernel") != kernel:
+                continue
+            try:
+                src, _, prefix = fields["source"].partition(" sha256 prefix ")
+                digest = hashlib.sha256(open(os.path.join(ROOT, src), "rb").read()).hexdigest()
+                if not digest.startswith(prefix):
+                    return None
+                return int(fields["traffic_bytes_per_launch"])
+            except (KeyError, OSError, ValueError):
                 return None
-            return int(fields["traffic_bytes_per_launch"])
-        except (KeyError, OSError, ValueError):
-            return None
     return None
 
 
@@ -360,8 +367,7 @@ def run_ours(args, world, rank):
         b = work["gu_bytes"] if dom == "gate_up" else work["bytes"] - work["gu_bytes"]
         achieved = b / (dom_ms / 1e3) / 1e9
         peak_note = f"{pk_kind} hbm copy"
-    tc_path = fp8 and T * k >= 1024
-    traffic = ncu_traffic(args.workload, dom) if tc_path else None
+    traffic = ncu_traffic(args.workload, dom)
     roofline = {"bound": bound, "kernel": dom, "achieved": round(achieved, 2), "peak": peak,
                 "unit": unit, "frac": round(achieved / peak, 4), "traffic": traffic,
                 "peak_source": peak_note, "kernel_ms": round(dom_ms, 5)}
