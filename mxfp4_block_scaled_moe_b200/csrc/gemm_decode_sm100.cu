@@ -820,7 +820,6 @@ __global__ void __launch_bounds__(kSplitThreads) split_tokens_kernel(
     uint8_t* __restrict__ xs, uint8_t* __restrict__ sfb, int max_chunks) {
   __shared__ float s_max[kSplitThreads / 32];
   __shared__ int s_pos[kMaxTopK];
-  griddep_launch_dependents();   // the gate_up GEMM may start its setup and weight stream
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int t = blockIdx.x;
   const int i0 = kSplitVals * static_cast<int>(threadIdx.x);
@@ -831,6 +830,12 @@ __global__ void __launch_bounds__(kSplitThreads) split_tokens_kernel(
     raw[0] = ld_nc_v4(src);
     raw[1] = ld_nc_v4(src + 1);
   }
+  // This kernel starts during the routing kernel (programmatic dependent launch): the row
+  // above is the layer input, the routing lookups below are that kernel's output. Only
+  // once routing is complete may the gate_up GEMM launch, since its setup reads the
+  // routing's expert offsets before it waits for this kernel.
+  griddep_wait();
+  griddep_launch_dependents();
   // thread j < k: the token's routed row j (its scale record is written by this thread)
   uint8_t* rec = nullptr;
   int jr = 0;
@@ -990,9 +995,17 @@ cudaError_t launch_split_tokens(bool fp8, const uint16_t* x, const int32_t* topk
                                 cudaStream_t st) {
   if (T <= 0) return cudaSuccess;
   if (k > dec::kMaxTopK || H > dec::kSplitThreads * dec::kSplitVals || H % 64) return cudaErrorInvalidValue;
-  dec::split_tokens_kernel<<<static_cast<unsigned>(T), dec::kSplitThreads, 0, st>>>(
-      x, topk_idx, inv, offsets, E, static_cast<int64_t>(T) * k, H, k, s0, fp8 ? 1 : 0, xs, sfb, max_chunks_for(T));
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(T));
+  cfg.blockDim = dim3(dec::kSplitThreads);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, dec::split_tokens_kernel, x, topk_idx, inv, offsets, E, static_cast<int64_t>(T) * k, H,
+                            k, s0, fp8 ? 1 : 0, xs, sfb, max_chunks_for(T));
 }
 
 // gate_up (gate_up = true): A = gu weights, B = xs (4 parts per routed row), writes xs_mid

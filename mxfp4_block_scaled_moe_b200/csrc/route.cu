@@ -411,6 +411,9 @@ __global__ void __launch_bounds__(kPermThreads) route_small_kernel(
   __shared__ PermuteSmem sm;
   __shared__ unsigned s_last;
   __shared__ int s_tok[kPermThreads / 32], s_ntok;
+  // the decode token split may launch now and load its rows; it waits for this kernel
+  // before reading any routing output
+  griddep_launch_dependents();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   const int64_t wid = static_cast<int64_t>(blockIdx.x) * nwarps + warp;
   if (wid < static_cast<int64_t>(T) * E) {
