@@ -167,6 +167,7 @@ struct Carve {
 struct LayerBuffers {
   unsigned* tickets;
   float* logits;
+  float* logits_rest;
   int32_t* topk_idx;
   float* topk_w;
   int32_t* counts;
@@ -191,13 +192,16 @@ struct LayerBuffers {
   float* part;         // tensor-core decode: split-K partial accumulators
 };
 
-size_t layout(int T, int E, int k, int H, int I, bool fp8, bool tc, bool dtc, LayerBuffers* b, char* base) {
+// n_rest: the tensor-core router's extra K-range partials of the logits (T x E each)
+size_t layout(int T, int E, int k, int H, int I, bool fp8, bool tc, bool dtc, int n_rest, LayerBuffers* b,
+              char* base) {
   const int64_t P = static_cast<int64_t>(T) * k;
   Carve c;
   size_t o_tickets = c.take<uint8_t>(kTicketBytes);
   size_t o_dtick = c.take<unsigned>(dtc ? static_cast<int64_t>(mxmoe::decode_tc_ticket_count(H, I)) : 0);
   const size_t tickets_end = c.off;
   size_t o_logits = c.take<float>(static_cast<int64_t>(T) * E);
+  size_t o_lrest = c.take<float>(static_cast<int64_t>(n_rest) * T * E);
   size_t o_idx = c.take<int32_t>(P), o_w = c.take<float>(P);
   size_t o_counts = c.take<int32_t>(static_cast<int64_t>(mxmoe::permute_chunks(P)) * E);
   size_t o_off = c.take<int32_t>(E + 1), o_act = c.take<int32_t>(E), o_nact = c.take<int32_t>(1);
@@ -219,6 +223,7 @@ size_t layout(int T, int E, int k, int H, int I, bool fp8, bool tc, bool dtc, La
     b->part = reinterpret_cast<float*>(base + o_part);
     b->tickets = reinterpret_cast<unsigned*>(base + o_tickets);
     b->logits = reinterpret_cast<float*>(base + o_logits);
+    b->logits_rest = n_rest > 0 ? reinterpret_cast<float*>(base + o_lrest) : nullptr;
     b->topk_idx = reinterpret_cast<int32_t*>(base + o_idx);
     b->topk_w = reinterpret_cast<float*>(base + o_w);
     b->counts = reinterpret_cast<int32_t*>(base + o_counts);
@@ -294,7 +299,14 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
                   tc_gemm_supported(a.H, a.I, a.gu_blocks, a.d_blocks, a.gu_scales, a.d_scales);
   const bool dtc = !tc && !calib_out && decode_tc_supported(a.H, a.I, a.T, a.gu_blocks, a.d_blocks, a.gu_scales,
                                                              a.d_scales);
-  const size_t need = layout(a.T, a.E, a.k, a.H, a.I, fp8, tc, dtc, nullptr, nullptr);
+  // routing: one fused launch for small batches; else the router GEMM (on the tensor cores
+  // when the shapes allow, split over K ranges) and a top-k kernel that adds the ranges
+  const bool small = route_small_supported(a.T, a.E, a.k);
+  const int ksplit = !small && router_tc_supported(a.T, a.H, a.E, a.x, a.router_w, nullptr)
+                         ? router_tc_ksplit(a.T, a.H, ws->sms)
+                         : 0;
+  const int n_rest = ksplit > 1 ? ksplit - 1 : 0;
+  const size_t need = layout(a.T, a.E, a.k, a.H, a.I, fp8, tc, dtc, n_rest, nullptr, nullptr);
   if (int rc = ensure_capacity(ws, need)) return rc;
   if (std::max(a.H, a.I) > ws->smem_K) {
     cudaError_t e = expert_mma_set_smem_limits(std::max(a.H, a.I));
@@ -312,7 +324,7 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
     ws->dtc_ready = true;
   }
   LayerBuffers b;
-  layout(a.T, a.E, a.k, a.H, a.I, fp8, tc, dtc, &b, ws->base);
+  layout(a.T, a.E, a.k, a.H, a.I, fp8, tc, dtc, n_rest, &b, ws->base);
   // The decode path's tickets follow the fixed ticket block, where other layouts keep
   // ordinary buffers: they are known to be zero only after a decode-path call, which
   // leaves them at zero. Clear them when that is not known.
@@ -326,7 +338,7 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
   const float s0 = fp8 ? act_scale[0] : 1.0f, s1 = fp8 ? act_scale[1] : 1.0f;
 
   StageTimer tm(st);
-  if (route_small_supported(a.T, a.E, a.k)) {
+  if (small) {
     // small batch: router, top-k and permutation in one CTA, one launch
     if ((e = launch_route_small(a.x, a.router_w, a.router_b, a.T, a.H, a.E, a.k, b.logits,
                                 b.tickets + kRouteTicket, b.tickets + kRouteTokTickets, b.topk_idx, b.topk_w,
@@ -335,10 +347,17 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
     ++launches;
     tm.mark("route");
   } else {
-    if ((e = launch_router(a.x, a.router_w, a.router_b, a.T, a.H, a.E, b.logits, st))) return cuda_fail(e, "router");
+    if (ksplit > 0) {
+      if ((e = launch_router_tc(a.x, a.router_w, a.router_b, a.T, a.H, a.E, ksplit, b.logits, b.logits_rest, ws->err,
+                                st)))
+        return cuda_fail(e, "router");
+    } else if ((e = launch_router(a.x, a.router_w, a.router_b, a.T, a.H, a.E, b.logits, st))) {
+      return cuda_fail(e, "router");
+    }
     ++launches;
     tm.mark("router");
-    if ((e = launch_topk(b.logits, a.T, a.E, a.k, b.topk_idx, b.topk_w, st))) return cuda_fail(e, "topk");
+    if ((e = launch_topk(b.logits, b.logits_rest, n_rest, a.T, a.E, a.k, b.topk_idx, b.topk_w, st)))
+      return cuda_fail(e, "topk");
     ++launches;
     tm.mark("topk");
     if ((e = launch_permute(b.topk_idx, a.T, a.E, a.k, b.counts, b.offsets, b.perm_token, b.perm_slot,
@@ -504,15 +523,20 @@ int moe_route_topk(const uint16_t* x, const uint16_t* router_w, const uint16_t* 
   Workspace* ws = nullptr;
   if (int rc = current_device_ws(&ws)) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  float* logits = logits_out;
-  if (!logits) {
-    if (int rc = ensure_capacity(ws, kTicketBytes + static_cast<size_t>(T) * E * sizeof(float))) return rc;
-    logits = reinterpret_cast<float*>(ws->base + kTicketBytes);
-    ws->tickets_zeroed = kTicketBytes;   // the decode path's tickets may lie here
-  }
-  cudaError_t e = mxmoe::launch_router(x, router_w, router_b, T, H, E, logits, st);
+  // workspace: the logits (unless the caller keeps them) and the tensor-core router's extra
+  // K-range partials
+  const bool rtc = T > 32 && mxmoe::router_tc_supported(T, H, E, x, router_w, logits_out);
+  const int ksplit = rtc ? mxmoe::router_tc_ksplit(T, H, ws->sms) : 0;
+  const int n_rest = ksplit > 1 ? ksplit - 1 : 0;
+  const size_t lbytes = (static_cast<size_t>(T) * E * sizeof(float) + 255) & ~static_cast<size_t>(255);
+  if (int rc = ensure_capacity(ws, kTicketBytes + (logits_out ? 0 : lbytes) + n_rest * lbytes)) return rc;
+  ws->tickets_zeroed = kTicketBytes;   // the decode path's tickets may lie here
+  float* logits = logits_out ? logits_out : reinterpret_cast<float*>(ws->base + kTicketBytes);
+  float* rest = reinterpret_cast<float*>(ws->base + kTicketBytes + (logits_out ? 0 : lbytes));
+  cudaError_t e = rtc ? mxmoe::launch_router_tc(x, router_w, router_b, T, H, E, ksplit, logits, rest, ws->err, st)
+                      : mxmoe::launch_router(x, router_w, router_b, T, H, E, logits, st);
   if (e) return cuda_fail(e, "router launch");
-  e = mxmoe::launch_topk(logits, T, E, k, topk_idx, topk_w, st);
+  e = mxmoe::launch_topk(logits, rest, n_rest, T, E, k, topk_idx, topk_w, st);
   return e ? cuda_fail(e, "topk launch") : MXMOE_OK;
 }
 
@@ -522,7 +546,8 @@ int moe_topk_from_logits(const float* logits, int T, int E, int k, int32_t* topk
   if (int rc = check_routing_args(T, E, k)) return rc;
   if (T == 0) return MXMOE_OK;
   if (!logits || !topk_idx || !topk_w) return fail(MXMOE_EINVAL, "null pointer");
-  cudaError_t e = mxmoe::launch_topk(logits, T, E, k, topk_idx, topk_w, static_cast<cudaStream_t>(stream));
+  cudaError_t e = mxmoe::launch_topk(const_cast<float*>(logits), nullptr, 0, T, E, k, topk_idx, topk_w,
+                                     static_cast<cudaStream_t>(stream));
   return e ? cuda_fail(e, "topk launch") : MXMOE_OK;
 }
 

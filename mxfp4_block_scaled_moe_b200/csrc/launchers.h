@@ -13,7 +13,9 @@ cudaError_t launch_dequantize(const uint8_t* blocks, const uint8_t* scales, int6
 
 cudaError_t launch_router(const uint16_t* x, const uint16_t* wr, const uint16_t* br, int T, int H,
                           int E, float* logits, cudaStream_t st);
-cudaError_t launch_topk(const float* logits, int T, int E, int k, int32_t* idx, float* w,
+// rest / n_rest: further K-range partials of the logits (see launch_router_tc), summed into
+// logits in range order before the selection; n_rest = 0 for complete logits.
+cudaError_t launch_topk(float* logits, const float* rest, int n_rest, int T, int E, int k, int32_t* idx, float* w,
                         cudaStream_t st);
 int permute_chunks(int64_t P);
 cudaError_t launch_permute(const int32_t* idx, int T, int E, int k, int32_t* counts_ws,
@@ -21,6 +23,14 @@ cudaError_t launch_permute(const int32_t* idx, int T, int E, int k, int32_t* cou
                            int32_t* inv, int32_t* active, int32_t* n_active, int* err,
                            cudaStream_t st, int* launches);
 bool route_small_supported(int T, int E, int k);
+// Router GEMM on the tensor cores (csrc/router_sm100.cu): H % 64 == 0, 8 <= E <= 256 with
+// E % 8 == 0, 16-byte aligned x / router_w / logits. It splits K into ksplit ranges
+// (router_tc_ksplit): range 0 (with the bias) goes to logits, range s > 0 to
+// logits_rest + (s-1)*T*E; launch_topk adds them.
+bool router_tc_supported(int T, int H, int E, const void* x, const void* wr, const void* logits);
+int router_tc_ksplit(int T, int H, int sms);
+cudaError_t launch_router_tc(const uint16_t* x, const uint16_t* wr, const uint16_t* br, int T, int H, int E,
+                             int ksplit, float* logits, float* logits_rest, int* err, cudaStream_t st);
 cudaError_t launch_route_small(const uint16_t* x, const uint16_t* wr, const uint16_t* br, int T, int H, int E,
                                int k, float* logits, unsigned* ticket, unsigned* tok_tickets, int32_t* topk_idx,
                                float* topk_w, int32_t* offsets, int32_t* perm_token, int32_t* perm_slot, int32_t* inv,

@@ -227,13 +227,29 @@ __device__ __forceinline__ void topk_warp(const float* __restrict__ l, int E, in
   }
 }
 
-__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E,
-                                                    int k, int32_t* __restrict__ idx,
+// n_rest > 0: the router wrote its logits as 1 + n_rest partials over K ranges (rest:
+// n_rest arrays of T*E after logits); a token's logits are their sum in range order,
+// written back to logits before the selection.
+__global__ void __launch_bounds__(256) topk_kernel(float* __restrict__ logits, const float* __restrict__ rest,
+                                                    int n_rest, int T, int E, int k, int32_t* __restrict__ idx,
                                                     float* __restrict__ wts) {
+  __shared__ float s_row[8][256];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (t >= T) return;
-  topk_warp(logits + static_cast<int64_t>(t) * E, E, k, idx + static_cast<int64_t>(t) * k,
-            wts + static_cast<int64_t>(t) * k);
+  const float* row = logits + static_cast<int64_t>(t) * E;
+  if (n_rest > 0) {
+    float* rw = logits + static_cast<int64_t>(t) * E;
+    for (int e = lane; e < E; e += 32) {
+      float v = rw[e];
+      for (int s = 0; s < n_rest; ++s) v += rest[(static_cast<int64_t>(s) * T + t) * E + e];
+      rw[e] = v;
+      s_row[warp][e] = v;
+    }
+    __syncwarp();
+    row = s_row[warp];
+  }
+  topk_warp(row, E, k, idx + static_cast<int64_t>(t) * k, wts + static_cast<int64_t>(t) * k);
 }
 
 // --------------------------------------------------------------------- permute -----
@@ -628,9 +644,11 @@ cudaError_t launch_router(const uint16_t* x, const uint16_t* wr, const uint16_t*
   return cudaGetLastError();
 }
 
-cudaError_t launch_topk(const float* logits, int T, int E, int k, int32_t* idx, float* w,
+cudaError_t launch_topk(float* logits, const float* rest, int n_rest, int T, int E, int k, int32_t* idx, float* w,
                         cudaStream_t st) {
-  topk_kernel<<<static_cast<unsigned>(cdiv(static_cast<int64_t>(T) * 32, 256)), 256, 0, st>>>(logits, T, E, k, idx, w);
+  if (n_rest > 0 && E > 256) return cudaErrorInvalidValue;
+  topk_kernel<<<static_cast<unsigned>(cdiv(static_cast<int64_t>(T) * 32, 256)), 256, 0, st>>>(logits, rest, n_rest, T,
+                                                                                             E, k, idx, w);
   return cudaGetLastError();
 }
 
