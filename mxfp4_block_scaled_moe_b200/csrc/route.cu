@@ -240,11 +240,23 @@ __global__ void __launch_bounds__(256) topk_kernel(float* __restrict__ logits, c
   const float* row = logits + static_cast<int64_t>(t) * E;
   if (n_rest > 0) {
     float* rw = logits + static_cast<int64_t>(t) * E;
-    for (int e = lane; e < E; e += 32) {
-      float v = rw[e];
-      for (int s = 0; s < n_rest; ++s) v += rest[(static_cast<int64_t>(s) * T + t) * E + e];
-      rw[e] = v;
-      s_row[warp][e] = v;
+    if ((E & 3) == 0) {   // four consecutive logits per lane, 16-byte loads (rows are 16-byte aligned)
+      for (int e = 4 * lane; e < E; e += 128) {
+        float4 v = *reinterpret_cast<const float4*>(rw + e);
+        for (int s = 0; s < n_rest; ++s) {
+          const float4 u = *reinterpret_cast<const float4*>(rest + (static_cast<int64_t>(s) * T + t) * E + e);
+          v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
+        }
+        *reinterpret_cast<float4*>(rw + e) = v;
+        s_row[warp][e] = v.x; s_row[warp][e + 1] = v.y; s_row[warp][e + 2] = v.z; s_row[warp][e + 3] = v.w;
+      }
+    } else {
+      for (int e = lane; e < E; e += 32) {
+        float v = rw[e];
+        for (int s = 0; s < n_rest; ++s) v += rest[(static_cast<int64_t>(s) * T + t) * E + e];
+        rw[e] = v;
+        s_row[warp][e] = v;
+      }
     }
     __syncwarp();
     row = s_row[warp];
