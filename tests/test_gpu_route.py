@@ -37,9 +37,15 @@ def test_topk_from_identical_logits_bit_exact(B, T, E, k):
     assert np.allclose(gw[ok], ow[ok], rtol=2e-6, atol=1e-7)
 
 
+# T <= 32: the GEMV router; T > 32 with H % 64 == 0, E % 8 == 0, E <= 256: the tensor-core
+# router, split over K ranges (T = 129 ragged second tile, E = 256 the widest MMA, H = 64 a
+# single K range, T = 4096 the prefill shape); otherwise the mma.sync router (E = 23,
+# H = 2912 not a multiple of 64).
 @pytest.mark.parametrize("T,E,H,bias", [(1, 32, 2880, False), (8, 32, 2880, False),
                                         (64, 32, 2880, False), (200, 128, 2880, False),
-                                        (37, 23, 2880, True), (5, 4, 256, True)])
+                                        (37, 23, 2880, True), (5, 4, 256, True),
+                                        (129, 256, 2880, True), (300, 64, 64, True),
+                                        (150, 128, 2912, False), (4096, 128, 2880, True)])
 def test_router_logits_and_indices(B, T, E, H, bias):
     lay = inputs.small_layer(E=E, k=4 if E >= 4 else E, T=T, H=H, I=32, seed=T + E,
                              router_std=1.0 / np.sqrt(H), router_bias=bias, device="cuda")
