@@ -31,9 +31,9 @@
 //
 // The gate_up epilogue applies bias + SwiGLU and writes a directly as the down GEMM's B
 // operand (its 32-row warp is exactly one 32-value block of the down contraction, so a
-// part's block amax is a warp reduction); the down epilogue writes y and, for a few
-// tokens, the weighted combine of each 32-row slice, by the last of the slice's row
-// groups to finish.
+// part's block amax stays inside the warp: after a four-row transpose through shared
+// memory it is three xor-shuffles); the down epilogue writes y and, for a few tokens, the
+// weighted combine of each 32-row slice, by the last of the slice's row groups to finish.
 //
 // Scale-factor records of the B operand ("SFB"): for row group g and 128-wide k-tile kt,
 // 1024 bytes = two 512-byte tcgen05.cp atoms (B rows 0..127, 128..255), row r at byte

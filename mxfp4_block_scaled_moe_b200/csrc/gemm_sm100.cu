@@ -21,10 +21,10 @@
 // K = 2880 is 22.5 tiles of 128: the last tile reads the final 128 values through a
 // second tensor map and issues only its last two K-steps.
 //
-// Scale factors: a converter warp copies the tile's raw scale rows into shared memory
-// once per output tile and, per pipeline stage, rewrites the stage's 4 k-blocks into the
-// layout the MMA reads from tensor memory: weight row n at column n/32, lane n%32 of every
-// 32-lane quarter, byte j for k-block j. The stage's 8 columns go in with ONE tcgen05.cp
+// Scale factors: two converter warps read the checkpoint's e8m0 bytes of the stage's 4
+// k-blocks for the tile's rows (L1-cached loads issued kStages stages ahead) and write them
+// in the layout the MMA reads from tensor memory: weight row n at column n/32, lane n%32 of
+// every 32-lane quarter, byte j for k-block j. The stage's 8 columns go in with ONE tcgen05.cp
 // 128x256b from a 4 KB source that repeats the 32 lanes for each quarter: in the tensor
 // pipe a scale copy costs about as much as an MMA whatever its size (measured: 4 MMAs of
 // N = 240 take ~550 cycles; adding two 32x128b.warpx4 copies ~880, one 128x256b ~730).
