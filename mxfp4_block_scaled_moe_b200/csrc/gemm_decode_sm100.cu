@@ -580,7 +580,10 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
       // so no instruction waits for them early) and stored as the 128x256b copy
       // source: k-tile 0's word of row 32i + l at 16*L + 4*i, k-tile 1's at 2048 + 16*L + 4*i,
       // for each tensor-memory lane L = 32*q + l.
-      constexpr int kRing = 3;
+      // two sets: each unrolled copy of the loop body is more code fetched cold at every
+      // launch (measured on one B200 against three sets: 2-5 us faster at T = 1 / 8 / 64;
+      // five sets were 18 us slower)
+      constexpr int kRing = 2;
       int stage = 0;
       uint32_t phase = 0;
       const uint16_t* rp[4] = {nullptr, nullptr, nullptr, nullptr};
