@@ -577,13 +577,14 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
       // are four aligned 16-bit words (nb is even). They are loaded kRing stages ahead
       // into an unrolled ring of register sets (never moved, always from a valid address,
       // with a mask of the words that exist beside them, and combined only at the store,
-      // so no instruction waits for them early) and stored as the 128x256b copy
+      // so no instruction waits for them before that) and stored as the 128x256b copy
       // source: k-tile 0's word of row 32i + l at 16*L + 4*i, k-tile 1's at 2048 + 16*L + 4*i,
       // for each tensor-memory lane L = 32*q + l.
-      // two sets: each unrolled copy of the loop body is more code fetched cold at every
-      // launch (measured on one B200 against three sets: 2-5 us faster at T = 1 / 8 / 64;
-      // five sets were 18 us slower)
-      constexpr int kRing = 2;
+      // one set: each unrolled copy of the loop body is more code fetched cold at every
+      // launch, and after a unit's first stages the rows' scale bytes hit L1 (measured on one
+      // B200, layer forward at T = 1 / 8 / 64: one set 98 / 151 / 190 us, two 107 / 157 /
+      // 196, three 110 / 161 / 201, five 18 us slower than three)
+      constexpr int kRing = 1;
       int stage = 0;
       uint32_t phase = 0;
       const uint16_t* rp[4] = {nullptr, nullptr, nullptr, nullptr};
