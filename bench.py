@@ -5,7 +5,9 @@ permute, expert gate_up + SwiGLU, down, weighted combine. Default workload: the
 120B-shaped prefill layer with FP8 activations (E=128, top-4, H=I=2880, T=4096, static
 per-tensor scales from a 256-token calibration batch). Other workloads (--workload):
 decode1/decode8/decode64 (20B shape, E=32, bf16 activations), zipf (T=16384, skewed
-routing).
+routing), codec (the standalone MXFP4 codec over the 120B-shaped expert set: a step is
+one quantize of all gate_up + down weights from fp32 and one dequantize each to bf16 and
+fp32; metric GB/s of algorithmic bytes).
 
 Metric: MoE-layer tokens/s (whole job = sum over ranks). Inputs are resident in HBM
 when the timed region starts; L2 is flushed before every timed step, outside the step's
@@ -42,6 +44,7 @@ sys.path.insert(0, ROOT)
 from mxfp4_block_scaled_moe_b200 import inputs  # noqa: E402
 
 METRIC = "MoE-layer tokens/s"
+CODEC_METRIC = "MXFP4 codec GB/s"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -53,6 +56,7 @@ WORKLOADS = {
     "decode8": (lambda dev: inputs.decode_layer(T=8, E=32, device=dev), False),
     "decode64": (lambda dev: inputs.decode_layer(T=64, E=32, device=dev), False),
 }
+CODEC = "codec"
 
 PER_EXPERT_PACKED = lambda H, I: 2 * I * H // 2 + 2 * I * H // 32 + H * I // 2 + H * I // 32
 
@@ -431,6 +435,216 @@ def run_ours(args, world, rank):
     return res
 
 
+# ---------------------------------------------------------------- codec sweep -----
+
+CODEC_H = 2880   # H = I = 2880: gate_up (E, 2I, H) and down (E, H, I) share K = 2880
+
+
+def codec_sweep(n_experts, device):
+    """The codec sweep's fp32 weights as ONE (rows, 2880) tensor: the gate_up rows of all
+    experts (n_experts * 2I), then the down rows (n_experts * H). Both have K = 2880, and
+    the codec treats a tensor as a flat run of 32-value blocks, so one launch per leg
+    covers the whole set. Values: N(0, 0.02) with a Bernoulli(0.01) mask of outliers x 8
+    (the same draws as the codec tests)."""
+    K = CODEC_H
+    rows_gu, rows_d = n_experts * 2 * K, n_experts * K
+    w = torch.empty(rows_gu + rows_d, K, dtype=torch.float32, device=device)
+    w[:rows_gu] = inputs.codec_tensor(rows_gu, K, seed=0, tag="gate_up", device=device)
+    w[rows_gu:] = inputs.codec_tensor(rows_d, K, seed=0, tag="down", device=device)
+    return w
+
+
+def codec_leg_bytes(rows, K):
+    """Algorithmic bytes of each codec leg over (rows, K) values: quantize reads fp32 and
+    writes blocks + scales; dequantize reads blocks + scales and writes bf16 or fp32."""
+    n = rows * K
+    packed = n // 2 + n // 32
+    return {"quantize": 4 * n + packed, "dequantize_bf16": packed + 2 * n,
+            "dequantize_f32": packed + 4 * n}
+
+
+def oracle_codec_gbs(w_host, budget_s):
+    """The oracle's quantize + both dequantizes over the given rows, repeated until about
+    budget_s seconds have passed; returns (GB/s, rows, repetitions, seconds)."""
+    import oracle
+    rows, K = w_host.shape
+    reps = 0
+    t0 = time.perf_counter()
+    while True:
+        blk, sc = oracle.quantize(w_host)
+        oracle.dequantize(blk, sc, out="bf16")
+        oracle.dequantize(blk, sc, out="f32")
+        reps += 1
+        dt = time.perf_counter() - t0
+        if dt >= budget_s:
+            break
+    return sum(codec_leg_bytes(rows, K).values()) * reps / dt / 1e9, rows, reps, dt
+
+
+def run_codec(args, world, rank):
+    from mxfp4_block_scaled_moe_b200 import binding as B
+    pk, pk_kind = peaks()
+    w = codec_sweep(args.codec_experts, "cuda")
+    torch.cuda.empty_cache()              # the draws' temporaries
+    R, K = w.shape
+    blocks = torch.empty(R, K // 2, dtype=torch.uint8, device="cuda")
+    scales = torch.empty(R, K // 32, dtype=torch.uint8, device="cuda")
+    out16 = torch.empty(R, K, dtype=torch.bfloat16, device="cuda")
+    out32 = torch.empty(R, K, dtype=torch.float32, device="cuda")
+    legs = [("quantize", lambda: B.mxfp4_quantize(w, blocks, scales)),
+            ("dequantize_bf16", lambda: B.mxfp4_dequantize(blocks, scales, torch.bfloat16, out=out16)),
+            ("dequantize_f32", lambda: B.mxfp4_dequantize(blocks, scales, torch.float32, out=out32))]
+    leg_bytes = codec_leg_bytes(R, K)
+    step_bytes = sum(leg_bytes.values())
+    launches = 0
+    for _ in range(args.warmup):
+        for _, f in legs:
+            f()
+            launches += B.mxmoe_last_launch_count()
+    B.mxmoe_check()
+    launches_per_step = launches // max(args.warmup, 1)
+
+    # every step reads 12.7 GB of fp32 and writes 19 GB: far larger than L2, no flush needed
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(legs) + 1)] for _ in range(args.steps)]
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t_end = time.perf_counter() + 1.0
+        while time.perf_counter() < t_end:
+            for _, f in legs:
+                f()
+            torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+        torch.cuda.nvtx.range_push("mxmoe_timed")
+        for i in range(args.steps):
+            ev[i][0].record()
+            for j, (_, f) in enumerate(legs):
+                f()
+                ev[i][j + 1].record()
+        torch.cuda.synchronize()
+        torch.cuda.nvtx.range_pop()
+        barrier(world)
+    B.mxmoe_check()
+    leg_ms = {n: sum(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(args.steps))
+              for j, (n, _) in enumerate(legs)}
+    total_ms = max_over_ranks(sum(leg_ms.values()), world)
+    value = step_bytes * world * args.steps / (total_ms / 1e3) / 1e9
+    dom = max(leg_ms, key=leg_ms.get)
+    dom_ms = leg_ms[dom] / args.steps
+    achieved = leg_bytes[dom] / (dom_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 2), "peak": pk["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4),
+                "traffic": ncu_traffic(f"codec{args.codec_experts}", dom),
+                "peak_source": f"{pk_kind} hbm copy", "kernel_ms": round(dom_ms, 5)}
+
+    # ---- end to end through the C ABI from pinned host memory: the first experts' rows
+    # in chunks of one expert's rows (gate_up or down); per chunk the fp32 rows go in,
+    # the three legs run, and the packed, bf16 and fp32 results come back
+    chunk = 2 * K
+    rows_e2e = min(R, args.codec_e2e_chunks * chunk)
+    w_host = w[:rows_e2e].cpu().pin_memory()
+    blk_h = torch.empty(rows_e2e, K // 2, dtype=torch.uint8).pin_memory()
+    sc_h = torch.empty(rows_e2e, K // 32, dtype=torch.uint8).pin_memory()
+    o16_h = torch.empty(rows_e2e, K, dtype=torch.bfloat16).pin_memory()
+    o32_h = torch.empty(rows_e2e, K, dtype=torch.float32).pin_memory()
+    w_dev = torch.empty(chunk, K, dtype=torch.float32, device="cuda")
+
+    def e2e_step():
+        for r0 in range(0, rows_e2e, chunk):
+            r1 = min(rows_e2e, r0 + chunk)
+            n = r1 - r0
+            w_dev[:n].copy_(w_host[r0:r1], non_blocking=True)
+            B.mxfp4_quantize(w_dev[:n], blocks[:n], scales[:n])
+            B.mxfp4_dequantize(blocks[:n], scales[:n], torch.bfloat16, out=out16[:n])
+            B.mxfp4_dequantize(blocks[:n], scales[:n], torch.float32, out=out32[:n])
+            blk_h[r0:r1].copy_(blocks[:n], non_blocking=True)
+            sc_h[r0:r1].copy_(scales[:n], non_blocking=True)
+            o16_h[r0:r1].copy_(out16[:n], non_blocking=True)
+            o32_h[r0:r1].copy_(out32[:n], non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e_bytes = sum(codec_leg_bytes(rows_e2e, K).values())
+    e2e_value = e2e_bytes * world * args.steps / (e2e_ms / 1e3) / 1e9
+
+    res = {
+        "metric": CODEC_METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32 -> e2m1 + e8m0 -> bf16 / f32",
+        "data": "synthetic (seeded; N(0,0.02) with 1% outliers x 8)",
+        "config": {"workload": f"codec: 120B-shaped expert set, {args.codec_experts} experts, "
+                               f"gate_up ({args.codec_experts}, 5760, 2880) + down ({args.codec_experts}, 2880, 2880)",
+                   "rows": R, "K": K, "values": R * K,
+                   "l2": "not flushed: every step streams 12.7 GB in and 19 GB out at 128 experts, "
+                         "far above the 126 MB L2",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": roofline,
+        "stages_ms_per_step": {n: round(v / args.steps, 5) for n, v in leg_ms.items()},
+        "algorithmic": {"bytes_per_step": step_bytes, "bytes_per_leg": leg_bytes},
+        "e2e": {"value": round(e2e_value, 1), "unit": "GB/s",
+                "h2d_bytes_per_step": rows_e2e * K * 4,
+                "d2h_bytes_per_step": rows_e2e * (K // 2 + K // 32 + 2 * K + 4 * K),
+                "timing": f"the sweep's first {rows_e2e} rows in chunks of {chunk} from pinned host "
+                          "memory; per chunk the copy in, the three legs and the four copies out run "
+                          "in order on one stream"},
+        "gpu_launches": launches_per_step * args.steps,
+        "timing": "CUDA events around each leg of every step, K steps back to back",
+    }
+    res["clocks"] = clk.summary()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        v, rows, reps, dt = oracle_codec_gbs(w[: min(R, 1 << 16)].cpu().numpy(), args.cpu_budget)
+        res["cpu_baseline"] = {"value": round(v, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+                               "kind": "oracle",
+                               "sample": f"first {rows} of {R} rows of the same sweep, {reps} passes "
+                                         f"(quantize + both dequantizes) in {dt:.1f} s"}
+    return res
+
+
+def run_reference_codec(args, world, rank):
+    """The oracle's codec over bounded row samples of the sweep, on the host cores."""
+    if rank != 0:
+        return None
+    import oracle
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    K = CODEC_H
+    # rows drawn like the sweep's gate_up rows (same recipe and seed)
+    rows_all = args.codec_experts * 3 * K
+    w = inputs.codec_tensor(min(rows_all, 1 << 14), K, seed=0, tag="gate_up", device=dev).cpu().numpy()
+    oracle_codec_gbs(w, 0.0)                     # one untimed pass
+    for _ in range(args.warmup - 1):
+        oracle_codec_gbs(w, 0.0)
+    t0 = time.perf_counter()
+    reps = 0
+    for _ in range(args.steps):                  # a step: passes over the sample for ~ref_step_s
+        reps += oracle_codec_gbs(w, args.ref_step_s)[2]
+    dt = time.perf_counter() - t0
+    rows = w.shape[0]
+    value = sum(codec_leg_bytes(rows, K).values()) * reps / dt / 1e9
+    return {
+        "impl": "reference", "metric": CODEC_METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32 -> e2m1 + e8m0 -> bf16 / f32 (CPU oracle)",
+        "data": "synthetic (seeded)",
+        "config": {"workload": f"codec: 120B-shaped expert set, {args.codec_experts} experts",
+                   "rows": rows_all, "K": K},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": f"{rows} rows drawn like the sweep's, {reps} passes in {args.steps} steps"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
 def run_reference(args, world, rank):
     """The oracle as it stands, on the host cores, over bounded samples of the workload."""
     if rank != 0:
@@ -501,7 +715,11 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="prefill")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + [CODEC], default="prefill")
+    ap.add_argument("--codec-experts", type=int, default=128,
+                    help="codec workload: experts of the 120B-shaped set to sweep")
+    ap.add_argument("--codec-e2e-chunks", type=int, default=8,
+                    help="codec workload: chunks of one expert's rows in the end-to-end leg")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
     ap.add_argument("--ref-step-s", type=float, default=4.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -514,11 +732,11 @@ def main():
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))
-        res = run_reference(args, world, rank)
+        res = (run_reference_codec if args.workload == CODEC else run_reference)(args, world, rank)
     else:
         world, rank = dist_init()
         try:
-            res = run_ours(args, world, rank)
+            res = (run_codec if args.workload == CODEC else run_ours)(args, world, rank)
         finally:
             if world > 1:
                 import torch.distributed as dist

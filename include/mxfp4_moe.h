@@ -171,8 +171,9 @@ int mxmoe_check(void* stream);
  * The string stays valid until the next library call on the same thread. */
 const char* mxmoe_last_error(void);
 
-/* mxmoe_last_launch_count -- number of kernels the last successful moe_mxfp4_forward
- * on this host thread launched. */
+/* mxmoe_last_launch_count -- number of kernels the last successful moe_mxfp4_forward,
+ * mxfp4_quantize or mxfp4_dequantize on this host thread launched (a codec call launches
+ * one kernel, none when it fails or has no work). */
 int mxmoe_last_launch_count(void);
 
 /* mxmoe_profile_enable -- on != 0: from now on every moe_mxfp4_forward on this host

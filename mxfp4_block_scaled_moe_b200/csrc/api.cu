@@ -482,6 +482,7 @@ extern "C" {
 int mxfp4_quantize(const float* w, int64_t rows, int64_t K, uint8_t* blocks, uint8_t* scales,
                    void* stream) {
   t_last_error.clear();
+  t_last_launches = 0;
   if (rows < 0 || K < 0) return fail(MXMOE_EINVAL, "negative size rows=%lld K=%lld", (long long)rows, (long long)K);
   if (K % 32) return fail(MXMOE_EALIGN, "K = %lld is not a multiple of 32 (MXFP4 block size)", (long long)K);
   if (rows == 0 || K == 0) return MXMOE_OK;
@@ -490,12 +491,15 @@ int mxfp4_quantize(const float* w, int64_t rows, int64_t K, uint8_t* blocks, uin
   Workspace* ws = nullptr;
   if (int rc = current_device_ws(&ws)) return rc;
   cudaError_t e = mxmoe::launch_quantize(w, rows, K, blocks, scales, static_cast<cudaStream_t>(stream), ws->sms);
-  return e ? cuda_fail(e, "quantize launch") : MXMOE_OK;
+  if (e) return cuda_fail(e, "quantize launch");
+  t_last_launches = 1;
+  return MXMOE_OK;
 }
 
 int mxfp4_dequantize(const uint8_t* blocks, const uint8_t* scales, int64_t rows, int64_t K,
                      void* out, int out_dtype, void* stream) {
   t_last_error.clear();
+  t_last_launches = 0;
   if (rows < 0 || K < 0) return fail(MXMOE_EINVAL, "negative size rows=%lld K=%lld", (long long)rows, (long long)K);
   if (K % 32) return fail(MXMOE_EALIGN, "K = %lld is not a multiple of 32 (MXFP4 block size)", (long long)K);
   if (out_dtype != MXMOE_OUT_F32 && out_dtype != MXMOE_OUT_BF16)
@@ -507,7 +511,9 @@ int mxfp4_dequantize(const uint8_t* blocks, const uint8_t* scales, int64_t rows,
   if (int rc = current_device_ws(&ws)) return rc;
   cudaError_t e = mxmoe::launch_dequantize(blocks, scales, rows, K, out, out_dtype,
                                            static_cast<cudaStream_t>(stream), ws->sms);
-  return e ? cuda_fail(e, "dequantize launch") : MXMOE_OK;
+  if (e) return cuda_fail(e, "dequantize launch");
+  t_last_launches = 1;
+  return MXMOE_OK;
 }
 
 int moe_route_topk(const uint16_t* x, const uint16_t* router_w, const uint16_t* router_b, int T,

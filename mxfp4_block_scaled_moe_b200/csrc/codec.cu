@@ -9,7 +9,10 @@
 //
 // Memory layout per thread: quantize reads one float4 (4 values) per lane, 8 lanes per
 // block, so every warp-wide load is 512 contiguous bytes; dequantize reads one 32-bit
-// word (8 values) per lane, 4 lanes per block. Both kernels are HBM-bound streams.
+// word (8 values) per lane, 4 lanes per block. Both kernels are HBM-bound streams with
+// several loads in flight per thread (quantize 4 float4, dequantize 8 words).
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace mxmoe {
@@ -84,47 +87,69 @@ __device__ __forceinline__ uint32_t e2m1_mag_bits(uint32_t c) {
   return c < 2u ? c * 0x3F000000u : (((126u + (c >> 1)) << 23) | ((c & 1u) << 22));
 }
 
+constexpr int kDeqUnroll = 8;
+
 template <bool kBf16>
 __global__ void __launch_bounds__(256) dequantize_kernel(const uint32_t* __restrict__ blocks32,
                                                           const uint8_t* __restrict__ scales,
                                                           int64_t nwords, void* __restrict__ out) {
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; u < nwords;
-       u += stride) {
-    const uint32_t wd = __ldcs(&blocks32[u]);
-    const uint32_t s = scales[u >> 2];
-    // value = c * 2^(s-127) = (c * s1) * s2 with every factor exact in fp32
-    const float s1 = s == 255u ? __uint_as_float(254u << 23) : e8m0_to_f32(s);
-    float v[8];
+  // kDeqUnroll words per thread and iteration, stride apart (each warp-wide access stays
+  // contiguous), all loaded before the first is decoded
+  for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; base < nwords;
+       base += kDeqUnroll * stride) {
+    uint32_t wds[kDeqUnroll], scs[kDeqUnroll];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint32_t nib = (wd >> (4 * i)) & 15u;
-      const float c = __uint_as_float(e2m1_mag_bits(nib & 7u) | ((nib & 8u) << 28));
-      v[i] = c * s1;
+    for (int j = 0; j < kDeqUnroll; ++j) {
+      const int64_t u = base + j * stride;
+      wds[j] = u < nwords ? __ldcs(&blocks32[u]) : 0u;
+      scs[j] = u < nwords ? scales[u >> 2] : 127u;
     }
-    if (s == 255u) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] *= 2.0f;
-    }
-    if constexpr (kBf16) {
-      // every value has at most two significant bits: its bf16 is the top half of fp32
-      uint4 o;
-      o.x = (__float_as_uint(v[0]) >> 16) | (__float_as_uint(v[1]) & 0xFFFF0000u);
-      o.y = (__float_as_uint(v[2]) >> 16) | (__float_as_uint(v[3]) & 0xFFFF0000u);
-      o.z = (__float_as_uint(v[4]) >> 16) | (__float_as_uint(v[5]) & 0xFFFF0000u);
-      o.w = (__float_as_uint(v[6]) >> 16) | (__float_as_uint(v[7]) & 0xFFFF0000u);
-      __stcs(reinterpret_cast<uint4*>(out) + u, o);
-    } else {
-      float4* o = reinterpret_cast<float4*>(out) + 2 * u;
-      __stcs(o, make_float4(v[0], v[1], v[2], v[3]));
-      __stcs(o + 1, make_float4(v[4], v[5], v[6], v[7]));
+    for (int j = 0; j < kDeqUnroll; ++j) {
+      const int64_t u = base + j * stride;
+      if (u >= nwords) break;
+      const uint32_t wd = wds[j], s = scs[j];
+      // value = c * 2^(s-127) = (c * s1) * s2 with every factor exact in fp32
+      const float s1 = s == 255u ? __uint_as_float(254u << 23) : e8m0_to_f32(s);
+      float v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t nib = (wd >> (4 * i)) & 15u;
+        const float c = __uint_as_float(e2m1_mag_bits(nib & 7u) | ((nib & 8u) << 28));
+        v[i] = c * s1;
+      }
+      if (s == 255u) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] *= 2.0f;
+      }
+      if constexpr (kBf16) {
+        // every value has at most two significant bits: its bf16 is the top half of fp32
+        uint4 o;
+        o.x = (__float_as_uint(v[0]) >> 16) | (__float_as_uint(v[1]) & 0xFFFF0000u);
+        o.y = (__float_as_uint(v[2]) >> 16) | (__float_as_uint(v[3]) & 0xFFFF0000u);
+        o.z = (__float_as_uint(v[4]) >> 16) | (__float_as_uint(v[5]) & 0xFFFF0000u);
+        o.w = (__float_as_uint(v[6]) >> 16) | (__float_as_uint(v[7]) & 0xFFFF0000u);
+        __stcs(reinterpret_cast<uint4*>(out) + u, o);
+      } else {
+        float4* o = reinterpret_cast<float4*>(out) + 2 * u;
+        __stcs(o, make_float4(v[0], v[1], v[2], v[3]));
+        __stcs(o + 1, make_float4(v[4], v[5], v[6], v[7]));
+      }
     }
   }
 }
 
-int grid_for(int64_t work_items, int threads, int sms) {
-  int64_t g = cdiv(work_items, threads);
-  int64_t cap = static_cast<int64_t>(sms) * 8;
+// Grid of a grid-stride stream kernel: at most the CTAs that fit on the GPU at once, so
+// every CTA of the grid is resident from the start (a second, partial wave would run the
+// last share of the stream at lower occupancy).
+template <typename Kernel>
+int grid_for(Kernel kernel, int64_t work_items, int threads, int sms) {
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) != cudaSuccess || per_sm < 1)
+    per_sm = 1;
+  const int64_t g = cdiv(work_items, threads);
+  const int64_t cap = static_cast<int64_t>(sms) * per_sm;
   return static_cast<int>(g < 1 ? 1 : (g > cap ? cap : g));
 }
 
@@ -134,7 +159,12 @@ cudaError_t launch_quantize(const float* w, int64_t rows, int64_t K, uint8_t* bl
                             uint8_t* scales, cudaStream_t st, int sms) {
   const int64_t nquads = rows * K / 4;
   if (nquads == 0) return cudaSuccess;
-  const int grid = grid_for(cdiv(nquads, kQuantUnroll), 256, sms);
+  // 8 CTAs per SM although fewer are resident at once (48 registers a thread): measured
+  // on one B200 over the 12.7 GB fp32 expert set, 3.60 ms against 3.74 ms on the grid of
+  // resident CTAs, and a variant that loads the next iteration's values before encoding
+  // this one's was slower still (3.90 ms)
+  const int64_t want = std::max<int64_t>(cdiv(cdiv(nquads, kQuantUnroll), 256), 1);
+  const int grid = static_cast<int>(std::min<int64_t>(want, static_cast<int64_t>(sms) * 8));
   quantize_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const float4*>(w), nquads,
                                         reinterpret_cast<uint16_t*>(blocks), scales);
   return cudaGetLastError();
@@ -144,7 +174,8 @@ cudaError_t launch_dequantize(const uint8_t* blocks, const uint8_t* scales, int6
                               int64_t K, void* out, int out_dtype, cudaStream_t st, int sms) {
   const int64_t nwords = rows * K / 8;
   if (nwords == 0) return cudaSuccess;
-  const int grid = grid_for(nwords, 256, sms);
+  const int grid = out_dtype == MXMOE_OUT_BF16 ? grid_for(dequantize_kernel<true>, cdiv(nwords, kDeqUnroll), 256, sms)
+                                               : grid_for(dequantize_kernel<false>, cdiv(nwords, kDeqUnroll), 256, sms);
   if (out_dtype == MXMOE_OUT_BF16)
     dequantize_kernel<true><<<grid, 256, 0, st>>>(reinterpret_cast<const uint32_t*>(blocks),
                                                   scales, nwords, out);

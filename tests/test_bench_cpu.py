@@ -1,0 +1,43 @@
+"""bench.py's host-side accounting and its CPU reference arm for the codec workload (no GPU).
+
+The byte counts are the codec's algorithmic traffic ("quantization_mxfp4" (KerasFormers),
+Primitives: one 16-byte block of e2m1 pairs and one e8m0 scale byte per 32 values), and
+the per-expert packed size is the 120B-shaped expert set's (4.25 bits per weight)."""
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def test_codec_leg_bytes_closed_forms():
+    # one row of one 32-value block: 128 B of fp32, 16 B of blocks, 1 scale byte
+    b = bench.codec_leg_bytes(1, 32)
+    assert b == {"quantize": 128 + 16 + 1, "dequantize_bf16": 16 + 1 + 64, "dequantize_f32": 16 + 1 + 128}
+    # the full sweep: 128 experts x (5760 + 2880) rows x 2880 values
+    n = 128 * 8640 * 2880
+    full = bench.codec_leg_bytes(128 * 8640, 2880)
+    assert full["quantize"] == 4 * n + n // 2 + n // 32
+    assert full["dequantize_f32"] == full["quantize"]
+    assert full["dequantize_bf16"] == n // 2 + n // 32 + 2 * n
+
+
+def test_per_expert_packed_bytes():
+    # gate_up 8,294,400 B of blocks + 518,400 B of scales, down half of each
+    assert bench.PER_EXPERT_PACKED(2880, 2880) == 8_812_800 + 4_406_400 == 13_219_200
+
+
+def test_codec_reference_arm_runs_on_cpu_and_only_on_rank_0():
+    class A:
+        workload, steps, warmup, ref_step_s, codec_experts = "codec", 1, 3, 0.0, 128
+
+    assert bench.run_reference_codec(A(), world=2, rank=1) is None
+    res = bench.run_reference_codec(A(), world=1, rank=0)
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "config", "cpu_baseline", "e2e"):
+        assert key in res
+    assert res["impl"] == "reference" and res["metric"] == bench.CODEC_METRIC and res["unit"] == "GB/s"
+    assert res["value"] > 0 and res["cpu_baseline"]["kind"] == "oracle"
+    assert res["e2e"]["h2d_bytes_per_step"] == 0 and res["e2e"]["d2h_bytes_per_step"] == 0
