@@ -88,3 +88,44 @@ def to_device(p: Packed, device="cuda"):
 def gpu_bits(t) -> np.ndarray:
     """bf16 CUDA tensor -> numpy uint16 bits."""
     return inputs.bits(t)
+
+
+# ------------------------------------------------- exhaustive round-to-grid blocks ----
+
+GRID_ANCHOR = 4.0   # a block holding 4.0 and values below 8 has amax in [4, 8): scale 2^0
+
+
+class AnchoredBlocks:
+    """fp32 bit patterns [lo, hi) (with the sign bit when ``negative``) as (nb, 32) blocks:
+    column 0 is the anchor 4.0, columns 1..31 the values in pattern order (the last block
+    padded with zeros). With patterns below 8.0 every block's scale exponent is 0, so each
+    value's nibble is the round-to-grid of the value itself. The storage for chunks of up
+    to ``step`` patterns is allocated once and refilled by ``fill``."""
+
+    def __init__(self, step: int):
+        self.idx = np.arange(step, dtype=np.uint32)
+        nb = -(-step // 31)
+        self.body = np.zeros(nb * 31, np.uint32)
+        self.buf = np.empty((nb, 32), np.uint32)
+        self.buf[:, 0] = np.float32(GRID_ANCHOR).view(np.uint32)
+
+    def fill(self, lo: int, hi: int, negative: bool) -> np.ndarray:
+        n = hi - lo
+        nb = -(-n // 31)
+        body = self.body[: nb * 31]
+        np.add(self.idx[:n], np.uint32(lo), out=body[:n])
+        if negative:
+            np.bitwise_or(body[:n], np.uint32(0x80000000), out=body[:n])
+        body[n:] = 0
+        self.buf[:nb, 1:] = body.reshape(nb, 31)
+        return self.buf[:nb].view(np.float32)
+
+
+def anchored_blocks(lo: int, hi: int, negative: bool) -> np.ndarray:
+    """AnchoredBlocks for one range, as a fresh array."""
+    return AnchoredBlocks(hi - lo).fill(lo, hi, negative).copy()
+
+
+def nibble_codes(blocks_packed: np.ndarray) -> np.ndarray:
+    """(nb, 16) packed bytes -> (nb, 32) nibbles, element 2j in the low nibble of byte j."""
+    return np.stack([blocks_packed & 15, blocks_packed >> 4], axis=-1).reshape(blocks_packed.shape[0], 32)

@@ -136,3 +136,20 @@ def test_codec_sweep_full_size_sampled(B):
             del out
         del rb, rs, blk, sc
         torch.cuda.empty_cache()
+
+
+def test_quantize_round_to_grid_exhaustive_fp32(B):
+    """Every fp32 value in (-8, 8), both signs, through the GPU quantizer at scale 2^0
+    (blocks anchored by 4.0): nibbles bit-identical to the oracle's. The oracle's own
+    rounding is pinned against brute force in tests/test_oracle_codec.py."""
+    import helpers
+    top = int(np.float32(8.0).view(np.uint32))
+    step = 1 << 26
+    buf = helpers.AnchoredBlocks(step)
+    for negative in (False, True):
+        for lo in range(0, top, step):
+            blocks = buf.fill(lo, min(top, lo + step), negative)
+            oblk, osc = oracle.quantize(blocks)
+            gblk, gsc = B.mxfp4_quantize(torch.from_numpy(blocks).cuda())
+            assert np.array_equal(gsc.cpu().numpy(), osc), (negative, lo)
+            assert np.array_equal(gblk.cpu().numpy(), oblk), (negative, lo)

@@ -209,3 +209,51 @@ def test_quantize_then_dequantize_error_bound():
     err = np.abs(back - x) / np.ldexp(1.0, e)
     unsat = r <= 6
     assert (err[unsat] <= step[unsat]).all()
+
+
+# ------------------------------------------- round-to-grid against brute force ------
+
+_GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def _brute_force_codes(vals: np.ndarray) -> np.ndarray:
+    """E2M1 code of each fp32 value at scale 2^0 by exhaustive search: the grid point at
+    the least distance (ties to the point with the even code), sign bit from the value's
+    own sign bit (so -0 and tiny negatives keep it)."""
+    r = np.abs(vals.astype(np.float64))
+    d = np.abs(r[:, None] - _GRID[None, :])
+    cand = d == d.min(axis=1, keepdims=True)
+    even = cand & (np.arange(8) % 2 == 0)
+    mag = np.where(even.any(axis=1), even.argmax(axis=1), cand.argmax(axis=1)).astype(np.uint8)
+    return mag | ((vals.view(np.uint32) >> 31).astype(np.uint8) << 3)
+
+
+def _pattern_ranges():
+    """fp32 bit-pattern ranges below 8.0 that hold every decision of the rounding: 2^18
+    patterns on each side of each midpoint between grid points and of each grid point,
+    every 251st pattern of the whole range, and the subnormals' first 2^16."""
+    f = lambda x: int(np.float32(x).view(np.uint32))
+    mids = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]
+    ranges = [(f(m) - (1 << 18), f(m) + (1 << 18)) for m in mids]
+    ranges += [(max(f(g) - (1 << 18), 0), f(g) + (1 << 18)) for g in _GRID[1:]]
+    ranges += [(0, 1 << 16), (f(8.0) - (1 << 18), f(8.0))]
+    return ranges
+
+
+@pytest.mark.parametrize("negative", [False, True])
+def test_round_to_grid_matches_brute_force(negative):
+    import helpers
+    stride = np.arange(0, int(np.float32(8.0).view(np.uint32)), 251, dtype=np.uint32)
+    chunks = [helpers.anchored_blocks(lo, hi, negative) for lo, hi in _pattern_ranges()]
+    s = stride | np.uint32(0x80000000) if negative else stride
+    body = np.zeros(-(-s.size // 31) * 31, np.float32)
+    body[: s.size] = s.view(np.float32)
+    sb = np.empty((body.size // 31, 32), np.float32)
+    sb[:, 0], sb[:, 1:] = helpers.GRID_ANCHOR, body.reshape(-1, 31)
+    chunks.append(sb)
+    for blocks in chunks:
+        packed, scales = oracle.quantize(blocks)
+        assert (scales == 127).all()                       # amax in [4, 8): exponent 0
+        codes = helpers.nibble_codes(packed)
+        assert (codes[:, 0] == 6).all()                    # the anchor 4.0
+        assert np.array_equal(codes[:, 1:], _brute_force_codes(blocks[:, 1:].reshape(-1)).reshape(-1, 31))
