@@ -66,7 +66,7 @@ extern "C" {
  * of +-{0, 0.5, 1, 1.5, 2, 3, 4, 6} * 2^e with ties to the even code, magnitudes past 6
  * saturating; the sign bit is copied from the input (so -0.0 packs as nibble 8).
  * Errors: MXMOE_EALIGN if K % 32 != 0 ("As a quantize_model scheme": a clear error);
- * MXMOE_EINVAL for null pointers or negative sizes. */
+ * MXMOE_EINVAL for null pointers, negative sizes, or w / blocks not 16-byte aligned. */
 int mxfp4_quantize(const float* w, int64_t rows, int64_t K, uint8_t* blocks, uint8_t* scales,
                    void* stream);
 
@@ -74,8 +74,9 @@ int mxfp4_quantize(const float* w, int64_t rows, int64_t K, uint8_t* blocks, uin
  * out[r, k] = codebook[nibble] * 2^(scale - 127), written as fp32 (out_dtype
  * MXMOE_OUT_F32) or bf16 bits (MXMOE_OUT_BF16) into device memory out (rows, K).
  * Every finite result is exact in both types (subnormals included); results at or
- * beyond 2^128 are +-inf (scale bytes 253..255). Errors as mxfp4_quantize, plus
- * MXMOE_EUNSUPPORTED for an unknown out_dtype. */
+ * beyond 2^128 are +-inf (scale bytes 253..255). Errors as mxfp4_quantize (with blocks
+ * and out the pointers that must be 16-byte aligned), plus MXMOE_EUNSUPPORTED for an
+ * unknown out_dtype. */
 int mxfp4_dequantize(const uint8_t* blocks, const uint8_t* scales, int64_t rows, int64_t K,
                      void* out, int out_dtype, void* stream);
 
