@@ -41,3 +41,23 @@ def test_codec_reference_arm_runs_on_cpu_and_only_on_rank_0():
     assert res["impl"] == "reference" and res["metric"] == bench.CODEC_METRIC and res["unit"] == "GB/s"
     assert res["value"] > 0 and res["cpu_baseline"]["kind"] == "oracle"
     assert res["e2e"]["h2d_bytes_per_step"] == 0 and res["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_ncu_traffic_reads_the_matching_block_and_drops_stale_sources(tmp_path, monkeypatch):
+    import hashlib
+    (tmp_path / "profiles").mkdir()
+    src = tmp_path / "k.cu"
+    src.write_text("kernel source\n")
+    digest = hashlib.sha256(src.read_bytes()).hexdigest()[:16]
+    (tmp_path / "profiles" / "p.md").write_text(
+        "# summary\n\n"
+        "- workload: prefill\n- kernel: gate_up\n- traffic_bytes_per_launch: 123\n"
+        f"- source: k.cu sha256 prefix {digest}\n\n"
+        "- workload: prefill\n- kernel: down\n- traffic_bytes_per_launch: 45\n"
+        f"- source: k.cu sha256 prefix {digest}\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.ncu_traffic("prefill", "gate_up") == 123
+    assert bench.ncu_traffic("prefill", "down") == 45
+    assert bench.ncu_traffic("decode1", "gate_up") is None
+    src.write_text("kernel source, edited\n")          # the counters no longer describe it
+    assert bench.ncu_traffic("prefill", "gate_up") is None
