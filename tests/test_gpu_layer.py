@@ -165,6 +165,23 @@ def test_fp8_prefill_tcgen05_path(B, H, I, E, k, T):
     check_rows(B, p, d, rows, act_scale=s, out=out)
 
 
+@pytest.mark.parametrize("E,k,H,I,T,fp8", [
+    (1, 1, 64, 32, 5, False),        # one expert: every token routes to it with weight 1
+    (8, 8, 128, 96, 40, False),      # k = E: every expert selected, the routed path is the dense one
+    (8, 8, 128, 96, 40, True),
+    (256, 8, 256, 256, 200, False),  # the largest E and k the library takes
+    (256, 8, 256, 256, 200, True),   # 1600 routed pairs: the tcgen05 FP8 path, ~6 rows per expert
+    (16, 4, 32, 32, 70, False),      # the smallest contracting dims: one 32-value block
+])
+def test_degenerate_and_maximum_shapes(B, E, k, H, I, T, fp8):
+    lay = inputs.small_layer(E=E, k=k, T=T, H=H, I=I, seed=11, router_bias=True,
+                             router_std=1.0 / np.sqrt(H))
+    p = pack(lay)
+    d = to_device(p)
+    s = oracle.calibrate(p.x, p.router_w, p.router_b, *p.weights, k) if fp8 else None
+    check_rows(B, p, d, np.arange(T), act_scale=s)
+
+
 def _sample_rows(T, n, seed):
     rng = np.random.default_rng(seed)
     rows = np.sort(rng.choice(T, size=n, replace=False))
