@@ -92,11 +92,12 @@ struct Workspace {
   int smem_K = 0;      // largest K the expert kernels were configured for
   bool tc_ready = false;  // tcgen05 GEMM shared-memory limit raised
   bool dtc_ready = false; // tensor-core decode kernels' shared-memory limit raised
+  bool tcb_ready = false; // two-part (bf16 activation) tcgen05 GEMM's shared-memory limit raised
   size_t tickets_zeroed = 0;  // bytes at the start of the workspace known to be zero
 };
 
-// Routed pairs from which the FP8 path runs on the tcgen05 grouped GEMM (fewer pairs use
-// the register-dequant kernels). MXMOE_TC_MIN_PAIRS overrides it (0 = always when the
+// Routed pairs from which the prefill paths (FP8, and bf16 as two e4m3 parts) run on the
+// tcgen05 grouped GEMMs (fewer pairs use the tensor-core decode or register-dequant kernels). MXMOE_TC_MIN_PAIRS overrides it (0 = always when the
 // shapes allow, a huge value = never).
 int64_t tc_min_pairs() {
   static int64_t v = [] {
@@ -181,8 +182,11 @@ struct LayerBuffers {
   uint16_t* act_mid;   // (P, I) bf16 bits of the down-projection input
   float* y;            // (P, H) fp32 expert outputs
   unsigned* amax;      // 2 x fp32 bits (calibration)
-  uint8_t* a1;         // tcgen05 path: gate_up input rows grouped by expert, (P, H)
-  uint8_t* a2;         // tcgen05 path: down input rows, (P, I)
+  uint8_t* a1;         // tcgen05 path: gate_up input rows grouped by expert, (P, H); two-part
+                       // path: their e4m3 parts, (2, P, H)
+  uint8_t* a2;         // tcgen05 path: down input rows, (P, I); two-part path: (2, P, I)
+  uint8_t* sa1;        // two-part path: the parts' e8m0 scales, (2, P, H/32)
+  uint8_t* sa2;        // (2, P, I/32)
   uint8_t* xs;         // tensor-core decode: gate_up B rows (P*4, H/2) packed e2m1 parts
   uint8_t* sfb;        // their scale records
   uint8_t* xs_mid;     // down B rows (P*4, I/2)
@@ -193,8 +197,8 @@ struct LayerBuffers {
 };
 
 // n_rest: the tensor-core router's extra K-range partials of the logits (T x E each)
-size_t layout(int T, int E, int k, int H, int I, bool fp8, bool tc, bool dtc, int n_rest, LayerBuffers* b,
-              char* base) {
+size_t layout(int T, int E, int k, int H, int I, bool fp8, bool tc, bool tcb, bool dtc, int n_rest,
+              LayerBuffers* b, char* base) {
   const int64_t P = static_cast<int64_t>(T) * k;
   Carve c;
   size_t o_tickets = c.take<uint8_t>(kTicketBytes);
@@ -210,8 +214,10 @@ size_t layout(int T, int E, int k, int H, int I, bool fp8, bool tc, bool dtc, in
   size_t o_mid = c.take<uint16_t>(tc ? 0 : P * I);
   size_t o_y = c.take<float>(P * H);
   size_t o_amax = c.take<unsigned>(2);
-  size_t o_a1 = c.take<uint8_t>(tc ? P * H : 0);
-  size_t o_a2 = c.take<uint8_t>(tc ? P * I : 0);
+  size_t o_a1 = c.take<uint8_t>(tc ? P * H : tcb ? 2 * P * H : 0);
+  size_t o_a2 = c.take<uint8_t>(tc ? P * I : tcb ? 2 * P * I : 0);
+  size_t o_sa1 = c.take<uint8_t>(tcb ? 2 * P * (H / 32) : 0);
+  size_t o_sa2 = c.take<uint8_t>(tcb ? 2 * P * (I / 32) : 0);
   size_t o_xs = c.take<uint8_t>(dtc ? static_cast<int64_t>(mxmoe::decode_tc_xs_bytes(P, H)) : 0);
   size_t o_sfb = c.take<uint8_t>(dtc ? static_cast<int64_t>(mxmoe::decode_tc_sfb_row_bytes(E, T)) : 0);
   size_t o_xsm = c.take<uint8_t>(dtc ? static_cast<int64_t>(mxmoe::decode_tc_xs_bytes(P, I)) : 0);
@@ -239,6 +245,8 @@ size_t layout(int T, int E, int k, int H, int I, bool fp8, bool tc, bool dtc, in
     b->amax = reinterpret_cast<unsigned*>(base + o_amax);
     b->a1 = reinterpret_cast<uint8_t*>(base + o_a1);
     b->a2 = reinterpret_cast<uint8_t*>(base + o_a2);
+    b->sa1 = reinterpret_cast<uint8_t*>(base + o_sa1);
+    b->sa2 = reinterpret_cast<uint8_t*>(base + o_sa2);
     b->xs = reinterpret_cast<uint8_t*>(base + o_xs);
     b->sfb = reinterpret_cast<uint8_t*>(base + o_sfb);
     b->xs_mid = reinterpret_cast<uint8_t*>(base + o_xsm);
@@ -297,8 +305,12 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
   const int64_t P = static_cast<int64_t>(a.T) * a.k;
   const bool tc = fp8 && !calib_out && P >= tc_min_pairs() && std::max(a.H, a.I) / 32 <= kTcMaxNb &&
                   tc_gemm_supported(a.H, a.I, a.gu_blocks, a.d_blocks, a.gu_scales, a.d_scales);
-  const bool dtc = !tc && !calib_out && decode_tc_supported(a.H, a.I, a.T, a.gu_blocks, a.d_blocks, a.gu_scales,
-                                                             a.d_scales);
+  // bf16 activations with many routed pairs: the same GEMMs with each activation as two
+  // e4m3 parts (exact for the activations' significant bits)
+  const bool tcb = !fp8 && !calib_out && P >= tc_min_pairs() && std::max(a.H, a.I) / 32 <= kTcMaxNb &&
+                   tc_gemm_supported(a.H, a.I, a.gu_blocks, a.d_blocks, a.gu_scales, a.d_scales);
+  const bool dtc = !tc && !tcb && !calib_out &&
+                   decode_tc_supported(a.H, a.I, a.T, a.gu_blocks, a.d_blocks, a.gu_scales, a.d_scales);
   // routing: one fused launch for small batches; else the router GEMM (on the tensor cores
   // when the shapes allow, split over K ranges) and a top-k kernel that adds the ranges
   const bool small = route_small_supported(a.T, a.E, a.k);
@@ -306,7 +318,7 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
                          ? router_tc_ksplit(a.T, a.H, ws->sms)
                          : 0;
   const int n_rest = ksplit > 1 ? ksplit - 1 : 0;
-  const size_t need = layout(a.T, a.E, a.k, a.H, a.I, fp8, tc, dtc, n_rest, nullptr, nullptr);
+  const size_t need = layout(a.T, a.E, a.k, a.H, a.I, fp8, tc, tcb, dtc, n_rest, nullptr, nullptr);
   if (int rc = ensure_capacity(ws, need)) return rc;
   if (std::max(a.H, a.I) > ws->smem_K) {
     cudaError_t e = expert_mma_set_smem_limits(std::max(a.H, a.I));
@@ -318,13 +330,18 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (tcgen05 GEMM)");
     ws->tc_ready = true;
   }
+  if (tcb && !ws->tcb_ready) {
+    cudaError_t e = tc_parts_gemm_prepare(256);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (two-part tcgen05 GEMM)");
+    ws->tcb_ready = true;
+  }
   if (dtc && !ws->dtc_ready) {
     cudaError_t e = decode_tc_prepare();
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (tensor-core decode)");
     ws->dtc_ready = true;
   }
   LayerBuffers b;
-  layout(a.T, a.E, a.k, a.H, a.I, fp8, tc, dtc, n_rest, &b, ws->base);
+  layout(a.T, a.E, a.k, a.H, a.I, fp8, tc, tcb, dtc, n_rest, &b, ws->base);
   // The decode path's tickets follow the fixed ticket block, where other layouts keep
   // ordinary buffers: they are known to be zero only after a decode-path call, which
   // leaves them at zero. Clear them when that is not known.
@@ -379,6 +396,33 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
     if ((e = launch_tc_gemm(false, b.a2, P, a.I, a.d_blocks, a.d_scales, a.d_bias, a.E, a.H, b.offsets, s1, 0.0f,
                             nullptr, b.y, ws->err, ws->sms, st)))
       return cuda_fail(e, "down (tcgen05)");
+    ++launches;
+    tm.mark("down");
+    if ((e = launch_combine(b.y, b.topk_idx, b.topk_w, b.inv, a.T, a.H, a.k, out, st, ws->sms)))
+      return cuda_fail(e, "combine");
+    ++launches;
+    tm.mark("combine");
+    t_last_launches = launches;
+    return MXMOE_OK;
+  }
+  if (tcb) {
+    // bf16 activations as two e4m3 parts per value (block scales as the MMA's A scales)
+    if ((e = launch_split_parts(a.x, b.perm_token, a.T, P, a.H, b.a1, b.sa1, ws->sms, st)))
+      return cuda_fail(e, "activation split");
+    ++launches;
+    tm.mark("act_split");
+    if ((e = launch_tc_parts_gemm(true, b.a1, b.sa1, P, a.H, a.gu_blocks, a.gu_scales, a.gu_bias, a.E, a.I,
+                                  b.offsets, b.act_mid, nullptr, ws->err, ws->sms, st)))
+      return cuda_fail(e, "gate_up (tcgen05, two parts)");
+    ++launches;
+    tm.mark("gate_up");
+    if ((e = launch_split_parts(b.act_mid, nullptr, a.T, P, a.I, b.a2, b.sa2, ws->sms, st)))
+      return cuda_fail(e, "intermediate split");
+    ++launches;
+    tm.mark("mid_split");
+    if ((e = launch_tc_parts_gemm(false, b.a2, b.sa2, P, a.I, a.d_blocks, a.d_scales, a.d_bias, a.E, a.H,
+                                  b.offsets, nullptr, b.y, ws->err, ws->sms, st)))
+      return cuda_fail(e, "down (tcgen05, two parts)");
     ++launches;
     tm.mark("down");
     if ((e = launch_combine(b.y, b.topk_idx, b.topk_w, b.inv, a.T, a.H, a.k, out, st, ws->sms)))

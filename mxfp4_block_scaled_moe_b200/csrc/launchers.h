@@ -71,6 +71,16 @@ cudaError_t launch_tc_gemm(bool gate_up, const uint8_t* a, int64_t P_rows, int K
                            float s_in, float s_out, uint8_t* a_out, float* y_out, int* err, int sms,
                            cudaStream_t st);
 
+// bf16 activations on the tcgen05 grouped GEMM: each activation row as two e4m3 parts with
+// e8m0 scales per 32-value block (csrc/gemm_bf16_sm100.cu)
+cudaError_t launch_split_parts(const uint16_t* src, const int32_t* perm, int T, int64_t P, int K, uint8_t* parts,
+                               uint8_t* scales, int sms, cudaStream_t st);
+cudaError_t tc_parts_gemm_prepare(int E);
+cudaError_t launch_tc_parts_gemm(bool gate_up, const uint8_t* parts, const uint8_t* a_scales, int64_t P_rows, int K,
+                                 const uint8_t* blocks, const uint8_t* scales, const float* bias, int E, int n_out,
+                                 const int32_t* offsets, uint16_t* a_out, float* y_out, int* err, int sms,
+                                 cudaStream_t st);
+
 struct DecodeGemmArgs {   // tensor-core decode path (kind::mxf4: packed e2m1 weights x e2m1 token parts)
   const uint8_t* gu_blocks;
   const uint8_t* gu_scales;

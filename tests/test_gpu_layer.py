@@ -182,6 +182,30 @@ def test_degenerate_and_maximum_shapes(B, E, k, H, I, T, fp8):
     check_rows(B, p, d, np.arange(T), act_scale=s)
 
 
+@pytest.mark.parametrize("H,I,E,k,T", [(512, 512, 8, 2, 600), (320, 320, 8, 3, 600),
+                                       (2880, 2880, 6, 4, 300)])
+def test_bf16_prefill_two_part_tcgen05_path(B, H, I, E, k, T):
+    """T*k >= 1024 routed pairs with bf16 activations run the tcgen05 grouped GEMMs with each
+    activation split into two e4m3 parts: K a multiple of 128, K with a 64-value tail,
+    partial N tiles, ragged expert loads."""
+    lay = inputs.small_layer(E=E, k=k, T=T, H=H, I=I, seed=7, router_bias=True,
+                             router_std=1.0 / np.sqrt(H))
+    p = pack(lay)
+    d = to_device(p)
+    out = run_gpu(B, d, k)
+    rows = np.arange(T) if H <= 512 else _sample_rows(T, 24, 3)
+    check_rows(B, p, d, rows, out=out)
+
+
+def test_prefill_120b_shape_bf16_sampled(B):
+    lay = inputs.prefill_layer(T=4096, E=128, device="cuda")
+    p, d = layer_case(lay)
+    out1 = run_gpu(B, d, lay.k)
+    out2 = run_gpu(B, d, lay.k)
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))   # run-to-run identical
+    check_rows(B, p, d, _sample_rows(4096, 24, 4), out=out1)
+
+
 def _sample_rows(T, n, seed):
     rng = np.random.default_rng(seed)
     rows = np.sort(rng.choice(T, size=n, replace=False))
