@@ -236,6 +236,26 @@ def algorithmic_work(lay, idx):
     return dict(bytes=bytes_, flops=flops, distinct=distinct, gu_bytes=gu_bytes, gu_flops=gu_flops)
 
 
+NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "fp8_tflops": 4500.0, "bf16_tflops": 2250.0}
+
+
+def step_roofline(bytes_, flops, ms_per_step, pk, fp8):
+    """The whole step against the slower of its two bounds: algorithmic bytes over the HBM
+    bandwidth and algorithmic FLOPs over the tensor peak (FP8 with FP8 activations, else
+    bf16), with the measured peaks (the FP8 one as 2x the measured bf16) and the nominal
+    ones. frac = that bound's time / the measured step time."""
+    meas_t = pk.get("bf16_tflops_sustained", pk["bf16_tflops"]) * (2.0 if fp8 else 1.0)
+    nom_t = NOMINAL_PEAKS["fp8_tflops" if fp8 else "bf16_tflops"]
+    out = {}
+    for name, bw, tp in (("measured", pk["hbm_gbs"], meas_t), ("nominal", NOMINAL_PEAKS["hbm_gbs"], nom_t)):
+        t_mem = bytes_ / (bw * 1e9) * 1e3
+        t_fl = flops / (tp * 1e12) * 1e3
+        t = max(t_mem, t_fl)
+        out[name] = {"bound": "hbm" if t_mem >= t_fl else "tensor", "hbm_gbs": bw, "tensor_tflops": tp,
+                     "t_bound_ms": round(t, 5), "frac": round(t / ms_per_step, 4)}
+    return out
+
+
 # ------------------------------------------------------------- CPU baseline -----
 
 def oracle_tokens_per_s(lay, d, act, budget_s, host_weights=None):
@@ -419,6 +439,7 @@ def run_ours(args, world, rank):
                    "l2": "flushed before every timed step (512 MiB write, then a 256 MiB read)",
                    "parallelism": f"replicas x{world}"},
         "roofline": roofline,
+        "step_roofline": step_roofline(work["bytes"], work["flops"], ms_per_step, pk, fp8),
         "stages_ms_per_step": {s: round(v[0] / max(v[1], 1), 5) for s, v in stages.items()},
         "algorithmic": {"bytes_per_step": work["bytes"], "flops_per_step": work["flops"],
                         "distinct_experts": work["distinct"]},
