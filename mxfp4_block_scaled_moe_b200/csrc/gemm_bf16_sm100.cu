@@ -12,7 +12,8 @@
 // of x's ulp no larger than half of part 1's ulp, i.e. at most 4 significant bits, and
 // part 2 = e4m3(r / 2^s2) with s2 = floor(log2(max |r|)) - 7 holds it exactly wherever it
 // lies in e4m3's range under s2. So the two parts reproduce every element down to about
-// 2^-14 of its block's maximum exactly, and smaller ones to within 2^(s2 - 10). Both parts
+// 2^-14 of its block's maximum exactly, and smaller ones to within max(2^(s2 - 10),
+// 2^(s1 - 14)), about 2^-21 of the block's maximum. Both parts
 // are A operands of kind::mxf8f6f4 block-scaled MMAs with their e8m0 bytes as the A scale
 // factors, accumulating into one fp32 accumulator: the MMA sees x * w exactly (up to the
 // tiny elements above), at twice the FP8 path's MMA count (the bf16 MMA rate).
