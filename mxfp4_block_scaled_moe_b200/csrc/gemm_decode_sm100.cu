@@ -9,10 +9,11 @@
 //   A = 128 weight rows (gate_up: 128 gate rows and, in a second MMA, the 128 matching up
 //       rows; down: 128 rows of down_proj) with the checkpoint's e8m0 scales;
 //   B = the routed token rows as four MXFP4 "parts" each: p1 = e2m1(x / 2^s1), p2 the same
-//       on the residual x - p1, and so on, each s chosen from its 32-value block's largest
-//       residual so that nothing saturates. Every part keeps about two more bits of the
-//       block, and four parts reproduce a bf16 row to about 1e-5 of a dot product's size
-//       (the per-tensor FP8 path splits the e4m3 value of x / s0 the same way).
+//       on the residual x - p1, and so on, each s chosen from its group's largest residual
+//       (the whole row for gate_up's input, each 32-value block for down's) so that nothing
+//       saturates. Every part removes about three bits of the residual, and four parts
+//       change a 2880-long dot product by about 2e-4 of the largest output (the
+//       per-tensor FP8 path splits the e4m3 value of x / s0 the same way).
 //   D = 128 x N fp32 in tensor memory, N = 4 * rows rounded up to 16; the epilogue adds a
 //       token's four columns.
 // Why not FP8 tokens against FP4 weights (kind::mxf8f6f4): a block-scaled MMA costs the
