@@ -206,6 +206,19 @@ def test_prefill_120b_shape_bf16_sampled(B):
     check_rows(B, p, d, _sample_rows(4096, 24, 4), out=out1)
 
 
+@pytest.mark.skip(reason="H != I on the tensor-core paths has not run on a GPU yet")
+@pytest.mark.parametrize("T,fp8", [(400, True), (400, False), (8, False), (8, True)])
+def test_tensor_core_paths_with_H_ne_I(B, T, fp8):
+    """H = 320 (2.5 k-tiles of 128), I = 192 (1.5): 1600 routed pairs take the tcgen05
+    prefill GEMMs (FP8, or bf16 as two e4m3 parts), T = 8 the tensor-core decode GEMMs."""
+    lay = inputs.small_layer(E=8, k=4, T=T, H=320, I=192, seed=13, router_bias=True,
+                             router_std=1.0 / np.sqrt(320))
+    p = pack(lay)
+    d = to_device(p)
+    s = oracle.calibrate(p.x, p.router_w, p.router_b, *p.weights, p.lay.k) if fp8 else None
+    check_rows(B, p, d, np.arange(T), act_scale=s)
+
+
 def _sample_rows(T, n, seed):
     rng = np.random.default_rng(seed)
     rows = np.sort(rng.choice(T, size=n, replace=False))
