@@ -1,13 +1,19 @@
 """Benchmark of the MXFP4 MoE expert layer on B200 (one JSON line on rank 0).
 
 A step is one moe_mxfp4_forward over one batch of synthetic tokens: router + top-k,
-permute, expert gate_up + SwiGLU, down, weighted combine. Default workload: the
-120B-shaped prefill layer with FP8 activations (E=128, top-4, H=I=2880, T=4096, static
-per-tensor scales from a 256-token calibration batch). Other workloads (--workload):
-decode1/decode8/decode64 (20B shape, E=32, bf16 activations), zipf (T=16384, skewed
-routing), prefill_bf16 (the prefill layer with bf16 activations), codec (the standalone MXFP4 codec over the 120B-shaped expert set: a step is
-one quantize of all gate_up + down weights from fp32 and one dequantize each to bf16 and
-fp32; metric GB/s of algorithmic bytes).
+permute, expert gate_up + SwiGLU, down, weighted combine. Default workload (the line's
+`value`): the largest single-GPU configuration, the 120B-shaped prefill layer with
+Zipf(1.1)-skewed routing and FP8 activations (E=128, top-4, H=I=2880, T=16384, static
+per-tensor scales from a 256-token calibration batch). In the same run, under
+`other_configs`, the 120B prefill at T=4096 (uniform routing) and the 20B decode batches
+T=1/8/64 (E=32, bf16 activations), each with its own step time, stage times, rooflines
+and clocks. Other workloads (--workload): prefill, decode1/decode8/decode64,
+prefill_bf16 (the prefill layer with bf16 activations), codec (the standalone MXFP4 codec
+over the 120B-shaped expert set: a step is one quantize of all gate_up + down weights
+from fp32 and one dequantize each to bf16 and fp32; metric GB/s of algorithmic bytes).
+
+The FP8 tensor roofline divides by this GPU's measured rate for the MMA the prefill
+GEMMs issue (the library's kind::mxf8f6f4 rate probe, run at the start of the bench).
 
 Metric: MoE-layer tokens/s (whole job = sum over ranks). Inputs are resident in HBM
 when the timed region starts; L2 is flushed before every timed step, outside the step's
@@ -58,6 +64,11 @@ WORKLOADS = {
     "decode64": (lambda dev: inputs.decode_layer(T=64, E=32, device=dev), False),
 }
 CODEC = "codec"
+# The default line: the largest single-GPU configuration (120B-shaped prefill, T = 16384,
+# Zipf-skewed routing), then the 120B prefill at T = 4096 and the 20B decode batches
+# measured in the same run.
+DEFAULT_WORKLOAD = "zipf"
+DEFAULT_EXTRAS = ("prefill", "decode1", "decode8", "decode64")
 
 PER_EXPERT_PACKED = lambda H, I: 2 * I * H // 2 + 2 * I * H // 32 + H * I // 2 + H * I // 32
 
@@ -142,23 +153,74 @@ def job_tokens_per_s(tokens_per_rank_step: int, world: int, steps: int, max_ms: 
 
 # ----------------------------------------------------------------------- setup ----
 
-def build_layer(name, device):
+def tensor_peak(B, seconds=1.0):
+    """The FP8 block-scaled MMA rate of this GPU, measured with the library's rate probe
+    (kind::mxf8f6f4, E4M3 x E2M1, M = 128, K = 32, one CTA per SM, operands resident in
+    shared memory): `burst` = one ~10 ms launch on a GPU that has idled for a moment,
+    `sustained` = the last second of back-to-back launches (the power cap's clock), both
+    for N = 256, plus the prefill GEMM's own pattern (N = 240 with one scale-factor copy
+    per four MMAs) at the sustained clock. TFLOP/s."""
+    stream = torch.cuda.current_stream()
+    B.mxmoe_tc_rate_probe(256, False, 100)            # load the kernel
+    torch.cuda.synchronize()
+    time.sleep(0.5)
+
+    def timed(n, copy, iters):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        f = B.mxmoe_tc_rate_probe(n, copy, iters)
+        e1.record(stream)
+        return f, e0, e1
+
+    f, e0, e1 = timed(256, False, 20000)
+    torch.cuda.synchronize()
+    burst = f / (e0.elapsed_time(e1) / 1e3) / 1e12
+    t_end = time.perf_counter() + seconds
+    runs = []
+    while time.perf_counter() < t_end:
+        runs.append(timed(256, False, 20000))
+        torch.cuda.synchronize()
+    last = runs[-5:]
+    sustained = sum(r[0] for r in last) / (sum(r[1].elapsed_time(r[2]) for r in last) / 1e3) / 1e12
+    f, e0, e1 = timed(240, True, 20000)
+    torch.cuda.synchronize()
+    pattern = f / (e0.elapsed_time(e1) / 1e3) / 1e12
+    B.mxmoe_check()
+    return {"peak_tflops": round(max(burst, sustained), 1),
+            "burst_tflops": round(burst, 1), "sustained_tflops": round(sustained, 1),
+            "n240_with_scale_copy_tflops": round(pattern, 1),
+            "probe": "tcgen05.mma kind::mxf8f6f4 block_scale, E4M3 x E2M1, M=128 N=256 K=32, "
+                     "one CTA per SM, operands in shared memory"}
+
+
+def layer_weights(lay, device, cache):
+    """MXFP4 expert weights of a synthetic layer, quantized by the library's own kernel
+    (cached per (E, H, I, seed): the prefill and Zipf layers share their experts)."""
+    from mxfp4_block_scaled_moe_b200 import binding as B
+    key = (lay.E, lay.H, lay.I, lay.seed)
+    if key not in cache:
+        E, H, I = lay.E, lay.H, lay.I
+        gu_b = torch.empty(E, 2 * I, H // 2, dtype=torch.uint8, device=device)
+        gu_s = torch.empty(E, 2 * I, H // 32, dtype=torch.uint8, device=device)
+        d_b = torch.empty(E, H, I // 2, dtype=torch.uint8, device=device)
+        d_s = torch.empty(E, H, I // 32, dtype=torch.uint8, device=device)
+        for e in range(E):   # weights: fp32 draws quantized by the library's own kernel
+            B.mxfp4_quantize(lay.gate_up(e), gu_b[e], gu_s[e])
+            B.mxfp4_quantize(lay.down(e), d_b[e], d_s[e])
+        cache[key] = (gu_b, gu_s, d_b, d_s)
+    return cache[key]
+
+
+def build_layer(name, device, cache=None):
     from mxfp4_block_scaled_moe_b200 import binding as B
     make, fp8 = WORKLOADS[name]
     lay = make(device)
-    E, H, I = lay.E, lay.H, lay.I
-    gu_b = torch.empty(E, 2 * I, H // 2, dtype=torch.uint8, device=device)
-    gu_s = torch.empty(E, 2 * I, H // 32, dtype=torch.uint8, device=device)
-    d_b = torch.empty(E, H, I // 2, dtype=torch.uint8, device=device)
-    d_s = torch.empty(E, H, I // 32, dtype=torch.uint8, device=device)
-    for e in range(E):   # weights: fp32 draws quantized by the library's own kernel
-        B.mxfp4_quantize(lay.gate_up(e), gu_b[e], gu_s[e])
-        B.mxfp4_quantize(lay.down(e), d_b[e], d_s[e])
+    gu_b, gu_s, d_b, d_s = layer_weights(lay, device, {} if cache is None else cache)
     d = dict(x=lay.x, router_w=lay.router_w, router_b=lay.router_b, gu_blocks=gu_b,
              gu_scales=gu_s, gu_bias=lay.gu_bias, d_blocks=d_b, d_scales=d_s, d_bias=lay.d_bias)
     act = None
     if fp8:
-        xc = inputs.calibration_x(H=H, device=device)
+        xc = inputs.calibration_x(H=lay.H, device=device)
         act = B.moe_mxfp4_calibrate(xc, lay.router_w, lay.router_b, gu_b, gu_s, lay.gu_bias,
                                     d_b, d_s, lay.d_bias, lay.k).cpu().tolist()
     torch.cuda.synchronize()
@@ -176,6 +238,7 @@ class ClockSampler:
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
@@ -239,12 +302,17 @@ def algorithmic_work(lay, idx):
 NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "fp8_tflops": 4500.0, "bf16_tflops": 2250.0}
 
 
-def step_roofline(bytes_, flops, ms_per_step, pk, fp8):
+def step_roofline(bytes_, flops, ms_per_step, pk, fp8, fp8_peak=None):
     """The whole step against the slower of its two bounds: algorithmic bytes over the HBM
     bandwidth and algorithmic FLOPs over the tensor peak (FP8 with FP8 activations, else
-    bf16), with the measured peaks (the FP8 one as 2x the measured bf16) and the nominal
-    ones. frac = that bound's time / the measured step time."""
-    meas_t = pk.get("bf16_tflops_sustained", pk["bf16_tflops"]) * (2.0 if fp8 else 1.0)
+    bf16), with the measured peaks and the nominal ones. The measured FP8 peak is the rate
+    probe's (fp8_peak, TFLOP/s); without it, 2x the measured bf16 peak (the nominal
+    fp8/bf16 ratio). The measured bf16 peak is the burst figure. frac = that bound's time /
+    the measured step time."""
+    if fp8:
+        meas_t = fp8_peak if fp8_peak else pk["bf16_tflops"] * 2.0
+    else:
+        meas_t = pk["bf16_tflops"]
     nom_t = NOMINAL_PEAKS["fp8_tflops" if fp8 else "bf16_tflops"]
     out = {}
     for name, bw, tp in (("measured", pk["hbm_gbs"], meas_t), ("nominal", NOMINAL_PEAKS["hbm_gbs"], nom_t)):
@@ -279,15 +347,67 @@ def oracle_tokens_per_s(lay, d, act, budget_s, host_weights=None):
 
 # ------------------------------------------------------------------------ main ----
 
-def run_ours(args, world, rank):
-    from mxfp4_block_scaled_moe_b200 import binding as B
-    pk, pk_kind = peaks()
-    lay, d, act = build_layer(args.workload, "cuda")
+class L2Flush:
+    """Evicts L2 between timed steps: a 512 MiB write, then a 256 MiB read that leaves L2
+    holding clean lines of an unrelated buffer (so a step does not pay the flush's
+    write-back)."""
+
+    def __init__(self):
+        self.flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+        self.clean = torch.zeros(32 << 20, dtype=torch.int64, device="cuda")     # 256 MiB
+        self.clean_sum = torch.empty((), dtype=torch.int64, device="cuda")
+
+    def __call__(self, i):
+        self.flush.fill_(i & 0xFF)
+        torch.sum(self.clean, dim=0, out=self.clean_sum)
+
+
+def kernel_roofline(name, lay, work, stages, act, pk, pk_kind, tpk):
+    """The dominant kernel (the largest stage other than routing, casts and combine)
+    against its bound: tensor FLOPs at prefill sizes, packed-weight HBM bytes at decode."""
+    small = ("router", "topk", "router+topk", "route", "permute", "act_quant", "act_quant+scatter", "act_split",
+             "mid_split", "combine")
+    dom = max((s for s in stages if s not in small), key=lambda s: stages[s][0], default=None)
+    if dom is None:
+        dom = max(stages, key=lambda s: stages[s][0])
+    dom_ms = stages[dom][0] / max(stages[dom][1], 1)
+    fp8 = act is not None
+    extra = {}
+    if lay.T >= 1024:
+        bound, unit = "tensor", "TFLOP/s"
+        flops = work["gu_flops"] if dom == "gate_up" else work["flops"] - work["gu_flops"]
+        achieved = flops / (dom_ms / 1e3) / 1e12
+        if fp8 and tpk:
+            peak = tpk["peak_tflops"]
+            peak_note = "measured kind::mxf8f6f4 rate probe (this run, this GPU): the larger of burst and sustained"
+            extra = {"frac_of_nominal_fp8": round(achieved / NOMINAL_PEAKS["fp8_tflops"], 4)}
+        elif fp8:
+            peak = pk["bf16_tflops"] * 2.0
+            peak_note = f"{pk_kind} bf16 burst x 2 (nominal fp8/bf16 ratio)"
+        else:
+            # bf16 activations: a bf16 contraction (run as two e4m3 parts, the bf16 MMA rate)
+            peak = pk["bf16_tflops"]
+            peak_note = f"{pk_kind} bf16 burst (cuBLAS)"
+            extra = {"frac_of_nominal_bf16": round(achieved / NOMINAL_PEAKS["bf16_tflops"], 4)}
+    else:
+        bound, unit = "hbm", "GB/s"
+        peak = pk["hbm_gbs"]
+        b = work["gu_bytes"] if dom == "gate_up" else work["bytes"] - work["gu_bytes"]
+        achieved = b / (dom_ms / 1e3) / 1e9
+        peak_note = f"{pk_kind} hbm copy"
+        extra = {"frac_of_nominal_hbm": round(achieved / NOMINAL_PEAKS["hbm_gbs"], 4)}
+    r = {"bound": bound, "kernel": dom, "achieved": round(achieved, 2), "peak": peak,
+         "unit": unit, "frac": round(achieved / peak, 4), "traffic": ncu_traffic(name, dom),
+         "peak_source": peak_note, "kernel_ms": round(dom_ms, 5)}
+    r.update(extra)
+    return r
+
+
+def measure_layer(B, name, lay, d, act, args, world, flusher, pk, pk_kind, tpk, with_e2e):
+    """Device-timed steps of one workload (K steps in one CUDA graph, L2 flushed before
+    each), per-stage times, rooflines, clocks; with_e2e adds the end-to-end leg."""
     k, T, H = lay.k, lay.T, lay.H
     out = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
-    clean = torch.zeros(32 << 20, dtype=torch.int64, device="cuda")     # 256 MiB
-    clean_sum = torch.empty((), dtype=torch.int64, device="cuda")
     stream = torch.cuda.current_stream()
     idx, _ = B.moe_route_topk(d["x"], d["router_w"], d["router_b"], k)
     work = algorithmic_work(lay, idx.cpu().numpy())
@@ -298,8 +418,7 @@ def run_ours(args, world, rank):
     launches_per_step = B.mxmoe_last_launch_count()
 
     # ---- device-resident timed region: the K steps are captured into one CUDA graph as
-    # [L2 flush, event, forward, event] x K and replayed once; the library records its
-    # per-stage events inside the same graph.
+    # [L2 flush, event, forward, event] x K and replayed once
     ev = [(torch.cuda.Event(enable_timing=True, external=True),
            torch.cuda.Event(enable_timing=True, external=True)) for _ in range(args.steps)]
     graph = torch.cuda.CUDAGraph()
@@ -311,8 +430,7 @@ def run_ours(args, world, rank):
     B.mxmoe_profile_enable(args.stage_events_in_timed_graph)
     with torch.cuda.graph(graph, stream=side):
         for i in range(args.steps):
-            flush.fill_(i & 0xFF)                # evict L2 by writing 512 MiB ...
-            torch.sum(clean, dim=0, out=clean_sum)   # ... then refill it with clean lines
+            flusher(i)
             ev[i][0].record()
             forward(B, d, k, act, out)
             ev[i][1].record()
@@ -338,9 +456,49 @@ def run_ours(args, world, rank):
     value = job_tokens_per_s(T, world, args.steps, total_ms)
     del graph
 
-    # ---- end to end through the C ABI with host buffers, double-buffered: the copy of the
-    # next step's tokens in and of the previous step's output out run on their own streams
-    # beside the current step's forward; every step's two copies are inside the timed region
+    e2e = None
+    if with_e2e:
+        e2e = e2e_leg(B, d, k, act, out, args, world)
+    if not stages:   # stage times from an instrumented replay of the same graph shape
+        B.mxmoe_profile_enable(True)
+        g2 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g2, stream=side):
+            for i in range(args.steps):
+                flusher(i)
+                forward(B, d, k, act, out)
+        torch.cuda.synchronize()
+        g2.replay()
+        torch.cuda.synchronize()
+        stages = B.mxmoe_profile_read()
+        B.mxmoe_profile_enable(False)
+        del g2
+    fp8 = act is not None
+    res = {
+        "value": round(value, 1), "ms_per_step": round(ms_per_step, 5),
+        "roofline": kernel_roofline(name, lay, work, stages, act, pk, pk_kind, tpk),
+        "step_roofline": step_roofline(work["bytes"], work["flops"], ms_per_step, pk, fp8,
+                                       tpk["peak_tflops"] if (fp8 and tpk) else None),
+        "stages_ms_per_step": {s: round(v[0] / max(v[1], 1), 5) for s, v in stages.items()},
+        "algorithmic": {"bytes_per_step": work["bytes"], "flops_per_step": work["flops"],
+                        "distinct_experts": work["distinct"]},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+        "config": {"workload": f"{name}: {lay.name}", "E": lay.E, "k": k, "T": T,
+                   "H": H, "I": lay.I, "activations": "fp8_e4m3 static" if fp8 else "bf16",
+                   "l2": "flushed before every timed step (512 MiB write, then a 256 MiB read)",
+                   "parallelism": f"replicas x{world}"},
+    }
+    if e2e is not None:
+        res["e2e"] = e2e
+    return res
+
+
+def e2e_leg(B, d, k, act, out, args, world):
+    """End to end through the C ABI with host buffers, double-buffered: the copy of the
+    next step's tokens in and of the previous step's output out run on their own streams
+    beside the current step's forward; every step's two copies are inside the timed region."""
+    T, H = d["x"].shape
+    stream = torch.cuda.current_stream()
     x_host = d["x"].cpu().pin_memory()
     out_host = [torch.empty(T, H, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
     x_dev = [torch.empty_like(d["x"]) for _ in range(2)]
@@ -380,85 +538,56 @@ def run_ours(args, world, rank):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    e2e_value = job_tokens_per_s(T, world, args.steps, e2e_ms)
+    return {"value": round(job_tokens_per_s(T, world, args.steps, e2e_ms), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2,
+            "timing": "steps back to back, copies double-buffered on their own streams, L2 not "
+                      "flushed between steps (the routed experts' weights of a small batch can "
+                      "stay in L2)"}
 
-    if not stages:   # stage times from an instrumented replay of the same graph shape
-        B.mxmoe_profile_enable(True)
-        g2 = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g2, stream=side):
-            for i in range(args.steps):
-                flush.fill_(i & 0xFF)
-                torch.sum(clean, dim=0, out=clean_sum)
-                forward(B, d, k, act, out)
-        torch.cuda.synchronize()
-        g2.replay()
-        torch.cuda.synchronize()
-        stages = B.mxmoe_profile_read()
-        B.mxmoe_profile_enable(False)
-        del g2
-    # ---- roofline of the dominant kernel
-    small = ("router", "topk", "router+topk", "route", "permute", "act_quant", "act_quant+scatter", "act_split",
-             "mid_split", "combine")
-    dom = max((s for s in stages if s not in small),
-              key=lambda s: stages[s][0], default=None)
-    if dom is None:
-        dom = max(stages, key=lambda s: stages[s][0])
-    dom_ms = stages[dom][0] / max(stages[dom][1], 1)
+
+def run_ours(args, world, rank):
+    from mxfp4_block_scaled_moe_b200 import binding as B
+    pk, pk_kind = peaks()
+    cache = {}
+    tpk = tensor_peak(B) if not args.no_tc_probe else None
+    flusher = L2Flush()
+    lay, d, act = build_layer(args.workload, "cuda", cache)
+    head = measure_layer(B, args.workload, lay, d, act, args, world, flusher, pk, pk_kind, tpk, True)
     fp8 = act is not None
-    if lay.T >= 1024:
-        bound, unit = "tensor", "TFLOP/s"
-        if fp8:
-            # FP8 dense peak = measured bf16 peak x the nominal fp8/bf16 ratio (4.5 / 2.25 = 2)
-            peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"]) * 2.0
-            peak_note = f"{pk_kind} bf16 sustained x 2 (nominal fp8/bf16 ratio)"
-        else:
-            # bf16 activations: a bf16 contraction (run as two e4m3 parts, the bf16 MMA rate)
-            peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
-            peak_note = f"{pk_kind} bf16 sustained"
-        flops = work["gu_flops"] if dom == "gate_up" else work["flops"] - work["gu_flops"]
-        achieved = flops / (dom_ms / 1e3) / 1e12
-    else:
-        bound, unit = "hbm", "GB/s"
-        peak = pk["hbm_gbs"]
-        b = work["gu_bytes"] if dom == "gate_up" else work["bytes"] - work["gu_bytes"]
-        achieved = b / (dom_ms / 1e3) / 1e9
-        peak_note = f"{pk_kind} hbm copy"
-    traffic = ncu_traffic(args.workload, dom)
-    roofline = {"bound": bound, "kernel": dom, "achieved": round(achieved, 2), "peak": peak,
-                "unit": unit, "frac": round(achieved / peak, 4), "traffic": traffic,
-                "peak_source": peak_note, "kernel_ms": round(dom_ms, 5)}
-
     res = {
-        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3 x e2m1 -> f32" if fp8 else "bf16 x e2m1 -> f32",
         "data": "synthetic (seeded; weights N(0,0.02) quantized to MXFP4 on the GPU)",
-        "config": {"workload": f"{args.workload}: {lay.name}", "E": lay.E, "k": k, "T": T,
-                   "H": H, "I": lay.I, "activations": "fp8_e4m3 static" if fp8 else "bf16",
-                   "l2": "flushed before every timed step (512 MiB write, then a 256 MiB read)",
-                   "parallelism": f"replicas x{world}"},
-        "roofline": roofline,
-        "step_roofline": step_roofline(work["bytes"], work["flops"], ms_per_step, pk, fp8),
-        "stages_ms_per_step": {s: round(v[0] / max(v[1], 1), 5) for s, v in stages.items()},
-        "algorithmic": {"bytes_per_step": work["bytes"], "flops_per_step": work["flops"],
-                        "distinct_experts": work["distinct"]},
-        "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
-                "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2,
-                "timing": "steps back to back, copies double-buffered on their own streams, L2 not "
-                          "flushed between steps (the routed experts' weights of a small batch can "
-                          "stay in L2)"},
-        "gpu_launches": launches_per_step * args.steps,
+        "config": head["config"],
+        "roofline": head["roofline"],
+        "step_roofline": head["step_roofline"],
+        "stages_ms_per_step": head["stages_ms_per_step"],
+        "algorithmic": head["algorithmic"],
+        "e2e": head["e2e"],
+        "gpu_launches": head["gpu_launches"],
         "timing": "K steps captured in one CUDA graph (flush, forward) and replayed once; "
                   "stage times from a replay of the same graph with per-stage events",
+        "clocks": head["clocks"],
     }
-    res["clocks"] = clk.summary()
+    if tpk:
+        res["tensor_peak_probe"] = tpk
+    extras = [w for w in args.extra.split(",") if w and w != args.workload] if args.extra else []
+    if extras:
+        res["other_configs"] = {}
+        for name in extras:
+            lay2, d2, act2 = build_layer(name, "cuda", cache)
+            r = measure_layer(B, name, lay2, d2, act2, args, world, flusher, pk, pk_kind, tpk, False)
+            r["metric"], r["unit"] = METRIC, "tokens/s"
+            res["other_configs"][name] = r
+            del lay2, d2
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, n, dt, _ = oracle_tokens_per_s(lay, d, act, args.cpu_budget)
         import oracle
         res["cpu_baseline"] = {"value": round(v, 4), "unit": "tokens/s",
                                "cores": oracle.num_threads(), "kind": "oracle",
-                               "sample": f"first {n} of {T} tokens of the same workload, {dt:.1f} s"}
+                               "sample": f"first {n} of {lay.T} tokens of the same workload, {dt:.1f} s"}
     return res
 
 
@@ -742,7 +871,14 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS) + [CODEC], default="prefill")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + [CODEC], default=DEFAULT_WORKLOAD)
+    ap.add_argument("--extra", default=None,
+                    help="comma-separated workloads measured in the same run and reported under "
+                         "other_configs (default: the 120B prefill and the three decode batches "
+                         "with one GPU, none with several; '' for none)")
+    ap.add_argument("--no-tc-probe", action="store_true",
+                    help="skip the tensor-pipe rate probe (the FP8 roofline then uses 2x the "
+                         "measured bf16 peak)")
     ap.add_argument("--codec-experts", type=int, default=128,
                     help="codec workload: experts of the 120B-shaped set to sweep")
     ap.add_argument("--codec-e2e-chunks", type=int, default=8,
@@ -756,6 +892,9 @@ def main():
                          "from a separate replay of an instrumented copy of the graph")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.extra is None:
+        single = int(os.environ.get("WORLD_SIZE", "1")) == 1
+        args.extra = ",".join(DEFAULT_EXTRAS) if single and args.workload in WORKLOADS else ""
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))

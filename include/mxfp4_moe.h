@@ -120,11 +120,13 @@ int moe_permute(const int32_t* topk_idx, int T, int E, int k, int32_t* offsets,
  * Same arguments, outputs and ordering as moe_permute. Limits: T*k <= 262144 and
  * E <= 256; larger sizes return MXMOE_EUNSUPPORTED with a message and launch nothing.
  * Differences: a pair with an expert id outside [0, E) is dropped without touching the
- * device error word. The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress, with that device current), so make that first call before any
- * stream capture begins. All calls share the one array and each call rewrites what it
- * reads, so calls that overlap on the GPU (different streams, no ordering) race with each
- * other: order them. */
+ * device error word; offsets[E] then counts only the kept pairs, and perm_token /
+ * perm_slot positions from offsets[E] to T*k - 1 are left as they were (unwritten).
+ * Every call looks up the array's device address on the current device
+ * (cudaGetSymbolAddress; the first lookup in a process may load the library's device
+ * image), so make the first call before any stream capture begins. All calls share the
+ * one array and each call rewrites what it reads, so calls that overlap on the GPU
+ * (different streams, no ordering) race with each other: order them. */
 int moe_permute_noalloc(const int32_t* topk_idx, int T, int E, int k, int32_t* offsets,
                         int32_t* perm_token, int32_t* perm_slot, void* stream);
 
@@ -157,6 +159,23 @@ int moe_mxfp4_forward(const uint16_t* x, const uint16_t* router_w, const uint16_
                       const uint8_t* d_blocks, const uint8_t* d_scales, const float* d_bias,
                       int E, int k, int T, int H, int I, const float* act_scale, uint16_t* out,
                       void* stream);
+
+/* moe_mxfp4_forward_dense -- the dense all-experts path of the same layer ("quantization_
+ * mxfp4" (KerasFormers), As GPT-OSS's native format: long prefills may run all experts on
+ * every token instead of the routed ones, with identical output). Same arguments, layouts,
+ * activations (act_scale) and result definition as moe_mxfp4_forward: every token is
+ * multiplied through all E experts, each expert's output weighted by the token's gate
+ * (its softmax weight for the k selected experts, 0 for the others) and summed over all E
+ * experts in ascending id, fp32, one bf16 rounding. With finite values that sum equals the
+ * routed one term for term, so the output equals moe_mxfp4_forward's wherever both run
+ * the same expert kernels (T > 64). The work is E/k times the routed path's. Limits: H and
+ * I multiples of 64 in [128, 4608], 32-byte aligned blocks, E*T*max(H, I) < 2^31
+ * (MXMOE_EUNSUPPORTED otherwise). Uses the library workspace (E*T*(I + 4H) bytes and more). */
+int moe_mxfp4_forward_dense(const uint16_t* x, const uint16_t* router_w, const uint16_t* router_b,
+                            const uint8_t* gu_blocks, const uint8_t* gu_scales, const float* gu_bias,
+                            const uint8_t* d_blocks, const uint8_t* d_scales, const float* d_bias,
+                            int E, int k, int T, int H, int I, const float* act_scale, uint16_t* out,
+                            void* stream);
 
 /* moe_mxfp4_calibrate -- static per-tensor FP8 scales from a calibration batch with a
  * min-max observer ("gpt-oss-120b-mxfp4-fp8attn-v2", Quantization Recipe):
@@ -200,6 +219,21 @@ int mxmoe_profile_read(char* names, float* total_ms, int* calls, int max_entries
 /* mxmoe_release -- free the workspace of the current device (synchronizes the device).
  * Returns MXMOE_OK or MXMOE_ECUDA. */
 int mxmoe_release(void);
+
+/* mxmoe_tc_rate_probe -- measure the tensor pipe's rate for the block-scaled MMA the
+ * prefill GEMMs issue (tcgen05.mma kind::mxf8f6f4, E4M3 A with M = 128 against E2M1 B with
+ * N = n, K = 32, e8m0 block scales). The pages have no counterpart: the W-MXFP4 / A-FP8
+ * GEMMs are judged against the FP8 tensor peak ("amd/gpt-oss-20b-MoE-Quant-W-MXFP4-A-FP8-
+ * KV-FP8", Quantization schemes), and this call measures that peak for this instruction.
+ * Launches `ctas` CTAs (one per SM for ctas <= the SM count) on `stream`; in each, one
+ * thread issues `iters` x 4 MMAs back to back from operands resident in shared memory
+ * (with_scale_copy != 0: one tcgen05.cp.128x256b of B scales before every 4, as the
+ * prefill GEMM's per-stage scale copy). The caller times the launch (CUDA events on
+ * `stream`). flops (host, nullable) receives the FLOPs the launch performs,
+ * 2 * 128 * n * 32 * 4 * iters * ctas. n: multiple of 16 in [16, 256]; iters in
+ * [1, 1000000]; ctas in [1, 4096]. Returns MXMOE_OK, MXMOE_EINVAL or MXMOE_ECUDA; a
+ * bounded wait that expires sets MXMOE_ETIMEOUT for mxmoe_check. */
+int mxmoe_tc_rate_probe(int n, int with_scale_copy, int iters, int ctas, double* flops, void* stream);
 
 /* mxmoe_selftest_wait_timeout -- exercise the failure path of the library's bounded
  * device waits. The pages have no counterpart: every mbarrier wait in the tensor-core

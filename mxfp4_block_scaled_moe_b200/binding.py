@@ -32,12 +32,14 @@ _SIGS = {
     "moe_permute_noalloc": [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp],
     "moe_fp8_quantize": [_vp, _i64, _f32, _vp, _vp],
     "moe_mxfp4_forward": [_vp] * 9 + [_i32] * 5 + [_vp, _vp, _vp],
+    "moe_mxfp4_forward_dense": [_vp] * 9 + [_i32] * 5 + [_vp, _vp, _vp],
     "moe_mxfp4_calibrate": [_vp] * 9 + [_i32] * 5 + [_vp, _vp],
     "mxmoe_check": [_vp],
     "mxmoe_last_error": [],
     "mxmoe_last_launch_count": [],
     "mxmoe_release": [],
     "mxmoe_selftest_wait_timeout": [_vp],
+    "mxmoe_tc_rate_probe": [_i32, _i32, _i32, _i32, _vp, _vp],
     "mxmoe_profile_enable": [_i32],
     "mxmoe_profile_read": [_vp, _vp, _vp, _i32],
 }
@@ -202,9 +204,8 @@ def _layer_ptrs(x, router_w, router_b, gu_blocks, gu_scales, gu_bias, d_blocks, 
     return ptrs, E, T, H, I
 
 
-def moe_mxfp4_forward(x, router_w, router_b, gu_blocks, gu_scales, gu_bias, d_blocks, d_scales,
-                      d_bias, k, act_scale=None, out=None, stream=None):
-    """The MoE expert layer; act_scale = None (bf16 activations) or two floats {s0, s1}."""
+def _forward(name, x, router_w, router_b, gu_blocks, gu_scales, gu_bias, d_blocks, d_scales,
+             d_bias, k, act_scale, out, stream):
     ptrs, E, T, H, I = _layer_ptrs(x, router_w, router_b, gu_blocks, gu_scales, gu_bias,
                                    d_blocks, d_scales, d_bias)
     if out is None:
@@ -214,10 +215,25 @@ def moe_mxfp4_forward(x, router_w, router_b, gu_blocks, gu_scales, gu_bias, d_bl
     if act_scale is not None:
         s = [float(v) for v in act_scale]
         acts = (ctypes.c_float * 2)(s[0], s[1])
-    _call("moe_mxfp4_forward", *ptrs, E, k, T, H, I,
+    _call(name, *ptrs, E, k, T, H, I,
           ctypes.cast(acts, ctypes.c_void_p) if acts is not None else None, _ptr(out),
           _stream(stream))
     return out
+
+
+def moe_mxfp4_forward(x, router_w, router_b, gu_blocks, gu_scales, gu_bias, d_blocks, d_scales,
+                      d_bias, k, act_scale=None, out=None, stream=None):
+    """The MoE expert layer; act_scale = None (bf16 activations) or two floats {s0, s1}."""
+    return _forward("moe_mxfp4_forward", x, router_w, router_b, gu_blocks, gu_scales, gu_bias,
+                    d_blocks, d_scales, d_bias, k, act_scale, out, stream)
+
+
+def moe_mxfp4_forward_dense(x, router_w, router_b, gu_blocks, gu_scales, gu_bias, d_blocks,
+                            d_scales, d_bias, k, act_scale=None, out=None, stream=None):
+    """The same layer by the dense all-experts path (every token through all E experts,
+    zero gates off the top-k)."""
+    return _forward("moe_mxfp4_forward_dense", x, router_w, router_b, gu_blocks, gu_scales,
+                    gu_bias, d_blocks, d_scales, d_bias, k, act_scale, out, stream)
 
 
 def moe_mxfp4_calibrate(x, router_w, router_b, gu_blocks, gu_scales, gu_bias, d_blocks, d_scales,
@@ -240,6 +256,18 @@ def mxmoe_last_launch_count() -> int:
 
 def mxmoe_release():
     _call("mxmoe_release")
+
+
+def mxmoe_tc_rate_probe(n=256, with_scale_copy=False, iters=20000, ctas=None, stream=None) -> float:
+    """Launch the tensor-pipe rate probe (kind::mxf8f6f4 MMAs, M = 128, N = n) on `ctas`
+    CTAs (default: one per SM); returns the FLOPs the launch performs. Time it with CUDA
+    events on `stream`."""
+    if ctas is None:
+        ctas = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    f = ctypes.c_double(0.0)
+    _call("mxmoe_tc_rate_probe", int(n), 1 if with_scale_copy else 0, int(iters), int(ctas),
+          ctypes.byref(f), _stream(stream))
+    return f.value
 
 
 def mxmoe_selftest_wait_timeout(stream=None):

@@ -96,16 +96,10 @@ struct Workspace {
   size_t tickets_zeroed = 0;  // bytes at the start of the workspace known to be zero
 };
 
-// Routed pairs from which the prefill paths (FP8, and bf16 as two e4m3 parts) run on the
-// tcgen05 grouped GEMMs (fewer pairs use the tensor-core decode or register-dequant kernels). MXMOE_TC_MIN_PAIRS overrides it (0 = always when the
-// shapes allow, a huge value = never).
-int64_t tc_min_pairs() {
-  static int64_t v = [] {
-    const char* s = std::getenv("MXMOE_TC_MIN_PAIRS");
-    return s ? std::atoll(s) : 1024LL;
-  }();
-  return v;
-}
+// Batches above the tensor-core decode path's size (T > kDecodeMaxT) run on the tcgen05
+// grouped GEMMs whenever the shapes allow: FP8 activations directly, bf16 activations as
+// two e4m3 parts. The register-dequant kernels (mma.sync) remain for calibration and for
+// shapes neither tensor-core path takes.
 constexpr int kTcMaxNb = 144;   // K <= 4608: the range the tcgen05 GEMM is tested on
 
 constexpr int kMaxDevices = 64;
@@ -219,7 +213,7 @@ size_t layout(int T, int E, int k, int H, int I, bool fp8, bool tc, bool tcb, bo
   size_t o_sa1 = c.take<uint8_t>(tcb ? 2 * P * (H / 32) : 0);
   size_t o_sa2 = c.take<uint8_t>(tcb ? 2 * P * (I / 32) : 0);
   size_t o_xs = c.take<uint8_t>(dtc ? static_cast<int64_t>(mxmoe::decode_tc_xs_bytes(P, H)) : 0);
-  size_t o_sfb = c.take<uint8_t>(dtc ? static_cast<int64_t>(mxmoe::decode_tc_sfb_row_bytes(E, T)) : 0);
+  size_t o_sfb = c.take<uint8_t>(dtc ? static_cast<int64_t>(mxmoe::decode_tc_sfb_bytes(E, H, T)) : 0);
   size_t o_xsm = c.take<uint8_t>(dtc ? static_cast<int64_t>(mxmoe::decode_tc_xs_bytes(P, I)) : 0);
   size_t o_sfbm = c.take<uint8_t>(dtc ? static_cast<int64_t>(mxmoe::decode_tc_sfb_bytes(E, I, T)) : 0);
   size_t o_part = c.take<uint8_t>(dtc ? static_cast<int64_t>(mxmoe::decode_tc_part_bytes(P, H, I)) : 0);
@@ -303,11 +297,12 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
   if (int rc = current_device_ws(&ws)) return rc;
   const bool fp8 = act_scale != nullptr;
   const int64_t P = static_cast<int64_t>(a.T) * a.k;
-  const bool tc = fp8 && !calib_out && P >= tc_min_pairs() && std::max(a.H, a.I) / 32 <= kTcMaxNb &&
+  const bool large = a.T > kDecodeMaxT;
+  const bool tc = fp8 && !calib_out && large && std::max(a.H, a.I) / 32 <= kTcMaxNb &&
                   tc_gemm_supported(a.H, a.I, a.gu_blocks, a.d_blocks, a.gu_scales, a.d_scales);
   // bf16 activations with many routed pairs: the same GEMMs with each activation as two
   // e4m3 parts (exact for the activations' significant bits)
-  const bool tcb = !fp8 && !calib_out && P >= tc_min_pairs() && std::max(a.H, a.I) / 32 <= kTcMaxNb &&
+  const bool tcb = !fp8 && !calib_out && large && std::max(a.H, a.I) / 32 <= kTcMaxNb &&
                    tc_gemm_supported(a.H, a.I, a.gu_blocks, a.d_blocks, a.gu_scales, a.d_scales);
   const bool dtc = !tc && !tcb && !calib_out &&
                    decode_tc_supported(a.H, a.I, a.T, a.gu_blocks, a.d_blocks, a.gu_scales, a.d_scales);
@@ -519,6 +514,118 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
   return MXMOE_OK;
 }
 
+// The dense all-experts path: every token through all E experts (expert-major rows
+// e * T + t), the gates zero off the top-k, the weighted sum over all experts in ascending
+// order. The tcgen05 grouped GEMMs read the T activation rows once per expert (shared A
+// rows) instead of a gathered copy per routed pair.
+int run_layer_dense(const LayerArgs& a, const float* act_scale, uint16_t* out, cudaStream_t st) {
+  using namespace mxmoe;
+  Workspace* ws = nullptr;
+  if (int rc = current_device_ws(&ws)) return rc;
+  const bool fp8 = act_scale != nullptr;
+  const int64_t T = a.T, E = a.E, H = a.H, I = a.I;
+  const int64_t R = E * T;   // expert-major rows
+  if (!(std::max(a.H, a.I) / 32 <= kTcMaxNb &&
+        tc_gemm_supported(a.H, a.I, a.gu_blocks, a.d_blocks, a.gu_scales, a.d_scales)))
+    return fail(MXMOE_EUNSUPPORTED, "the dense path needs H and I multiples of 64 in [128, 4608] and 32-byte "
+                                    "aligned blocks (got H = %d, I = %d)", a.H, a.I);
+  if (R * std::max(H, I) >= (int64_t{1} << 31) || R >= (int64_t{1} << 24))
+    return fail(MXMOE_EUNSUPPORTED, "the dense path holds E*T*max(H, I) < 2^31 values (E = %d, T = %d)", a.E, a.T);
+  const bool rtc = a.T > 32 && router_tc_supported(a.T, a.H, a.E, a.x, a.router_w, nullptr);
+  const int ksplit = rtc ? router_tc_ksplit(a.T, a.H, ws->sms) : 0;
+  const int n_rest = ksplit > 1 ? ksplit - 1 : 0;
+  Carve c;
+  c.take<uint8_t>(kTicketBytes);
+  const size_t o_logits = c.take<float>(T * E), o_rest = c.take<float>(n_rest * T * E);
+  const size_t o_idx = c.take<int32_t>(T * a.k), o_w = c.take<float>(T * a.k);
+  const size_t o_g = c.take<float>(T * E), o_off = c.take<int32_t>(E + 1);
+  const size_t o_a1 = c.take<uint8_t>(fp8 ? T * H : 2 * T * H);
+  const size_t o_sa1 = c.take<uint8_t>(fp8 ? 0 : 2 * T * (H / 32));
+  const size_t o_mid = c.take<uint16_t>(fp8 ? 0 : R * I);
+  const size_t o_a2 = c.take<uint8_t>(fp8 ? R * I : 2 * R * I);
+  const size_t o_sa2 = c.take<uint8_t>(fp8 ? 0 : 2 * R * (I / 32));
+  const size_t o_y = c.take<float>(R * H);
+  if (int rc = ensure_capacity(ws, c.off)) return rc;
+  if (fp8 && !ws->tc_ready) {
+    cudaError_t e = tc_gemm_prepare(256);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (tcgen05 GEMM)");
+    ws->tc_ready = true;
+  }
+  if (!fp8 && !ws->tcb_ready) {
+    cudaError_t e = tc_parts_gemm_prepare(256);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (two-part tcgen05 GEMM)");
+    ws->tcb_ready = true;
+  }
+  ws->tickets_zeroed = kTicketBytes;
+  char* base = ws->base;
+  float* logits = reinterpret_cast<float*>(base + o_logits);
+  float* rest = n_rest ? reinterpret_cast<float*>(base + o_rest) : nullptr;
+  int32_t* idx = reinterpret_cast<int32_t*>(base + o_idx);
+  float* w = reinterpret_cast<float*>(base + o_w);
+  float* gates = reinterpret_cast<float*>(base + o_g);
+  int32_t* offsets = reinterpret_cast<int32_t*>(base + o_off);
+  uint8_t* a1 = reinterpret_cast<uint8_t*>(base + o_a1);
+  uint8_t* sa1 = reinterpret_cast<uint8_t*>(base + o_sa1);
+  uint16_t* mid = reinterpret_cast<uint16_t*>(base + o_mid);
+  uint8_t* a2 = reinterpret_cast<uint8_t*>(base + o_a2);
+  uint8_t* sa2 = reinterpret_cast<uint8_t*>(base + o_sa2);
+  float* y = reinterpret_cast<float*>(base + o_y);
+  const float s0 = fp8 ? act_scale[0] : 1.0f, s1 = fp8 ? act_scale[1] : 1.0f;
+  int launches = 0;
+  cudaError_t e;
+  StageTimer tm(st);
+  if ((e = rtc ? launch_router_tc(a.x, a.router_w, a.router_b, a.T, a.H, a.E, ksplit, logits, rest, ws->err, st)
+               : launch_router(a.x, a.router_w, a.router_b, a.T, a.H, a.E, logits, st)))
+    return cuda_fail(e, "router");
+  ++launches;
+  tm.mark("router");
+  if ((e = launch_topk(logits, rest, n_rest, a.T, a.E, a.k, idx, w, st))) return cuda_fail(e, "topk");
+  ++launches;
+  tm.mark("topk");
+  if ((e = launch_dense_setup(idx, w, a.T, a.E, a.k, gates, offsets, st, ws->sms))) return cuda_fail(e, "dense gates");
+  ++launches;
+  tm.mark("dense_gates");
+  if (fp8) {
+    if ((e = launch_fp8_quant(a.x, T * H, s0, a1, st, ws->sms))) return cuda_fail(e, "fp8 activation cast");
+    ++launches;
+    tm.mark("act_quant");
+    if ((e = launch_tc_gemm(true, a1, T, a.H, a.gu_blocks, a.gu_scales, a.gu_bias, a.E, a.I, offsets, s0, s1, a2,
+                            nullptr, ws->err, ws->sms, st, true)))
+      return cuda_fail(e, "gate_up (tcgen05, dense)");
+    ++launches;
+    tm.mark("gate_up");
+    if ((e = launch_tc_gemm(false, a2, R, a.I, a.d_blocks, a.d_scales, a.d_bias, a.E, a.H, offsets, s1, 0.0f,
+                            nullptr, y, ws->err, ws->sms, st)))
+      return cuda_fail(e, "down (tcgen05, dense)");
+    ++launches;
+    tm.mark("down");
+  } else {
+    if ((e = launch_split_parts(a.x, nullptr, a.T, T, a.H, a1, sa1, ws->sms, st)))
+      return cuda_fail(e, "activation split");
+    ++launches;
+    tm.mark("act_split");
+    if ((e = launch_tc_parts_gemm(true, a1, sa1, T, a.H, a.gu_blocks, a.gu_scales, a.gu_bias, a.E, a.I, offsets,
+                                  mid, nullptr, ws->err, ws->sms, st, true)))
+      return cuda_fail(e, "gate_up (tcgen05, two parts, dense)");
+    ++launches;
+    tm.mark("gate_up");
+    if ((e = launch_split_parts(mid, nullptr, a.T, R, a.I, a2, sa2, ws->sms, st)))
+      return cuda_fail(e, "intermediate split");
+    ++launches;
+    tm.mark("mid_split");
+    if ((e = launch_tc_parts_gemm(false, a2, sa2, R, a.I, a.d_blocks, a.d_scales, a.d_bias, a.E, a.H, offsets,
+                                  nullptr, y, ws->err, ws->sms, st)))
+      return cuda_fail(e, "down (tcgen05, two parts, dense)");
+    ++launches;
+    tm.mark("down");
+  }
+  if ((e = launch_dense_combine(y, gates, a.T, a.H, a.E, out, st, ws->sms))) return cuda_fail(e, "dense combine");
+  ++launches;
+  tm.mark("combine");
+  t_last_launches = launches;
+  return MXMOE_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -658,6 +765,24 @@ int moe_mxfp4_forward(const uint16_t* x, const uint16_t* router_w, const uint16_
   return run_layer(a, act_scale, out, nullptr, static_cast<cudaStream_t>(stream));
 }
 
+int moe_mxfp4_forward_dense(const uint16_t* x, const uint16_t* router_w, const uint16_t* router_b,
+                            const uint8_t* gu_blocks, const uint8_t* gu_scales, const float* gu_bias,
+                            const uint8_t* d_blocks, const uint8_t* d_scales, const float* d_bias,
+                            int E, int k, int T, int H, int I, const float* act_scale, uint16_t* out,
+                            void* stream) {
+  t_last_error.clear();
+  t_last_launches = 0;
+  LayerArgs a{x, router_w, router_b, gu_blocks, gu_scales, gu_bias, d_blocks, d_scales, d_bias,
+              E, k, T, H, I};
+  if (T == 0) return check_routing_args(T, E, k);
+  if (int rc = check_layer_args(a)) return rc;
+  if (!out) return fail(MXMOE_EINVAL, "out is NULL");
+  if (!aligned16(out)) return fail(MXMOE_EINVAL, "out is not 16-byte aligned");
+  if (act_scale && !(act_scale[0] > 0.0f && act_scale[1] > 0.0f))
+    return fail(MXMOE_EINVAL, "act_scale values must be > 0");
+  return run_layer_dense(a, act_scale, out, static_cast<cudaStream_t>(stream));
+}
+
 int moe_mxfp4_calibrate(const uint16_t* x, const uint16_t* router_w, const uint16_t* router_b,
                         const uint8_t* gu_blocks, const uint8_t* gu_scales, const float* gu_bias,
                         const uint8_t* d_blocks, const uint8_t* d_scales, const float* d_bias,
@@ -692,6 +817,22 @@ int mxmoe_selftest_wait_timeout(void* stream) {
   if (int rc = current_device_ws(&ws)) return rc;
   cudaError_t e = mxmoe::launch_wait_selftest(ws->err, static_cast<cudaStream_t>(stream));
   return e ? cuda_fail(e, "wait self-test launch") : MXMOE_OK;
+}
+
+int mxmoe_tc_rate_probe(int n, int with_scale_copy, int iters, int ctas, double* flops, void* stream) {
+  t_last_error.clear();
+  t_last_launches = 0;
+  if (n < 16 || n > 256 || n % 16) return fail(MXMOE_EINVAL, "n = %d must be a multiple of 16 in [16, 256]", n);
+  if (iters < 1 || iters > 1000000) return fail(MXMOE_EINVAL, "iters = %d outside [1, 1000000]", iters);
+  if (ctas < 1 || ctas > 4096) return fail(MXMOE_EINVAL, "ctas = %d outside [1, 4096]", ctas);
+  Workspace* ws = nullptr;
+  if (int rc = current_device_ws(&ws)) return rc;
+  cudaError_t e = mxmoe::launch_tc_rate(n, with_scale_copy ? 1 : 0, iters, ctas, ws->err,
+                                        static_cast<cudaStream_t>(stream));
+  if (e) return cuda_fail(e, "rate probe launch");
+  t_last_launches = 1;
+  if (flops) *flops = 2.0 * 128.0 * n * 32.0 * 4.0 * iters * ctas;
+  return MXMOE_OK;
 }
 
 const char* mxmoe_last_error(void) { return t_last_error.c_str(); }
@@ -757,7 +898,9 @@ int mxmoe_release(void) {
 // active-expert list) lives in a fixed array of this library's device image instead of
 // the cudaMalloc'd workspace. Host code may not pass `g_noalloc_scratch` itself to a
 // kernel (in host code the name stands for a host-side shadow, not a device address),
-// so the device address is looked up with cudaGetSymbolAddress once per device.
+// so every call looks the current device's address up with cudaGetSymbolAddress (it
+// allocates nothing). Looking it up per call rather than caching it keeps the address
+// valid after a context teardown (cudaDeviceReset) reloads the library's device image.
 namespace {
 
 constexpr int64_t kNoAllocMaxPairs = 262144;   // T * k accepted by the variant
@@ -767,9 +910,6 @@ constexpr int kNoAllocInts = kNoAllocMaxChunks * kNoAllocMaxExperts + kNoAllocMa
 
 // 256-byte aligned, 132,352 bytes; every GPU that loads the library keeps it until exit.
 static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocInts];
-
-int32_t* g_noalloc_dev[kMaxDevices] = {};
-std::mutex g_noalloc_mu;
 
 }  // namespace
 
@@ -785,21 +925,10 @@ extern "C" int moe_permute_noalloc(const int32_t* topk_idx, int T, int E, int k,
     return fail(MXMOE_EUNSUPPORTED, "moe_permute_noalloc: too many chunks");
   if (!offsets) return fail(MXMOE_EINVAL, "offsets is NULL");
   if (T > 0 && (!topk_idx || !perm_token || !perm_slot)) return fail(MXMOE_EINVAL, "null pointer");
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  if (dev < 0 || dev >= kMaxDevices) return fail(MXMOE_EUNSUPPORTED, "device %d beyond %d", dev, kMaxDevices);
-  int32_t* scratch = nullptr;
-  {
-    std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (!g_noalloc_dev[dev]) {
-      void* ptr = nullptr;
-      e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);   // this device is current
-      if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
-      g_noalloc_dev[dev] = static_cast<int32_t*>(ptr);
-    }
-    scratch = g_noalloc_dev[dev];
-  }
+  void* ptr = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);   // the current device's copy
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+  int32_t* scratch = static_cast<int32_t*>(ptr);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (T == 0) {
     e = cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), st);

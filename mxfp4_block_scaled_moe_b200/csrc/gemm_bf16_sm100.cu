@@ -70,7 +70,9 @@ struct Params {
   const uint8_t* a_scales;   // part scales, (2, P, nb): part p of grouped row m at (p * P + m) * nb
   const float* bias;         // (E, rows_total)
   const int32_t* offsets;    // (E+1)
-  int64_t P;                 // grouped rows
+  int64_t P;                 // rows of each part of A (grouped rows; a_shared: T)
+  int a_shared;              // 1: every expert reads the same A rows (the dense all-experts
+                             // path: A row = row within the expert), 0: A row = grouped row
   int E;
   int K;
   int nb;                    // K / 32
@@ -284,8 +286,9 @@ moe_gemm_parts_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_c
             dep_ready = true;
           }
           uint8_t* a_dst = sA + stage * kParts * kAStage;
-          tma_load_2d(a_dst, &tmap_a, &full[stage], kx, tl.m0);
-          tma_load_2d(a_dst + kAStage, &tmap_a, &full[stage], kx, static_cast<int>(p.P) + tl.m0);
+          const int arow = p.a_shared ? tl.m0 - p.offsets[tl.e] : tl.m0;
+          tma_load_2d(a_dst, &tmap_a, &full[stage], kx, arow);
+          tma_load_2d(a_dst + kAStage, &tmap_a, &full[stage], kx, static_cast<int>(p.P) + arow);
           if (++stage == kStages) { stage = 0; phase ^= 1; }
         }
       }
@@ -362,7 +365,7 @@ moe_gemm_parts_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_c
         rp[i] = reinterpret_cast<const uint16_t*>(
             p.b_scales + (in ? (static_cast<int64_t>(group) * p.rows_per_group + n0 + rr) * p.nb : 0));
         ok |= (in ? 1u : 0u) << i;
-        const int64_t m = static_cast<int64_t>(tl.m0) + lane + 32 * i;
+        const int64_t m = static_cast<int64_t>(p.a_shared ? tl.m0 - p.offsets[tl.e] : tl.m0) + lane + 32 * i;
         const bool ain = m < p.P;
         rp[4 + i] = reinterpret_cast<const uint16_t*>(
             p.a_scales + (ain ? (static_cast<int64_t>(w2) * p.P + m) * p.nb : 0));
@@ -581,7 +584,7 @@ cudaError_t tc_parts_gemm_prepare(int E) {
 cudaError_t launch_tc_parts_gemm(bool gate_up, const uint8_t* parts, const uint8_t* a_scales, int64_t P_rows, int K,
                                  const uint8_t* blocks, const uint8_t* scales, const float* bias, int E, int n_out,
                                  const int32_t* offsets, uint16_t* a_out, float* y_out, int* err, int sms,
-                                 cudaStream_t st) {
+                                 cudaStream_t st, bool a_shared) {
   using namespace g100b;
   const int rows_per_group = n_out;
   const int groups = gate_up ? 2 * E : E;
@@ -611,6 +614,7 @@ cudaError_t launch_tc_parts_gemm(bool gate_up, const uint8_t* parts, const uint8
   prm.bias = bias;
   prm.offsets = offsets;
   prm.P = P_rows;
+  prm.a_shared = a_shared ? 1 : 0;
   prm.E = E;
   prm.K = K;
   prm.nb = K / 32;

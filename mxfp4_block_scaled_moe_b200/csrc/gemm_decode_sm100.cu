@@ -9,11 +9,13 @@
 //   A = 128 weight rows (gate_up: 128 gate rows and, in a second MMA, the 128 matching up
 //       rows; down: 128 rows of down_proj) with the checkpoint's e8m0 scales;
 //   B = the routed token rows as four MXFP4 "parts" each: p1 = e2m1(x / 2^s1), p2 the same
-//       on the residual x - p1, and so on, each s chosen from its group's largest residual
-//       (the whole row for gate_up's input, each 32-value block for down's) so that nothing
-//       saturates. Every part removes about three bits of the residual, and four parts
-//       change a 2880-long dot product by about 2e-4 of the largest output (the
-//       per-tensor FP8 path splits the e4m3 value of x / s0 the same way).
+//       on the residual x - p1, and so on, each s chosen from the largest residual of its
+//       32-value block so that nothing saturates. Every part removes about three bits of
+//       the residual, and four parts change a 2880-long dot product by about 1.5e-4 of
+//       the largest output; a block scale keeps that bound when one channel is 1000x the
+//       others (a row-wide scale would not: the other values would keep only the bits
+//       below the outlier's). The per-tensor FP8 path splits the e4m3 value of x / s0 the
+//       same way.
 //   D = 128 x N fp32 in tensor memory, N = 4 * rows rounded up to 16; the epilogue adds a
 //       token's four columns.
 // Why not FP8 tokens against FP4 weights (kind::mxf8f6f4): a block-scaled MMA costs the
@@ -69,9 +71,9 @@ constexpr int kSfaCol = 480;       // A scales: tile h, atom a at 480 + 8h + 4a
 constexpr int kSfbCol = 496;       // B scales: k-tile t, atom b at 496 + 8t + 4b
 constexpr int kSfRecord = 1024;    // B scale record per (row group, 128-wide k-tile)
 // Per stage: the A (weight) scales of each tile as one 128x256b tcgen05.cp source (4 KB:
-// the two 128-wide k-tiles' atoms, repeated for the four 32-lane quarters), then the B
-// scale record(s): gate_up one 1 KB record per unit (copied once), down two per stage.
-__host__ __device__ constexpr int sf_stage_bytes(int kA) { return kA * 4096 + (kA == 2 ? 1024 : 2048); }
+// the two 128-wide k-tiles' atoms, repeated for the four 32-lane quarters), then the two
+// 1 KB B scale records of the stage's k-tiles.
+__host__ __device__ constexpr int sf_stage_bytes(int kA) { return kA * 4096 + 2 * 1024; }
 constexpr int kSfStageMax = sf_stage_bytes(2);
 constexpr int kMaxE = 256;
 constexpr int kMaxGrp = kDecodeMaxGroups;
@@ -463,12 +465,10 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
       bool dep_ready = false;
       for (int u = blockIdx.x; u < sc.units && ok; u += gridDim.x) {
         const Unit w = unit_at(sc, p, u);
-        // B scales: gate_up has one record per row group (the same for every k-tile); down
-        // one per 128-wide k-tile
-        const uint32_t sfb_bytes = kGateUp ? kSfRecord : 2 * kSfRecord;
+        // B scales: one record per 128-wide k-tile, two per stage
+        const uint32_t sfb_bytes = 2 * kSfRecord;
         const uint32_t tx = kA * BM * kRowBytes + w.nbox * p.box_rows * kRowBytes + sfb_bytes;
-        const uint8_t* rec = kGateUp ? p.sfb + (static_cast<int64_t>(w.e) * p.max_chunks + w.c) * kSfRecord
-                                     : p.sfb + (static_cast<int64_t>(w.e) * p.max_chunks + w.c) * 2 * p.nst * kSfRecord;
+        const uint8_t* rec = p.sfb + (static_cast<int64_t>(w.e) * p.max_chunks + w.c) * 2 * p.nst * kSfRecord;
         for (int kst = w.k0; kst < w.k1; ++kst) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[stage], tx);
@@ -483,7 +483,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
           for (int b = 0; b < w.nbox; ++b)
             tma_load_2d(sB(stage) + b * p.box_rows * kRowBytes, &map_x, &full[stage], kRowBytes * kst,
                         kParts * w.off + b * p.box_rows);
-          bulk_g2s(sSFB(stage), kGateUp ? rec : rec + 2 * kst * kSfRecord, sfb_bytes, &full[stage]);
+          bulk_g2s(sSFB(stage), rec + 2 * kst * kSfRecord, sfb_bytes, &full[stage]);
           if (++stage == S) { stage = 0; phase ^= 1; }
         }
       }
@@ -495,8 +495,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
     uint32_t use0 = 0u, use1 = 0u;   // completed uses of each accumulator slot
     int nxt = 0;
     bool ok = true;
-    int uj = 0;   // units issued by this CTA
-    for (int u = blockIdx.x; u < sc.units && ok; u += gridDim.x, ++uj) {
+    for (int u = blockIdx.x; u < sc.units && ok; u += gridDim.x) {
       const Unit w = unit_at(sc, p, u);
       const bool big = kGateUp && w.ncols > kBigCols;
       const int slot = big ? 0 : nxt;
@@ -512,9 +511,6 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
       const uint32_t du = big ? static_cast<uint32_t>(kSlot1) : dg + static_cast<uint32_t>(w.ncols);
       const uint32_t id0 = idesc_mxf4(BM, w.ncols);
       const int nat = w.ncols > 128 ? 2 : 1;   // B scale atoms per k-tile
-      // gate_up: the unit's B scale atoms, copied once at its first stage into the slot of
-      // this unit's parity (the previous unit may still be reading the other slot)
-      const uint32_t sfb_unit = tmem + kSfbCol + 8 * static_cast<uint32_t>(uj & 1);
       for (int kst = w.k0; kst < w.k1; ++kst) {
         if (!mbar_wait(&full[stage], phase, abort_flag, p.err)) { ok = false; break; }
         tc_fence_after();
@@ -526,15 +522,10 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
 #pragma unroll
           for (int h = 0; h < kA; ++h)
             tc_cp_128x256b(tmem + kSfaCol + 8 * h, smem_desc(smem_u32(sSFA(stage, h)), 2048, 128, 0));
-          for (int t = 0; t < nkt; ++t) {
-            if (!kGateUp)
-              for (int b = 0; b < nat; ++b)
-                tc_cp_32x128b_x4(tmem + kSfbCol + 8 * t + 4 * b,
-                                 smem_desc(smem_u32(sSFB(stage) + kSfRecord * t + 512 * b), 0, 128, 0));
-          }
-          if (kGateUp && kst == w.k0)
+          for (int t = 0; t < nkt; ++t)
             for (int b = 0; b < nat; ++b)
-              tc_cp_32x128b_x4(sfb_unit + 4 * b, smem_desc(smem_u32(sSFB(stage) + 512 * b), 0, 128, 0));
+              tc_cp_32x128b_x4(tmem + kSfbCol + 8 * t + 4 * b,
+                               smem_desc(smem_u32(sSFB(stage) + kSfRecord * t + 512 * b), 0, 128, 0));
           const uint32_t b0 = smem_u32(sB(stage));
           for (int sk = 0; sk < nks; ++sk) {
             const int t = sk >> 1;
@@ -547,7 +538,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
             for (int h = 0; h < kA; ++h) {
               const uint64_t ad = smem_desc(smem_u32(sA(stage, h)) + 32 * sk, 16, 1024, 2);
               tc_mma_mxf4(tmem + (h ? du : dg), ad, bd, id, (tmem + kSfaCol + 8 * h + 4 * t) | sel,
-                          (kGateUp ? sfb_unit : tmem + kSfbCol + 8 * t) | sel, acc);
+                          (tmem + kSfbCol + 8 * t) | sel, acc);
             }
           }
           tc_commit(&empty[stage]);
@@ -807,25 +798,24 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
 
 // ------------------------------------------------ token operand of the gate_up GEMM --
 // One CTA per token: the token's x (or, with FP8 activations, the e4m3 value of x / s0)
-// as four e2m1 parts, each with ONE e8m0 scale for the whole row (the smallest s with the
-// row's largest residual / 2^s <= 6), written to each of the token's k routed rows in
-// expert-grouped order (its position inv[t*k + j]). A row-wide scale costs a little
-// accuracy against per-block scales (a simulation of the 2880-long dot products: 1.2e-4
-// of the largest output instead of 4e-5, against a 2e-3 bar) and makes the gate_up GEMM's
-// B scale atom the same for every k-tile, so the GEMM copies it into tensor memory once
-// per unit instead of twice per stage. Its record: [expert][row group][two 512-byte
-// atoms], the four k-block bytes of a row all equal. The row's loads are issued first
-// (they depend on nothing), the routing lookups beside them; each thread holds 16
-// consecutive values, so a part leaves as one 8-byte store per routed row.
+// as four e2m1 parts, each 32-value block with its own e8m0 scale per part (the smallest
+// s with the block's largest residual / 2^s <= 6), written to each of the token's k
+// routed rows in expert-grouped order (its position inv[t*k + j]). Scale records: per
+// (expert, row group, 128-wide k-tile) one 1 KB record as the down GEMM's B operand has
+// them, row r at sf_atom_byte(r, k-block within the k-tile). The row's loads are issued
+// first (they depend on nothing), the routing lookups beside them; each thread holds 16
+// consecutive values (half a block: a block's maximum is one shuffle with the
+// neighbouring lane), so a part leaves as one 8-byte store per routed row.
 constexpr int kSplitThreads = 256;
 constexpr int kSplitVals = 16;   // values per thread: H <= 4096
 __global__ void __launch_bounds__(kSplitThreads) split_tokens_kernel(
     const uint16_t* __restrict__ x, const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ inv,
     const int32_t* __restrict__ offsets, int E, int64_t P, int H, int k, float s0, int fp8,
-    uint8_t* __restrict__ xs, uint8_t* __restrict__ sfb, int max_chunks) {
-  __shared__ float s_max[kSplitThreads / 32];
+    uint8_t* __restrict__ xs, uint8_t* __restrict__ sfb, int max_chunks, int nst) {
   __shared__ int s_pos[kMaxTopK];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __shared__ long long s_rec[kMaxTopK];   // byte offset of the routed row's first record, or -1
+  __shared__ int s_jr[kMaxTopK];          // the routed row within its row group
+  const int lane = threadIdx.x & 31;
   const int t = blockIdx.x;
   const int i0 = kSplitVals * static_cast<int>(threadIdx.x);
   const bool act = i0 < H;   // H % 64 == 0: a thread's 16 values are all in or all out
@@ -841,21 +831,21 @@ __global__ void __launch_bounds__(kSplitThreads) split_tokens_kernel(
   // routing's expert offsets before it waits for this kernel.
   griddep_wait();
   griddep_launch_dependents();
-  // thread j < k: the token's routed row j (its scale record is written by this thread)
-  uint8_t* rec = nullptr;
-  int jr = 0;
-  if (static_cast<int>(threadIdx.x) < k) {
+  if (static_cast<int>(threadIdx.x) < k) {   // thread j < k: the token's routed row j
     const int64_t pr = static_cast<int64_t>(t) * k + threadIdx.x;
     const int e = topk_idx[pr];
     const int pos = inv[pr];
-    int ps = -1;
+    int ps = -1, jr = 0;
+    long long rec = -1;
     if (e >= 0 && e < E && pos >= 0 && pos < P) {   // else the permutation has flagged it
       const int je = pos - offsets[e];   // row within the expert
-      rec = sfb + (static_cast<int64_t>(e) * max_chunks + je / kGroupRows) * kSfRecord;
+      rec = (static_cast<long long>(e) * max_chunks + je / kGroupRows) * 2 * nst * kSfRecord;
       jr = je % kGroupRows;
       ps = pos;
     }
     s_pos[threadIdx.x] = ps;
+    s_rec[threadIdx.x] = rec;
+    s_jr[threadIdx.x] = jr;
   }
   float r[kSplitVals];
 #pragma unroll
@@ -869,18 +859,16 @@ __global__ void __launch_bounds__(kSplitThreads) split_tokens_kernel(
     }
   }
   const int64_t row_bytes = H / 2;
-  __syncthreads();   // s_pos
+  const int kb = static_cast<int>(threadIdx.x) >> 1;   // this thread's 32-value block
+  const int64_t rec_kt = static_cast<int64_t>(kb >> 2) * kSfRecord;
+  const bool writes_scale = act && (lane & 1) == 0;
+  __syncthreads();   // s_pos, s_rec, s_jr
 #pragma unroll 1
   for (int pp = 0; pp < kParts; ++pp) {
     float m = 0.0f;
 #pragma unroll
     for (int v = 0; v < kSplitVals; ++v) m = fmaxf(m, fabsf(r[v]));
-    m = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(m)));
-    if (lane == 0) s_max[warp] = m;
-    __syncthreads();
-#pragma unroll
-    for (int w = 0; w < kSplitThreads / 32; ++w) m = fmaxf(m, s_max[w]);
-    __syncthreads();   // every thread has read s_max before the next part writes it
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));   // the other half of the block
     const int sc = e2m1_part_exponent(m);
     const float down = pow2f(-sc), up = pow2f(sc);
     uint32_t packed[2] = {0u, 0u};
@@ -896,12 +884,12 @@ __global__ void __launch_bounds__(kSplitThreads) split_tokens_kernel(
     if (act)
       for (int j = 0; j < k; ++j) {
         const int pos = s_pos[j];
-        if (pos >= 0)
-          *reinterpret_cast<uint2*>(xs + (static_cast<int64_t>(pos) * kParts + pp) * row_bytes + i0 / 2) =
-              make_uint2(packed[0], packed[1]);
+        if (pos < 0) continue;
+        *reinterpret_cast<uint2*>(xs + (static_cast<int64_t>(pos) * kParts + pp) * row_bytes + i0 / 2) =
+            make_uint2(packed[0], packed[1]);
+        if (writes_scale)
+          sfb[s_rec[j] + rec_kt + sf_atom_byte(kParts * s_jr[j] + pp, kb & 3)] = static_cast<uint8_t>(sc + 127);
       }
-    if (rec)   // the row's scale for all four k-blocks of the atom word
-      *reinterpret_cast<uint32_t*>(rec + sf_atom_byte(kParts * jr + pp, 0)) = 0x01010101u * static_cast<uint32_t>(sc + 127);
   }
 }
 
@@ -982,8 +970,6 @@ size_t decode_tc_sfb_bytes(int E, int K, int T) {
   return static_cast<size_t>(E) * max_chunks_for(T) * 2 * nst_for(K) * dec::kSfRecord;
 }
 
-size_t decode_tc_sfb_row_bytes(int E, int T) { return static_cast<size_t>(E) * max_chunks_for(T) * dec::kSfRecord; }
-
 size_t decode_tc_part_bytes(int64_t P, int H, int I) {
   const size_t gu = static_cast<size_t>(split_cap(2, P, I)) * 2 * P * dec::kParts * I * 4;
   const size_t d = static_cast<size_t>(split_cap(1, P, H)) * 1 * P * dec::kParts * H * 4;
@@ -1010,7 +996,7 @@ cudaError_t launch_split_tokens(bool fp8, const uint16_t* x, const int32_t* topk
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, dec::split_tokens_kernel, x, topk_idx, inv, offsets, E, static_cast<int64_t>(T) * k, H,
-                            k, s0, fp8 ? 1 : 0, xs, sfb, max_chunks_for(T));
+                            k, s0, fp8 ? 1 : 0, xs, sfb, max_chunks_for(T), nst_for(H));
 }
 
 // gate_up (gate_up = true): A = gu weights, B = xs (4 parts per routed row), writes xs_mid

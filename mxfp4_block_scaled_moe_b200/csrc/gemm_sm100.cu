@@ -77,6 +77,8 @@ struct Params {
   int tail_steps;            // K-steps of 32 in the final partial tile (0 or 2)
   float s_in;                // scale of the A operand (s0 gate_up / s1 down)
   float s_out;               // gate_up: quantization scale s1 of a
+  int a_shared;              // 1: every expert reads the same A rows (the dense all-experts
+                             // path: A row = row within the expert), 0: A row = grouped row
   uint8_t* a_out;            // gate_up output (P, I) e4m3
   float* y_out;              // down output (P, H) fp32
   int* err;
@@ -208,7 +210,7 @@ moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constan
             griddep_wait();
             dep_ready = true;
           }
-          tma_load_2d(sA + stage * kAStage, &tmap_a, &full[stage], kx, tl.m0);
+          tma_load_2d(sA + stage * kAStage, &tmap_a, &full[stage], kx, p.a_shared ? tl.m0 - p.offsets[tl.e] : tl.m0);
           if (++stage == kStages) { stage = 0; phase ^= 1; }
         }
       }
@@ -494,12 +496,13 @@ cudaError_t tc_gemm_prepare(int E) {
 }
 
 
-// a: grouped activation rows (P_rows, K) e4m3; blocks/scales: (E, rows_total, K/2) and
+// a: grouped activation rows (P_rows, K) e4m3 (a_shared: the T rows every expert reads);
+// blocks/scales: (E, rows_total, K/2) and
 // (E, rows_total, K/32); gate_up: rows_total = 2I, n_out = I; down: rows_total = n_out = H.
 cudaError_t launch_tc_gemm(bool gate_up, const uint8_t* a, int64_t P_rows, int K, const uint8_t* blocks,
                            const uint8_t* scales, const float* bias, int E, int n_out, const int32_t* offsets,
                            float s_in, float s_out, uint8_t* a_out, float* y_out, int* err, int sms,
-                           cudaStream_t st) {
+                           cudaStream_t st, bool a_shared) {
   using namespace g100;
   const int rows_per_group = n_out;          // one half of gate_up, or all of down
   const int groups = gate_up ? 2 * E : E;
@@ -538,6 +541,7 @@ cudaError_t launch_tc_gemm(bool gate_up, const uint8_t* a, int64_t P_rows, int K
   prm.tail_steps = (K % BK) / 32;
   prm.s_in = s_in;
   prm.s_out = s_out;
+  prm.a_shared = a_shared ? 1 : 0;
   prm.a_out = a_out;
   prm.y_out = y_out;
   prm.err = err;

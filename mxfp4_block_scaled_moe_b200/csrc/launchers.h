@@ -69,7 +69,7 @@ cudaError_t tc_gemm_prepare(int E);
 cudaError_t launch_tc_gemm(bool gate_up, const uint8_t* a, int64_t P_rows, int K, const uint8_t* blocks,
                            const uint8_t* scales, const float* bias, int E, int n_out, const int32_t* offsets,
                            float s_in, float s_out, uint8_t* a_out, float* y_out, int* err, int sms,
-                           cudaStream_t st);
+                           cudaStream_t st, bool a_shared = false);
 
 // bf16 activations on the tcgen05 grouped GEMM: each activation row as two e4m3 parts with
 // e8m0 scales per 32-value block (csrc/gemm_bf16_sm100.cu)
@@ -79,7 +79,7 @@ cudaError_t tc_parts_gemm_prepare(int E);
 cudaError_t launch_tc_parts_gemm(bool gate_up, const uint8_t* parts, const uint8_t* a_scales, int64_t P_rows, int K,
                                  const uint8_t* blocks, const uint8_t* scales, const float* bias, int E, int n_out,
                                  const int32_t* offsets, uint16_t* a_out, float* y_out, int* err, int sms,
-                                 cudaStream_t st);
+                                 cudaStream_t st, bool a_shared = false);
 
 struct DecodeGemmArgs {   // tensor-core decode path (kind::mxf4: packed e2m1 weights x e2m1 token parts)
   const uint8_t* gu_blocks;
@@ -99,7 +99,7 @@ struct DecodeGemmArgs {   // tensor-core decode path (kind::mxf4: packed e2m1 we
   const float* topk_w;
   const int32_t* inv;
   const uint8_t* xs;            // gate_up B operand: (P*4, H/2) packed e2m1 parts
-  const uint8_t* sfb;           // its scale records, one per row group (decode_tc_sfb_row_bytes)
+  const uint8_t* sfb;           // its scale records (decode_tc_sfb_bytes(E, H, T))
   uint8_t* xs_mid;              // down B operand: (P*4, I/2)
   uint8_t* sfb_mid;             // (decode_tc_sfb_bytes(E, I, T))
   float s0;                     // B scale of gate_up (FP8 s0, else 1)
@@ -120,8 +120,7 @@ bool decode_tc_supported(int H, int I, int T, const void* gu_blocks, const void*
                          const void* d_scales);
 cudaError_t decode_tc_prepare();
 size_t decode_tc_xs_bytes(int64_t P, int K);
-size_t decode_tc_sfb_bytes(int E, int K, int T);       // per 128-wide k-tile records (down's B)
-size_t decode_tc_sfb_row_bytes(int E, int T);          // one record per row group (gate_up's B)
+size_t decode_tc_sfb_bytes(int E, int K, int T);       // B scale records, one per 128-wide k-tile
 size_t decode_tc_part_bytes(int64_t P, int H, int I);
 size_t decode_tc_ticket_count(int H, int I);
 // offsets of the three ticket arrays inside the decode_tc_ticket_count block
@@ -134,10 +133,20 @@ cudaError_t launch_split_tokens(bool fp8, const uint16_t* x, const int32_t* topk
                                 cudaStream_t st);
 cudaError_t launch_decode_gemm(bool gate_up, const DecodeGemmArgs& a, cudaStream_t st);
 
+// dense all-experts path (csrc/dense.cu): gates (T, E) and offsets e * T; the weighted sum
+// over all experts of y laid out expert-major (E * T, H)
+cudaError_t launch_dense_setup(const int32_t* topk_idx, const float* topk_w, int T, int E, int k, float* gates,
+                               int32_t* offsets, cudaStream_t st, int sms);
+cudaError_t launch_dense_combine(const float* y, const float* gates, int T, int H, int E, uint16_t* out,
+                                 cudaStream_t st, int sms);
+
 cudaError_t launch_combine(const float* y, const int32_t* topk_idx, const float* topk_w,
                            const int32_t* inv, int T, int H, int k, uint16_t* out, cudaStream_t st,
                            int sms);
 
+
+// mxmoe_tc_rate_probe: back-to-back kind::mxf8f6f4 MMAs (M = 128, N = n) on `ctas` CTAs
+cudaError_t launch_tc_rate(int n, int with_copy, int iters, int ctas, int* err, cudaStream_t st);
 
 // mxmoe_selftest_wait_timeout: a bounded wait that expires (ETIMEOUT in *err)
 cudaError_t launch_wait_selftest(int* err, cudaStream_t st);

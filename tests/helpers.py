@@ -72,6 +72,48 @@ def output_tolerance_ok(out_bits: np.ndarray, ref_acc: np.ndarray, rel: float = 
     return bool(np.all(err <= bound)), float(np.max(err) / scale) if scale else 0.0, excess
 
 
+# ------------------------------------------------------------- row selection ----
+
+def covering_rows(idx: np.ndarray, E: int, tile: int = 128, extra=()):
+    """Tokens whose outputs, compared with the oracle, reach every expert's first and last
+    row tile of the grouped GEMMs (an expert's routed rows are its tokens in ascending
+    order, cut into tiles of `tile` rows; an expert with 1-3 rows is one partial tile).
+    Greedy: for each target tile not yet reached, the token of that tile that reaches the
+    most targets still open. Returns the sorted token ids (plus `extra`)."""
+    T, k = idx.shape
+    flat = idx.reshape(-1).astype(np.int64)
+    order = np.argsort(flat, kind="stable")             # pairs grouped by expert, ascending t
+    counts = np.bincount(flat, minlength=E)
+    starts = np.concatenate([[0], np.cumsum(counts)[:-1]])
+    rank = np.empty_like(flat)
+    rank[order] = np.arange(flat.size) - starts[flat[order]]
+    tile_of = (rank // tile).reshape(T, k)              # tile of each (token, slot) in its expert
+    open_ = set()
+    for e in np.nonzero(counts)[0]:
+        open_.add((int(e), 0))
+        open_.add((int(e), int((counts[e] - 1) // tile)))
+    members = {}                                        # target tile -> its tokens
+    for t in range(T):
+        for j in range(k):
+            key = (int(idx[t, j]), int(tile_of[t, j]))
+            if key in open_:
+                members.setdefault(key, []).append(t)
+    chosen = set(int(r) for r in extra)
+    for t in chosen:
+        for j in range(k):
+            open_.discard((int(idx[t, j]), int(tile_of[t, j])))
+    for key in sorted(open_):
+        if key not in open_:
+            continue
+        best = max(members[key], key=lambda t: sum((int(idx[t, j]), int(tile_of[t, j])) in open_
+                                                   for j in range(k)))
+        chosen.add(best)
+        for j in range(k):
+            open_.discard((int(idx[best, j]), int(tile_of[best, j])))
+    assert not open_
+    return np.array(sorted(chosen), dtype=np.int64)
+
+
 # ------------------------------------------------------------------ GPU helpers ----
 
 def to_device(p: Packed, device="cuda"):

@@ -98,3 +98,11 @@ def test_layer_argument_checks(L):
     assert cal(T=0) == EINVAL
     assert cal(tail=(None, None)) == EINVAL
     assert cal(dbias=None) == EINVAL and "d_bias" in err(L)
+
+
+def test_rate_probe_argument_checks(L):
+    f = ctypes.c_double(0.0)
+    assert L.mxmoe_tc_rate_probe(8, 0, 10, 1, ctypes.byref(f), None) == EINVAL and "multiple of 16" in err(L)
+    assert L.mxmoe_tc_rate_probe(264, 0, 10, 1, ctypes.byref(f), None) == EINVAL
+    assert L.mxmoe_tc_rate_probe(256, 0, 0, 1, ctypes.byref(f), None) == EINVAL and "iters" in err(L)
+    assert L.mxmoe_tc_rate_probe(256, 0, 10, 0, ctypes.byref(f), None) == EINVAL and "ctas" in err(L)

@@ -66,13 +66,16 @@ def test_ncu_traffic_reads_the_matching_block_and_drops_stale_sources(tmp_path, 
 def test_step_roofline_against_both_bounds():
     pk = {"hbm_gbs": 6538.6, "bf16_tflops": 1628.9, "bf16_tflops_sustained": 1376.3}
     # the 120B prefill step: 1,744,404,480 B and 818,392,596,480 FLOP
-    r = bench.step_roofline(1_744_404_480, 818_392_596_480, 0.85, pk, fp8=True)
+    r = bench.step_roofline(1_744_404_480, 818_392_596_480, 0.85, pk, fp8=True, fp8_peak=2500.0)
     m, n = r["measured"], r["nominal"]
-    assert m["bound"] == "tensor" and abs(m["t_bound_ms"] - 818.392596480 / 2752.6) < 1e-5
+    assert m["bound"] == "tensor" and abs(m["t_bound_ms"] - 818.392596480 / 2500.0) < 1e-5
+    # without a probe figure: twice the measured bf16 burst peak
+    r2 = bench.step_roofline(1_744_404_480, 818_392_596_480, 0.85, pk, fp8=True)
+    assert r2["measured"]["tensor_tflops"] == 2 * 1628.9
     assert abs(m["frac"] - m["t_bound_ms"] / 0.85) < 1e-4
     # nominal: 218 us of bytes at 8 TB/s against 182 us of FP8 FLOPs at 4.5 PF
     assert n["bound"] == "hbm" and abs(n["t_bound_ms"] - 0.2180506) < 1e-6
     # bf16 activations take the bf16 peaks
     b = bench.step_roofline(1_744_404_480, 818_392_596_480, 1.52, pk, fp8=False)
-    assert b["measured"]["tensor_tflops"] == 1376.3 and b["nominal"]["tensor_tflops"] == 2250.0
+    assert b["measured"]["tensor_tflops"] == 1628.9 and b["nominal"]["tensor_tflops"] == 2250.0
     assert b["nominal"]["bound"] == "tensor"

@@ -3,11 +3,14 @@ CPU (no GPU, no library code).
 
 Part p of a value is the residual left by parts 0..p-1, rounded to the nearest e2m1 grid
 point (ties to the even code) under a power-of-two scale 2^s, s the smallest exponent with
-max|residual| / 2^s <= 6 over the scale's group: the whole row for the gate_up input, each
-32-value block for the down input. The claim checked: over 2880-long dot products with
-N(0, 0.02) weights, the four-part expansion changes the result by about 2e-4 of the largest
-output (row scales: 2.2e-4 here) and less with block scales (1.5e-4), an order of magnitude
-inside the layer's 2e-3 bar; each part removes about three bits of the residual."""
+max|residual| / 2^s <= 6 over the scale's group. The decode GEMMs give every 32-value block
+its own scale per part (gate_up's input x and down's input a alike). The claims checked:
+over 2880-long dot products with N(0, 0.02) weights the four-part expansion changes the
+result by about 1.5e-4 of the largest output, an order of magnitude inside the layer's 2e-3
+bar; each part removes about three bits of the residual; and with an outlier channel (one
+value 1000x the rest of its row) block scales keep the error near that bound while one
+scale for the whole row would not (the other values would keep only the bits left below
+the outlier's, 4e-3 of the output)."""
 import numpy as np
 
 _GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
@@ -56,10 +59,21 @@ def test_four_e2m1_parts_keep_dot_products_within_3e4_of_their_size():
     K = 2880
     x = rng.standard_normal((8, K)).astype(np.float32).astype(np.float64)
     w = rng.normal(0.0, 0.02, (512, K))
-    row = _rel_err(x, w, K)               # gate_up input: one scale per part per row
-    blk = _rel_err(x, w, 32)              # down input: one scale per part per 32 values
+    row = _rel_err(x, w, K)               # one scale per part for the whole row
+    blk = _rel_err(x, w, 32)              # one scale per part per 32 values (the kernels')
     assert row < 3e-4 and blk < 2e-4 and blk < row
-    assert row < 2e-3 / 5                 # well inside the layer bar
+    assert blk < 2e-3 / 10                # well inside the layer bar
+
+
+def test_block_scales_absorb_outlier_channels():
+    rng = np.random.default_rng(9)
+    K = 2880
+    x = rng.standard_normal((8, K))
+    x[:, 17] *= 1000.0                    # one channel 10^3 x the rest
+    x[:, 1000] *= 300.0
+    w = rng.normal(0.0, 0.02, (512, K))
+    assert _rel_err(x, w, 32) < 1e-3      # block scales: inside the bar with room
+    assert _rel_err(x, w, K) > 2e-3       # a row-wide scale would break it
 
 
 def test_parts_converge_and_keep_small_values():

@@ -11,12 +11,14 @@ bit-exactly wherever the k-th and (k+1)-th router logits are not a near tie.
 
 Weights are MXFP4-packed by the oracle's quantizer; the GPU consumes the same bytes.
 """
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
 
 import oracle
-from helpers import Packed, output_tolerance_ok, pack, to_device
+from helpers import Packed, covering_rows, output_tolerance_ok, pack, to_device
 from mxfp4_block_scaled_moe_b200 import inputs
 
 pytestmark = pytest.mark.gpu
@@ -93,9 +95,13 @@ def test_tiny_fp8_all_outputs(B):
 
 
 @pytest.mark.parametrize("fp8", [False, True])
-def test_small_ragged_layer(B, fp8):
-    # H = 320 (10 blocks), I = 192 (6 blocks): neither a multiple of the 64-row tiles
-    p = pack(inputs.small_layer(E=8, k=3, T=77, H=320, I=192, seed=5, router_bias=True))
+@pytest.mark.parametrize("H,I", [(320, 192), (352, 224)])
+def test_small_ragged_layer(B, fp8, H, I):
+    # T = 77 > 64 with a handful of rows per expert. H = 320 (10 blocks), I = 192 (6): the
+    # tcgen05 grouped GEMMs with H != I and K tails (2.5 and 1.5 k-tiles of 128). H = 352,
+    # I = 224 (odd multiples of 32, which neither tensor-core path takes): the register-
+    # dequant kernels with H != I.
+    p = pack(inputs.small_layer(E=8, k=3, T=77, H=H, I=I, seed=5, router_bias=True))
     d = to_device(p)
     s = oracle.calibrate(p.x, p.router_w, p.router_b, *p.weights, p.lay.k) if fp8 else None
     check_rows(B, p, d, np.arange(p.lay.T), act_scale=s)
@@ -197,16 +203,21 @@ def test_bf16_prefill_two_part_tcgen05_path(B, H, I, E, k, T):
     check_rows(B, p, d, rows, out=out)
 
 
-def test_prefill_120b_shape_bf16_sampled(B):
+def _gpu_idx(B, d, k):
+    idx, _ = B.moe_route_topk(d["x"], d["router_w"], d["router_b"], k)
+    return idx.cpu().numpy()
+
+
+def test_prefill_120b_shape_bf16_every_expert_tile(B):
     lay = inputs.prefill_layer(T=4096, E=128, device="cuda")
     p, d = layer_case(lay)
     out1 = run_gpu(B, d, lay.k)
     out2 = run_gpu(B, d, lay.k)
     assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))   # run-to-run identical
-    check_rows(B, p, d, _sample_rows(4096, 24, 4), out=out1)
+    rows = covering_rows(_gpu_idx(B, d, lay.k), lay.E, extra=(0, 4095))
+    check_rows(B, p, d, rows, out=out1)
 
 
-@pytest.mark.skip(reason="H != I on the tensor-core paths has not run on a GPU yet")
 @pytest.mark.parametrize("T,fp8", [(400, True), (400, False), (8, False), (8, True)])
 def test_tensor_core_paths_with_H_ne_I(B, T, fp8):
     """H = 320 (2.5 k-tiles of 128), I = 192 (1.5): 1600 routed pairs take the tcgen05
@@ -226,7 +237,7 @@ def _sample_rows(T, n, seed):
     return rows
 
 
-def test_prefill_120b_shape_fp8_sampled(B):
+def test_prefill_120b_shape_fp8_every_expert_tile(B):
     lay = inputs.prefill_layer(T=4096, E=128, device="cuda")
     p, d = layer_case(lay)
     xc = inputs.calibration_x(device="cuda")
@@ -234,20 +245,19 @@ def test_prefill_120b_shape_fp8_sampled(B):
     out1 = run_gpu(B, d, lay.k, act_scale=s)
     out2 = run_gpu(B, d, lay.k, act_scale=s)
     assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))   # run-to-run identical
-    check_rows(B, p, d, _sample_rows(4096, 24, 1), act_scale=s, out=out1)
+    rows = covering_rows(_gpu_idx(B, d, lay.k), lay.E, extra=(0, 4095))
+    check_rows(B, p, d, rows, act_scale=s, out=out1)
 
 
-def test_prefill_zipf_skew_sampled(B):
+def test_prefill_zipf_skew_every_expert_tile(B):
     lay = inputs.zipf_layer(T=16384, E=128, device="cuda")
     p, d = layer_case(lay)
-    idx, _ = B.moe_route_topk(d["x"], d["router_w"], d["router_b"], lay.k)
-    load = np.bincount(idx.cpu().numpy().reshape(-1), minlength=lay.E)
+    idx = _gpu_idx(B, d, lay.k)
+    load = np.bincount(idx.reshape(-1), minlength=lay.E)
     assert (load == 0).sum() >= 3 and load.max() > 10 * load.mean()
     xc = inputs.calibration_x(device="cuda")
     s = oracle.calibrate(inputs.bits(xc), p.router_w, p.router_b, *p.weights, lay.k)
-    hot = int(np.argmax(load))
-    rows = np.unique(np.concatenate([_sample_rows(16384, 12, 2),
-                                     np.nonzero((idx.cpu().numpy() == hot).any(1))[0][:4]]))
+    rows = covering_rows(idx, lay.E, extra=(0, 16383))
     check_rows(B, p, d, rows, act_scale=s)
 
 
@@ -285,3 +295,95 @@ def test_empty_batch_and_bad_arguments(B):
     c_bad[0] = ctypes.c_void_p(args[0] + 2)
     assert L.moe_mxfp4_forward(*c_bad, 4, 2, 16, 256, 256, None, ctypes.c_void_p(o.data_ptr()), None) == B.EINVAL
     assert L.moe_mxfp4_forward(*c, 4, 2, 16, 256, 256, None, None, None) == B.EINVAL
+
+
+# ------------------------------------------------ activation outliers, wide scale ranges --
+
+_OUTLIER_CHANNELS = ((17, 1000.0), (1000, 300.0))
+
+
+def _with_outliers(x: torch.Tensor) -> torch.Tensor:
+    """x with two channels scaled up (one 10^3 x, one 300 x the rest), as bf16."""
+    y = x.float().clone()
+    for c, m in _OUTLIER_CHANNELS:
+        y[:, c % x.shape[1]] *= m
+    return y.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("path,T,fp8", [("decode", 1, False), ("decode", 8, False), ("decode", 64, False),
+                                        ("decode", 1, True), ("decode", 8, True),
+                                        ("parts", 300, False), ("fp8", 300, True)])
+def test_activation_outlier_channels(B, path, T, fp8):
+    """Tokens whose row holds one channel 1000x and one 300x the others. On the decode
+    path (T <= 64) each activation becomes four e2m1 parts under per-32-value block scales
+    (a row-wide scale would leave the other values only the bits below the outlier's); on
+    the bf16 prefill path two e4m3 parts under block scales; FP8 activations saturate at
+    +-448 s0 with the scales of a calibration batch that has the same outlier channels."""
+    if path == "decode":
+        lay = inputs.decode_layer(T=T, E=32, device="cuda")
+        rows = np.arange(T)
+    else:
+        lay = inputs.small_layer(E=6, k=4, T=T, H=2880, I=2880, seed=7, router_bias=True,
+                                 router_std=1.0 / np.sqrt(2880), device="cuda")
+        rows = _sample_rows(T, 24, 5)
+    lay = dataclasses.replace(lay, x=_with_outliers(lay.x))
+    p, d = layer_case(lay)
+    s = None
+    if fp8:
+        xc = _with_outliers(inputs.calibration_x(device="cuda"))
+        s = oracle.calibrate(inputs.bits(xc), p.router_w, p.router_b, *p.weights, p.lay.k)
+    check_rows(B, p, d, rows, act_scale=s)
+
+
+def _wide_scale_pack(lay: inputs.Layer, mode: str) -> Packed:
+    """The layer's weights with C2's outliers (1% of values x 8) before the oracle's
+    quantizer, then scale bytes rewritten: mode "tiny" sets 2% of the blocks to bytes 0-3
+    (2^-127 .. 2^-124: subnormal products), mode "huge" sets 0.3% of them to bytes 136-140
+    (2^9 .. 2^13 times the others' range) while outputs stay finite. Oracle and GPU consume
+    the same bytes."""
+    E, H, I = lay.E, lay.H, lay.I
+    rng = np.random.default_rng(1234 + (mode == "huge"))
+    gu_b = np.empty((E, 2 * I, H // 2), np.uint8)
+    gu_s = np.empty((E, 2 * I, H // 32), np.uint8)
+    d_b = np.empty((E, H, I // 2), np.uint8)
+    d_s = np.empty((E, H, I // 32), np.uint8)
+
+    def one(w):
+        w = w.cpu().numpy().copy()
+        w[rng.random(w.shape) < 0.01] *= 8.0
+        b, sc = oracle.quantize(w)
+        if mode == "tiny":
+            m = rng.random(sc.shape) < 0.02
+            sc[m] = rng.integers(0, 4, size=int(m.sum()))
+        else:
+            m = rng.random(sc.shape) < 0.003
+            sc[m] = rng.integers(136, 141, size=int(m.sum()))
+        return b, sc
+
+    for e in range(E):
+        gu_b[e], gu_s[e] = one(lay.gate_up(e))
+        d_b[e], d_s[e] = one(lay.down(e))
+    rb = None if lay.router_b is None else inputs.bits(lay.router_b)
+    return Packed(lay, inputs.bits(lay.x), inputs.bits(lay.router_w), rb, gu_b, gu_s,
+                  lay.gu_bias.cpu().numpy(), d_b, d_s, lay.d_bias.cpu().numpy())
+
+
+@pytest.mark.parametrize("mode", ["tiny", "huge"])
+@pytest.mark.parametrize("T,k,H,fp8", [(600, 2, 512, True), (600, 2, 512, False), (8, 4, 512, False),
+                                       (8, 4, 512, True), (100, 2, 480, False)])
+def test_wide_e8m0_weight_scales(B, mode, T, k, H, fp8):
+    """Weights whose e8m0 scale bytes span the format: blocks at bytes 0-3 beside ordinary
+    ones near 120, or a few blocks at 136-140, on every path: the tcgen05 prefill GEMMs
+    (T = 600, FP8 and bf16 as two parts), the tensor-core decode GEMMs (T = 8) and the
+    register-dequant kernels (H = I = 480, not a multiple of 64, which neither tensor-core
+    path takes)."""
+    lay = inputs.small_layer(E=8, k=k, T=T, H=H, I=H, seed=21, router_bias=True,
+                             router_std=1.0 / np.sqrt(H), device="cuda")
+    p = _wide_scale_pack(lay, mode)
+    d = to_device(p)
+    s = None
+    if fp8:
+        s = oracle.calibrate(p.x[: min(T, 256)], p.router_w, p.router_b, *p.weights, k)
+    out = run_gpu(B, d, k, act_scale=s)
+    assert torch.isfinite(out.float()).all()
+    check_rows(B, p, d, np.arange(T), act_scale=s, out=out)

@@ -1,0 +1,31 @@
+"""The tensor-pipe rate probe (mxmoe_tc_rate_probe) that gives the benchmark its FP8
+roofline denominator: it runs to completion without a device error, reports the FLOPs
+of its MMAs, and measures a rate within the physically possible range for a B200 (the
+tensor pipe of 148 SMs between ~1 and ~2 GHz)."""
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+
+def _rate(B, n, copy, iters=4000):
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    f = B.mxmoe_tc_rate_probe(n, copy, iters)
+    e1.record()
+    torch.cuda.synchronize()
+    B.mxmoe_check()
+    return f, f / (e0.elapsed_time(e1) / 1e3) / 1e12
+
+
+def test_rate_probe_runs_and_reports_its_flops():
+    from mxfp4_block_scaled_moe_b200 import binding as B
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    B.mxmoe_tc_rate_probe(256, False, 10)          # load
+    f, tf = _rate(B, 256, False)
+    assert f == 2.0 * 128 * 256 * 32 * 4 * 4000 * sms
+    # a block-scaled M=128 N=256 K=32 MMA moves at most 2*128*256*32 / 128 = 16384 FLOP per
+    # SM cycle; 148 SMs at 1.0-2.1 GHz bound the measured rate
+    assert 0.2 * 16384 * sms * 1.0e9 / 1e12 < tf < 16384 * sms * 2.1e9 / 1e12 * 1.05
+    _, tf_copy = _rate(B, 240, True)
+    assert 0.0 < tf_copy < tf * 1.05               # the scale copy only takes pipe time

@@ -62,3 +62,27 @@ def test_noalloc_permute_rejects_sizes_beyond_its_scratch():
     rc = L.moe_permute_noalloc(ctypes.c_void_p(idx.data_ptr()), 65537, 8, 4, None, None, None, None)
     assert rc == B.EUNSUPPORTED
     assert b"262144" in L.mxmoe_last_error()
+
+
+def test_noalloc_permute_drops_an_out_of_range_expert_id():
+    """A pair whose expert id lies outside [0, E) is left out: offsets[E] counts the other
+    T*k - 1 pairs, which are grouped exactly as moe_permute groups them; the positions from
+    offsets[E] on stay unwritten, and the device error word stays clear (moe_permute itself
+    reports the same input as MXMOE_EDEVICE)."""
+    from mxfp4_block_scaled_moe_b200 import binding as B
+    L = B.lib()
+    T, E, k = 300, 32, 4
+    idx = _routing(T, E, k, 0.3, seed=5)
+    idx[123, 2] = E                      # one id past the last expert
+    B.mxmoe_check()                      # start from a clear error word
+    off, pt, ps = _noalloc(L, idx, E)
+    assert L.mxmoe_check(None) == 0
+    n = T * k - 1
+    assert int(off[E]) == n
+    assert torch.all(pt[n:] == -1) and torch.all(ps[n:] == -1)
+    ref = B.moe_permute(idx, E)
+    with pytest.raises(B.MxmoeError) as ei:
+        B.mxmoe_check()
+    assert ei.value.rc == B.EDEVICE
+    assert torch.equal(off, ref[0])
+    assert torch.equal(pt[:n], ref[1][:n]) and torch.equal(ps[:n], ref[2][:n])
