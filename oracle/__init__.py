@@ -214,6 +214,78 @@ def calibrate(x, router_w, router_b, gu_blocks, gu_scales, gu_bias, d_blocks, d_
     return s
 
 
+def quantize_axis(w, axis):
+    """MXFP4 along one contracting axis, moved to the end ("quantization_mxfp4",
+    Primitives: MXFP4Quantizer.quantize(w, axis)). Returns blocks (shape with `axis` moved
+    last, K/2 there) and scales (K/32 there)."""
+    w = _c(w, np.float32)
+    axis = axis % w.ndim
+    K = w.shape[axis]
+    outer = int(np.prod(w.shape[:axis])) if axis else 1
+    inner = int(np.prod(w.shape[axis + 1:])) if axis + 1 < w.ndim else 1
+    moved = w.shape[:axis] + w.shape[axis + 1:]
+    if K % 32:
+        _check(lib().orc_quantize_axis(None, _i64(outer), _i64(K), _i64(inner), None, None), "quantize_axis")
+    blocks = np.empty(moved + (K // 2,), np.uint8)
+    scales = np.empty(moved + (K // 32,), np.uint8)
+    _check(lib().orc_quantize_axis(_p(w), _i64(outer), _i64(K), _i64(inner), _p(blocks), _p(scales)),
+           "quantize_axis")
+    return blocks, scales
+
+
+def dequantize_axis(blocks, scales, axis, out="f32"):
+    """Inverse of quantize_axis: the packed axis (last) goes back to position `axis`."""
+    blocks = _c(blocks, np.uint8)
+    scales = _c(scales, np.uint8)
+    K = blocks.shape[-1] * 2
+    moved = blocks.shape[:-1]
+    nd = len(moved) + 1
+    axis = axis % nd
+    shape = moved[:axis] + (K,) + moved[axis:]
+    outer = int(np.prod(shape[:axis])) if axis else 1
+    inner = int(np.prod(shape[axis + 1:])) if axis + 1 < nd else 1
+    f32 = np.empty(shape, np.float32) if out == "f32" else None
+    b16 = np.empty(shape, np.uint16) if out == "bf16" else None
+    _check(lib().orc_dequantize_axis(_p(blocks), _p(scales), _i64(outer), _i64(K), _i64(inner), _p(f32),
+                                     _p(b16)), "dequantize_axis")
+    return f32 if out == "f32" else b16
+
+
+def linear(x, blocks, scales, bias=None, act_scale=None):
+    """MXFP4 weight-only linear, optional FP8 activations: out = bf16(fp32(s * x.W^T) + b).
+
+    ("quantization_mxfp4", As a quantize_model scheme.) Returns (out bf16 bits (T, N),
+    acc fp32 (T, N))."""
+    x = _c(x, np.uint16)
+    blocks = _c(blocks, np.uint8)
+    scales = _c(scales, np.uint8)
+    T, K = x.shape
+    N = blocks.shape[0]
+    b = None if bias is None else _c(bias, np.float32)
+    s = None if act_scale is None else np.array([act_scale], np.float32)
+    out = np.empty((T, N), np.uint16)
+    acc = np.empty((T, N), np.float32)
+    _check(lib().orc_linear(_p(x), T, K, _p(blocks), _p(scales), N, _p(b), _p(s), _p(out), _p(acc)), "linear")
+    return out, acc
+
+
+def fp8_linear(x, wq, s_x, s_w, bias=None):
+    """FP8 E4M3 static per-tensor linear: out = bf16(fp32(s_x s_w dec(xq).dec(wq)^T) + b).
+
+    ("gpt-oss-120b-mxfp4-fp8attn-v2", Model Details / Quantization Recipe.) Returns
+    (out bf16 bits (T, N), acc fp32 (T, N))."""
+    x = _c(x, np.uint16)
+    wq = _c(wq, np.uint8)
+    T, K = x.shape
+    N = wq.shape[0]
+    b = None if bias is None else _c(bias, np.float32)
+    out = np.empty((T, N), np.uint16)
+    acc = np.empty((T, N), np.float32)
+    _check(lib().orc_fp8_linear(_p(x), T, K, _p(wq), N, ctypes.c_float(s_x), ctypes.c_float(s_w), _p(b),
+                                _p(out), _p(acc)), "fp8_linear")
+    return out, acc
+
+
 def num_threads() -> int:
     """Threads the oracle's OpenMP loops use (OMP_NUM_THREADS, else all cores)."""
     v = os.environ.get("OMP_NUM_THREADS")

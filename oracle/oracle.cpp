@@ -20,7 +20,12 @@
 //  * "amd/gpt-oss-20b-MoE-Quant-W-MXFP4-A-FP8-KV-FP8", "Quantization schemes": weights
 //    OCP MXFP4, activations FP8 symmetric per-tensor, router not quantized.
 //  * "gpt-oss-120b-mxfp4-fp8attn-v2", "Model Details" / "Quantization Recipe": FP8 E4M3
-//    with static per-tensor scales from min-max calibration; router kept unquantized.
+//    with static per-tensor scales from min-max calibration; router kept unquantized;
+//    attention projections Q/K/V/O as FP8 E4M3 weights with a static per-tensor weight
+//    scale and input scale.
+//  * "quantization_mxfp4", "Primitives": MXFP4Quantizer quantizes along one arbitrary
+//    contracting axis, which it moves to the end; "As a quantize_model scheme": any
+//    Dense kernel can be stored MXFP4 (weight-only) and dequantized on the fly.
 //
 // Readings where the pages are silent (each listed in the design notes):
 //  - nibble order: element 2j sits in the low nibble of byte j;
@@ -447,6 +452,111 @@ int orc_calibrate(const uint16_t* x, const uint16_t* router_w, const uint16_t* r
   for (int t = 0; t < T; ++t) am = std::max(am, amid[t]);
   act_scale_out[0] = ax / 448.0f;
   act_scale_out[1] = am / 448.0f;
+  return ORC_OK;
+}
+
+// --------------------------------------------- quantizer along an arbitrary axis ---
+
+// "quantization_mxfp4", Primitives (MXFP4Quantizer.quantize(w, axis)): the tensor is
+// viewed as (outer, K, inner) with the contracting axis (length K) in the middle; that
+// axis moves to the end and every resulting row of K values is quantized as orc_quantize
+// does. blocks: (outer, inner, K/2); scales: (outer, inner, K/32).
+int orc_quantize_axis(const float* w, int64_t outer, int64_t K, int64_t inner, uint8_t* blocks,
+                      uint8_t* scales) {
+  if (outer < 0 || K < 0 || inner < 0) return ORC_EINVAL;
+  if (K % 32 != 0) return ORC_EALIGN;
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < outer * inner; ++r) {
+    const int64_t o = r / inner, i = r % inner;
+    std::vector<float> row(K);
+    for (int64_t k = 0; k < K; ++k) row[k] = w[(o * K + k) * inner + i];
+    orc_quantize(row.data(), 1, K, blocks + r * (K / 2), scales + r * (K / 32));
+  }
+  return ORC_OK;
+}
+
+// The inverse view: dequantize every (outer, inner) row of K values and put the axis
+// back in the middle: out (outer, K, inner). Either output may be null.
+int orc_dequantize_axis(const uint8_t* blocks, const uint8_t* scales, int64_t outer, int64_t K,
+                        int64_t inner, float* out_f32, uint16_t* out_bf16) {
+  if (outer < 0 || K < 0 || inner < 0) return ORC_EINVAL;
+  if (K % 32 != 0) return ORC_EALIGN;
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < outer * inner; ++r) {
+    const int64_t o = r / inner, i = r % inner;
+    std::vector<float> f(K);
+    std::vector<uint16_t> b(K);
+    orc_dequantize(blocks + r * (K / 2), scales + r * (K / 32), 1, K, f.data(), b.data());
+    for (int64_t k = 0; k < K; ++k) {
+      if (out_f32) out_f32[(o * K + k) * inner + i] = f[k];
+      if (out_bf16) out_bf16[(o * K + k) * inner + i] = b[k];
+    }
+  }
+  return ORC_OK;
+}
+
+// ------------------------------------------------------------------------ linear ---
+
+// MXFP4 weight-only linear ("quantization_mxfp4", As a quantize_model scheme), with the
+// optional FP8 E4M3 static per-tensor activations of the W-MXFP4 / A-FP8 scheme:
+// y[t, n] = fp32( fp32(s * sum_k xin[t, k] W[n, k]) + b[n] ), out = bf16(y), where xin is
+// the bf16 input (s = 1) or, with act_scale != null, e4m3(fp32(x / s)) with s = *act_scale.
+// x: (T, K) bf16; blocks (N, K/2), scales (N, K/32); bias (N) fp32 or null (zero).
+int orc_linear(const uint16_t* x, int T, int K, const uint8_t* blocks, const uint8_t* scales, int N,
+               const float* bias, const float* act_scale, uint16_t* out, float* acc_out) {
+  if (!x || !blocks || !scales || !out || T < 0 || K <= 0 || N <= 0) return ORC_EINVAL;
+  if (K % 32 != 0) return ORC_EALIGN;
+  const double s = act_scale ? static_cast<double>(*act_scale) : 1.0;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int t = 0; t < T; ++t) {
+    std::vector<double> xin(K), row(K);
+    for (int k = 0; k < K; ++k) {
+      const float v = bf16_to_f32(x[(int64_t)t * K + k]);
+      if (act_scale) {
+        volatile float q = v / *act_scale;
+        xin[k] = e4m3_value(e4m3_rne_satfinite(q));
+      } else {
+        xin[k] = v;
+      }
+    }
+    for (int n = 0; n < N; ++n) {
+      dequant_row(blocks + (int64_t)n * (K / 2), scales + (int64_t)n * (K / 32), K, row.data());
+      double acc = 0.0;
+      for (int k = 0; k < K; ++k) acc += xin[k] * row[k];
+      volatile float prod = static_cast<float>(s * acc);
+      const float y = prod + (bias ? bias[n] : 0.0f);
+      out[(int64_t)t * N + n] = bf16_rne(y);
+      if (acc_out) acc_out[(int64_t)t * N + n] = y;
+    }
+  }
+  return ORC_OK;
+}
+
+// FP8 E4M3 static per-tensor linear ("gpt-oss-120b-mxfp4-fp8attn-v2", Model Details and
+// Quantization Recipe: Q/K/V/O projections with FP8 E4M3 weights, a static per-tensor
+// weight_scale and a static per-tensor input_scale). The dequantized operands are
+// dec(xq) * s_x and dec(wq) * s_w, so
+// y[t, n] = fp32( s_x * s_w * sum_k dec(xq[t, k]) dec(wq[n, k]) ) + b[n], out = bf16(y),
+// with xq = e4m3(fp32(x / s_x)). x: (T, K) bf16; wq: (N, K) e4m3 codes; bias null = zero.
+int orc_fp8_linear(const uint16_t* x, int T, int K, const uint8_t* wq, int N, float s_x, float s_w,
+                   const float* bias, uint16_t* out, float* acc_out) {
+  if (!x || !wq || !out || T < 0 || K <= 0 || N <= 0 || !(s_x > 0.0f) || !(s_w > 0.0f)) return ORC_EINVAL;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int t = 0; t < T; ++t) {
+    std::vector<double> xin(K);
+    for (int k = 0; k < K; ++k) {
+      volatile float q = bf16_to_f32(x[(int64_t)t * K + k]) / s_x;
+      xin[k] = e4m3_value(e4m3_rne_satfinite(q));
+    }
+    for (int n = 0; n < N; ++n) {
+      double acc = 0.0;   // exact: e4m3 products have at most 8 significant bits
+      for (int k = 0; k < K; ++k) acc += xin[k] * e4m3_value(wq[(int64_t)n * K + k]);
+      volatile float prod = static_cast<float>(static_cast<double>(s_x) * static_cast<double>(s_w) * acc);
+      const float y = prod + (bias ? bias[n] : 0.0f);
+      out[(int64_t)t * N + n] = bf16_rne(y);
+      if (acc_out) acc_out[(int64_t)t * N + n] = y;
+    }
+  }
   return ORC_OK;
 }
 
