@@ -34,6 +34,7 @@ host cores (rank 0 only).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -64,6 +65,7 @@ WORKLOADS = {
     "decode64": (lambda dev: inputs.decode_layer(T=64, E=32, device=dev), False),
 }
 CODEC = "codec"
+CROSSOVER = "crossover"
 # The default line: the largest single-GPU configuration (120B-shaped prefill, T = 16384,
 # Zipf-skewed routing), then the 120B prefill at T = 4096 and the 20B decode batches
 # measured in the same run.
@@ -591,6 +593,84 @@ def run_ours(args, world, rank):
     return res
 
 
+# ------------------------------------------------------- routed / dense crossover -----
+
+CROSSOVER_GRID = ((32, 4, (16, 64, 128, 256, 512, 1024)), (128, 4, (64, 256, 512, 1024, 2048, 4096)),
+                  (8, 8, (128, 1024, 4096)), (4, 4, (128, 1024, 4096)))
+
+
+def time_steps(fn, steps, flusher):
+    """Mean device time of one call of fn over `steps` calls captured in one CUDA graph,
+    L2 flushed before each (CUDA events around every call)."""
+    ev = [(torch.cuda.Event(enable_timing=True, external=True),
+           torch.cuda.Event(enable_timing=True, external=True)) for _ in range(steps)]
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        for i in range(steps):
+            flusher(i)
+            ev[i][0].record()
+            fn()
+            ev[i][1].record()
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    del g
+    return ms
+
+
+def run_crossover(args, world, rank):
+    """The routed path (moe_mxfp4_forward) against the dense all-experts path
+    (moe_mxfp4_forward_dense) on the same layer, FP8 activations, uniform routing
+    (router N(0, 1/sqrt(H))), H = I = 2880, over a grid of (E, k, T): top-4 of 32 and of
+    128 experts, and k = E (every expert selected, where both paths do the same expert
+    work). Reports both step times; the dense path does E/k times the expert work but needs
+    no permutation, gather or scatter."""
+    from mxfp4_block_scaled_moe_b200 import binding as B
+    flusher = L2Flush()
+    cache = {}
+    rows = []
+    for E, k, Ts in CROSSOVER_GRID:
+        for T in Ts:
+            lay = dataclasses.replace(inputs.prefill_layer(T=T, E=E, device="cuda"), k=k)
+            gu_b, gu_s, d_b, d_s = layer_weights(lay, "cuda", cache)
+            d = dict(x=lay.x, router_w=lay.router_w, router_b=lay.router_b, gu_blocks=gu_b, gu_scales=gu_s,
+                     gu_bias=lay.gu_bias, d_blocks=d_b, d_scales=d_s, d_bias=lay.d_bias)
+            xc = inputs.calibration_x(H=lay.H, device="cuda")
+            act = B.moe_mxfp4_calibrate(xc, lay.router_w, lay.router_b, gu_b, gu_s, lay.gu_bias,
+                                        d_b, d_s, lay.d_bias, lay.k).cpu().tolist()
+            out = torch.empty(T, lay.H, dtype=torch.bfloat16, device="cuda")
+            out_d = torch.empty_like(out)
+            routed = lambda: forward(B, d, lay.k, act, out)
+            dense = lambda: B.moe_mxfp4_forward_dense(d["x"], d["router_w"], d["router_b"], d["gu_blocks"],
+                                                      d["gu_scales"], d["gu_bias"], d["d_blocks"], d["d_scales"],
+                                                      d["d_bias"], lay.k, act_scale=act, out=out_d)
+            for _ in range(args.warmup):
+                routed()
+                dense()
+            B.mxmoe_check()
+            t_r = time_steps(routed, args.steps, flusher)
+            t_d = time_steps(dense, args.steps, flusher)
+            B.mxmoe_check()
+            same = bool(torch.equal(out.view(torch.int16), out_d.view(torch.int16))) if T > 64 else None
+            rows.append({"E": E, "k": lay.k, "T": T, "routed_ms": round(t_r, 5), "dense_ms": round(t_d, 5),
+                         "dense_over_routed": round(t_d / t_r, 3), "outputs_bit_identical": same})
+            del d, lay
+    return {"metric": "routed vs dense all-experts MoE-layer step time", "unit": "ms", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": False,
+            "dtype": "e4m3 x e2m1 -> f32", "data": "synthetic (seeded; uniform routing)",
+            "config": {"workload": "crossover: H = I = 2880, FP8 activations",
+                       "l2": "flushed before every timed step"},
+            "table": rows}
+
+
 # ---------------------------------------------------------------- codec sweep -----
 
 CODEC_H = 2880   # H = I = 2880: gate_up (E, 2I, H) and down (E, H, I) share K = 2880
@@ -871,7 +951,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS) + [CODEC], default=DEFAULT_WORKLOAD)
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + [CODEC, CROSSOVER], default=DEFAULT_WORKLOAD)
     ap.add_argument("--extra", default=None,
                     help="comma-separated workloads measured in the same run and reported under "
                          "other_configs (default: the 120B prefill and the three decode batches "
@@ -898,11 +978,17 @@ def main():
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))
-        res = (run_reference_codec if args.workload == CODEC else run_reference)(args, world, rank)
+        if args.workload == CROSSOVER:
+            res = {"impl": "reference", "unavailable": "the crossover workload compares two GPU paths; "
+                                                       "the oracle has no counterpart to time"}
+            res = res if int(os.environ.get("RANK", "0")) == 0 else None
+        else:
+            res = (run_reference_codec if args.workload == CODEC else run_reference)(args, world, rank)
     else:
         world, rank = dist_init()
         try:
-            res = (run_codec if args.workload == CODEC else run_ours)(args, world, rank)
+            run = {CODEC: run_codec, CROSSOVER: run_crossover}.get(args.workload, run_ours)
+            res = run(args, world, rank)
         finally:
             if world > 1:
                 import torch.distributed as dist

@@ -80,6 +80,55 @@ int mxfp4_quantize(const float* w, int64_t rows, int64_t K, uint8_t* blocks, uin
 int mxfp4_dequantize(const uint8_t* blocks, const uint8_t* scales, int64_t rows, int64_t K,
                      void* out, int out_dtype, void* stream);
 
+/* mxfp4_quantize_axis / mxfp4_dequantize_axis -- the codec along an arbitrary contracting
+ * axis ("quantization_mxfp4" (KerasFormers), Primitives: MXFP4Quantizer.quantize(w, axis)
+ * quantizes along one axis, which it moves to the end). The tensor w is viewed as
+ * (outer, K, inner): K is the length of the contracting axis, outer the product of the
+ * dims before it, inner the product of the dims after it (inner = 1: the last axis, the
+ * same as mxfp4_quantize). The packed result has the axis last: blocks (outer, inner,
+ * K/2), scales (outer, inner, K/32), each row of K values quantized exactly as
+ * mxfp4_quantize does (same bits). mxfp4_dequantize_axis is the inverse view: it writes
+ * (outer, K, inner) fp32 (out_dtype MXMOE_OUT_F32) or bf16 (MXMOE_OUT_BF16) values, the
+ * same values as mxfp4_dequantize. All pointers are device memory, caller-owned; w,
+ * blocks and out 16-byte aligned. Errors: MXMOE_EALIGN if K % 32 != 0 (the clear error of
+ * "As a quantize_model scheme"), MXMOE_EINVAL for a negative size, a null or misaligned
+ * pointer, MXMOE_EUNSUPPORTED for an unknown out_dtype, MXMOE_ECUDA on a launch error.
+ * Any zero size is a no-op. */
+int mxfp4_quantize_axis(const float* w, int64_t outer, int64_t K, int64_t inner, uint8_t* blocks,
+                        uint8_t* scales, void* stream);
+int mxfp4_dequantize_axis(const uint8_t* blocks, const uint8_t* scales, int64_t outer, int64_t K,
+                          int64_t inner, void* out, int out_dtype, void* stream);
+
+/* mxfp4_linear -- a plain MXFP4 weight-only linear layer ("quantization_mxfp4", As a
+ * quantize_model scheme: a Dense kernel stored MXFP4 and dequantized on the fly), with the
+ * optional FP8 E4M3 static per-tensor activations of the W-MXFP4 / A-FP8 scheme ("amd/gpt-
+ * oss-20b-MoE-Quant-W-MXFP4-A-FP8-KV-FP8", Quantization schemes):
+ *   out[t, n] = bf16( fp32(s * sum_k xin[t, k] * W[n, k]) + bias[n] ),
+ * xin = x (bf16, s = 1) or, with act_scale != NULL, e4m3(fp32(x / s)) with s = *act_scale
+ * (a HOST pointer to one float). x: device bf16 (T, K); blocks (N, K/2) and scales
+ * (N, K/32) as mxfp4_quantize packs a (N, K) weight; bias: device fp32 (N) or NULL (zero);
+ * out: device bf16 (T, N). More than 64 tokens run on the tcgen05 grouped GEMM (one
+ * expert) when K and N are multiples of 64 (K <= 4608), else the register-dequant
+ * kernel. Errors: MXMOE_EALIGN (K % 32, N % 16), MXMOE_EINVAL (sizes, null or misaligned
+ * pointers: x, blocks, out and bias 16-byte aligned), MXMOE_ECUDA. Uses the library
+ * workspace; T = 0 is a no-op. */
+int mxfp4_linear(const uint16_t* x, int T, int K, const uint8_t* blocks, const uint8_t* scales, int N,
+                 const float* bias, const float* act_scale, uint16_t* out, void* stream);
+
+/* fp8_linear -- the FP8 E4M3 static per-tensor linear of the attention projections
+ * ("gpt-oss-120b-mxfp4-fp8attn-v2", Model Details and Quantization Recipe: Q/K/V/O with
+ * FP8 E4M3 weights, a static per-tensor weight scale and input scale):
+ *   out[t, n] = bf16( fp32(fp32(s_x * s_w) * sum_k xq[t, k] * wq[n, k]) + bias[n] ),
+ * xq = e4m3(fp32(x / s_x)) (round to nearest even, saturating at +-448). x: device bf16
+ * (T, K); wq: device E4M3 codes (N, K) (the checkpoint's FP8 weight); s_x, s_w: the
+ * static input and weight scales (> 0); bias: device fp32 (N) or NULL; out: device bf16
+ * (T, N). Runs on tcgen05 (kind::f8f6f4) with fp32 accumulation, K split over the SMs
+ * when there are few tokens. Errors: MXMOE_EALIGN (K % 32, N % 8), MXMOE_EINVAL (sizes,
+ * scales, null or misaligned pointers: x, wq, out, bias 16-byte aligned), MXMOE_ECUDA.
+ * Uses the library workspace; T = 0 is a no-op. */
+int fp8_linear(const uint16_t* x, int T, int K, const uint8_t* wq, int N, float s_x, float s_w,
+               const float* bias, uint16_t* out, void* stream);
+
 /* moe_route_topk -- router + top-k softmax (GPT-OSS top-k routing; router kept in bf16:
  * "gpt-oss-120b-mxfp4-fp8attn-v2", config.json modules_to_not_convert).
  * x: device bf16 (T, H); router_w: device bf16 (E, H); router_b: device bf16 (E) or NULL.
@@ -176,6 +225,32 @@ int moe_mxfp4_forward_dense(const uint16_t* x, const uint16_t* router_w, const u
                             const uint8_t* d_blocks, const uint8_t* d_scales, const float* d_bias,
                             int E, int k, int T, int H, int I, const float* act_scale, uint16_t* out,
                             void* stream);
+
+/* moe_mxfp4_experts -- the expert half of the layer on rows already grouped by expert:
+ * for every expert e and every row p in [offsets[e], offsets[e+1]),
+ *   y[p] = s1 * (ain . Wd[e]^T) + d_bias[e],  ain = the gated activation of
+ *   g = s0 * (xin . Wgu[e]^T) + gu_bias[e]  (bf16 or A-FP8 activations as in
+ *   moe_mxfp4_forward; act_scale a HOST pointer to {s0, s1} or NULL),
+ * fp32 (P, H). "quantization_mxfp4", As GPT-OSS's native format (per-expert gate_up /
+ * SwiGLU / down). For a partition of the experts over several ranks (expert parallelism):
+ * a rank runs its own experts on the rows the other ranks sent it. x_rows: device bf16
+ * (P, H); offsets: device int32 (E + 1), nondecreasing, offsets[E] = P; weights and
+ * biases of the E experts as in moe_mxfp4_forward. Runs the tcgen05 grouped GEMMs: H and
+ * I multiples of 64 in [128, 4608], blocks 32-byte aligned (MXMOE_EUNSUPPORTED
+ * otherwise). Errors as moe_mxfp4_forward. Uses the library workspace. */
+int moe_mxfp4_experts(const uint16_t* x_rows, const int32_t* offsets, int E, int P, int H, int I,
+                      const uint8_t* gu_blocks, const uint8_t* gu_scales, const float* gu_bias,
+                      const uint8_t* d_blocks, const uint8_t* d_scales, const float* d_bias,
+                      const float* act_scale, float* y, void* stream);
+
+/* moe_combine -- the weighted combine of the layer: out[t] = bf16( sum over the token's k
+ * slots, in ascending expert id, of topk_w[t, j] * y[inv[t*k + j]] ), fp32 with one
+ * rounding per multiply and add ("quantization_mxfp4", As GPT-OSS's native format: expert
+ * outputs summed with their router gates). y: device fp32 (rows, H); topk_idx / topk_w:
+ * device (T, k); inv: device int32 (T*k), the row of y that holds pair (t, j); out:
+ * device bf16 (T, H). H % 8 == 0 (MXMOE_EALIGN), 1 <= k <= 8. */
+int moe_combine(const float* y, const int32_t* topk_idx, const float* topk_w, const int32_t* inv,
+                int T, int H, int k, uint16_t* out, void* stream);
 
 /* moe_mxfp4_calibrate -- static per-tensor FP8 scales from a calibration batch with a
  * min-max observer ("gpt-oss-120b-mxfp4-fp8attn-v2", Quantization Recipe):

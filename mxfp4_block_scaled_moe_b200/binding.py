@@ -26,6 +26,10 @@ _vp, _i64, _i32, _f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_
 _SIGS = {
     "mxfp4_quantize": [_vp, _i64, _i64, _vp, _vp, _vp],
     "mxfp4_dequantize": [_vp, _vp, _i64, _i64, _vp, _i32, _vp],
+    "mxfp4_quantize_axis": [_vp, _i64, _i64, _i64, _vp, _vp, _vp],
+    "mxfp4_dequantize_axis": [_vp, _vp, _i64, _i64, _i64, _vp, _i32, _vp],
+    "mxfp4_linear": [_vp, _i32, _i32, _vp, _vp, _i32, _vp, _vp, _vp, _vp],
+    "fp8_linear": [_vp, _i32, _i32, _vp, _i32, _f32, _f32, _vp, _vp, _vp],
     "moe_route_topk": [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp],
     "moe_topk_from_logits": [_vp, _i32, _i32, _i32, _vp, _vp, _vp],
     "moe_permute": [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp],
@@ -34,6 +38,8 @@ _SIGS = {
     "moe_mxfp4_forward": [_vp] * 9 + [_i32] * 5 + [_vp, _vp, _vp],
     "moe_mxfp4_forward_dense": [_vp] * 9 + [_i32] * 5 + [_vp, _vp, _vp],
     "moe_mxfp4_calibrate": [_vp] * 9 + [_i32] * 5 + [_vp, _vp],
+    "moe_mxfp4_experts": [_vp, _vp, _i32, _i32, _i32, _i32] + [_vp] * 9,
+    "moe_combine": [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp],
     "mxmoe_check": [_vp],
     "mxmoe_last_error": [],
     "mxmoe_last_launch_count": [],
@@ -185,6 +191,77 @@ def moe_fp8_quantize(x, s, stream=None):
     return q
 
 
+def _axis_view(shape, axis):
+    axis = axis % len(shape)
+    K = int(shape[axis])
+    outer = 1
+    for d in shape[:axis]:
+        outer *= int(d)
+    inner = 1
+    for d in shape[axis + 1:]:
+        inner *= int(d)
+    return axis, outer, K, inner
+
+
+def mxfp4_quantize_axis(w: torch.Tensor, axis: int, stream=None):
+    """fp32 tensor -> (blocks, scales) along `axis`, moved to the end: blocks have the
+    shape of w with that axis last and K/2 long, scales K/32 long."""
+    _dev(w, torch.float32, "w")
+    axis, outer, K, inner = _axis_view(w.shape, axis)
+    moved = tuple(w.shape[:axis]) + tuple(w.shape[axis + 1:])
+    blocks = torch.empty(*moved, K // 2, dtype=torch.uint8, device=w.device)
+    scales = torch.empty(*moved, max(K // 32, 0), dtype=torch.uint8, device=w.device)
+    _call("mxfp4_quantize_axis", _ptr(w), outer, K, inner, _ptr(blocks), _ptr(scales), _stream(stream))
+    return blocks, scales
+
+
+def mxfp4_dequantize_axis(blocks: torch.Tensor, scales: torch.Tensor, axis: int, out_dtype=torch.float32,
+                          out=None, stream=None):
+    """Inverse of mxfp4_quantize_axis: the packed (last) axis goes back to position `axis`."""
+    _dev(blocks, torch.uint8, "blocks")
+    _dev(scales, torch.uint8, "scales")
+    K = blocks.shape[-1] * 2
+    moved = tuple(blocks.shape[:-1])
+    nd = len(moved) + 1
+    axis = axis % nd
+    shape = moved[:axis] + (K,) + moved[axis:]
+    _, outer, _, inner = _axis_view(shape, axis)
+    if out is None:
+        out = torch.empty(shape, dtype=out_dtype, device=blocks.device)
+    code = OUT_F32 if out.dtype == torch.float32 else OUT_BF16
+    _call("mxfp4_dequantize_axis", _ptr(blocks), _ptr(scales), outer, K, inner, _ptr(out), code, _stream(stream))
+    return out
+
+
+def mxfp4_linear(x, blocks, scales, bias=None, act_scale=None, out=None, stream=None):
+    """out (T, N) bf16 = x (T, K) bf16 . W^T + bias with W MXFP4 (blocks (N, K/2), scales
+    (N, K/32)); act_scale (one float) casts the input to FP8 E4M3 first."""
+    _dev(x, torch.bfloat16, "x")
+    _dev(blocks, torch.uint8, "blocks")
+    _dev(scales, torch.uint8, "scales")
+    _dev(bias, torch.float32, "bias")
+    T, K = x.shape
+    N = blocks.shape[0]
+    if out is None:
+        out = torch.empty(T, N, dtype=torch.bfloat16, device=x.device)
+    s = None if act_scale is None else ctypes.byref(ctypes.c_float(float(act_scale)))
+    _call("mxfp4_linear", _ptr(x), T, K, _ptr(blocks), _ptr(scales), N, _ptr(bias), s, _ptr(out), _stream(stream))
+    return out
+
+
+def fp8_linear(x, wq, s_x, s_w, bias=None, out=None, stream=None):
+    """out (T, N) bf16 = bf16(s_x s_w e4m3(x / s_x) . wq^T + bias); wq: (N, K) uint8 E4M3 codes."""
+    _dev(x, torch.bfloat16, "x")
+    _dev(wq, torch.uint8, "wq")
+    _dev(bias, torch.float32, "bias")
+    T, K = x.shape
+    N = wq.shape[0]
+    if out is None:
+        out = torch.empty(T, N, dtype=torch.bfloat16, device=x.device)
+    _call("fp8_linear", _ptr(x), T, K, _ptr(wq), N, float(s_x), float(s_w), _ptr(bias), _ptr(out), _stream(stream))
+    return out
+
+
 # ----------------------------------------------------------------------- layer -----
 
 def _layer_ptrs(x, router_w, router_b, gu_blocks, gu_scales, gu_bias, d_blocks, d_scales, d_bias):
@@ -243,6 +320,37 @@ def moe_mxfp4_calibrate(x, router_w, router_b, gu_blocks, gu_scales, gu_bias, d_
                                    d_blocks, d_scales, d_bias)
     out = torch.empty(2, dtype=torch.float32, device=x.device)
     _call("moe_mxfp4_calibrate", *ptrs, E, k, T, H, I, _ptr(out), _stream(stream))
+    return out
+
+
+def moe_mxfp4_experts(x_rows, offsets, gu_blocks, gu_scales, gu_bias, d_blocks, d_scales, d_bias,
+                      act_scale=None, y=None, stream=None):
+    """fp32 (P, H) expert outputs of rows grouped by expert (offsets: int32 (E+1))."""
+    _dev(x_rows, torch.bfloat16, "x_rows")
+    _dev(offsets, torch.int32, "offsets")
+    P, H = x_rows.shape
+    E = gu_blocks.shape[0]
+    I = d_blocks.shape[-1] * 2
+    if y is None:
+        y = torch.empty(P, H, dtype=torch.float32, device=x_rows.device)
+    acts = None
+    if act_scale is not None:
+        s = [float(v) for v in act_scale]
+        acts = (ctypes.c_float * 2)(s[0], s[1])
+    _call("moe_mxfp4_experts", _ptr(x_rows), _ptr(offsets), E, P, H, I, _ptr(gu_blocks), _ptr(gu_scales),
+          _ptr(gu_bias), _ptr(d_blocks), _ptr(d_scales), _ptr(d_bias),
+          ctypes.cast(acts, ctypes.c_void_p) if acts is not None else None, _ptr(y), _stream(stream))
+    return y
+
+
+def moe_combine(y, topk_idx, topk_w, inv, out=None, stream=None):
+    """bf16 (T, H): each token's k expert outputs y[inv] weighted and summed in ascending expert id."""
+    _dev(y, torch.float32, "y")
+    T, k = topk_idx.shape
+    H = y.shape[1]
+    if out is None:
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=y.device)
+    _call("moe_combine", _ptr(y), _ptr(topk_idx), _ptr(topk_w), _ptr(inv), T, H, k, _ptr(out), _stream(stream))
     return out
 
 

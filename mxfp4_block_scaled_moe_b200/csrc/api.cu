@@ -518,6 +518,17 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
 // e * T + t), the gates zero off the top-k, the weighted sum over all experts in ascending
 // order. The tcgen05 grouped GEMMs read the T activation rows once per expert (shared A
 // rows) instead of a gathered copy per routed pair.
+// Shapes the dense path takes: its expert kernels' (tcgen05 grouped GEMMs), with the
+// expert-major intermediate indexable in 32 bits.
+bool dense_kernels_take(const LayerArgs& a) {
+  return std::max(a.H, a.I) / 32 <= kTcMaxNb &&
+         mxmoe::tc_gemm_supported(a.H, a.I, a.gu_blocks, a.d_blocks, a.gu_scales, a.d_scales);
+}
+bool dense_fits(const LayerArgs& a) {
+  const int64_t R = static_cast<int64_t>(a.E) * a.T;
+  return R * std::max(a.H, a.I) < (int64_t{1} << 31) && R < (int64_t{1} << 24);
+}
+
 int run_layer_dense(const LayerArgs& a, const float* act_scale, uint16_t* out, cudaStream_t st) {
   using namespace mxmoe;
   Workspace* ws = nullptr;
@@ -525,11 +536,10 @@ int run_layer_dense(const LayerArgs& a, const float* act_scale, uint16_t* out, c
   const bool fp8 = act_scale != nullptr;
   const int64_t T = a.T, E = a.E, H = a.H, I = a.I;
   const int64_t R = E * T;   // expert-major rows
-  if (!(std::max(a.H, a.I) / 32 <= kTcMaxNb &&
-        tc_gemm_supported(a.H, a.I, a.gu_blocks, a.d_blocks, a.gu_scales, a.d_scales)))
+  if (!dense_kernels_take(a))
     return fail(MXMOE_EUNSUPPORTED, "the dense path needs H and I multiples of 64 in [128, 4608] and 32-byte "
                                     "aligned blocks (got H = %d, I = %d)", a.H, a.I);
-  if (R * std::max(H, I) >= (int64_t{1} << 31) || R >= (int64_t{1} << 24))
+  if (!dense_fits(a))
     return fail(MXMOE_EUNSUPPORTED, "the dense path holds E*T*max(H, I) < 2^31 values (E = %d, T = %d)", a.E, a.T);
   const bool rtc = a.T > 32 && router_tc_supported(a.T, a.H, a.E, a.x, a.router_w, nullptr);
   const int ksplit = rtc ? router_tc_ksplit(a.T, a.H, ws->sms) : 0;
@@ -667,6 +677,179 @@ int mxfp4_dequantize(const uint8_t* blocks, const uint8_t* scales, int64_t rows,
   return MXMOE_OK;
 }
 
+int mxfp4_quantize_axis(const float* w, int64_t outer, int64_t K, int64_t inner, uint8_t* blocks, uint8_t* scales,
+                        void* stream) {
+  t_last_error.clear();
+  t_last_launches = 0;
+  if (outer < 0 || K < 0 || inner < 0)
+    return fail(MXMOE_EINVAL, "negative size outer=%lld K=%lld inner=%lld", (long long)outer, (long long)K,
+                (long long)inner);
+  if (K % 32) return fail(MXMOE_EALIGN, "K = %lld is not a multiple of 32 (MXFP4 block size)", (long long)K);
+  if (outer == 0 || K == 0 || inner == 0) return MXMOE_OK;
+  if (!w || !blocks || !scales) return fail(MXMOE_EINVAL, "null pointer");
+  if (!aligned16(w) || !aligned16(blocks)) return fail(MXMOE_EINVAL, "w and blocks must be 16-byte aligned");
+  Workspace* ws = nullptr;
+  if (int rc = current_device_ws(&ws)) return rc;
+  cudaError_t e = mxmoe::launch_quantize_axis(w, outer, K, inner, blocks, scales, static_cast<cudaStream_t>(stream),
+                                              ws->sms);
+  if (e) return cuda_fail(e, "quantize launch");
+  t_last_launches = 1;
+  return MXMOE_OK;
+}
+
+int mxfp4_dequantize_axis(const uint8_t* blocks, const uint8_t* scales, int64_t outer, int64_t K, int64_t inner,
+                          void* out, int out_dtype, void* stream) {
+  t_last_error.clear();
+  t_last_launches = 0;
+  if (outer < 0 || K < 0 || inner < 0)
+    return fail(MXMOE_EINVAL, "negative size outer=%lld K=%lld inner=%lld", (long long)outer, (long long)K,
+                (long long)inner);
+  if (K % 32) return fail(MXMOE_EALIGN, "K = %lld is not a multiple of 32 (MXFP4 block size)", (long long)K);
+  if (out_dtype != MXMOE_OUT_F32 && out_dtype != MXMOE_OUT_BF16)
+    return fail(MXMOE_EUNSUPPORTED, "out_dtype %d is neither MXMOE_OUT_F32 nor MXMOE_OUT_BF16", out_dtype);
+  if (outer == 0 || K == 0 || inner == 0) return MXMOE_OK;
+  if (!blocks || !scales || !out) return fail(MXMOE_EINVAL, "null pointer");
+  if (!aligned16(blocks) || !aligned16(out)) return fail(MXMOE_EINVAL, "blocks and out must be 16-byte aligned");
+  Workspace* ws = nullptr;
+  if (int rc = current_device_ws(&ws)) return rc;
+  cudaError_t e = mxmoe::launch_dequantize_axis(blocks, scales, outer, K, inner, out, out_dtype,
+                                                static_cast<cudaStream_t>(stream), ws->sms);
+  if (e) return cuda_fail(e, "dequantize launch");
+  t_last_launches = 1;
+  return MXMOE_OK;
+}
+
+int mxfp4_linear(const uint16_t* x, int T, int K, const uint8_t* blocks, const uint8_t* scales, int N,
+                 const float* bias, const float* act_scale, uint16_t* out, void* stream) {
+  using namespace mxmoe;
+  t_last_error.clear();
+  t_last_launches = 0;
+  if (T < 0 || K <= 0 || N <= 0) return fail(MXMOE_EINVAL, "T = %d must be >= 0, K = %d and N = %d positive", T, K, N);
+  if (K % 32) return fail(MXMOE_EALIGN, "K = %d is not a multiple of 32 (MXFP4 block size)", K);
+  if (N % 16) return fail(MXMOE_EALIGN, "N = %d is not a multiple of 16", N);
+  if (T >= (1 << 24)) return fail(MXMOE_EUNSUPPORTED, "T = %d exceeds 2^24 - 1", T);
+  if (T == 0) return MXMOE_OK;
+  if (!x || !blocks || !scales || !out) return fail(MXMOE_EINVAL, "null pointer");
+  if (!aligned16(x) || !aligned16(blocks) || !aligned16(out) || (bias && !aligned16(bias)))
+    return fail(MXMOE_EINVAL, "x, blocks, out and bias must be 16-byte aligned");
+  if (act_scale && !(*act_scale > 0.0f)) return fail(MXMOE_EINVAL, "act_scale must be > 0");
+  Workspace* ws = nullptr;
+  if (int rc = current_device_ws(&ws)) return rc;
+  const bool fp8 = act_scale != nullptr;
+  const int64_t TK = static_cast<int64_t>(T) * K;
+  // more than a decode batch on the tcgen05 grouped GEMM (one expert), else the
+  // register-dequant kernel, which spreads the weight rows over every SM
+  const bool tc = T > kDecodeMaxT && K / 32 <= kTcMaxNb && tc_gemm_supported(N, K, blocks, blocks, scales, scales);
+  Carve c;
+  c.take<uint8_t>(kTicketBytes);
+  const size_t o_meta = c.take<int32_t>(8);
+  const size_t o_zb = c.take<float>(bias ? 0 : N);
+  const size_t o_a = c.take<uint8_t>(tc ? (fp8 ? TK : 2 * TK) : (fp8 ? 2 * TK : 0));
+  const size_t o_sa = c.take<uint8_t>(tc && !fp8 ? 2 * (TK / 32) : 0);
+  const size_t o_y = c.take<float>(static_cast<int64_t>(T) * N);
+  if (int rc = ensure_capacity(ws, c.off)) return rc;
+  ws->tickets_zeroed = kTicketBytes;
+  if (tc && fp8 && !ws->tc_ready) {
+    cudaError_t e = tc_gemm_prepare(256);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (tcgen05 GEMM)");
+    ws->tc_ready = true;
+  }
+  if (tc && !fp8 && !ws->tcb_ready) {
+    cudaError_t e = tc_parts_gemm_prepare(256);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (two-part tcgen05 GEMM)");
+    ws->tcb_ready = true;
+  }
+  if (!tc && K > ws->smem_K) {
+    cudaError_t e = expert_mma_set_smem_limits(K);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    ws->smem_K = K;
+  }
+  char* base = ws->base;
+  int32_t* offsets = reinterpret_cast<int32_t*>(base + o_meta);
+  int32_t* active = offsets + 2;
+  int32_t* n_active = offsets + 3;
+  float* zb = bias ? nullptr : reinterpret_cast<float*>(base + o_zb);
+  const float* b = bias ? bias : zb;
+  uint8_t* a = reinterpret_cast<uint8_t*>(base + o_a);
+  uint8_t* sa = reinterpret_cast<uint8_t*>(base + o_sa);
+  float* y = reinterpret_cast<float*>(base + o_y);
+  const float s = fp8 ? *act_scale : 1.0f;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int launches = 0;
+  cudaError_t e;
+  if ((e = launch_linear_setup(T, N, offsets, active, n_active, zb, st, ws->sms))) return cuda_fail(e, "linear set-up");
+  ++launches;
+  if (tc && fp8) {
+    if ((e = launch_fp8_quant(x, TK, s, a, st, ws->sms))) return cuda_fail(e, "fp8 activation cast");
+    if ((e = launch_tc_gemm(false, a, T, K, blocks, scales, b, 1, N, offsets, s, 0.0f, nullptr, y, ws->err, ws->sms,
+                            st)))
+      return cuda_fail(e, "linear (tcgen05)");
+    launches += 2;
+  } else if (tc) {
+    if ((e = launch_split_parts(x, nullptr, T, T, K, a, sa, ws->sms, st))) return cuda_fail(e, "activation split");
+    if ((e = launch_tc_parts_gemm(false, a, sa, T, K, blocks, scales, b, 1, N, offsets, nullptr, y, ws->err, ws->sms,
+                                  st)))
+      return cuda_fail(e, "linear (tcgen05, two parts)");
+    launches += 2;
+  } else {
+    const uint16_t* act = x;
+    if (fp8) {
+      if ((e = launch_fp8_quant_as_bf16(x, TK, s, reinterpret_cast<uint16_t*>(a), st, ws->sms)))
+        return cuda_fail(e, "fp8 activation cast");
+      act = reinterpret_cast<uint16_t*>(a);
+      ++launches;
+    }
+    if ((e = launch_expert_mma(blocks, scales, b, N, K, act, nullptr, offsets, active, n_active, 1, s, 1, K, 0.0f,
+                               nullptr, y, nullptr, T, ws->err, nullptr, st)))
+      return cuda_fail(e, "linear (register dequant)");
+    ++launches;
+  }
+  if ((e = launch_f32_to_bf16(y, static_cast<int64_t>(T) * N, out, st, ws->sms))) return cuda_fail(e, "bf16 output");
+  ++launches;
+  t_last_launches = launches;
+  return MXMOE_OK;
+}
+
+int fp8_linear(const uint16_t* x, int T, int K, const uint8_t* wq, int N, float s_x, float s_w, const float* bias,
+               uint16_t* out, void* stream) {
+  using namespace mxmoe;
+  t_last_error.clear();
+  t_last_launches = 0;
+  if (T < 0 || K <= 0 || N <= 0) return fail(MXMOE_EINVAL, "T = %d must be >= 0, K = %d and N = %d positive", T, K, N);
+  if (K % 32) return fail(MXMOE_EALIGN, "K = %d is not a multiple of 32", K);
+  if (N % 8) return fail(MXMOE_EALIGN, "N = %d is not a multiple of 8", N);
+  if (!(s_x > 0.0f) || !(s_w > 0.0f)) return fail(MXMOE_EINVAL, "s_x and s_w must be > 0");
+  if (T >= (1 << 24)) return fail(MXMOE_EUNSUPPORTED, "T = %d exceeds 2^24 - 1", T);
+  if (T == 0) return MXMOE_OK;
+  if (!x || !wq || !out) return fail(MXMOE_EINVAL, "null pointer");
+  if (!aligned16(x) || !aligned16(wq) || !aligned16(out) || (bias && !aligned16(bias)))
+    return fail(MXMOE_EINVAL, "x, wq, out and bias must be 16-byte aligned");
+  if (!fp8_linear_supported()) return fail(MXMOE_EUNSUPPORTED, "cuTensorMapEncodeTiled is unavailable");
+  Workspace* ws = nullptr;
+  if (int rc = current_device_ws(&ws)) return rc;
+  const int ksplit = fp8_linear_ksplit(T, K, N, ws->sms);
+  Carve c;
+  c.take<uint8_t>(kTicketBytes);
+  const size_t o_xq = c.take<uint8_t>(static_cast<int64_t>(T) * K);
+  const size_t o_part = c.take<float>(ksplit > 1 ? static_cast<int64_t>(ksplit) * T * N : 0);
+  if (int rc = ensure_capacity(ws, c.off)) return rc;
+  ws->tickets_zeroed = kTicketBytes;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* xq = reinterpret_cast<uint8_t*>(ws->base + o_xq);
+  float* part = reinterpret_cast<float*>(ws->base + o_part);
+  cudaError_t e;
+  StageTimer tm(st);
+  if ((e = launch_fp8_quant(x, static_cast<int64_t>(T) * K, s_x, xq, st, ws->sms)))
+    return cuda_fail(e, "fp8 activation cast");
+  tm.mark("act_quant");
+  const float s = s_x * s_w;
+  if ((e = launch_fp8_linear(xq, T, K, wq, N, s, bias, out, part, ksplit, ws->err, ws->sms, st)))
+    return cuda_fail(e, "fp8 linear");
+  tm.mark("fp8_gemm");
+  t_last_launches = ksplit > 1 ? 3 : 2;
+  return MXMOE_OK;
+}
+
 int moe_route_topk(const uint16_t* x, const uint16_t* router_w, const uint16_t* router_b, int T,
                    int H, int E, int k, float* logits_out, int32_t* topk_idx, float* topk_w,
                    void* stream) {
@@ -762,6 +945,16 @@ int moe_mxfp4_forward(const uint16_t* x, const uint16_t* router_w, const uint16_
   if (!aligned16(out)) return fail(MXMOE_EINVAL, "out is not 16-byte aligned");
   if (act_scale && !(act_scale[0] > 0.0f && act_scale[1] > 0.0f))
     return fail(MXMOE_EINVAL, "act_scale values must be > 0");
+  // Routed / dense crossover. With every expert selected (k == E) the dense all-experts
+  // path does the same expert work as the routed one, without the permutation, the
+  // gather into expert-grouped rows and the ordered combine (measured on B200, FP8, H = I =
+  // 2880: k = E = 4 and 8 at T = 128 .. 4096, dense 0.82-0.99x the routed time). With k < E
+  // it does E/k times the expert work and was slower at every measured size (top-4 of 32:
+  // 1.13x at T = 128 rising to 4.3x at 1024; of 128: 1.4x at T = 64 to 20x at 4096), so the
+  // routed path keeps those. Above the decode sizes both run the same expert kernels, so
+  // the output is the same bit for bit.
+  if (k == E && T > mxmoe::kDecodeMaxT && dense_kernels_take(a) && dense_fits(a))
+    return run_layer_dense(a, act_scale, out, static_cast<cudaStream_t>(stream));
   return run_layer(a, act_scale, out, nullptr, static_cast<cudaStream_t>(stream));
 }
 
@@ -781,6 +974,102 @@ int moe_mxfp4_forward_dense(const uint16_t* x, const uint16_t* router_w, const u
   if (act_scale && !(act_scale[0] > 0.0f && act_scale[1] > 0.0f))
     return fail(MXMOE_EINVAL, "act_scale values must be > 0");
   return run_layer_dense(a, act_scale, out, static_cast<cudaStream_t>(stream));
+}
+
+int moe_mxfp4_experts(const uint16_t* x_rows, const int32_t* offsets, int E, int P, int H, int I,
+                      const uint8_t* gu_blocks, const uint8_t* gu_scales, const float* gu_bias,
+                      const uint8_t* d_blocks, const uint8_t* d_scales, const float* d_bias,
+                      const float* act_scale, float* y, void* stream) {
+  using namespace mxmoe;
+  t_last_error.clear();
+  t_last_launches = 0;
+  if (E < 1 || E > 256) return fail(MXMOE_EUNSUPPORTED, "E = %d outside [1, 256]", E);
+  if (P < 0 || H <= 0 || I <= 0) return fail(MXMOE_EINVAL, "P = %d must be >= 0, H = %d and I = %d positive", P, H, I);
+  if (H % 32 || I % 32) return fail(MXMOE_EALIGN, "H = %d and I = %d must be multiples of 32", H, I);
+  if (P >= (1 << 24)) return fail(MXMOE_EUNSUPPORTED, "P = %d exceeds 2^24 - 1", P);
+  if (P == 0) return MXMOE_OK;
+  const void* ptrs[] = {x_rows, offsets, gu_blocks, gu_scales, gu_bias, d_blocks, d_scales, d_bias, y};
+  for (const void* q : ptrs)
+    if (!q) return fail(MXMOE_EINVAL, "null pointer");
+  if (!aligned16(x_rows) || !aligned16(y) || !aligned16(gu_blocks) || !aligned16(d_blocks) || !aligned16(gu_bias) ||
+      !aligned16(d_bias))
+    return fail(MXMOE_EINVAL, "x_rows, y, blocks and biases must be 16-byte aligned");
+  if (act_scale && !(act_scale[0] > 0.0f && act_scale[1] > 0.0f))
+    return fail(MXMOE_EINVAL, "act_scale values must be > 0");
+  if (!(std::max(H, I) / 32 <= kTcMaxNb && tc_gemm_supported(H, I, gu_blocks, d_blocks, gu_scales, d_scales)))
+    return fail(MXMOE_EUNSUPPORTED, "the grouped expert GEMMs need H and I multiples of 64 in [128, 4608] and "
+                                    "32-byte aligned blocks (got H = %d, I = %d)", H, I);
+  Workspace* ws = nullptr;
+  if (int rc = current_device_ws(&ws)) return rc;
+  const bool fp8 = act_scale != nullptr;
+  const int64_t PH = static_cast<int64_t>(P) * H, PI = static_cast<int64_t>(P) * I;
+  Carve c;
+  c.take<uint8_t>(kTicketBytes);
+  const size_t o_a1 = c.take<uint8_t>(fp8 ? PH : 2 * PH);
+  const size_t o_sa1 = c.take<uint8_t>(fp8 ? 0 : 2 * (PH / 32));
+  const size_t o_mid = c.take<uint16_t>(fp8 ? 0 : PI);
+  const size_t o_a2 = c.take<uint8_t>(fp8 ? PI : 2 * PI);
+  const size_t o_sa2 = c.take<uint8_t>(fp8 ? 0 : 2 * (PI / 32));
+  if (int rc = ensure_capacity(ws, c.off)) return rc;
+  ws->tickets_zeroed = kTicketBytes;
+  if (fp8 && !ws->tc_ready) {
+    cudaError_t e = tc_gemm_prepare(256);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (tcgen05 GEMM)");
+    ws->tc_ready = true;
+  }
+  if (!fp8 && !ws->tcb_ready) {
+    cudaError_t e = tc_parts_gemm_prepare(256);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (two-part tcgen05 GEMM)");
+    ws->tcb_ready = true;
+  }
+  char* base = ws->base;
+  uint8_t* a1 = reinterpret_cast<uint8_t*>(base + o_a1);
+  uint8_t* sa1 = reinterpret_cast<uint8_t*>(base + o_sa1);
+  uint16_t* mid = reinterpret_cast<uint16_t*>(base + o_mid);
+  uint8_t* a2 = reinterpret_cast<uint8_t*>(base + o_a2);
+  uint8_t* sa2 = reinterpret_cast<uint8_t*>(base + o_sa2);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (fp8) {
+    const float s0 = act_scale[0], s1 = act_scale[1];
+    if ((e = launch_fp8_quant(x_rows, PH, s0, a1, st, ws->sms))) return cuda_fail(e, "fp8 activation cast");
+    if ((e = launch_tc_gemm(true, a1, P, H, gu_blocks, gu_scales, gu_bias, E, I, offsets, s0, s1, a2, nullptr, ws->err,
+                            ws->sms, st)))
+      return cuda_fail(e, "gate_up (tcgen05)");
+    if ((e = launch_tc_gemm(false, a2, P, I, d_blocks, d_scales, d_bias, E, H, offsets, s1, 0.0f, nullptr, y, ws->err,
+                            ws->sms, st)))
+      return cuda_fail(e, "down (tcgen05)");
+  } else {
+    if ((e = launch_split_parts(x_rows, nullptr, P, P, H, a1, sa1, ws->sms, st))) return cuda_fail(e, "activation split");
+    if ((e = launch_tc_parts_gemm(true, a1, sa1, P, H, gu_blocks, gu_scales, gu_bias, E, I, offsets, mid, nullptr,
+                                  ws->err, ws->sms, st)))
+      return cuda_fail(e, "gate_up (tcgen05, two parts)");
+    if ((e = launch_split_parts(mid, nullptr, P, P, I, a2, sa2, ws->sms, st))) return cuda_fail(e, "intermediate split");
+    if ((e = launch_tc_parts_gemm(false, a2, sa2, P, I, d_blocks, d_scales, d_bias, E, H, offsets, nullptr, y, ws->err,
+                                  ws->sms, st)))
+      return cuda_fail(e, "down (tcgen05, two parts)");
+  }
+  t_last_launches = fp8 ? 3 : 4;
+  return MXMOE_OK;
+}
+
+int moe_combine(const float* y, const int32_t* topk_idx, const float* topk_w, const int32_t* inv, int T, int H, int k,
+                uint16_t* out, void* stream) {
+  t_last_error.clear();
+  t_last_launches = 0;
+  if (T < 0 || H <= 0) return fail(MXMOE_EINVAL, "T = %d must be >= 0 and H = %d positive", T, H);
+  if (k < 1 || k > 8) return fail(MXMOE_EUNSUPPORTED, "k = %d outside [1, 8]", k);
+  if (H % 8) return fail(MXMOE_EALIGN, "H = %d is not a multiple of 8", H);
+  if (T == 0) return MXMOE_OK;
+  if (!y || !topk_idx || !topk_w || !inv || !out) return fail(MXMOE_EINVAL, "null pointer");
+  if (!aligned16(y) || !aligned16(out)) return fail(MXMOE_EINVAL, "y and out must be 16-byte aligned");
+  Workspace* ws = nullptr;
+  if (int rc = current_device_ws(&ws)) return rc;
+  cudaError_t e = mxmoe::launch_combine(y, topk_idx, topk_w, inv, T, H, k, out, static_cast<cudaStream_t>(stream),
+                                        ws->sms);
+  if (e) return cuda_fail(e, "combine launch");
+  t_last_launches = 1;
+  return MXMOE_OK;
 }
 
 int moe_mxfp4_calibrate(const uint16_t* x, const uint16_t* router_w, const uint16_t* router_b,

@@ -140,6 +140,76 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint32_t* __restr
   }
 }
 
+// ------------------------------------------------ along an arbitrary contracting axis --
+// The tensor as (outer, K, inner) with the contracting axis in the middle; the packed
+// result has that axis last: blocks (outer, inner, K/2), scales (outer, inner, K/32)
+// ("quantization_mxfp4" (KerasFormers), Primitives: MXFP4Quantizer quantizes along one
+// axis, moved to the end). One thread per (outer, block, inner) with inner fastest, so a
+// warp reads each of its 32 values as one contiguous run across inner; it writes its 16
+// block bytes as one 16-byte store. The same exponent and rounding as quantize_kernel.
+__global__ void __launch_bounds__(256) quantize_axis_kernel(const float* __restrict__ w, int64_t outer, int64_t K,
+                                                             int64_t inner, uint8_t* __restrict__ blocks,
+                                                             uint8_t* __restrict__ scales) {
+  const int64_t nb = K / 32;
+  const int64_t n = outer * nb * inner;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < n; idx += stride) {
+    const int64_t i = idx % inner, ob = idx / inner;
+    const int64_t b = ob % nb, o = ob / nb;
+    const float* src = w + (o * K + 32 * b) * inner + i;
+    float v[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = __ldcs(src + j * inner);
+    float m = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) m = fmaxf(m, fabsf(v[j]));
+    int e = (m > 0.0f) ? floor_log2_pos(m) - 2 : -127;
+    e = max(-127, min(127, e));
+    const float inv = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+    uint32_t wd[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const uint32_t sign = (__float_as_uint(v[j]) >> 31) << 3;
+      wd[j >> 3] |= (e2m1_code(fabsf(v[j]) * inv) | sign) << (4 * (j & 7));
+    }
+    const int64_t r = o * inner + i;
+    *reinterpret_cast<uint4*>(blocks + r * (K / 2) + 16 * b) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+    scales[r * nb + b] = static_cast<uint8_t>(e + 127);
+  }
+}
+
+// The inverse: (outer, inner, K/2) + (outer, inner, K/32) -> (outer, K, inner) fp32 or
+// bf16, the values of dequantize_kernel; a warp's stores of each value index are one
+// contiguous run across inner.
+template <bool kBf16>
+__global__ void __launch_bounds__(256) dequantize_axis_kernel(const uint8_t* __restrict__ blocks,
+                                                               const uint8_t* __restrict__ scales, int64_t outer,
+                                                               int64_t K, int64_t inner, void* __restrict__ out) {
+  const int64_t nb = K / 32;
+  const int64_t n = outer * nb * inner;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < n; idx += stride) {
+    const int64_t i = idx % inner, ob = idx / inner;
+    const int64_t b = ob % nb, o = ob / nb;
+    const int64_t r = o * inner + i;
+    const uint4 q = *reinterpret_cast<const uint4*>(blocks + r * (K / 2) + 16 * b);
+    const uint32_t s = scales[r * nb + b];
+    const float s1 = s == 255u ? __uint_as_float(254u << 23) : e8m0_to_f32(s);
+    const uint32_t wd[4] = {q.x, q.y, q.z, q.w};
+    const int64_t dst = (o * K + 32 * b) * inner + i;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const uint32_t nib = (wd[j >> 3] >> (4 * (j & 7))) & 15u;
+      float v = __uint_as_float(e2m1_mag_bits(nib & 7u) | ((nib & 8u) << 28)) * s1;
+      if (s == 255u) v *= 2.0f;
+      if constexpr (kBf16)
+        reinterpret_cast<uint16_t*>(out)[dst + j * inner] = static_cast<uint16_t>(__float_as_uint(v) >> 16);
+      else
+        reinterpret_cast<float*>(out)[dst + j * inner] = v;
+    }
+  }
+}
+
 // Grid of a grid-stride stream kernel: at most the CTAs that fit on the GPU at once, so
 // every CTA of the grid is resident from the start (a second, partial wave would run the
 // last share of the stream at lower occupancy).
@@ -182,6 +252,30 @@ cudaError_t launch_dequantize(const uint8_t* blocks, const uint8_t* scales, int6
   else
     dequantize_kernel<false><<<grid, 256, 0, st>>>(reinterpret_cast<const uint32_t*>(blocks),
                                                    scales, nwords, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_axis(const float* w, int64_t outer, int64_t K, int64_t inner, uint8_t* blocks,
+                                 uint8_t* scales, cudaStream_t st, int sms) {
+  if (inner == 1) return launch_quantize(w, outer, K, blocks, scales, st, sms);
+  const int64_t n = outer * (K / 32) * inner;
+  if (n == 0) return cudaSuccess;
+  quantize_axis_kernel<<<grid_for(quantize_axis_kernel, n, 256, sms), 256, 0, st>>>(w, outer, K, inner, blocks,
+                                                                                   scales);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dequantize_axis(const uint8_t* blocks, const uint8_t* scales, int64_t outer, int64_t K,
+                                   int64_t inner, void* out, int out_dtype, cudaStream_t st, int sms) {
+  if (inner == 1) return launch_dequantize(blocks, scales, outer, K, out, out_dtype, st, sms);
+  const int64_t n = outer * (K / 32) * inner;
+  if (n == 0) return cudaSuccess;
+  if (out_dtype == MXMOE_OUT_BF16)
+    dequantize_axis_kernel<true><<<grid_for(dequantize_axis_kernel<true>, n, 256, sms), 256, 0, st>>>(
+        blocks, scales, outer, K, inner, out);
+  else
+    dequantize_axis_kernel<false><<<grid_for(dequantize_axis_kernel<false>, n, 256, sms), 256, 0, st>>>(
+        blocks, scales, outer, K, inner, out);
   return cudaGetLastError();
 }
 

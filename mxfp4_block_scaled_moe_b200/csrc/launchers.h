@@ -11,6 +11,12 @@ cudaError_t launch_quantize(const float* w, int64_t rows, int64_t K, uint8_t* bl
 cudaError_t launch_dequantize(const uint8_t* blocks, const uint8_t* scales, int64_t rows,
                               int64_t K, void* out, int out_dtype, cudaStream_t st, int sms);
 
+// the codec along an arbitrary axis: the tensor as (outer, K, inner), packed (outer, inner, K/2)
+cudaError_t launch_quantize_axis(const float* w, int64_t outer, int64_t K, int64_t inner, uint8_t* blocks,
+                                 uint8_t* scales, cudaStream_t st, int sms);
+cudaError_t launch_dequantize_axis(const uint8_t* blocks, const uint8_t* scales, int64_t outer, int64_t K,
+                                   int64_t inner, void* out, int out_dtype, cudaStream_t st, int sms);
+
 cudaError_t launch_router(const uint16_t* x, const uint16_t* wr, const uint16_t* br, int T, int H,
                           int E, float* logits, cudaStream_t st);
 // rest / n_rest: further K-range partials of the logits (see launch_router_tc), summed into
@@ -140,10 +146,22 @@ cudaError_t launch_dense_setup(const int32_t* topk_idx, const float* topk_w, int
 cudaError_t launch_dense_combine(const float* y, const float* gates, int T, int H, int E, uint16_t* out,
                                  cudaStream_t st, int sms);
 
+// a plain MXFP4 linear as a one-expert grouped GEMM (csrc/dense.cu)
+cudaError_t launch_linear_setup(int T, int N, int32_t* offsets, int32_t* active, int32_t* n_active, float* zero_bias,
+                                cudaStream_t st, int sms);
+cudaError_t launch_f32_to_bf16(const float* y, int64_t n, uint16_t* out, cudaStream_t st, int sms);
+
 cudaError_t launch_combine(const float* y, const int32_t* topk_idx, const float* topk_w,
                            const int32_t* inv, int T, int H, int k, uint16_t* out, cudaStream_t st,
                            int sms);
 
+
+// FP8 E4M3 static per-tensor linear (csrc/linear_sm100.cu): xq (T, K) e4m3, wq (N, K) e4m3,
+// out = bf16(fp32(s * xq.wq^T) + bias); ksplit > 1 needs part = (ksplit, T, N) fp32
+int fp8_linear_ksplit(int T, int K, int N, int sms);
+bool fp8_linear_supported();
+cudaError_t launch_fp8_linear(const uint8_t* xq, int T, int K, const uint8_t* wq, int N, float s, const float* bias,
+                              uint16_t* out, float* part, int ksplit, int* err, int sms, cudaStream_t st);
 
 // mxmoe_tc_rate_probe: back-to-back kind::mxf8f6f4 MMAs (M = 128, N = n) on `ctas` CTAs
 cudaError_t launch_tc_rate(int n, int with_copy, int iters, int ctas, int* err, cudaStream_t st);

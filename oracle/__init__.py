@@ -194,6 +194,23 @@ def moe_forward(x, router_w, router_b, gu_blocks, gu_scales, gu_bias, d_blocks, 
     return out, acc, idx, w
 
 
+def expert_rows(x, expert, gu_blocks, gu_scales, gu_bias, d_blocks, d_scales, d_bias, act_scale=None):
+    """y (P, H) fp32 = the expert FFN of each (row, expert) pair, with the layer's arithmetic
+    ("quantization_mxfp4", As GPT-OSS's native format)."""
+    x = _c(x, np.uint16)
+    expert = _c(expert, np.int32)
+    P, H = x.shape
+    E = np.asarray(gu_blocks).shape[0]
+    I = np.asarray(d_blocks).shape[-1] * 2
+    acts = None if act_scale is None else np.ascontiguousarray(np.asarray(act_scale, np.float32))
+    y = np.empty((P, H), np.float32)
+    _check(lib().orc_expert_rows(_p(x), _p(expert), P, _p(_c(gu_blocks, np.uint8)), _p(_c(gu_scales, np.uint8)),
+                                 _p(_c(gu_bias, np.float32)), _p(_c(d_blocks, np.uint8)),
+                                 _p(_c(d_scales, np.uint8)), _p(_c(d_bias, np.float32)), E, H, I, _p(acts), _p(y)),
+           "expert_rows")
+    return y
+
+
 def calibrate(x, router_w, router_b, gu_blocks, gu_scales, gu_bias, d_blocks, d_scales, d_bias,
               k):
     """Static per-tensor FP8 scales {s0, s1} = {amax|x|, amax|a|} / 448 (min-max observer).

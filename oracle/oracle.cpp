@@ -421,6 +421,25 @@ int orc_moe_forward(const uint16_t* x, const uint16_t* router_w, const uint16_t*
   return ORC_OK;
 }
 
+// The expert FFN of given (row, expert) pairs: y[p] = expert_ffn(x[p], expert[p]) with the
+// arithmetic of orc_moe_forward (bf16 or A-FP8 activations). x: (P, H) bf16 rows; expert:
+// (P) ids in [0, E); y: (P, H) fp32. The per-pair half of the layer, for checking a
+// partition of the experts over several ranks against the whole layer.
+int orc_expert_rows(const uint16_t* x, const int32_t* expert, int P, const uint8_t* gu_blocks,
+                    const uint8_t* gu_scales, const float* gu_bias, const uint8_t* d_blocks,
+                    const uint8_t* d_scales, const float* d_bias, int E, int H, int I,
+                    const float* act_scale, float* y) {
+  LayerArgs A{x, x, nullptr, gu_blocks, gu_scales, gu_bias, d_blocks, d_scales, d_bias,
+              E, 1, P, H, I, act_scale};
+  int rc = check_layer(A);
+  if (rc) return rc;
+  for (int p = 0; p < P; ++p)
+    if (expert[p] < 0 || expert[p] >= E) return ORC_EINVAL;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int p = 0; p < P; ++p) expert_ffn(A, p, expert[p], y + (int64_t)p * H, nullptr);
+  return ORC_OK;
+}
+
 // Static per-tensor activation scales from a calibration batch (min-max observer):
 // s0 = amax|x| / 448; s1 = amax over routed (token, expert) pairs of the bf16-path gated
 // activation (fp32, before rounding) / 448.

@@ -74,3 +74,22 @@ def test_dense_rejects_shapes_its_kernels_do_not_take(B):
     with pytest.raises(B.MxmoeError) as ei:
         _run(B, B.moe_mxfp4_forward_dense, d, 2)
     assert ei.value.rc == B.EUNSUPPORTED
+
+
+@pytest.mark.parametrize("fp8", [True, False])
+def test_every_expert_selected_runs_dense_and_matches_the_oracle(B, fp8):
+    """k == E above the decode sizes: moe_mxfp4_forward takes the dense path (the measured
+    crossover); the result still matches the oracle's routed (= dense) layer."""
+    lay = inputs.small_layer(E=8, k=8, T=150, H=256, I=256, seed=35, router_bias=True,
+                             router_std=1.0 / np.sqrt(256))
+    p = pack(lay)
+    d = to_device(p)
+    s = oracle.calibrate(p.x, p.router_w, p.router_b, *p.weights, 8) if fp8 else None
+    got = _run(B, B.moe_mxfp4_forward, d, 8, s)
+    dense_launches = B.mxmoe_last_launch_count()
+    dense = _run(B, B.moe_mxfp4_forward_dense, d, 8, s)
+    assert dense_launches == B.mxmoe_last_launch_count()
+    assert torch.equal(got.view(torch.int16), dense.view(torch.int16))
+    _, oacc, _, _ = p.oracle_forward(act_scale=s)
+    ok, rel, excess = output_tolerance_ok(inputs.bits(got), oacc)
+    assert ok, f"max|d|/max|ref| = {rel:.3e}, worst excess {excess:.3e}"
