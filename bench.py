@@ -66,6 +66,7 @@ WORKLOADS = {
 }
 CODEC = "codec"
 CROSSOVER = "crossover"
+ATTN = "attn_fp8"
 # The default line: the largest single-GPU configuration (120B-shaped prefill, T = 16384,
 # Zipf-skewed routing), then the 120B prefill at T = 4096 and the 20B decode batches
 # measured in the same run.
@@ -593,6 +594,104 @@ def run_ours(args, world, rank):
     return res
 
 
+# --------------------------------------------- FP8 attention projections (fp8_linear) -----
+
+ATTN_T = 4096
+ATTN_SHAPES = (("qkv", 2880, 5120), ("o", 4096, 2880))   # (name, K in, N out)
+
+
+def attn_weights(device):
+    """FP8 E4M3 weights of the 120B model's attention projections with static per-tensor
+    scales (min-max observer: s_w = amax / 448), drawn N(0, 0.02) and cast by the library."""
+    from mxfp4_block_scaled_moe_b200 import binding as B
+    ws = {}
+    for name, K, N in ATTN_SHAPES:
+        w = inputs.normal((N, K), 0.02, 0, "attn_" + name, 0, device)
+        s_w = float(w.abs().max()) / 448.0
+        wq = B.moe_fp8_quantize(w.to(torch.bfloat16), s_w)
+        b = inputs.normal((N,), 0.01, 0, "attn_b_" + name, 0, device)
+        ws[name] = (wq, s_w, b)
+    torch.cuda.synchronize()
+    return ws
+
+
+def run_attn_fp8(args, world, rank):
+    """A step = the fused Q/K/V projection (2880 -> 5120) and the O projection (4096 ->
+    2880) of T tokens through fp8_linear (FP8 E4M3 weights and inputs, static per-tensor
+    scales; "gpt-oss-120b-mxfp4-fp8attn-v2", Model Details). Metric tokens/s; roofline
+    of the larger GEMM against the measured FP8 MMA rate (kind::f8f6f4 runs at the same
+    rate as the probe's kind::mxf8f6f4, 16384 FLOP per SM cycle)."""
+    from mxfp4_block_scaled_moe_b200 import binding as B
+    pk, pk_kind = peaks()
+    tpk = tensor_peak(B) if not args.no_tc_probe else None
+    T = args.attn_tokens
+    ws = attn_weights("cuda")
+    xs = {name: inputs.normal((T, K), 1.0, 1, "attn_x_" + name, 0, "cuda", torch.bfloat16)
+          for name, K, N in ATTN_SHAPES}
+    s_x = {name: float(xs[name].float().abs().max()) / 448.0 for name, _, _ in ATTN_SHAPES}
+    outs = {name: torch.empty(T, N, dtype=torch.bfloat16, device="cuda") for name, K, N in ATTN_SHAPES}
+    flusher = L2Flush()
+
+    def step():
+        for name, K, N in ATTN_SHAPES:
+            wq, s_w, b = ws[name]
+            B.fp8_linear(xs[name], wq, s_x[name], s_w, b, out=outs[name])
+
+    for _ in range(args.warmup):
+        step()
+    B.mxmoe_check()
+    launches = 2 * len(ATTN_SHAPES)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t_end = time.perf_counter() + 1.0
+        while time.perf_counter() < t_end:
+            step()
+            torch.cuda.synchronize()
+        barrier(world)
+        ms = time_steps(step, args.steps, flusher)
+        barrier(world)
+    ms = max_over_ranks(ms, world)
+    per = {}
+    for name, K, N in ATTN_SHAPES:
+        wq, s_w, b = ws[name]
+        per[name] = time_steps(lambda: B.fp8_linear(xs[name], wq, s_x[name], s_w, b, out=outs[name]),
+                               args.steps, flusher)
+    flops = {name: 2.0 * T * K * N for name, K, N in ATTN_SHAPES}
+    dom = max(per, key=per.get)
+    achieved = flops[dom] / (per[dom] / 1e3) / 1e12
+    peak = tpk["peak_tflops"] if tpk else pk["bf16_tflops"] * 2.0
+    res = {
+        "metric": "FP8 attention-projection tokens/s", "value": round(T * world / (ms / 1e3), 1), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 x e4m3 -> f32",
+        "data": "synthetic (seeded; weights N(0,0.02) cast to FP8 E4M3 with a per-tensor min-max scale)",
+        "config": {"workload": f"attn_fp8: fused QKV 2880->5120 and O 4096->2880, T={T}",
+                   "l2": "flushed before every timed step (512 MiB write, then a 256 MiB read)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "tensor", "kernel": f"fp8_linear {dom}", "achieved": round(achieved, 2),
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                     "peak_source": "measured kind::mxf8f6f4 rate probe (this run, this GPU)" if tpk
+                     else f"{pk_kind} bf16 burst x 2", "kernel_ms": round(per[dom], 5),
+                     "frac_of_nominal_fp8": round(achieved / NOMINAL_PEAKS["fp8_tflops"], 4)},
+        "stages_ms_per_step": {k: round(v, 5) for k, v in per.items()},
+        "gpu_launches": launches * args.steps,
+        "clocks": clk.summary(),
+    }
+    if tpk:
+        res["tensor_peak_probe"] = tpk
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        n = 4
+        t0 = time.perf_counter()
+        for name, K, N in ATTN_SHAPES:
+            wq, s_w, b = ws[name]
+            oracle.fp8_linear(inputs.bits(xs[name][:n]), wq.cpu().numpy(), np.float32(s_x[name]),
+                              np.float32(s_w), b.cpu().numpy())
+        dt = time.perf_counter() - t0
+        res["cpu_baseline"] = {"value": round(n / dt, 4), "unit": "tokens/s", "cores": oracle.num_threads(),
+                               "kind": "oracle", "sample": f"first {n} of {T} tokens, both projections, {dt:.1f} s"}
+    return res
+
+
 # ------------------------------------------------------- routed / dense crossover -----
 
 CROSSOVER_GRID = ((32, 4, (16, 64, 128, 256, 512, 1024)), (128, 4, (64, 256, 512, 1024, 2048, 4096)),
@@ -951,7 +1050,8 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS) + [CODEC, CROSSOVER], default=DEFAULT_WORKLOAD)
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + [CODEC, CROSSOVER, ATTN], default=DEFAULT_WORKLOAD)
+    ap.add_argument("--attn-tokens", type=int, default=ATTN_T, help="attn_fp8 workload: tokens per step")
     ap.add_argument("--extra", default=None,
                     help="comma-separated workloads measured in the same run and reported under "
                          "other_configs (default: the 120B prefill and the three decode batches "
@@ -978,16 +1078,16 @@ def main():
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))
-        if args.workload == CROSSOVER:
-            res = {"impl": "reference", "unavailable": "the crossover workload compares two GPU paths; "
-                                                       "the oracle has no counterpart to time"}
+        if args.workload in (CROSSOVER, ATTN):
+            res = {"impl": "reference", "unavailable": "the crossover and attention workloads report the oracle "
+                                                       "as the cpu_baseline of their own line"}
             res = res if int(os.environ.get("RANK", "0")) == 0 else None
         else:
             res = (run_reference_codec if args.workload == CODEC else run_reference)(args, world, rank)
     else:
         world, rank = dist_init()
         try:
-            run = {CODEC: run_codec, CROSSOVER: run_crossover}.get(args.workload, run_ours)
+            run = {CODEC: run_codec, CROSSOVER: run_crossover, ATTN: run_attn_fp8}.get(args.workload, run_ours)
             res = run(args, world, rank)
         finally:
             if world > 1:
