@@ -680,13 +680,19 @@ def run_attn_fp8(args, world, rank):
         res["tensor_peak_probe"] = tpk
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
-        n = 4
-        t0 = time.perf_counter()
-        for name, K, N in ATTN_SHAPES:
-            wq, s_w, b = ws[name]
-            oracle.fp8_linear(inputs.bits(xs[name][:n]), wq.cpu().numpy(), np.float32(s_x[name]),
-                              np.float32(s_w), b.cpu().numpy())
-        dt = time.perf_counter() - t0
+        host = {name: (inputs.bits(xs[name]), ws[name][0].cpu().numpy(), ws[name][2].cpu().numpy())
+                for name, _, _ in ATTN_SHAPES}
+
+        def oracle_step(n):
+            t0 = time.perf_counter()
+            for name, K, N in ATTN_SHAPES:
+                xb, wq_h, b_h = host[name]
+                oracle.fp8_linear(xb[:n], wq_h, np.float32(s_x[name]), np.float32(ws[name][1]), b_h)
+            return time.perf_counter() - t0
+
+        t1 = oracle_step(1)   # one token per thread-slot: scale the sample to ~cpu_budget seconds
+        n = int(max(1, min(T, args.cpu_budget * oracle.num_threads() / max(t1, 1e-6))))
+        dt = oracle_step(n)
         res["cpu_baseline"] = {"value": round(n / dt, 4), "unit": "tokens/s", "cores": oracle.num_threads(),
                                "kind": "oracle", "sample": f"first {n} of {T} tokens, both projections, {dt:.1f} s"}
     return res

@@ -490,9 +490,7 @@ moe_gemm_parts_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_c
 #pragma unroll
           for (int i = 0; i < 8; ++i) o[i] = __fadd_rn(__uint_as_float(v[i]), bb[i]);
           if (valid && live) {
-            float4* dst = reinterpret_cast<float4*>(p.y_out + pos * p.n_out + n0 + c0);
-            dst[0] = make_float4(o[0], o[1], o[2], o[3]);
-            dst[1] = make_float4(o[4], o[5], o[6], o[7]);
+            st_global_v8(p.y_out + pos * p.n_out + n0 + c0, o);
           }
         }
       }

@@ -139,6 +139,7 @@ cudaError_t launch_split_tokens(bool fp8, const uint16_t* x, const int32_t* topk
                                 cudaStream_t st);
 cudaError_t launch_decode_gemm(bool gate_up, const DecodeGemmArgs& a, cudaStream_t st);
 
+
 // dense all-experts path (csrc/dense.cu): gates (T, E) and offsets e * T; the weighted sum
 // over all experts of y laid out expert-major (E * T, H)
 cudaError_t launch_dense_setup(const int32_t* topk_idx, const float* topk_w, int T, int E, int k, float* gates,

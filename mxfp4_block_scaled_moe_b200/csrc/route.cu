@@ -10,6 +10,7 @@
 #include <atomic>
 
 #include "common.cuh"
+#include "topk.cuh"
 
 namespace mxmoe {
 
@@ -166,66 +167,7 @@ __global__ void __launch_bounds__(128) router_gemm_kernel(const uint16_t* __rest
 }
 
 // ----------------------------------------------------------------------- top-k -----
-// Ranking: larger logit first, NaN after every number, equal values -> lower id first.
-__device__ __forceinline__ bool ranks_before(float a, int ia, float b, int ib) {
-  const bool na = isnan(a), nb = isnan(b);
-  if (na != nb) return nb;
-  if (!na && a != b) return a > b;
-  return ia < ib;
-}
-
-// One warp selects the k largest of a token's E logits (E <= 256, each lane holds up to 8)
-// and writes the indices and the softmax over them.
-__device__ __forceinline__ void topk_warp(const float* __restrict__ l, int E, int k,
-                                          int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
-  const int lane = threadIdx.x & 31;
-  float v[8];
-  int taken = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int e = lane + 32 * i;
-    v[i] = e < E ? l[e] : 0.0f;
-  }
-  float sel[8];
-  int sidx[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    if (j >= k) break;
-    float bv = 0.0f;
-    int bi = -1;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E && !((taken >> i) & 1) && (bi < 0 || ranks_before(v[i], e, bv, bi))) {
-        bv = v[i];
-        bi = e;
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (oi >= 0 && (bi < 0 || ranks_before(ov, oi, bv, bi))) { bv = ov; bi = oi; }
-    }
-    sel[j] = bv;
-    sidx[j] = bi;
-    if ((bi & 31) == lane) taken |= 1 << (bi >> 5);
-  }
-  // softmax over the k selected logits: lane j < k takes term j; every lane adds the terms
-  // in order j = 0 .. k-1 (the same sum as a sequential loop)
-  float my_sel = sel[0];
-  int my_idx = sidx[0];
-#pragma unroll
-  for (int j = 1; j < 8; ++j)
-    if (j < k && lane == j) { my_sel = sel[j]; my_idx = sidx[j]; }
-  const float pj = lane < k ? expf(my_sel - sel[0]) : 0.0f;
-  float z = 0.0f;
-  for (int j = 0; j < k; ++j) z += __shfl_sync(0xffffffffu, pj, j);
-  if (lane < k) {
-    idx_out[lane] = my_idx;
-    w_out[lane] = __fdiv_rn(pj, z);
-  }
-}
+// topk_warp (csrc/topk.cuh): one warp per token.
 
 // n_rest > 0: the router wrote its logits as 1 + n_rest partials over K ranges (rest:
 // n_rest arrays of T*E after logits); a token's logits are their sum in range order,
@@ -428,6 +370,7 @@ __global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(
 // single-CTA permutation. Every counter is reset by the CTA that consumed it. Saves two
 // launches on the latency-bound decode path.
 constexpr int kSmallT = 64, kSmallE = 256;
+constexpr int kSmallPairs = 64;   // routed pairs placed by the direct count in route_small_kernel
 
 __global__ void __launch_bounds__(kPermThreads) route_small_kernel(
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ wr, const uint16_t* __restrict__ br,
@@ -520,6 +463,50 @@ __global__ void __launch_bounds__(kPermThreads) route_small_kernel(
   if (!s_last) return;
   __threadfence();
   __syncthreads();   // the CTA's global writes of topk_idx are visible to all its threads
+  const int P = T * k;
+  if (P <= kSmallPairs) {
+    // A handful of pairs (a decode step): each pair's position is the number of valid pairs
+    // with a smaller expert id plus the earlier valid pairs with the same one -- the order of
+    // the general scatter, without its passes and barriers.
+    int* s_e = sm.scan_tmp;   // P <= 256 expert ids
+    int* s_off = &sm.wc[0][0];   // E + 1 <= 257 offsets
+    for (int q = threadIdx.x; q < P; q += blockDim.x) {
+      int e = __ldcg(topk_idx + q);
+      if (e < 0 || e >= E) {
+        set_device_error(err, MXMOE_EDEVICE);
+        e = -1;
+      }
+      s_e[q] = e;
+    }
+    __syncthreads();
+    for (int q = threadIdx.x; q < P; q += blockDim.x) {
+      const int e = s_e[q];
+      if (e < 0) continue;
+      int pos = 0;
+      for (int r = 0; r < P; ++r) {
+        const int f = s_e[r];
+        pos += (f >= 0 && (f < e || (f == e && r < q))) ? 1 : 0;
+      }
+      perm_token[pos] = q / k;
+      perm_slot[pos] = q % k;
+      inv[q] = pos;
+    }
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) {
+      int c = 0;
+      for (int r = 0; r < P; ++r) c += (s_e[r] >= 0 && s_e[r] < e) ? 1 : 0;
+      s_off[e] = c;
+      offsets[e] = c;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int n = 0;
+      for (int e = 0; e < E; ++e)
+        if (s_off[e + 1] > s_off[e]) active[n++] = e;
+      *n_active = n;
+      *ticket = 0u;
+    }
+    return;
+  }
   permute_scatter_body(sm, 0, topk_idx, static_cast<int64_t>(T) * k, E, k, nullptr, offsets, perm_token,
                        perm_slot, inv, active, n_active, err);
   if (threadIdx.x == 0) *ticket = 0u;
