@@ -33,8 +33,9 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
       const int j = ord[q];
       const float w = topk_w[static_cast<int64_t>(t) * k + j];
       const int64_t pos = inv[static_cast<int64_t>(t) * k + j];
-      float v[8];
-      ld_global_v8(y + pos * H + 8 * c, v);   // H % 8 == 0: 32-byte aligned
+      const float4* src = reinterpret_cast<const float4*>(y + pos * H) + 2 * c;
+      const float4 a = src[0], b = src[1];
+      const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
       for (int r = 0; r < 8; ++r) acc[r] = __fadd_rn(acc[r], __fmul_rn(w, v[r]));
     }

@@ -72,13 +72,6 @@ __device__ __forceinline__ void st_global_v8(float* dst, const float (&v)[8]) {
                : "memory");
 }
 
-// One 32-byte load of eight fp32 values (256-bit global load); src 32-byte aligned.
-__device__ __forceinline__ void ld_global_v8(const float* src, float (&v)[8]) {
-  asm volatile("ld.global.v8.f32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n"
-               : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7])
-               : "l"(src));
-}
-
 // Programmatic dependent launch: a kernel launched with programmatic stream serialization
 // may start once every CTA of the previous kernel in the stream has called
 // griddep_launch_dependents() (or exited); griddep_wait() returns once that kernel has

@@ -428,17 +428,15 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
       sc.stage_bytes = stage_bytes_for(kA, b_rows);
       const int avail = static_cast<int>((smem_raw + p.smem_bytes) - ring);
       sc.stages = min(kMaxStages, avail / (sc.stage_bytes + sf_stage_bytes(kA)));
-      // K split: fewest stages on the busiest CTA, counting for each split unit's partial
-      // write, ticket and the finisher's reduction about four stages when the unit is wide
-      // (its partial is up to 128 x 224 fp32 per tile) and one when it holds a few tokens
-      // (one token: 92 tiles for 148 SMs; three splits of four stages bring the busiest CTA
-      // from twelve stages to eight)
+      // K split: fewest stages on the busiest CTA, counting about four stages for each
+      // split unit's partial write, ticket and the finisher's reduction (measured: at one
+      // token, three splits of four stages instead of one unit of twelve made gate_up
+      // slower, 39.7 against 26.7 us)
       const int tiles = ng * p.n_m, G = gridDim.x;
-      const int pen = maxcols <= 32 ? 1 : 4;
       int best = 1, best_cost = INT_MAX;
       for (int s = 1; s <= min(p.split_cap, p.nst); ++s) {
         const int per = (tiles * s + G - 1) / G;
-        const int cost = per * ((p.nst + s - 1) / s) + (s > 1 ? pen * per : 0);
+        const int cost = per * ((p.nst + s - 1) / s) + (s > 1 ? 4 * per : 0);
         if (cost < best_cost) { best_cost = cost; best = s; }
       }
       sc.nsplit = best;
