@@ -367,7 +367,8 @@ class L2Flush:
 
 def kernel_roofline(name, lay, work, stages, act, pk, pk_kind, tpk):
     """The dominant kernel (the largest stage other than routing, casts and combine)
-    against its bound: tensor FLOPs at prefill sizes, packed-weight HBM bytes at decode."""
+    against its bound: tensor FLOPs at prefill sizes, packed-weight HBM bytes at decode
+    (the whole step's bytes when the step is the one-launch decode layer)."""
     small = ("router", "topk", "router+topk", "route", "permute", "act_quant", "act_quant+scatter", "act_split",
              "mid_split", "combine")
     dom = max((s for s in stages if s not in small), key=lambda s: stages[s][0], default=None)
@@ -378,7 +379,8 @@ def kernel_roofline(name, lay, work, stages, act, pk, pk_kind, tpk):
     extra = {}
     if lay.T >= 1024:
         bound, unit = "tensor", "TFLOP/s"
-        flops = work["gu_flops"] if dom == "gate_up" else work["flops"] - work["gu_flops"]
+        flops = work["gu_flops"] if dom == "gate_up" else work["flops"] if dom == "layer" else \
+            work["flops"] - work["gu_flops"]
         achieved = flops / (dom_ms / 1e3) / 1e12
         if fp8 and tpk:
             peak = tpk["peak_tflops"]
@@ -395,7 +397,9 @@ def kernel_roofline(name, lay, work, stages, act, pk, pk_kind, tpk):
     else:
         bound, unit = "hbm", "GB/s"
         peak = pk["hbm_gbs"]
-        b = work["gu_bytes"] if dom == "gate_up" else work["bytes"] - work["gu_bytes"]
+        # "layer": the one-launch decode layer moves the whole step's bytes
+        b = work["gu_bytes"] if dom == "gate_up" else work["bytes"] if dom == "layer" else \
+            work["bytes"] - work["gu_bytes"]
         achieved = b / (dom_ms / 1e3) / 1e9
         peak_note = f"{pk_kind} hbm copy"
         extra = {"frac_of_nominal_hbm": round(achieved / NOMINAL_PEAKS["hbm_gbs"], 4)}

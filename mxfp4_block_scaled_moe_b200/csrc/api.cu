@@ -92,6 +92,7 @@ struct Workspace {
   int smem_K = 0;      // largest K the expert kernels were configured for
   bool tc_ready = false;  // tcgen05 GEMM shared-memory limit raised
   bool dtc_ready = false; // tensor-core decode kernels' shared-memory limit raised
+  bool dl_ready = false;  // one-launch decode layer's shared-memory limit raised
   bool tcb_ready = false; // two-part (bf16 activation) tcgen05 GEMM's shared-memory limit raised
   size_t tickets_zeroed = 0;  // bytes at the start of the workspace known to be zero
 };
@@ -188,15 +189,25 @@ struct LayerBuffers {
   unsigned* dtickets;  // tensor-core decode: split-K and combine tickets (zero between calls)
   size_t tickets_end;  // bytes from the workspace start that hold tickets
   float* part;         // tensor-core decode: split-K partial accumulators
+  // one-launch decode layer (T <= kDecodeLayerMaxT)
+  unsigned* dl_counters;   // zero between calls
+  uint8_t* dl_xs;
+  uint8_t* dl_sfx;
+  uint8_t* dl_xs_mid;
+  uint8_t* dl_sf_mid;
+  float* dl_part;
+  float* dl_dpart;
 };
 
 // n_rest: the tensor-core router's extra K-range partials of the logits (T x E each)
-size_t layout(int T, int E, int k, int H, int I, bool fp8, bool tc, bool tcb, bool dtc, int n_rest,
-              LayerBuffers* b, char* base) {
+size_t layout(int T, int E, int k, int H, int I, bool fp8, bool tc, bool tcb, bool dtc, bool dlay, int sms,
+              int n_rest, LayerBuffers* b, char* base) {
   const int64_t P = static_cast<int64_t>(T) * k;
+  const mxmoe::DecodeLayerSizes dls = dlay ? mxmoe::decode_layer_sizes(T, H, I, sms) : mxmoe::DecodeLayerSizes{};
   Carve c;
   size_t o_tickets = c.take<uint8_t>(kTicketBytes);
   size_t o_dtick = c.take<unsigned>(dtc ? static_cast<int64_t>(mxmoe::decode_tc_ticket_count(H, I)) : 0);
+  size_t o_dlc = c.take<unsigned>(static_cast<int64_t>(dls.counters));
   const size_t tickets_end = c.off;
   size_t o_logits = c.take<float>(static_cast<int64_t>(T) * E);
   size_t o_lrest = c.take<float>(static_cast<int64_t>(n_rest) * T * E);
@@ -217,7 +228,20 @@ size_t layout(int T, int E, int k, int H, int I, bool fp8, bool tc, bool tcb, bo
   size_t o_xsm = c.take<uint8_t>(dtc ? static_cast<int64_t>(mxmoe::decode_tc_xs_bytes(P, I)) : 0);
   size_t o_sfbm = c.take<uint8_t>(dtc ? static_cast<int64_t>(mxmoe::decode_tc_sfb_bytes(E, I, T)) : 0);
   size_t o_part = c.take<uint8_t>(dtc ? static_cast<int64_t>(mxmoe::decode_tc_part_bytes(P, H, I)) : 0);
+  size_t o_dlxs = c.take<uint8_t>(static_cast<int64_t>(dls.xs));
+  size_t o_dlsfx = c.take<uint8_t>(static_cast<int64_t>(dls.sfx));
+  size_t o_dlmid = c.take<uint8_t>(static_cast<int64_t>(dls.xs_mid));
+  size_t o_dlsfm = c.take<uint8_t>(static_cast<int64_t>(dls.sf_mid));
+  size_t o_dlp = c.take<uint8_t>(static_cast<int64_t>(dls.part));
+  size_t o_dldp = c.take<uint8_t>(static_cast<int64_t>(dls.dpart));
   if (b) {
+    b->dl_counters = reinterpret_cast<unsigned*>(base + o_dlc);
+    b->dl_xs = reinterpret_cast<uint8_t*>(base + o_dlxs);
+    b->dl_sfx = reinterpret_cast<uint8_t*>(base + o_dlsfx);
+    b->dl_xs_mid = reinterpret_cast<uint8_t*>(base + o_dlmid);
+    b->dl_sf_mid = reinterpret_cast<uint8_t*>(base + o_dlsfm);
+    b->dl_part = reinterpret_cast<float*>(base + o_dlp);
+    b->dl_dpart = reinterpret_cast<float*>(base + o_dldp);
     b->dtickets = reinterpret_cast<unsigned*>(base + o_dtick);
     b->tickets_end = tickets_end;
     b->part = reinterpret_cast<float*>(base + o_part);
@@ -304,16 +328,19 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
   // e4m3 parts (exact for the activations' significant bits)
   const bool tcb = !fp8 && !calib_out && large && std::max(a.H, a.I) / 32 <= kTcMaxNb &&
                    tc_gemm_supported(a.H, a.I, a.gu_blocks, a.d_blocks, a.gu_scales, a.d_scales);
-  const bool dtc = !tc && !tcb && !calib_out &&
+  // a handful of tokens: the whole layer in one launch
+  const bool dlay = !tc && !tcb && !calib_out && a.T <= kDecodeLayerMaxT &&
+                    decode_layer_supported(a.H, a.I, a.T, a.E, a.k, a.gu_blocks, a.d_blocks, a.gu_scales, a.d_scales);
+  const bool dtc = !tc && !tcb && !dlay && !calib_out &&
                    decode_tc_supported(a.H, a.I, a.T, a.gu_blocks, a.d_blocks, a.gu_scales, a.d_scales);
   // routing: one fused launch for small batches; else the router GEMM (on the tensor cores
   // when the shapes allow, split over K ranges) and a top-k kernel that adds the ranges
-  const bool small = route_small_supported(a.T, a.E, a.k);
+  const bool small = !dlay && route_small_supported(a.T, a.E, a.k);
   const int ksplit = !small && router_tc_supported(a.T, a.H, a.E, a.x, a.router_w, nullptr)
                          ? router_tc_ksplit(a.T, a.H, ws->sms)
                          : 0;
   const int n_rest = ksplit > 1 ? ksplit - 1 : 0;
-  const size_t need = layout(a.T, a.E, a.k, a.H, a.I, fp8, tc, tcb, dtc, n_rest, nullptr, nullptr);
+  const size_t need = layout(a.T, a.E, a.k, a.H, a.I, fp8, tc, tcb, dtc, dlay, ws->sms, n_rest, nullptr, nullptr);
   if (int rc = ensure_capacity(ws, need)) return rc;
   if (std::max(a.H, a.I) > ws->smem_K) {
     cudaError_t e = expert_mma_set_smem_limits(std::max(a.H, a.I));
@@ -330,26 +357,52 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (two-part tcgen05 GEMM)");
     ws->tcb_ready = true;
   }
+  if (dlay && !ws->dl_ready) {
+    cudaError_t e = decode_layer_prepare();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (decode layer)");
+    ws->dl_ready = true;
+  }
   if (dtc && !ws->dtc_ready) {
     cudaError_t e = decode_tc_prepare();
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (tensor-core decode)");
     ws->dtc_ready = true;
   }
   LayerBuffers b;
-  layout(a.T, a.E, a.k, a.H, a.I, fp8, tc, tcb, dtc, n_rest, &b, ws->base);
-  // The decode path's tickets follow the fixed ticket block, where other layouts keep
+  layout(a.T, a.E, a.k, a.H, a.I, fp8, tc, tcb, dtc, dlay, ws->sms, n_rest, &b, ws->base);
+  // The decode paths' tickets follow the fixed ticket block, where other layouts keep
   // ordinary buffers: they are known to be zero only after a decode-path call, which
   // leaves them at zero. Clear them when that is not known.
-  if (dtc && b.tickets_end > ws->tickets_zeroed) {
+  const bool counted = dtc || dlay;
+  if (counted && b.tickets_end > ws->tickets_zeroed) {
     cudaError_t e = cudaMemsetAsync(ws->base, 0, b.tickets_end, st);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync (tickets)");
   }
-  ws->tickets_zeroed = dtc ? b.tickets_end : kTicketBytes;
+  ws->tickets_zeroed = counted ? b.tickets_end : kTicketBytes;
   int launches = 0;
   cudaError_t e;
   const float s0 = fp8 ? act_scale[0] : 1.0f, s1 = fp8 ? act_scale[1] : 1.0f;
 
   StageTimer tm(st);
+  if (dlay) {
+    DecodeLayerArgs d{};
+    d.x = a.x; d.router_w = a.router_w; d.router_b = a.router_b;
+    d.gu_blocks = a.gu_blocks; d.gu_scales = a.gu_scales; d.gu_bias = a.gu_bias;
+    d.d_blocks = a.d_blocks; d.d_scales = a.d_scales; d.d_bias = a.d_bias;
+    d.E = a.E; d.H = a.H; d.I = a.I; d.T = a.T; d.k = a.k;
+    d.fp8 = fp8; d.s0 = s0; d.s1 = s1;
+    d.sms = ws->sms;
+    d.logits = b.logits;
+    d.xs = b.dl_xs; d.sfx = b.dl_sfx; d.xs_mid = b.dl_xs_mid; d.sf_mid = b.dl_sf_mid;
+    d.part = b.dl_part; d.dpart = b.dl_dpart; d.counters = b.dl_counters;
+    d.topk_idx = b.topk_idx; d.topk_w = b.topk_w;
+    d.out = out;
+    d.err = ws->err;
+    if ((e = launch_decode_layer(d, st))) return cuda_fail(e, "decode layer");
+    ++launches;
+    tm.mark("layer");
+    t_last_launches = launches;
+    return MXMOE_OK;
+  }
   if (small) {
     // small batch: router, top-k and permutation in one CTA, one launch
     if ((e = launch_route_small(a.x, a.router_w, a.router_b, a.T, a.H, a.E, a.k, b.logits,
@@ -1095,6 +1148,8 @@ int mxmoe_check(void* stream) {
   if ((e = cudaMemcpy(&v, ws->err, sizeof(int), cudaMemcpyDeviceToHost))) return cuda_fail(e, "read error word");
   if (v != 0) {
     if ((e = cudaMemset(ws->err, 0, sizeof(int)))) return cuda_fail(e, "clear error word");
+    // a kernel that stopped early may have left its counters short of zero
+    ws->tickets_zeroed = 0;
     return fail(v, "device error word = %d", v);
   }
   return MXMOE_OK;

@@ -43,6 +43,7 @@
 
 #include "common.cuh"
 #include "tc_common.cuh"
+#include "tmap.h"
 
 namespace mxmoe {
 namespace g100b {
@@ -522,38 +523,6 @@ size_t smem_bytes(int E) {
 }  // namespace g100b
 
 // ---------------------------------------------------------------- host side -------
-namespace {
-
-using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiled encoder() {
-  static EncodeTiled fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiled>(p);
-  }
-  return fn;
-}
-
-bool encode(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
-            const uint64_t* strides_bytes, const uint32_t* box) {
-  EncodeTiled fn = encoder();
-  if (!fn) return false;
-  cuuint64_t d[3], s[2];
-  cuuint32_t b[3], es[3] = {1, 1, 1};
-  for (int i = 0; i < rank; ++i) { d[i] = dims[i]; b[i] = box[i]; }
-  for (int i = 0; i + 1 < rank; ++i) s[i] = strides_bytes[i];
-  return fn(m, dt, rank, const_cast<void*>(base), d, s, b, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-}  // namespace
 
 // src rows (bf16, K values) -> two e4m3 parts (2, P, K) + e8m0 scales (2, P, K/32); row m
 // is src[perm[m]] when perm is given (tokens in expert-grouped order), else src[m].
@@ -592,7 +561,7 @@ cudaError_t launch_tc_parts_gemm(bool gate_up, const uint8_t* parts, const uint8
     const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(P_rows > 0 ? 2 * P_rows : 1)};
     const uint64_t strides[1] = {static_cast<uint64_t>(K)};
     const uint32_t box[2] = {BK, BM};
-    if (!encode(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, parts, dims, strides, box)) return cudaErrorInvalidValue;
+    if (!tmap_encode(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, parts, dims, strides, box)) return cudaErrorInvalidValue;
   }
   {
     const uint64_t row_bytes = static_cast<uint64_t>(K) / 2;
@@ -600,10 +569,10 @@ cudaError_t launch_tc_parts_gemm(bool gate_up, const uint8_t* parts, const uint8
                               static_cast<uint64_t>(groups)};
     const uint64_t strides[2] = {row_bytes, row_bytes * rows_per_group};
     const uint32_t box[3] = {BK, static_cast<uint32_t>(bn_rows), 1};
-    if (!encode(&mb, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, blocks, dims, strides, box))
+    if (!tmap_encode(&mb, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, blocks, dims, strides, box))
       return cudaErrorInvalidValue;
     const uint64_t tdims[3] = {BK, static_cast<uint64_t>(rows_per_group), static_cast<uint64_t>(groups)};
-    if (!encode(&mbt, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, blocks + (K - BK) / 2, tdims, strides, box))
+    if (!tmap_encode(&mbt, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, blocks + (K - BK) / 2, tdims, strides, box))
       return cudaErrorInvalidValue;
   }
   Params prm;

@@ -48,7 +48,9 @@
 
 #include "common.cuh"
 #include "launchers.h"
+#include "mx_parts.cuh"
 #include "tc_common.cuh"
+#include "tmap.h"
 
 namespace mxmoe {
 namespace dec {
@@ -81,29 +83,8 @@ constexpr int kMaxSplit = 8;
 constexpr int kMaxTopK = 8;
 constexpr int kSmemBytes = 227 * 1024;
 
-// instruction descriptor, kind::mxf4 block-scaled (scale_vec::2X): A = B = E2M1 (1),
-// e8m0 scales; sf_id (0 or 2) selects the scale-byte pair of a K = 64 step.
-__host__ __device__ constexpr uint32_t idesc_mxf4(int M, int N) {
-  return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
-         (static_cast<uint32_t>(M >> 4) << 24);
-}
-
 __host__ __device__ __forceinline__ int sf_atom_byte(int r, int j) {   // r < 256
   return (r >> 7) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + j;
-}
-
-__device__ __forceinline__ float pow2f(int s) {   // exact 2^s for s in [-126, 127]
-  return __uint_as_float(static_cast<uint32_t>(s + 127) << 23);
-}
-
-// Scale exponent of an e2m1 part: the smallest s with amax / 2^s <= 6 (the e2m1 maximum),
-// clamped to [-126, 125]; amax == 0 gives 0. Branch-free: a subnormal amax reads as
-// floor(log2) = -127, which the clamp maps to -126 exactly as its true exponent would.
-__device__ __forceinline__ int e2m1_part_exponent(float amax) {
-  const int fl = static_cast<int>(__float_as_uint(amax) >> 23) - 127;   // amax >= 0
-  int s = max(-126, min(125, fl - 2));                                   // amax / 2^s in [4, 8)
-  s = (amax > 6.0f * pow2f(s)) ? min(125, s + 1) : s;
-  return amax > 0.0f ? s : 0;
 }
 
 struct Params {
@@ -900,35 +881,6 @@ __global__ void __launch_bounds__(kSplitThreads) split_tokens_kernel(
 
 namespace {
 
-using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiled encoder() {
-  static EncodeTiled fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiled>(ptr);
-  }
-  return fn;
-}
-
-bool encode(CUtensorMap* m, int rank, const void* base, const uint64_t* dims, const uint64_t* strides_bytes,
-            const uint32_t* box) {
-  EncodeTiled fn = encoder();
-  if (!fn) return false;
-  cuuint64_t d[3], s[2];
-  cuuint32_t b[3], es[3] = {1, 1, 1};
-  for (int i = 0; i < rank; ++i) { d[i] = dims[i]; b[i] = box[i]; }
-  for (int i = 0; i + 1 < rank; ++i) s[i] = strides_bytes[i];
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, const_cast<void*>(base), d, s, b, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 constexpr size_t kPartBudget = 16u << 20;   // split-K partials, bytes
 
 int split_cap(int kA, int64_t P, int n_out) {
@@ -957,7 +909,7 @@ bool decode_tc_supported(int H, int I, int T, const void* gu_blocks, const void*
   // the widest B tile must still leave two pipeline stages
   const int worst = dec::ring_offset() + 2 * (dec::stage_bytes_for(2, dec::kMaxN) + dec::kSfStageMax);
   if (worst + 1024 > dec::kSmemBytes) return false;
-  return encoder() != nullptr;
+  return tmap_available();
 }
 
 cudaError_t decode_tc_prepare() {
@@ -1022,13 +974,13 @@ cudaError_t launch_decode_gemm(bool gate_up, const DecodeGemmArgs& a, cudaStream
     const uint64_t dims[3] = {row_bytes, static_cast<uint64_t>(n_out), static_cast<uint64_t>(groups)};
     const uint64_t strides[2] = {row_bytes, row_bytes * n_out};
     const uint32_t box[3] = {static_cast<uint32_t>(kRowBytes), BM, static_cast<uint32_t>(kA)};
-    if (!encode(&mw, 3, gate_up ? a.gu_blocks : a.d_blocks, dims, strides, box)) return cudaErrorInvalidValue;
+    if (!tmap_encode(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, gate_up ? a.gu_blocks : a.d_blocks, dims, strides, box)) return cudaErrorInvalidValue;
   }
   {
     const uint64_t dims[2] = {static_cast<uint64_t>(K) / 2, static_cast<uint64_t>(b_rows > 0 ? b_rows : 1)};
     const uint64_t strides[1] = {static_cast<uint64_t>(K) / 2};
     const uint32_t box[2] = {static_cast<uint32_t>(kRowBytes), static_cast<uint32_t>(box_rows)};
-    if (!encode(&mx, 2, gate_up ? a.xs : a.xs_mid, dims, strides, box)) return cudaErrorInvalidValue;
+    if (!tmap_encode(&mx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, gate_up ? a.xs : a.xs_mid, dims, strides, box)) return cudaErrorInvalidValue;
   }
   Params prm{};
   prm.w_scales = gate_up ? a.gu_scales : a.d_scales;

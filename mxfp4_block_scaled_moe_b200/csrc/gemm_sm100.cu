@@ -40,6 +40,7 @@
 
 #include "common.cuh"
 #include "tc_common.cuh"
+#include "tmap.h"
 
 namespace mxmoe {
 namespace g100 {
@@ -440,38 +441,6 @@ size_t smem_bytes(int E) {
 }  // namespace g100
 
 // ---------------------------------------------------------------- host side -------
-namespace {
-
-using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiled encoder() {
-  static EncodeTiled fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiled>(p);
-  }
-  return fn;
-}
-
-bool encode(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
-            const uint64_t* strides_bytes, const uint32_t* box) {
-  EncodeTiled fn = encoder();
-  if (!fn) return false;
-  cuuint64_t d[3], s[2];
-  cuuint32_t b[3], es[3] = {1, 1, 1};
-  for (int i = 0; i < rank; ++i) { d[i] = dims[i]; b[i] = box[i]; }
-  for (int i = 0; i + 1 < rank; ++i) s[i] = strides_bytes[i];
-  return fn(m, dt, rank, const_cast<void*>(base), d, s, b, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-}  // namespace
 
 // Whether the tcgen05 path can run these shapes/pointers (else the register-dequant path).
 bool tc_gemm_supported(int H, int I, const void* gu_blocks, const void* d_blocks, const void* gu_scales,
@@ -481,7 +450,7 @@ bool tc_gemm_supported(int H, int I, const void* gu_blocks, const void* d_blocks
   if ((reinterpret_cast<uintptr_t>(gu_blocks) | reinterpret_cast<uintptr_t>(d_blocks)) & 31u) return false;
   // the scale converters read the e8m0 bytes as 16-bit words
   if ((reinterpret_cast<uintptr_t>(gu_scales) | reinterpret_cast<uintptr_t>(d_scales)) & 1u) return false;
-  return encoder() != nullptr;
+  return tmap_available();
 }
 
 cudaError_t tc_gemm_prepare(int E) {
@@ -510,7 +479,7 @@ cudaError_t launch_tc_gemm(bool gate_up, const uint8_t* a, int64_t P_rows, int K
     const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(P_rows > 0 ? P_rows : 1)};
     const uint64_t strides[1] = {static_cast<uint64_t>(K)};
     const uint32_t box[2] = {BK, BM};
-    if (!encode(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a, dims, strides, box)) return cudaErrorInvalidValue;
+    if (!tmap_encode(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a, dims, strides, box)) return cudaErrorInvalidValue;
   }
   {
     const uint64_t row_bytes = static_cast<uint64_t>(K) / 2;
@@ -518,10 +487,10 @@ cudaError_t launch_tc_gemm(bool gate_up, const uint8_t* a, int64_t P_rows, int K
                               static_cast<uint64_t>(groups)};
     const uint64_t strides[2] = {row_bytes, row_bytes * rows_per_group};
     const uint32_t box[3] = {BK, static_cast<uint32_t>(bn_rows), 1};
-    if (!encode(&mb, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, blocks, dims, strides, box))
+    if (!tmap_encode(&mb, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, blocks, dims, strides, box))
       return cudaErrorInvalidValue;
     const uint64_t tdims[3] = {BK, static_cast<uint64_t>(rows_per_group), static_cast<uint64_t>(groups)};
-    if (!encode(&mbt, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, blocks + (K - BK) / 2, tdims, strides, box))
+    if (!tmap_encode(&mbt, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, blocks + (K - BK) / 2, tdims, strides, box))
       return cudaErrorInvalidValue;
   }
   Params prm;

@@ -122,6 +122,46 @@ struct DecodeGemmArgs {   // tensor-core decode path (kind::mxf4: packed e2m1 we
 constexpr int kDecodeMaxT = 64;      // tokens the tensor-core decode path takes
 constexpr int kDecodeMaxGroups = 320;  // row groups (an expert's routed rows, 56 at a time)
 constexpr int kDecodeFoldMaxT = 8;   // the down kernel folds the combine up to this many tokens
+// One-launch decode layer (csrc/decode_layer_sm100.cu): routing, token operand, gate_up,
+// down and combine of at most kDecodeLayerMaxT tokens in one persistent grid of one CTA
+// per SM.
+constexpr int kDecodeLayerMaxT = 8;
+struct DecodeLayerSizes {   // workspace pieces, bytes (counters: unsigned words, zero between calls)
+  size_t xs, sfx, xs_mid, sf_mid, part, dpart, counters;
+};
+struct DecodeLayerArgs {
+  const uint16_t* x;
+  const uint16_t* router_w;
+  const uint16_t* router_b;     // nullable
+  const uint8_t* gu_blocks;
+  const uint8_t* gu_scales;
+  const float* gu_bias;
+  const uint8_t* d_blocks;
+  const uint8_t* d_scales;
+  const float* d_bias;
+  int E, H, I, T, k;
+  bool fp8;                     // static per-tensor FP8 activations (s0, s1)
+  float s0, s1;
+  int sms;                      // grid size: every CTA must be resident at once
+  float* logits;                // (T, E)
+  uint8_t* xs;
+  uint8_t* sfx;
+  uint8_t* xs_mid;
+  uint8_t* sf_mid;
+  float* part;
+  float* dpart;
+  unsigned* counters;           // decode_layer_sizes().counters words, zero between calls
+  int32_t* topk_idx;            // (T, k), nullable
+  float* topk_w;
+  uint16_t* out;                // (T, H) bf16
+  int* err;
+};
+bool decode_layer_supported(int H, int I, int T, int E, int k, const void* gu_blocks, const void* d_blocks,
+                            const void* gu_scales, const void* d_scales);
+cudaError_t decode_layer_prepare();
+DecodeLayerSizes decode_layer_sizes(int T, int H, int I, int sms);
+cudaError_t launch_decode_layer(const DecodeLayerArgs& a, cudaStream_t st);
+
 bool decode_tc_supported(int H, int I, int T, const void* gu_blocks, const void* d_blocks, const void* gu_scales,
                          const void* d_scales);
 cudaError_t decode_tc_prepare();

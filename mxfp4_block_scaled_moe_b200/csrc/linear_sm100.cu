@@ -28,6 +28,7 @@
 #include "common.cuh"
 #include "launchers.h"
 #include "tc_common.cuh"
+#include "tmap.h"
 
 namespace mxmoe {
 namespace lin {
@@ -261,33 +262,12 @@ __global__ void __launch_bounds__(256) fp8_linear_reduce_kernel(const float* __r
 
 namespace {
 
-using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiled lin_encoder() {
-  static EncodeTiled fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiled>(ptr);
-  }
-  return fn;
-}
-
 // (rows, K) bytes, K-major, box (BK, box_rows), 128-byte swizzle, zero fill outside
 bool encode_rows(CUtensorMap* m, const void* base, int64_t rows, int64_t K, uint32_t box_rows) {
-  EncodeTiled fn = lin_encoder();
-  if (!fn) return false;
-  cuuint64_t d[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows > 0 ? rows : 1)};
-  cuuint64_t s[1] = {static_cast<cuuint64_t>(K)};
-  cuuint32_t b[2] = {static_cast<cuuint32_t>(lin::BK), box_rows};
-  cuuint32_t es[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), d, s, b, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(rows > 0 ? rows : 1)};
+  const uint64_t strides[1] = {static_cast<uint64_t>(K)};
+  const uint32_t box[2] = {static_cast<uint32_t>(lin::BK), box_rows};
+  return tmap_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box);
 }
 
 constexpr size_t kLinPartBudget = 64u << 20;   // bytes of split-K partials at most
@@ -341,6 +321,6 @@ cudaError_t launch_fp8_linear(const uint8_t* xq, int T, int K, const uint8_t* wq
   return cudaGetLastError();
 }
 
-bool fp8_linear_supported() { return lin_encoder() != nullptr; }
+bool fp8_linear_supported() { return tmap_available(); }
 
 }  // namespace mxmoe

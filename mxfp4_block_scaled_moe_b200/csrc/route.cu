@@ -389,31 +389,7 @@ __global__ void __launch_bounds__(kPermThreads) route_small_kernel(
   const int64_t wid = static_cast<int64_t>(blockIdx.x) * nwarps + warp;
   if (wid < static_cast<int64_t>(T) * E) {
     const int t = static_cast<int>(wid / E), e = static_cast<int>(wid % E);
-    const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(t) * H);
-    const uint4* wrow = reinterpret_cast<const uint4*>(wr + static_cast<int64_t>(e) * H);
-    float acc = 0.0f;
-    // four 16-byte chunks of each operand in flight per lane, then their FMAs in chunk
-    // order (the same order as one chunk at a time)
-    for (int c0 = lane; c0 < H / 8; c0 += 4 * 32) {
-      uint4 a[4], b[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int c = c0 + 32 * u;
-        if (c < H / 8) { a[u] = ld_nc_v4(xr + c); b[u] = ld_nc_v4(wrow + c); }
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        if (c0 + 32 * u >= H / 8) break;
-        const uint32_t av[4] = {a[u].x, a[u].y, a[u].z, a[u].w}, bv[4] = {b[u].x, b[u].y, b[u].z, b[u].w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          acc = fmaf(__uint_as_float(av[i] << 16), __uint_as_float(bv[i] << 16), acc);
-          acc = fmaf(__uint_as_float(av[i] & 0xFFFF0000u), __uint_as_float(bv[i] & 0xFFFF0000u), acc);
-        }
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    const float acc = router_logit_warp(x + static_cast<int64_t>(t) * H, wr + static_cast<int64_t>(e) * H, H);
     if (lane == 0) logits[wid] = br ? acc + bf16_bits_to_f32(br[e]) : acc;
   }
   // tokens whose logits this CTA helped compute: the last of a token's CTAs runs its top-k
