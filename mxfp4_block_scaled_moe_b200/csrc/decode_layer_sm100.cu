@@ -352,20 +352,20 @@ __device__ __forceinline__ void split_block(float v, uint8_t* row0, int64_t row_
 }
 
 // ------------------------------------------------------------- routing, per CTA ----
-// One warp: the routed experts in ascending id, each one's token mask, and each token's
-// experts in ascending id with their weights, from sc.tk_idx / sc.tk_w. g_idx / g_w
-// (nullable): the top-k written out as (T, k).
+// One warp: the routed experts in ascending id and each one's token mask, from
+// sc.tk_idx (the masks gather by shared-memory atomics in sc.a_of, which then takes the
+// experts' active indices). g_idx / g_w (nullable): the top-k written out as (T, k).
 __device__ __forceinline__ void build_sched(Sched& sc, int T, int E, int k, int* err, int32_t* g_idx, float* g_w) {
   const int lane = threadIdx.x & 31;
-  for (int e = lane; e < E; e += 32) sc.a_of[e] = -1;
-  for (int a = lane; a < kMaxActive; a += 32) sc.tmask[a] = 0u;
+  unsigned* mask_of = reinterpret_cast<unsigned*>(sc.a_of);
+  for (int e = lane; e < E; e += 32) mask_of[e] = 0u;
   __syncwarp();
   for (int q = lane; q < T * k; q += 32) {
-    const int t = q / k, j = q % k;
+    const int t = q / k, j = q - t * k;
     const int e = sc.tk_idx[t][j];
     if (e >= 0 && e < E) {
-      sc.a_of[e] = 0;   // routed; numbered below
-    } else if (err) {
+      atomicOr(&mask_of[e], 1u << t);
+    } else {
       set_device_error(err, MXMOE_EDEVICE);
     }
     if (g_idx) {
@@ -375,43 +375,44 @@ __device__ __forceinline__ void build_sched(Sched& sc, int T, int E, int k, int*
   }
   __syncwarp();
   int base = 0;
-  for (int e0 = 0; e0 < E; e0 += 32) {
-    const int e = e0 + lane;
-    const bool f = e < E && sc.a_of[e] == 0;
-    const unsigned bal = __ballot_sync(0xffffffffu, f);
-    if (f) {
+#pragma unroll
+  for (int i = 0; i < kMaxE / 32; ++i) {
+    if (32 * i >= E) break;
+    const int e = lane + 32 * i;
+    const unsigned tm = e < E ? mask_of[e] : 0u;
+    const unsigned bal = __ballot_sync(0xffffffffu, tm != 0u);
+    if (tm) {
       const int a = base + __popc(bal & ((1u << lane) - 1u));
       sc.a_of[e] = a;
       sc.act[a] = e;
+      sc.tmask[a] = tm;
     }
     base += __popc(bal);
   }
   if (lane == 0) sc.na = base;
   __syncwarp();
-  for (int q = lane; q < T * k; q += 32) {
-    const int t = q / k, e = sc.tk_idx[t][q % k];
-    if (e >= 0 && e < E) atomicOr(&sc.tmask[sc.a_of[e]], 1u << t);
-  }
-  if (lane < T) {
-    // the token's experts in ascending id (the combine's order); an id out of range,
-    // flagged above, stays in the list as expert slot 0 with weight 0
-    const int t = lane;
-    for (int j = 0; j < k; ++j) {
-      const int e = sc.tk_idx[t][j];
-      const bool valid = e >= 0 && e < E;
-      const int a = valid ? sc.a_of[e] : 0;
-      const float w = valid ? sc.tk_w[t][j] : 0.0f;
-      int i = j;
-      while (i > 0 && sc.cb_a[t][i - 1] > a) {
-        sc.cb_a[t][i] = sc.cb_a[t][i - 1];
-        sc.cb_w[t][i] = sc.cb_w[t][i - 1];
-        --i;
-      }
-      sc.cb_a[t][i] = a;
-      sc.cb_w[t][i] = w;
+}
+
+// Lanes t < T: token t's experts in ascending id with their weights (the output's order);
+// an id out of range (flagged by build_sched) stays in the list as expert slot 0 with
+// weight 0.
+__device__ __forceinline__ void build_token_lists(Sched& sc, int T, int E, int k) {
+  const int t = threadIdx.x & 31;
+  if (t >= T) return;
+  for (int j = 0; j < k; ++j) {
+    const int e = sc.tk_idx[t][j];
+    const bool valid = e >= 0 && e < E;
+    const int a = valid ? sc.a_of[e] : 0;
+    const float w = valid ? sc.tk_w[t][j] : 0.0f;
+    int i = j;
+    while (i > 0 && sc.cb_a[t][i - 1] > a) {
+      sc.cb_a[t][i] = sc.cb_a[t][i - 1];
+      sc.cb_w[t][i] = sc.cb_w[t][i - 1];
+      --i;
     }
+    sc.cb_a[t][i] = a;
+    sc.cb_w[t][i] = w;
   }
-  __syncwarp();
 }
 
 // ------------------------------------------------------------------ epilogue piece --
@@ -423,13 +424,6 @@ template <int kTp>
 __device__ __forceinline__ void epi_gate_up(const Params& p, const Sched& sc, const Phase& d, const Piece& pc,
                                             float (&g0)[kTp], float (&g1)[kTp], int q, int lane) {
   const int T = p.T;
-  const int e = sc.act[pc.a];
-  const int rr0 = pc.m * BM + 32 * q;   // the warp's first intermediate row
-  float bias0 = 0.0f, bias1 = 0.0f;
-  if (rr0 < p.I) {
-    bias0 = __ldg(p.gu_bias + static_cast<int64_t>(e) * 2 * p.I + rr0 + lane);
-    bias1 = __ldg(p.gu_bias + static_cast<int64_t>(e) * 2 * p.I + p.I + rr0 + lane);
-  }
   if (!pc.whole) {
     // park this piece's per-token values; the last piece adds the CTAs' values in CTA order
     const int64_t per = 2 * static_cast<int64_t>(T) * BM;
@@ -480,11 +474,15 @@ __device__ __forceinline__ void epi_gate_up(const Params& p, const Sched& sc, co
     }
     if (lane == 0) *tk = 0u;   // ready for the next call
   }
-  const unsigned mask = sc.tmask[pc.a];
+  const int rr0 = pc.m * BM + 32 * q;   // the warp's first intermediate row
+  const int nst_d = (p.I + 255) / 256;
   if (rr0 < p.I) {
+    const int e = sc.act[pc.a];
+    const float bias0 = __ldg(p.gu_bias + static_cast<int64_t>(e) * 2 * p.I + rr0 + lane);
+    const float bias1 = __ldg(p.gu_bias + static_cast<int64_t>(e) * 2 * p.I + p.I + rr0 + lane);
+    const unsigned mask = sc.tmask[pc.a];
     const int kb = rr0 / 32;   // the warp's block of the down contraction
     const int64_t row_stride = p.I / 2;
-    const int nst_d = (p.I + 255) / 256;
     uint8_t* rows = p.xs_mid + static_cast<int64_t>(pc.a) * p.npad * row_stride + 16 * kb;
     uint8_t* sf = p.sf_mid + (static_cast<int64_t>(pc.a) * nst_d + (kb >> 3)) * kSfSrc + ((kb >> 2) & 1) * 2048 +
                   (kb & 3);
@@ -504,7 +502,7 @@ __device__ __forceinline__ void epi_gate_up(const Params& p, const Sched& sc, co
   fence_proxy_async_global();
   __threadfence();
   __syncwarp();
-  if (lane == 0) atomicAdd(&p.done_gu[pc.a * ((p.I + 255) / 256) + (pc.m >> 1)], 1u);
+  if (lane == 0) atomicAdd(&p.done_gu[pc.a * nst_d + (pc.m >> 1)], 1u);
 }
 
 // The down side: every piece parks its per-token values of both row tiles (no bias),
@@ -527,41 +525,65 @@ __device__ __forceinline__ void epi_down(const Params& p, const Sched& sc, const
 
 // One (32-row slice, token) item of the output, by one warp (lane = row): the token's
 // experts in ascending id, each y = s * (the expert tile's pieces added in CTA order) +
-// bias, weighted and added. All of a token's expert pieces (kPc each) and biases are in
-// flight at once; every warp of the grid takes items, so this is one round trip.
+// bias, weighted and added. All of a token's expert pieces (kCombinePc each) and biases
+// are in flight at once, and every warp of the grid takes items.
+// Not inlined, and with plain arguments, so that its one copy of code serves the real
+// items and a dry run (dry: the same loads, no store) that every CTA makes early on: the
+// output runs once per call, right after the weights have streamed through the caches,
+// and its instructions would otherwise come from memory there, a few microseconds.
+struct ItemArgs {
+  const float* dpart;
+  const float* d_bias;
+  uint16_t* out;
+  int H, T, k, nm;
+  float s_in;
+};
 constexpr int kCombinePc = 6;
-__device__ __forceinline__ void combine_item(const Params& p, const Sched& sc, int nm, int s, int t, int lane) {
-  const int T = p.T, k = p.k;
+__device__ __noinline__ void combine_item(const ItemArgs x, const Sched* __restrict__ sc, int s, int t, bool dry) {
+  const int lane = threadIdx.x & 31;
   const int r = 32 * s + lane;
   const int m = s / 8, h = (s / 4) & 1;                 // tile pair, row tile within it
-  const int off = (h * T + t) * BM + 32 * (s & 3) + lane;
-  const float s_in = p.fp8 ? p.s1 : 1.0f;
+  const int off = (h * x.T + t) * BM + 32 * (s & 3) + lane;
+  const int per = 2 * x.T * BM;
   float v[kMaxK][kCombinePc], bd[kMaxK];
   int np[kMaxK];
   const float* src[kMaxK];
 #pragma unroll
   for (int j = 0; j < kMaxK; ++j) {
-    const bool on = j < k;
-    const int a = sc.cb_a[t][on ? j : 0];
-    const int tile = a * nm + m;
-    np[j] = on ? sc.dcn[tile] : 0;
-    src[j] = p.dpart + static_cast<int64_t>(sc.poff[tile]) * 2 * T * BM + off;
-    bd[j] = on ? __ldg(p.d_bias + static_cast<int64_t>(sc.act[a]) * p.H + r) : 0.0f;
+    const bool on = j < x.k;
+    const int a = sc->cb_a[t][on ? j : 0];
+    const int tile = a * x.nm + m;
+    np[j] = on ? sc->dcn[tile] : 0;
+    src[j] = x.dpart + static_cast<int64_t>(sc->poff[tile]) * per + off;
+    bd[j] = on ? __ldg(x.d_bias + static_cast<int64_t>(sc->act[a]) * x.H + r) : 0.0f;
 #pragma unroll
-    for (int i = 0; i < kCombinePc; ++i) v[j][i] = i < np[j] ? __ldcg(src[j] + i * 2 * T * BM) : 0.0f;
+    for (int i = 0; i < kCombinePc; ++i) v[j][i] = i < np[j] ? __ldcg(src[j] + i * per) : 0.0f;
   }
   float acc = 0.0f;
 #pragma unroll
   for (int j = 0; j < kMaxK; ++j) {
-    if (j >= k) break;
+    if (j >= x.k) break;
     float y = 0.0f;
 #pragma unroll
     for (int i = 0; i < kCombinePc; ++i)
       if (i < np[j]) y += v[j][i];
-    for (int i = kCombinePc; i < np[j]; ++i) y += __ldcg(src[j] + i * 2 * T * BM);   // a tile in more pieces
-    acc = __fadd_rn(acc, __fmul_rn(sc.cb_w[t][j], __fadd_rn(__fmul_rn(s_in, y), bd[j])));
+    for (int i = kCombinePc; i < np[j]; ++i) y += __ldcg(src[j] + i * per);   // a tile in more pieces
+    acc = __fadd_rn(acc, __fmul_rn(sc->cb_w[t][j], __fadd_rn(__fmul_rn(x.s_in, y), bd[j])));
   }
-  p.out[static_cast<int64_t>(t) * p.H + r] = f32_to_bf16_bits_rn(acc);
+  if (!dry) x.out[static_cast<int64_t>(t) * x.H + r] = f32_to_bf16_bits_rn(acc);
+}
+
+__device__ __forceinline__ ItemArgs item_args(const Params& p, int nm) {
+  ItemArgs x;
+  x.dpart = p.dpart;
+  x.d_bias = p.d_bias;
+  x.out = p.out;
+  x.H = p.H;
+  x.T = p.T;
+  x.k = p.k;
+  x.nm = nm;
+  x.s_in = p.fp8 ? p.s1 : 1.0f;
+  return x;
 }
 
 // ---------------------------------------------------------------------- the kernel --
@@ -577,9 +599,10 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap map_gu, const __grid_con
   uint64_t* empty = full + kStages;
   uint64_t* acc_full = empty + kStages;
   uint64_t* acc_empty = acc_full + 2;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(acc_empty + 2);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_empty + 2) + 1;
-  volatile unsigned* last_out = reinterpret_cast<volatile unsigned*>(acc_empty + 2) + 2;
+  uint64_t* down_ready = acc_empty + 2;         // down's work list and the output's tables are built
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(down_ready + 1);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(down_ready + 1) + 1;
+  volatile unsigned* last_out = reinterpret_cast<volatile unsigned*>(down_ready + 1) + 2;
   uint8_t* ring = smem + kRingOffset;
   auto sA = [&](int s, int h) { return ring + s * kStageBytes + h * (BM * kRowBytes); };
   auto sB = [&](int s) { return ring + s * kStageBytes + kOffB; };
@@ -603,6 +626,7 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap map_gu, const __grid_con
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], kEpiWarps);
     }
+    mbar_init(down_ready, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
@@ -653,12 +677,11 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap map_gu, const __grid_con
     if (warp == 0) {
       build_sched(sc, T, E, k, p.err, blockIdx.x == 0 ? p.topk_idx : nullptr, blockIdx.x == 0 ? p.topk_w : nullptr);
       __syncwarp();
-#pragma unroll 1
-      for (int ph = 0; ph < 2; ++ph) {
-        const Phase d = phase_of(p, sc.na, ph);
-        if (lane == 0) sc.phs[ph] = d;
-        build_pieces(sc, d, ph, p.err);
-      }
+      // gate_up's work list now; down's, the token lists and the output's tables are the
+      // epilogue warps' first job (they wait for the first accumulator anyway)
+      const Phase d = phase_of(p, sc.na, 0);
+      if (lane == 0) sc.phs[0] = d;
+      build_pieces(sc, d, 0, p.err);
     }
   }
   tc_fence_before();
@@ -681,6 +704,7 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap map_gu, const __grid_con
       uint32_t phase = 0;
       bool ok = true;
       for (int ph = 0; ph < 2 && ok; ++ph) {
+        if (ph == 1 && !mbar_wait(down_ready, 0, abort_flag, p.err)) { ok = false; break; }
         for (int ip = 0; ok && ip < sc.npc[ph]; ++ip) {
           const Piece pc = piece_at(sc, ph, ip);
           const int e = sc.act[pc.a];
@@ -707,6 +731,7 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap map_gu, const __grid_con
       bool ok = true;
       const uint32_t tx = static_cast<uint32_t>(npad * kRowBytes + kSfSrc);
       for (int ph = 0; ph < 2 && ok; ++ph) {
+        if (ph == 1 && !mbar_wait(down_ready, 0, abort_flag, p.err)) { ok = false; break; }
         for (int ip = 0; ok && ip < sc.npc[ph]; ++ip) {
           const Piece pc = piece_at(sc, ph, ip);
           for (int kst = pc.k0; kst < pc.k1; ++kst) {
@@ -740,6 +765,7 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap map_gu, const __grid_con
     bool ok = true;
     const uint32_t id0 = idesc_mxf4(BM, npad);
     for (int ph = 0; ph < 2 && ok; ++ph) {
+      if (ph == 1 && !mbar_wait(down_ready, 0, abort_flag, p.err)) { ok = false; break; }
       const Phase& d = sc.phs[ph];
       for (int ip = 0; ok && ip < sc.npc[ph]; ++ip) {
         const Piece pc = piece_at(sc, ph, ip);
@@ -791,6 +817,7 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap map_gu, const __grid_con
     uint32_t phase = 0;
     bool ok = true;
     for (int ph = 0; ph < 2 && ok; ++ph) {
+      if (ph == 1 && !mbar_wait(down_ready, 0, abort_flag, p.err)) { ok = false; break; }
       const Phase& d = sc.phs[ph];
       const int nb = d.K / 32;
       for (int ip = 0; ok && ip < sc.npc[ph]; ++ip) {
@@ -848,8 +875,16 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap map_gu, const __grid_con
     {
       // the down pieces' layout for the combine (needed only after gate_up; the four
       // epilogue warps work it out while the first weights load)
-      const Phase& dd = sc.phs[1];
       const int et = static_cast<int>(threadIdx.x) - 4 * 32;
+      if (et < 32) {
+        const Phase d1 = phase_of(p, na, 1);
+        if (et == 0) sc.phs[1] = d1;
+        build_pieces(sc, d1, 1, p.err);
+      } else if (et < 64) {
+        build_token_lists(sc, T, E, k);
+      }
+      asm volatile("bar.sync 1, 128;\n" ::: "memory");
+      const Phase& dd = sc.phs[1];
       const int nt = na * dd.nm;
       for (int i = et; i < nt; i += 4 * 32) {
         const unsigned s0 = static_cast<unsigned>(i * dd.nst);
@@ -888,6 +923,8 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap map_gu, const __grid_con
         }
       }
       asm volatile("bar.sync 1, 128;\n" ::: "memory");
+      if (et == 0) mbar_arrive(down_ready);
+      if (et < 32) combine_item(item_args(p, dd.nm), &sc, 0, 0, true);   // the output's code, early
     }
     uint32_t use[2] = {0u, 0u};
     int slot = 0;
@@ -956,8 +993,9 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap map_gu, const __grid_con
     __syncthreads();
     if (!*abort_flag) {
       const int items = p.H / 32 * T;
-      for (int it = blockIdx.x * kWarps + warp; it < items; it += G * kWarps)
-        combine_item(p, sc, sc.phs[1].nm, it / T, it % T, lane);
+      // items one per CTA before any CTA takes a second
+      const ItemArgs xa = item_args(p, sc.phs[1].nm);
+      for (int it = warp * G + blockIdx.x; it < items; it += G * kWarps) combine_item(xa, &sc, it / T, it % T, false);
     }
   }
 
