@@ -6,8 +6,10 @@
 // once per layer.
 //
 // Operands of one expert e (or one group of at most 56 of its routed rows):
-//   A = 128 weight rows (gate_up: 128 gate rows and, in a second MMA, the 128 matching up
-//       rows; down: 128 rows of down_proj) with the checkpoint's e8m0 scales;
+//   A = two 128-row weight tiles per stage, each its own MMA and accumulator (gate_up: 128
+//       gate rows and the 128 matching up rows; down: 256 consecutive rows of down_proj),
+//       with the checkpoint's e8m0 scales; both share the stage's B tile, so a stage moves
+//       32 KB of weights for one B load and one set of B-scale copies;
 //   B = the routed token rows as four MXFP4 "parts" each: p1 = e2m1(x / 2^s1), p2 the same
 //       on the residual x - p1, and so on, each s chosen from the largest residual of its
 //       32-value block so that nothing saturates. Every part removes about three bits of
@@ -116,7 +118,8 @@ struct Params {
   const int32_t* inv;
   int T, k;
   // split-K
-  float* part;               // [split][kA][P * 4][n_out] fp32 partial accumulators
+  float* part;               // [split][planes][P * 4][n_out] fp32 partial accumulators
+                             // (gate_up: planes gate and up; down: one, rows as they are)
   unsigned* split_tickets;   // [kMaxGrp][n_m][4], zero between calls
   unsigned* comb_tickets;    // [n_m][4], zero between calls
   int* err;
@@ -195,8 +198,8 @@ __device__ __forceinline__ void read_tmem8(uint32_t tg, uint32_t tu, int j0, flo
 }
 
 // Address of the fp32 partial of (split s, accumulator h, global column c, row).
-__device__ __forceinline__ float* part_at(const Params& p, int kA, int s, int h, int64_t c, int row) {
-  return p.part + ((static_cast<int64_t>(s) * kA + h) * (p.P * kParts) + c) * p.n_out + row;
+__device__ __forceinline__ float* part_at(const Params& p, int planes, int s, int h, int64_t c, int row) {
+  return p.part + ((static_cast<int64_t>(s) * planes + h) * (p.P * kParts) + c) * p.n_out + row;
 }
 
 // Sum a row's kParts part columns (in part order) for the 8 rows of a group.
@@ -322,7 +325,9 @@ __device__ __forceinline__ void combine_slice(const Params& p, int row) {
 template <bool kGateUp>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x, Params p) {
-  constexpr int kA = kGateUp ? 2 : 1;   // A tiles (accumulators) per unit
+  constexpr int kA = 2;                       // A tiles (accumulators) per unit
+  constexpr int kPlanes = kGateUp ? 2 : 1;    // planes of the split-K partials
+  constexpr int kUnitRows = kGateUp ? BM : 2 * BM;   // output rows a unit covers
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Sched& sc = *reinterpret_cast<Sched*>(smem);
@@ -455,7 +460,8 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
         for (int kst = w.k0; kst < w.k1; ++kst) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[stage], tx);
-          tma_load_3d(sA(stage, 0), &map_w, &full[stage], kRowBytes * kst, w.m * BM, kA * w.e);
+          // gate_up: rows m*128.. of gate (matrix 2e) and up (2e+1); down: rows m*256 .. +255
+          tma_load_3d(sA(stage, 0), &map_w, &full[stage], kRowBytes * kst, w.m * kUnitRows, kGateUp ? 2 * w.e : w.e);
           if (!dep_ready) {
             // the token operand and its scales are the previous kernel's output: everything
             // before this point (setup, the first weight stage, the scale converters' start)
@@ -480,7 +486,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
     bool ok = true;
     for (int u = blockIdx.x; u < sc.units && ok; u += gridDim.x) {
       const Unit w = unit_at(sc, p, u);
-      const bool big = kGateUp && w.ncols > kBigCols;
+      const bool big = w.ncols > kBigCols;
       const int slot = big ? 0 : nxt;
       if (big) {
         ok = mbar_wait(&acc_empty[0], (use0 & 1u) ^ 1u, abort_flag, p.err) &&
@@ -546,7 +552,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
     }
   } else if (warp == 2 || warp == 3) {
     // ------------------------------------------------ A (weight) scale converters -----
-    const int h = warp - 2;   // 0: gate / down rows, 1: up rows
+    const int h = warp - 2;   // gate_up: 0 gate rows, 1 up rows; down: the unit's first / second 128 rows
     if (h < kA) {
       // lane l owns rows l, l+32, l+64, l+96 of the tile; a stage's 8 scale bytes of a row
       // are four aligned 16-bit words (nb is even). They are loaded kRing stages ahead
@@ -567,9 +573,11 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
       int lu = blockIdx.x, lk = 0, lk1 = 0;   // load cursor: unit, stage, end stage
       auto start_unit = [&](int u) {
         const Unit w = unit_at(sc, p, u);
-        const int valid = min(BM, p.rows_per_group - w.m * BM);
+        const int row0 = w.m * kUnitRows + (kGateUp ? 0 : h * BM);
+        const int valid = max(0, min(BM, p.rows_per_group - row0));
         const int group = kGateUp ? 2 * w.e + h : w.e;
-        const uint8_t* blk = p.w_scales + (static_cast<int64_t>(group) * p.rows_per_group + w.m * BM) * p.nb;
+        // a tile wholly past the last row (down's last pair) reads the group's first row, masked
+        const uint8_t* blk = p.w_scales + (static_cast<int64_t>(group) * p.rows_per_group + (valid > 0 ? row0 : 0)) * p.nb;
         rows_ok = 0u;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -658,13 +666,18 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
     int nxt = 0;
     for (int u = blockIdx.x; u < sc.units; u += gridDim.x) {
       const Unit w = unit_at(sc, p, u);
-      const bool big = kGateUp && w.ncols > kBigCols;
+      const bool big = w.ncols > kBigCols;
       const int slot = big ? 0 : nxt;
+      // this warp's rows: gate_up one row of both accumulators (gate, up); down row0 of the
+      // first accumulator and row1 = row0 + 128 of the second
+      const int row0 = w.m * kUnitRows + 32 * q + lane;
+      const int row1 = kGateUp ? row0 : row0 + BM;
+      const bool live0 = (w.m * kUnitRows + 32 * q) < p.n_out;   // n_out % 64 == 0: whole warps
+      const bool live1 = kGateUp ? live0 : (w.m * kUnitRows + BM + 32 * q) < p.n_out;
       // this warp's biases, loaded before the wait so that their latency overlaps the MMAs
-      const int brow = min(w.m * BM + 32 * q + lane, p.n_out - 1);
       const float* bias_e = p.bias + static_cast<int64_t>(w.e) * p.rows_total;
-      const float bias0 = __ldg(bias_e + brow);
-      const float bias1 = kGateUp ? __ldg(bias_e + p.n_out + brow) : 0.0f;
+      const float bias0 = __ldg(bias_e + min(row0, p.n_out - 1));
+      const float bias1 = __ldg(bias_e + (kGateUp ? p.n_out : 0) + min(row1, p.n_out - 1));
       bool ok = mbar_wait(&acc_full[slot], (slot ? use1 : use0) & 1u, abort_flag, p.err);
       if (ok && big) ok = mbar_wait(&acc_full[1], use1 & 1u, abort_flag, p.err);
       if (!ok) break;
@@ -673,20 +686,21 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
       const uint32_t tg = lane_base + (big ? 0u : static_cast<uint32_t>(slot * kSlot1));
       const uint32_t tu = lane_base + (big ? static_cast<uint32_t>(kSlot1)
                                            : static_cast<uint32_t>(slot * kSlot1 + w.ncols));
-      const int row = w.m * BM + 32 * q + lane;
-      const bool live = (w.m * BM + 32 * q) < p.n_out;   // n_out % 64 == 0: whole warps
+      const bool live = live0 || live1;
       const bool split = sc.nsplit > 1;
       const int64_t col0 = static_cast<int64_t>(w.off) * kParts;
+      // the partial of accumulator h: gate_up plane h at the shared row, down plane 0 at its own row
+      const int ph1 = kGateUp ? 1 : 0;
       if (live && split) {
         // this split's partials
         for (int j0 = 0; j0 < w.n; j0 += 8) {
           float vg[8 * kParts], vu[8 * kParts];
-          read_tmem8<kGateUp>(tg, tu, j0, vg, vu);
+          read_tmem8<true>(tg, tu, j0, vg, vu);
 #pragma unroll
           for (int f = 0; f < 8 * kParts; ++f) {
             if (j0 + f / kParts < w.n) {
-              *part_at(p, kA, w.s, 0, col0 + kParts * j0 + f, row) = vg[f];
-              if (kGateUp) *part_at(p, kA, w.s, 1, col0 + kParts * j0 + f, row) = vu[f];
+              if (live0) *part_at(p, kPlanes, w.s, 0, col0 + kParts * j0 + f, row0) = vg[f];
+              if (live1) *part_at(p, kPlanes, w.s, ph1, col0 + kParts * j0 + f, row1) = vu[f];
             }
           }
         }
@@ -707,7 +721,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
         for (int j0 = 0; j0 < w.n; j0 += 8) {
           float vg[8 * kParts], vu[8 * kParts];
           if (!split) {
-            read_tmem8<kGateUp>(tg, tu, j0, vg, vu);
+            read_tmem8<true>(tg, tu, j0, vg, vu);
           } else {
 #pragma unroll
             for (int f = 0; f < 8 * kParts; ++f) { vg[f] = 0.0f; vu[f] = 0.0f; }
@@ -715,20 +729,21 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
 #pragma unroll
               for (int f = 0; f < 8 * kParts; ++f) {
                 if (j0 + f / kParts < w.n) {
-                  vg[f] += __ldcg(part_at(p, kA, s, 0, col0 + kParts * j0 + f, row));
-                  if (kGateUp) vu[f] += __ldcg(part_at(p, kA, s, 1, col0 + kParts * j0 + f, row));
+                  if (live0) vg[f] += __ldcg(part_at(p, kPlanes, s, 0, col0 + kParts * j0 + f, row0));
+                  if (live1) vu[f] += __ldcg(part_at(p, kPlanes, s, ph1, col0 + kParts * j0 + f, row1));
                 }
               }
             }
           }
           float gs[8], us[8];
           sum_parts(vg, gs);
+          sum_parts(vu, us);
           if (kGateUp) {
-            sum_parts(vu, us);
             finish_gate_up(p.xs_out, p.sfb_out, epi_stage, p.n_out, p.nst_out, p.max_chunks, p.s_in, p.s_out, w.e, w.c, w.off,
-                           w.n, j0, gs, us, bias0, bias1, row, lane, false);
+                           w.n, j0, gs, us, bias0, bias1, row0, lane, false);
           } else {
-            finish_down(p, w, j0, gs, bias0, row);
+            if (live0) finish_down(p, w, j0, gs, bias0, row0);
+            if (live1) finish_down(p, w, j0, us, bias1, row1);
           }
         }
         if (split && lane == 0) *stk = 0u;   // ready for the next call
@@ -758,7 +773,8 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
         t = __shfl_sync(0xffffffffu, t, 0);
         if (t == static_cast<unsigned>(sc.n_grp - 1)) {
           __threadfence();
-          combine_slice(p, row);
+          if (live0) combine_slice(p, row0);
+          if (live1) combine_slice(p, row1);
           if (lane == 0) *tk = 0u;
         }
       }
@@ -959,12 +975,12 @@ cudaError_t launch_split_tokens(bool fp8, const uint16_t* x, const int32_t* topk
 // combine of a few tokens.
 cudaError_t launch_decode_gemm(bool gate_up, const DecodeGemmArgs& a, cudaStream_t st) {
   using namespace dec;
-  const int kA = gate_up ? 2 : 1;
   const int K = gate_up ? a.H : a.I;
   const int n_out = gate_up ? a.I : a.H;
   const int groups = gate_up ? 2 * a.E : a.E;
   const int64_t b_rows = a.P * kParts;
-  const int n_m = (n_out + BM - 1) / BM;
+  const int unit_rows = gate_up ? BM : 2 * BM;   // output rows per unit (down: two 128-row tiles)
+  const int n_m = (n_out + unit_rows - 1) / unit_rows;
   const int box_rows = box_rows_for(a.T);
   if (a.E > kMaxE || a.k > kMaxTopK || a.T > kDecodeMaxT || (!gate_up && a.out && a.T > kDecodeFoldMaxT))
     return cudaErrorInvalidValue;
@@ -973,7 +989,9 @@ cudaError_t launch_decode_gemm(bool gate_up, const DecodeGemmArgs& a, cudaStream
     const uint64_t row_bytes = static_cast<uint64_t>(K) / 2;
     const uint64_t dims[3] = {row_bytes, static_cast<uint64_t>(n_out), static_cast<uint64_t>(groups)};
     const uint64_t strides[2] = {row_bytes, row_bytes * n_out};
-    const uint32_t box[3] = {static_cast<uint32_t>(kRowBytes), BM, static_cast<uint32_t>(kA)};
+    // gate_up: 128 rows of gate (matrix 2e) and of up (2e+1); down: 256 rows of matrix e
+    const uint32_t box[3] = {static_cast<uint32_t>(kRowBytes), static_cast<uint32_t>(gate_up ? BM : 2 * BM),
+                             gate_up ? 2u : 1u};
     if (!tmap_encode(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, gate_up ? a.gu_blocks : a.d_blocks, dims, strides, box)) return cudaErrorInvalidValue;
   }
   {
@@ -994,7 +1012,7 @@ cudaError_t launch_decode_gemm(bool gate_up, const DecodeGemmArgs& a, cudaStream
   prm.nst = nst_for(K);
   prm.n_m = n_m;
   prm.box_rows = box_rows;
-  prm.split_cap = split_cap(kA, a.P, n_out);
+  prm.split_cap = split_cap(gate_up ? 2 : 1, a.P, n_out);
   prm.max_chunks = max_chunks_for(a.T);
   prm.smem_bytes = kSmemBytes;
   prm.P = a.P;

@@ -218,10 +218,12 @@ def test_prefill_120b_shape_bf16_every_expert_tile(B):
     check_rows(B, p, d, rows, out=out1)
 
 
-@pytest.mark.parametrize("T,fp8", [(400, True), (400, False), (8, False), (8, True)])
+@pytest.mark.parametrize("T,fp8", [(400, True), (400, False), (8, False), (8, True), (24, False), (24, True)])
 def test_tensor_core_paths_with_H_ne_I(B, T, fp8):
     """H = 320 (2.5 k-tiles of 128), I = 192 (1.5): 1600 routed pairs take the tcgen05
-    prefill GEMMs (FP8, or bf16 as two e4m3 parts), T = 8 the tensor-core decode GEMMs."""
+    prefill GEMMs (FP8, or bf16 as two e4m3 parts), T = 8 the one-launch decode layer,
+    T = 24 the tensor-core decode GEMMs (down's second 256-row unit holds 64 live rows in
+    its first tile and none in its second)."""
     lay = inputs.small_layer(E=8, k=4, T=T, H=320, I=192, seed=13, router_bias=True,
                              router_std=1.0 / np.sqrt(320))
     p = pack(lay)
@@ -370,11 +372,12 @@ def _wide_scale_pack(lay: inputs.Layer, mode: str) -> Packed:
 
 @pytest.mark.parametrize("mode", ["tiny", "huge"])
 @pytest.mark.parametrize("T,k,H,fp8", [(600, 2, 512, True), (600, 2, 512, False), (8, 4, 512, False),
-                                       (8, 4, 512, True), (100, 2, 480, False)])
+                                       (8, 4, 512, True), (24, 4, 512, False), (100, 2, 480, False)])
 def test_wide_e8m0_weight_scales(B, mode, T, k, H, fp8):
     """Weights whose e8m0 scale bytes span the format: blocks at bytes 0-3 beside ordinary
     ones near 120, or a few blocks at 136-140, on every path: the tcgen05 prefill GEMMs
-    (T = 600, FP8 and bf16 as two parts), the tensor-core decode GEMMs (T = 8) and the
+    (T = 600, FP8 and bf16 as two parts), the one-launch decode layer (T = 8), the
+    tensor-core decode GEMMs (T = 24) and the
     register-dequant kernels (H = I = 480, not a multiple of 64, which neither tensor-core
     path takes)."""
     lay = inputs.small_layer(E=8, k=k, T=T, H=H, I=H, seed=21, router_bias=True,
