@@ -40,9 +40,16 @@
 // memory it is three xor-shuffles); the down epilogue writes y and, for a few tokens, the
 // weighted combine of each 32-row slice, by the last of the slice's row groups to finish.
 //
-// Scale-factor records of the B operand ("SFB"): for row group g and 128-wide k-tile kt,
-// 1024 bytes = two 512-byte tcgen05.cp atoms (B rows 0..127, 128..255), row r at byte
-// 512*(r/128) + 16*(r%32) + 4*((r/32)%4) + j for the tile's k-block j.
+// Scale-factor records of the B operand ("SFB"), one of 5 KB per (row group, 256-deep
+// stage). Tensor memory holds a 128-wide k-tile's scales of B rows 0..127 in four columns
+// (column i, lane 32q + l: the four k-block scales of row 32i + l, the same for the four
+// 32-lane quarters q). The first 4 KB are the tcgen05.cp.128x256b source of the stage's
+// two k-tiles for rows 0..127 (k-tile kt's 16 bytes of lane L at 2048 kt + 16 L): one
+// copy per stage for B tiles of at most 128 rows. Wider tiles (up to 224 rows) take the
+// four 32x128b.warpx4 atoms instead: rows 0..127 of k-tile kt from the first 512 bytes of
+// its 2 KB, rows 128..255 from the 512 bytes at 4096 + 512 kt. Row r < 128, k-block j of
+// k-tile kt: bytes 2048 kt + 512 q + 16 (r % 32) + 4 (r / 32) + j for q = 0..3; row
+// r >= 128: byte 4096 + 512 kt + 16 (r % 32) + 4 ((r - 128) / 32) + j.
 #include <climits>
 
 #include <cuda.h>
@@ -72,12 +79,14 @@ constexpr int kTmemCols = 512;
 constexpr int kSlot1 = 240;        // accumulator slot 1 starts here (slot 0 at column 0)
 constexpr int kBigCols = 112;      // gate_up units wider than this take both slots
 constexpr int kSfaCol = 480;       // A scales: tile h, atom a at 480 + 8h + 4a
-constexpr int kSfbCol = 496;       // B scales: k-tile t, atom b at 496 + 8t + 4b
-constexpr int kSfRecord = 1024;    // B scale record per (row group, 128-wide k-tile)
+constexpr int kSfbCol = 496;       // B scales: tiles <= 128 rows: k-tile t at 496 + 4t;
+                                   // wider: k-tile t, atom b at 496 + 8t + 4b
+constexpr int kSfRecord = 5120;    // B scale record per (row group, 256-deep stage)
+constexpr int kSfNarrow = 4096;    // its part that B tiles of at most 128 rows use
 // Per stage: the A (weight) scales of each tile as one 128x256b tcgen05.cp source (4 KB:
-// the two 128-wide k-tiles' atoms, repeated for the four 32-lane quarters), then the two
-// 1 KB B scale records of the stage's k-tiles.
-__host__ __device__ constexpr int sf_stage_bytes(int kA) { return kA * 4096 + 2 * 1024; }
+// the two 128-wide k-tiles' atoms, repeated for the four 32-lane quarters), then the
+// stage's B scale record.
+__host__ __device__ constexpr int sf_stage_bytes(int kA) { return kA * 4096 + kSfRecord; }
 constexpr int kSfStageMax = sf_stage_bytes(2);
 constexpr int kMaxE = 256;
 constexpr int kMaxGrp = kDecodeMaxGroups;
@@ -85,8 +94,16 @@ constexpr int kMaxSplit = 8;
 constexpr int kMaxTopK = 8;
 constexpr int kSmemBytes = 227 * 1024;
 
-__host__ __device__ __forceinline__ int sf_atom_byte(int r, int j) {   // r < 256
-  return (r >> 7) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + j;
+// Store the e8m0 byte v of B row r (< 256), k-block j of k-tile ktl (0 or 1) of a stage
+// into the stage's record (every copy of it: four for rows below 128).
+__device__ __forceinline__ void sfb_store(uint8_t* rec, int r, int ktl, int j, uint8_t v) {
+  if (r < 128) {
+    uint8_t* b = rec + 2048 * ktl + 16 * (r & 31) + 4 * (r >> 5) + j;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) b[512 * q] = v;
+  } else {
+    rec[4096 + 512 * ktl + 16 * (r & 31) + 4 * ((r - 128) >> 5) + j] = v;
+  }
 }
 
 struct Params {
@@ -103,7 +120,7 @@ struct Params {
   const int32_t* offsets;
   const int32_t* active;
   const int32_t* n_active;
-  const uint8_t* sfb;        // B scale records [E][max_chunks][2*nst][1024]
+  const uint8_t* sfb;        // B scale records [E][max_chunks][nst][kSfRecord]
   float s_in;                // per-tensor scale of the B operand (FP8) or 1
   // gate_up outputs (the down GEMM's B operand)
   uint8_t* xs_out;           // (P * 4, I / 2) packed e2m1 parts
@@ -233,7 +250,7 @@ __device__ __noinline__ void finish_gate_up(uint8_t* xs_out, uint8_t* sfb_out, f
                                             int row, int lane, bool dry) {
   const int kb = row >> 5;   // the warp's 32 rows: one 32-value block of the down contraction
   const int nv = min(8, n - j0);
-  uint8_t* rec = sfb_out + ((static_cast<int64_t>(e) * max_chunks + c) * 2 * nst_out + (kb >> 2)) * kSfRecord;
+  uint8_t* rec = sfb_out + ((static_cast<int64_t>(e) * max_chunks + c) * nst_out + (kb >> 3)) * kSfRecord;
   const int64_t row_bytes = n_out / 2;
   float a[8];
 #pragma unroll
@@ -274,7 +291,7 @@ __device__ __noinline__ void finish_gate_up(uint8_t* xs_out, uint8_t* sfb_out, f
       v[3] -= __half2float(__half(__half_raw{h1.y})) * up;
       if (mine) {
         *reinterpret_cast<uint16_t*>(dst + pp * row_bytes) = static_cast<uint16_t>(b0 | (b1 << 8));
-        if (sub == 0) rec[sf_atom_byte(kParts * (j0 + p0 + j) + pp, kb & 3)] = static_cast<uint8_t>(sc + 127);
+        if (sub == 0) sfb_store(rec, kParts * (j0 + p0 + j) + pp, (kb >> 2) & 1, kb & 3, static_cast<uint8_t>(sc + 127));
       }
     }
   }
@@ -453,10 +470,10 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
       bool dep_ready = false;
       for (int u = blockIdx.x; u < sc.units && ok; u += gridDim.x) {
         const Unit w = unit_at(sc, p, u);
-        // B scales: one record per 128-wide k-tile, two per stage
-        const uint32_t sfb_bytes = 2 * kSfRecord;
+        // B scales: the stage's record (its first 4 KB for B tiles of at most 128 rows)
+        const uint32_t sfb_bytes = w.ncols > 128 ? kSfRecord : kSfNarrow;
         const uint32_t tx = kA * BM * kRowBytes + w.nbox * p.box_rows * kRowBytes + sfb_bytes;
-        const uint8_t* rec = p.sfb + (static_cast<int64_t>(w.e) * p.max_chunks + w.c) * 2 * p.nst * kSfRecord;
+        const uint8_t* rec = p.sfb + (static_cast<int64_t>(w.e) * p.max_chunks + w.c) * p.nst * kSfRecord;
         for (int kst = w.k0; kst < w.k1; ++kst) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[stage], tx);
@@ -472,7 +489,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
           for (int b = 0; b < w.nbox; ++b)
             tma_load_2d(sB(stage) + b * p.box_rows * kRowBytes, &map_x, &full[stage], kRowBytes * kst,
                         kParts * w.off + b * p.box_rows);
-          bulk_g2s(sSFB(stage), rec + 2 * kst * kSfRecord, sfb_bytes, &full[stage]);
+          bulk_g2s(sSFB(stage), rec + static_cast<int64_t>(kst) * kSfRecord, sfb_bytes, &full[stage]);
           if (++stage == S) { stage = 0; phase ^= 1; }
         }
       }
@@ -499,7 +516,8 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
       const uint32_t dg = big ? 0u : static_cast<uint32_t>(slot * kSlot1);
       const uint32_t du = big ? static_cast<uint32_t>(kSlot1) : dg + static_cast<uint32_t>(w.ncols);
       const uint32_t id0 = idesc_mxf4(BM, w.ncols);
-      const int nat = w.ncols > 128 ? 2 : 1;   // B scale atoms per k-tile
+      const bool wide = w.ncols > 128;   // B rows past 128: per-k-tile atoms, 8 columns a k-tile
+      const int sfb_step = wide ? 8 : 4;  // tensor-memory columns of B scales per k-tile
       for (int kst = w.k0; kst < w.k1; ++kst) {
         if (!mbar_wait(&full[stage], phase, abort_flag, p.err)) { ok = false; break; }
         tc_fence_after();
@@ -511,10 +529,15 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
 #pragma unroll
           for (int h = 0; h < kA; ++h)
             tc_cp_128x256b(tmem + kSfaCol + 8 * h, smem_desc(smem_u32(sSFA(stage, h)), 2048, 128, 0));
-          for (int t = 0; t < nkt; ++t)
-            for (int b = 0; b < nat; ++b)
-              tc_cp_32x128b_x4(tmem + kSfbCol + 8 * t + 4 * b,
-                               smem_desc(smem_u32(sSFB(stage) + kSfRecord * t + 512 * b), 0, 128, 0));
+          if (!wide) {
+            tc_cp_128x256b(tmem + kSfbCol, smem_desc(smem_u32(sSFB(stage)), 2048, 128, 0));
+          } else {
+            for (int t = 0; t < nkt; ++t) {
+              tc_cp_32x128b_x4(tmem + kSfbCol + 8 * t, smem_desc(smem_u32(sSFB(stage) + 2048 * t), 0, 128, 0));
+              tc_cp_32x128b_x4(tmem + kSfbCol + 8 * t + 4,
+                               smem_desc(smem_u32(sSFB(stage) + 4096 + 512 * t), 0, 128, 0));
+            }
+          }
           const uint32_t b0 = smem_u32(sB(stage));
           for (int sk = 0; sk < nks; ++sk) {
             const int t = sk >> 1;
@@ -527,7 +550,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
             for (int h = 0; h < kA; ++h) {
               const uint64_t ad = smem_desc(smem_u32(sA(stage, h)) + 32 * sk, 16, 1024, 2);
               tc_mma_mxf4(tmem + (h ? du : dg), ad, bd, id, (tmem + kSfaCol + 8 * h + 4 * t) | sel,
-                          (tmem + kSfbCol + 8 * t) | sel, acc);
+                          (tmem + kSfbCol + sfb_step * t) | sel, acc);
             }
           }
           tc_commit(&empty[stage]);
@@ -800,8 +823,8 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
 // as four e2m1 parts, each 32-value block with its own e8m0 scale per part (the smallest
 // s with the block's largest residual / 2^s <= 6), written to each of the token's k
 // routed rows in expert-grouped order (its position inv[t*k + j]). Scale records: per
-// (expert, row group, 128-wide k-tile) one 1 KB record as the down GEMM's B operand has
-// them, row r at sf_atom_byte(r, k-block within the k-tile). The row's loads are issued
+// (expert, row group, 256-deep stage) one record as the down GEMM's B operand has them
+// (sfb_store). The row's loads are issued
 // first (they depend on nothing), the routing lookups beside them; each thread holds 16
 // consecutive values (half a block: a block's maximum is one shuffle with the
 // neighbouring lane), so a part leaves as one 8-byte store per routed row.
@@ -839,7 +862,7 @@ __global__ void __launch_bounds__(kSplitThreads) split_tokens_kernel(
     long long rec = -1;
     if (e >= 0 && e < E && pos >= 0 && pos < P) {   // else the permutation has flagged it
       const int je = pos - offsets[e];   // row within the expert
-      rec = (static_cast<long long>(e) * max_chunks + je / kGroupRows) * 2 * nst * kSfRecord;
+      rec = (static_cast<long long>(e) * max_chunks + je / kGroupRows) * nst * kSfRecord;
       jr = je % kGroupRows;
       ps = pos;
     }
@@ -860,7 +883,7 @@ __global__ void __launch_bounds__(kSplitThreads) split_tokens_kernel(
   }
   const int64_t row_bytes = H / 2;
   const int kb = static_cast<int>(threadIdx.x) >> 1;   // this thread's 32-value block
-  const int64_t rec_kt = static_cast<int64_t>(kb >> 2) * kSfRecord;
+  const int64_t rec_st = static_cast<int64_t>(kb >> 3) * kSfRecord;   // this block's stage record
   const bool writes_scale = act && (lane & 1) == 0;
   __syncthreads();   // s_pos, s_rec, s_jr
 #pragma unroll 1
@@ -888,7 +911,7 @@ __global__ void __launch_bounds__(kSplitThreads) split_tokens_kernel(
         *reinterpret_cast<uint2*>(xs + (static_cast<int64_t>(pos) * kParts + pp) * row_bytes + i0 / 2) =
             make_uint2(packed[0], packed[1]);
         if (writes_scale)
-          sfb[s_rec[j] + rec_kt + sf_atom_byte(kParts * s_jr[j] + pp, kb & 3)] = static_cast<uint8_t>(sc + 127);
+          sfb_store(sfb + s_rec[j] + rec_st, kParts * s_jr[j] + pp, (kb >> 2) & 1, kb & 3, static_cast<uint8_t>(sc + 127));
       }
   }
 }
@@ -938,7 +961,7 @@ cudaError_t decode_tc_prepare() {
 size_t decode_tc_xs_bytes(int64_t P, int K) { return static_cast<size_t>(P) * dec::kParts * (K / 2); }
 
 size_t decode_tc_sfb_bytes(int E, int K, int T) {
-  return static_cast<size_t>(E) * max_chunks_for(T) * 2 * nst_for(K) * dec::kSfRecord;
+  return static_cast<size_t>(E) * max_chunks_for(T) * nst_for(K) * dec::kSfRecord;
 }
 
 size_t decode_tc_part_bytes(int64_t P, int H, int I) {

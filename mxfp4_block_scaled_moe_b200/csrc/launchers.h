@@ -166,7 +166,7 @@ bool decode_tc_supported(int H, int I, int T, const void* gu_blocks, const void*
                          const void* d_scales);
 cudaError_t decode_tc_prepare();
 size_t decode_tc_xs_bytes(int64_t P, int K);
-size_t decode_tc_sfb_bytes(int E, int K, int T);       // B scale records, one per 128-wide k-tile
+size_t decode_tc_sfb_bytes(int E, int K, int T);       // B scale records, one per 256-deep stage
 size_t decode_tc_part_bytes(int64_t P, int H, int I);
 size_t decode_tc_ticket_count(int H, int I);
 // offsets of the three ticket arrays inside the decode_tc_ticket_count block
