@@ -493,32 +493,23 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
     d.max_active = static_cast<int>(std::min<int64_t>(a.E, P));
     d.sms = ws->sms;
     d.offsets = b.offsets; d.active = b.active; d.n_active = b.n_active;
-    d.topk_idx = b.topk_idx; d.topk_w = b.topk_w; d.inv = b.inv;
     d.xs = b.xs; d.sfb = b.sfb; d.xs_mid = b.xs_mid; d.sfb_mid = b.sfb_mid;
     d.s0 = s0; d.s1_quant = fp8 ? s1 : 0.0f; d.s1_in = s1;
     d.y = b.y;
-    const bool fold = a.T <= kDecodeFoldMaxT;
-    d.out = fold ? out : nullptr;
     d.part = b.part;
     d.split_tickets_gu = b.dtickets;
     d.split_tickets_d = b.dtickets + decode_tc_tickets_d(a.I);
-    d.comb_tickets = b.dtickets + decode_tc_tickets_comb(a.H, a.I);
     d.err = ws->err;
     if ((e = launch_decode_gemm(true, d, st))) return cuda_fail(e, "gate_up (tensor-core decode)");
     ++launches;
     tm.mark("gate_up");
     if ((e = launch_decode_gemm(false, d, st))) return cuda_fail(e, "down (tensor-core decode)");
     ++launches;
-    if (!fold) {
-      tm.mark("down");
-      if ((e = launch_combine(b.y, b.topk_idx, b.topk_w, b.inv, a.T, a.H, a.k, out, st, ws->sms)))
-        return cuda_fail(e, "combine");
-      ++launches;
-      tm.mark("combine");
-      t_last_launches = launches;
-      return MXMOE_OK;
-    }
-    tm.mark("down+combine");
+    tm.mark("down");
+    if ((e = launch_combine(b.y, b.topk_idx, b.topk_w, b.inv, a.T, a.H, a.k, out, st, ws->sms)))
+      return cuda_fail(e, "combine");
+    ++launches;
+    tm.mark("combine");
     t_last_launches = launches;
     return MXMOE_OK;
   }

@@ -37,8 +37,8 @@
 // The gate_up epilogue applies bias + SwiGLU and writes a directly as the down GEMM's B
 // operand (its 32-row warp is exactly one 32-value block of the down contraction, so a
 // part's block amax stays inside the warp: after a four-row transpose through shared
-// memory it is three xor-shuffles); the down epilogue writes y and, for a few tokens, the
-// weighted combine of each 32-row slice, by the last of the slice's row groups to finish.
+// memory it is three xor-shuffles); the down epilogue writes y (fp32), which the combine
+// kernel reduces per token.
 //
 // Scale-factor records of the B operand ("SFB"), one of 5 KB per (row group, 256-deep
 // stage). Tensor memory holds a 128-wide k-tile's scales of B rows 0..127 in four columns
@@ -127,18 +127,12 @@ struct Params {
   uint8_t* sfb_out;          // [E][max_chunks][2*nst_out][1024]
   int nst_out;
   float s_out;               // FP8: static scale of a; 0: bf16 intermediate
-  // down outputs
+  // down output
   float* y_out;              // (P, H) fp32
-  uint16_t* out;             // (T, H) bf16, combine (nullable: no fold)
-  const int32_t* topk_idx;
-  const float* topk_w;
-  const int32_t* inv;
-  int T, k;
   // split-K
   float* part;               // [split][planes][P * 4][n_out] fp32 partial accumulators
                              // (gate_up: planes gate and up; down: one, rows as they are)
   unsigned* split_tickets;   // [kMaxGrp][n_m][4], zero between calls
-  unsigned* comb_tickets;    // [n_m][4], zero between calls
   int* err;
 };
 
@@ -305,37 +299,6 @@ __device__ __forceinline__ void finish_down(const Params& p, const Unit& w, int 
   for (int jj = 0; jj < 8; ++jj)
     if (j0 + jj < w.n)
       p.y_out[static_cast<int64_t>(w.off + j0 + jj) * p.n_out + row] = __fadd_rn(__fmul_rn(p.s_in, ys[jj]), bd);
-}
-
-// Weighted combine of one 32-row slice of the output (lane = row) for every token: the
-// token's k expert outputs in ascending expert id, which is ascending position in the
-// expert-grouped order.
-__device__ __forceinline__ void combine_slice(const Params& p, int row) {
-  for (int t = 0; t < p.T; ++t) {
-    int pos[kMaxTopK];
-    float wt[kMaxTopK];
-#pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j) {
-      const bool v = j < p.k;
-      pos[j] = v ? p.inv[static_cast<int64_t>(t) * p.k + j] : INT_MAX;
-      wt[j] = v ? p.topk_w[static_cast<int64_t>(t) * p.k + j] : 0.0f;
-    }
-#pragma unroll
-    for (int r = 0; r < kMaxTopK; ++r) {
-#pragma unroll
-      for (int j = (r & 1); j + 1 < kMaxTopK; j += 2) {
-        if (pos[j] > pos[j + 1]) {
-          const int tp = pos[j]; pos[j] = pos[j + 1]; pos[j + 1] = tp;
-          const float tw = wt[j]; wt[j] = wt[j + 1]; wt[j + 1] = tw;
-        }
-      }
-    }
-    float acc = 0.0f;
-#pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j)
-      if (j < p.k) acc = __fadd_rn(acc, __fmul_rn(wt[j], __ldcg(p.y_out + static_cast<int64_t>(pos[j]) * p.n_out + row)));
-    p.out[static_cast<int64_t>(t) * p.n_out + row] = f32_to_bf16_bits_rn(acc);
-  }
 }
 
 // ---------------------------------------------------------------------- the kernel --
@@ -786,21 +749,6 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
         if (slot) ++use1; else ++use0;
         nxt ^= 1;
       }
-      if (!kGateUp && finished && p.out != nullptr) {
-        // the last row group to finish this 32-row slice combines it for every token
-        __threadfence();
-        __syncwarp();
-        unsigned* tk = p.comb_tickets + w.m * 4 + q;
-        unsigned t = 0;
-        if (lane == 0) t = atomicAdd(tk, 1u);
-        t = __shfl_sync(0xffffffffu, t, 0);
-        if (t == static_cast<unsigned>(sc.n_grp - 1)) {
-          __threadfence();
-          if (live0) combine_slice(p, row0);
-          if (live1) combine_slice(p, row1);
-          if (lane == 0) *tk = 0u;
-        }
-      }
     }
   }
 
@@ -971,8 +919,10 @@ size_t decode_tc_part_bytes(int64_t P, int H, int I) {
 }
 
 size_t decode_tc_ticket_count(int H, int I) {
+  // split-K tickets per (row group, unit rows, epilogue warp): gate_up units of 128 rows of
+  // I, down units of 256 rows of H (sized here for 128, a bound)
   const size_t m_gu = (I + dec::BM - 1) / dec::BM, m_d = (H + dec::BM - 1) / dec::BM;
-  return static_cast<size_t>(dec::kMaxGrp) * (m_gu + m_d) * 4 + m_d * 4;
+  return static_cast<size_t>(dec::kMaxGrp) * (m_gu + m_d) * 4;
 }
 
 cudaError_t launch_split_tokens(bool fp8, const uint16_t* x, const int32_t* topk_idx, const int32_t* inv,
@@ -994,8 +944,7 @@ cudaError_t launch_split_tokens(bool fp8, const uint16_t* x, const int32_t* topk
 }
 
 // gate_up (gate_up = true): A = gu weights, B = xs (4 parts per routed row), writes xs_mid
-// / sfb_mid for the down GEMM. down: A = d weights, B = xs_mid, writes y and (a.out) the
-// combine of a few tokens.
+// / sfb_mid for the down GEMM. down: A = d weights, B = xs_mid, writes y.
 cudaError_t launch_decode_gemm(bool gate_up, const DecodeGemmArgs& a, cudaStream_t st) {
   using namespace dec;
   const int K = gate_up ? a.H : a.I;
@@ -1005,7 +954,7 @@ cudaError_t launch_decode_gemm(bool gate_up, const DecodeGemmArgs& a, cudaStream
   const int unit_rows = gate_up ? BM : 2 * BM;   // output rows per unit (down: two 128-row tiles)
   const int n_m = (n_out + unit_rows - 1) / unit_rows;
   const int box_rows = box_rows_for(a.T);
-  if (a.E > kMaxE || a.k > kMaxTopK || a.T > kDecodeMaxT || (!gate_up && a.out && a.T > kDecodeFoldMaxT))
+  if (a.E > kMaxE || a.k > kMaxTopK || a.T > kDecodeMaxT)
     return cudaErrorInvalidValue;
   CUtensorMap mw, mx;
   {
@@ -1049,15 +998,8 @@ cudaError_t launch_decode_gemm(bool gate_up, const DecodeGemmArgs& a, cudaStream
   prm.nst_out = nst_for(a.I);
   prm.s_out = a.s1_quant;
   prm.y_out = a.y;
-  prm.out = gate_up ? nullptr : a.out;
-  prm.topk_idx = a.topk_idx;
-  prm.topk_w = a.topk_w;
-  prm.inv = a.inv;
-  prm.T = a.T;
-  prm.k = a.k;
   prm.part = a.part;
   prm.split_tickets = gate_up ? a.split_tickets_gu : a.split_tickets_d;
-  prm.comb_tickets = a.comb_tickets;
   prm.err = a.err;
   const int64_t max_grp = std::min<int64_t>(kMaxGrp, static_cast<int64_t>(a.max_active) + a.P / kGroupRows + 1);
   const int64_t max_units = max_grp * n_m * prm.split_cap;

@@ -101,9 +101,6 @@ struct DecodeGemmArgs {   // tensor-core decode path (kind::mxf4: packed e2m1 we
   const int32_t* offsets;
   const int32_t* active;
   const int32_t* n_active;
-  const int32_t* topk_idx;
-  const float* topk_w;
-  const int32_t* inv;
   const uint8_t* xs;            // gate_up B operand: (P*4, H/2) packed e2m1 parts
   const uint8_t* sfb;           // its scale records (decode_tc_sfb_bytes(E, H, T))
   uint8_t* xs_mid;              // down B operand: (P*4, I/2)
@@ -112,16 +109,13 @@ struct DecodeGemmArgs {   // tensor-core decode path (kind::mxf4: packed e2m1 we
   float s1_quant;               // FP8: scale of a's e4m3 cast; 0: bf16 intermediate
   float s1_in;                  // B scale of down (FP8 s1, else 1)
   float* y;                     // (P, H) fp32
-  uint16_t* out;                // (T, H) bf16: combine folded into the down kernel (nullable)
   float* part;                  // split-K partials (decode_tc_part_bytes)
-  unsigned* split_tickets_gu;   // zero between calls (decode_tc_ticket_count covers all three)
+  unsigned* split_tickets_gu;   // zero between calls (decode_tc_ticket_count covers both)
   unsigned* split_tickets_d;
-  unsigned* comb_tickets;
   int* err;
 };
 constexpr int kDecodeMaxT = 64;      // tokens the tensor-core decode path takes
 constexpr int kDecodeMaxGroups = 320;  // row groups (an expert's routed rows, 56 at a time)
-constexpr int kDecodeFoldMaxT = 8;   // the down kernel folds the combine up to this many tokens
 // One-launch decode layer (csrc/decode_layer_sm100.cu): routing, token operand, gate_up,
 // down and combine of at most kDecodeLayerMaxT tokens in one persistent grid of one CTA
 // per SM.
@@ -171,9 +165,6 @@ size_t decode_tc_part_bytes(int64_t P, int H, int I);
 size_t decode_tc_ticket_count(int H, int I);
 // offsets of the three ticket arrays inside the decode_tc_ticket_count block
 inline size_t decode_tc_tickets_d(int I) { return static_cast<size_t>(kDecodeMaxGroups) * ((I + 127) / 128) * 4; }
-inline size_t decode_tc_tickets_comb(int H, int I) {
-  return decode_tc_tickets_d(I) + static_cast<size_t>(kDecodeMaxGroups) * ((H + 127) / 128) * 4;
-}
 cudaError_t launch_split_tokens(bool fp8, const uint16_t* x, const int32_t* topk_idx, const int32_t* inv,
                                 const int32_t* offsets, int T, int E, int H, int k, float s0, uint8_t* xs, uint8_t* sfb,
                                 cudaStream_t st);
