@@ -500,14 +500,47 @@ def measure_layer(B, name, lay, d, act, args, world, flusher, pk, pk_kind, tpk, 
     return res
 
 
+def _cpulist(text):
+    cpus = set()
+    for part in text.strip().split(","):
+        if part:
+            lo, _, hi = part.partition("-")
+            cpus.update(range(int(lo), int(hi or lo) + 1))
+    return cpus
+
+
+def gpu_numa_cpus(dev):
+    """(node, CPUs) of the NUMA node the GPU's PCI device sits on, the CPUs limited to those
+    this process may run on; (None, None) when the topology is not visible."""
+    try:
+        p = torch.cuda.get_device_properties(dev)
+        bdf = f"{p.pci_domain_id:04x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+        node = int(open(f"/sys/bus/pci/devices/{bdf}/numa_node").read())
+        if node < 0:
+            return None, None
+        cpus = _cpulist(open(f"/sys/devices/system/node/node{node}/cpulist").read()) & os.sched_getaffinity(0)
+        return (node, cpus) if cpus else (None, None)
+    except (OSError, ValueError, AttributeError):
+        return None, None
+
+
 def e2e_leg(B, d, k, act, out, args, world):
     """End to end through the C ABI with host buffers, double-buffered: the copy of the
     next step's tokens in and of the previous step's output out run on their own streams
     beside the current step's forward; every step's two copies are inside the timed region."""
     T, H = d["x"].shape
     stream = torch.cuda.current_stream()
-    x_host = d["x"].cpu().pin_memory()
-    out_host = [torch.empty(T, H, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    # pinned host buffers on the GPU's own NUMA node (a buffer on the other socket crosses
+    # the inter-socket link on every copy): pages are placed where the allocating thread runs
+    node, cpus = gpu_numa_cpus(torch.cuda.current_device())
+    allowed = os.sched_getaffinity(0)
+    if cpus:
+        os.sched_setaffinity(0, cpus)
+    try:
+        x_host = d["x"].cpu().pin_memory()
+        out_host = [torch.empty(T, H, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    finally:
+        os.sched_setaffinity(0, allowed)
     x_dev = [torch.empty_like(d["x"]) for _ in range(2)]
     out_dev = [torch.empty_like(out) for _ in range(2)]
     d_e2e = [dict(d, x=x_dev[s]) for s in range(2)]
@@ -547,9 +580,11 @@ def e2e_leg(B, d, k, act, out, args, world):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
     return {"value": round(job_tokens_per_s(T, world, args.steps, e2e_ms), 1), "unit": "tokens/s",
             "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2,
+            "host_numa_node": node,
             "timing": "steps back to back, copies double-buffered on their own streams, L2 not "
                       "flushed between steps (the routed experts' weights of a small batch can "
-                      "stay in L2)"}
+                      "stay in L2); pinned host buffers allocated on the GPU's NUMA node when "
+                      "the topology is visible"}
 
 
 def run_ours(args, world, rank):
@@ -886,11 +921,18 @@ def run_codec(args, world, rank):
     # the three legs run, and the packed, bf16 and fp32 results come back
     chunk = 2 * K
     rows_e2e = min(R, args.codec_e2e_chunks * chunk)
-    w_host = w[:rows_e2e].cpu().pin_memory()
-    blk_h = torch.empty(rows_e2e, K // 2, dtype=torch.uint8).pin_memory()
-    sc_h = torch.empty(rows_e2e, K // 32, dtype=torch.uint8).pin_memory()
-    o16_h = torch.empty(rows_e2e, K, dtype=torch.bfloat16).pin_memory()
-    o32_h = torch.empty(rows_e2e, K, dtype=torch.float32).pin_memory()
+    node, cpus = gpu_numa_cpus(torch.cuda.current_device())   # pinned buffers near the GPU
+    allowed = os.sched_getaffinity(0)
+    if cpus:
+        os.sched_setaffinity(0, cpus)
+    try:
+        w_host = w[:rows_e2e].cpu().pin_memory()
+        blk_h = torch.empty(rows_e2e, K // 2, dtype=torch.uint8).pin_memory()
+        sc_h = torch.empty(rows_e2e, K // 32, dtype=torch.uint8).pin_memory()
+        o16_h = torch.empty(rows_e2e, K, dtype=torch.bfloat16).pin_memory()
+        o32_h = torch.empty(rows_e2e, K, dtype=torch.float32).pin_memory()
+    finally:
+        os.sched_setaffinity(0, allowed)
     w_dev = torch.empty(chunk, K, dtype=torch.float32, device="cuda")
 
     def e2e_step():
