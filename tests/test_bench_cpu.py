@@ -79,3 +79,14 @@ def test_step_roofline_against_both_bounds():
     b = bench.step_roofline(1_744_404_480, 818_392_596_480, 1.52, pk, fp8=False)
     assert b["measured"]["tensor_tflops"] == 1628.9 and b["nominal"]["tensor_tflops"] == 2250.0
     assert b["nominal"]["bound"] == "tensor"
+
+
+def test_cpulist_and_numa_fallback(monkeypatch):
+    assert bench._cpulist("0-3,8-11,16\n") == {0, 1, 2, 3, 8, 9, 10, 11, 16}
+    assert bench._cpulist("5") == {5}
+
+    class Props:   # a device whose PCI node file does not exist: no placement, no error
+        pci_domain_id, pci_bus_id, pci_device_id = 0xFFFF, 0xFF, 0x1F
+
+    monkeypatch.setattr(bench.torch.cuda, "get_device_properties", lambda dev: Props())
+    assert bench.gpu_numa_cpus(0) == (None, None)
