@@ -159,22 +159,30 @@ def job_tokens_per_s(tokens_per_rank_step: int, world: int, steps: int, max_ms: 
 def tensor_peak(B, seconds=1.0):
     """The FP8 block-scaled MMA rate of this GPU, measured with the library's rate probe
     (kind::mxf8f6f4, E4M3 x E2M1, M = 128, K = 32, one CTA per SM, operands resident in
-    shared memory): `burst` = one ~10 ms launch on a GPU that has idled for a moment,
-    `sustained` = the last second of back-to-back launches (the power cap's clock), both
-    for N = 256, plus the prefill GEMM's own pattern (N = 240 with one scale-factor copy
-    per four MMAs) at the sustained clock. TFLOP/s."""
+    shared memory, pseudo-random operand bytes like a GEMM's data): `burst` = one ~10 ms
+    launch on a GPU that has idled for a moment, `sustained` = the last second of
+    back-to-back launches (the power cap's clock), both for N = 256, plus the prefill GEMM's
+    own pattern (N = 240 with one scale-factor copy per four MMAs) at the sustained clock.
+    Zero operands (which switch fewer bits and run faster under the power cap) are timed
+    too, for reference. TFLOP/s."""
     stream = torch.cuda.current_stream()
     B.mxmoe_tc_rate_probe(256, False, 100)            # load the kernel
     torch.cuda.synchronize()
     time.sleep(0.5)
 
-    def timed(n, copy, iters):
+    def timed(n, copy, iters, rnd=True):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        f = B.mxmoe_tc_rate_probe(n, copy, iters)
+        f = B.mxmoe_tc_rate_probe(n, copy, iters, random_operands=rnd)
         e1.record(stream)
         return f, e0, e1
 
+    def rate(r):
+        return r[0] / (r[1].elapsed_time(r[2]) / 1e3) / 1e12
+
+    zero = timed(256, False, 20000, rnd=False)      # from idle, as the burst below
+    torch.cuda.synchronize()
+    time.sleep(0.5)
     f, e0, e1 = timed(256, False, 20000)
     torch.cuda.synchronize()
     burst = f / (e0.elapsed_time(e1) / 1e3) / 1e12
@@ -185,15 +193,16 @@ def tensor_peak(B, seconds=1.0):
         torch.cuda.synchronize()
     last = runs[-5:]
     sustained = sum(r[0] for r in last) / (sum(r[1].elapsed_time(r[2]) for r in last) / 1e3) / 1e12
-    f, e0, e1 = timed(240, True, 20000)
+    pat = timed(240, True, 20000)
     torch.cuda.synchronize()
-    pattern = f / (e0.elapsed_time(e1) / 1e3) / 1e12
     B.mxmoe_check()
     return {"peak_tflops": round(max(burst, sustained), 1),
             "burst_tflops": round(burst, 1), "sustained_tflops": round(sustained, 1),
-            "n240_with_scale_copy_tflops": round(pattern, 1),
+            "n240_with_scale_copy_tflops": round(rate(pat), 1),
+            "zero_operands_burst_tflops": round(rate(zero), 1),
             "probe": "tcgen05.mma kind::mxf8f6f4 block_scale, E4M3 x E2M1, M=128 N=256 K=32, "
-                     "one CTA per SM, operands in shared memory"}
+                     "one CTA per SM, operands in shared memory: pseudo-random bytes (E4M3 "
+                     "without NaN), unit scales"}
 
 
 def layer_weights(lay, device, cache):
@@ -384,7 +393,7 @@ def kernel_roofline(name, lay, work, stages, act, pk, pk_kind, tpk):
         achieved = flops / (dom_ms / 1e3) / 1e12
         if fp8 and tpk:
             peak = tpk["peak_tflops"]
-            peak_note = "measured kind::mxf8f6f4 rate probe (this run, this GPU): the larger of burst and sustained"
+            peak_note = "measured kind::mxf8f6f4 rate probe on random operands (this run, this GPU): the larger of burst and sustained"
             extra = {"frac_of_nominal_fp8": round(achieved / NOMINAL_PEAKS["fp8_tflops"], 4)}
         elif fp8:
             peak = pk["bf16_tflops"] * 2.0
@@ -708,7 +717,7 @@ def run_attn_fp8(args, world, rank):
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "tensor", "kernel": f"fp8_linear {dom}", "achieved": round(achieved, 2),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
-                     "peak_source": "measured kind::mxf8f6f4 rate probe (this run, this GPU)" if tpk
+                     "peak_source": "measured kind::mxf8f6f4 rate probe on random operands (this run, this GPU)" if tpk
                      else f"{pk_kind} bf16 burst x 2", "kernel_ms": round(per[dom], 5),
                      "frac_of_nominal_fp8": round(achieved / NOMINAL_PEAKS["fp8_tflops"], 4)},
         "stages_ms_per_step": {k: round(v, 5) for k, v in per.items()},

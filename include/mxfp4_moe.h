@@ -303,12 +303,16 @@ int mxmoe_release(void);
  * Launches `ctas` CTAs (one per SM for ctas <= the SM count) on `stream`; in each, one
  * thread issues `iters` x 4 MMAs back to back from operands resident in shared memory
  * (with_scale_copy != 0: one tcgen05.cp.128x256b of B scales before every 4, as the
- * prefill GEMM's per-stage scale copy). The caller times the launch (CUDA events on
- * `stream`). flops (host, nullable) receives the FLOPs the launch performs,
- * 2 * 128 * n * 32 * 4 * iters * ctas. n: multiple of 16 in [16, 256]; iters in
- * [1, 1000000]; ctas in [1, 4096]. Returns MXMOE_OK, MXMOE_EINVAL or MXMOE_ECUDA; a
- * bounded wait that expires sets MXMOE_ETIMEOUT for mxmoe_check. */
-int mxmoe_tc_rate_probe(int n, int with_scale_copy, int iters, int ctas, double* flops, void* stream);
+ * prefill GEMM's per-stage scale copy). random_operands: 1 fills the operands with
+ * pseudo-random bytes (E4M3 without NaN encodings against E2M1 containers, unit scales),
+ * the rate on data like a GEMM's; 0 with zeros, which draw less power and run faster
+ * under the power cap. The caller times the launch (CUDA events on `stream`). flops
+ * (host, nullable) receives the FLOPs the launch performs, 2 * 128 * n * 32 * 4 * iters
+ * * ctas. n: multiple of 16 in [16, 256]; random_operands 0 or 1; iters in [1, 1000000];
+ * ctas in [1, 4096]. Returns MXMOE_OK, MXMOE_EINVAL or MXMOE_ECUDA; a bounded wait that
+ * expires sets MXMOE_ETIMEOUT for mxmoe_check. */
+int mxmoe_tc_rate_probe(int n, int with_scale_copy, int random_operands, int iters, int ctas, double* flops,
+                        void* stream);
 
 /* mxmoe_selftest_wait_timeout -- exercise the failure path of the library's bounded
  * device waits. The pages have no counterpart: every mbarrier wait in the tensor-core

@@ -45,7 +45,7 @@ _SIGS = {
     "mxmoe_last_launch_count": [],
     "mxmoe_release": [],
     "mxmoe_selftest_wait_timeout": [_vp],
-    "mxmoe_tc_rate_probe": [_i32, _i32, _i32, _i32, _vp, _vp],
+    "mxmoe_tc_rate_probe": [_i32, _i32, _i32, _i32, _i32, _vp, _vp],
     "mxmoe_profile_enable": [_i32],
     "mxmoe_profile_read": [_vp, _vp, _vp, _i32],
 }
@@ -366,15 +366,16 @@ def mxmoe_release():
     _call("mxmoe_release")
 
 
-def mxmoe_tc_rate_probe(n=256, with_scale_copy=False, iters=20000, ctas=None, stream=None) -> float:
+def mxmoe_tc_rate_probe(n=256, with_scale_copy=False, iters=20000, ctas=None, stream=None,
+                        random_operands=True) -> float:
     """Launch the tensor-pipe rate probe (kind::mxf8f6f4 MMAs, M = 128, N = n) on `ctas`
-    CTAs (default: one per SM); returns the FLOPs the launch performs. Time it with CUDA
-    events on `stream`."""
+    CTAs (default: one per SM), on pseudo-random operands (or zeros); returns the FLOPs the
+    launch performs. Time it with CUDA events on `stream`."""
     if ctas is None:
         ctas = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
     f = ctypes.c_double(0.0)
-    _call("mxmoe_tc_rate_probe", int(n), 1 if with_scale_copy else 0, int(iters), int(ctas),
-          ctypes.byref(f), _stream(stream))
+    _call("mxmoe_tc_rate_probe", int(n), 1 if with_scale_copy else 0, 1 if random_operands else 0, int(iters),
+          int(ctas), ctypes.byref(f), _stream(stream))
     return f.value
 
 

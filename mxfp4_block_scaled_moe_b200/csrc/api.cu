@@ -1154,15 +1154,18 @@ int mxmoe_selftest_wait_timeout(void* stream) {
   return e ? cuda_fail(e, "wait self-test launch") : MXMOE_OK;
 }
 
-int mxmoe_tc_rate_probe(int n, int with_scale_copy, int iters, int ctas, double* flops, void* stream) {
+int mxmoe_tc_rate_probe(int n, int with_scale_copy, int random_operands, int iters, int ctas, double* flops,
+                        void* stream) {
   t_last_error.clear();
   t_last_launches = 0;
   if (n < 16 || n > 256 || n % 16) return fail(MXMOE_EINVAL, "n = %d must be a multiple of 16 in [16, 256]", n);
+  if (random_operands != 0 && random_operands != 1)
+    return fail(MXMOE_EINVAL, "random_operands = %d must be 0 or 1", random_operands);
   if (iters < 1 || iters > 1000000) return fail(MXMOE_EINVAL, "iters = %d outside [1, 1000000]", iters);
   if (ctas < 1 || ctas > 4096) return fail(MXMOE_EINVAL, "ctas = %d outside [1, 4096]", ctas);
   Workspace* ws = nullptr;
   if (int rc = current_device_ws(&ws)) return rc;
-  cudaError_t e = mxmoe::launch_tc_rate(n, with_scale_copy ? 1 : 0, iters, ctas, ws->err,
+  cudaError_t e = mxmoe::launch_tc_rate(n, with_scale_copy ? 1 : 0, random_operands, iters, ctas, ws->err,
                                         static_cast<cudaStream_t>(stream));
   if (e) return cuda_fail(e, "rate probe launch");
   t_last_launches = 1;

@@ -196,7 +196,7 @@ cudaError_t launch_fp8_linear(const uint8_t* xq, int T, int K, const uint8_t* wq
                               uint16_t* out, float* part, int ksplit, int* err, int sms, cudaStream_t st);
 
 // mxmoe_tc_rate_probe: back-to-back kind::mxf8f6f4 MMAs (M = 128, N = n) on `ctas` CTAs
-cudaError_t launch_tc_rate(int n, int with_copy, int iters, int ctas, int* err, cudaStream_t st);
+cudaError_t launch_tc_rate(int n, int with_copy, int random, int iters, int ctas, int* err, cudaStream_t st);
 
 // mxmoe_selftest_wait_timeout: a bounded wait that expires (ETIMEOUT in *err)
 cudaError_t launch_wait_selftest(int* err, cudaStream_t st);

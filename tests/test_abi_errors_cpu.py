@@ -102,7 +102,8 @@ def test_layer_argument_checks(L):
 
 def test_rate_probe_argument_checks(L):
     f = ctypes.c_double(0.0)
-    assert L.mxmoe_tc_rate_probe(8, 0, 10, 1, ctypes.byref(f), None) == EINVAL and "multiple of 16" in err(L)
-    assert L.mxmoe_tc_rate_probe(264, 0, 10, 1, ctypes.byref(f), None) == EINVAL
-    assert L.mxmoe_tc_rate_probe(256, 0, 0, 1, ctypes.byref(f), None) == EINVAL and "iters" in err(L)
-    assert L.mxmoe_tc_rate_probe(256, 0, 10, 0, ctypes.byref(f), None) == EINVAL and "ctas" in err(L)
+    assert L.mxmoe_tc_rate_probe(8, 0, 1, 10, 1, ctypes.byref(f), None) == EINVAL and "multiple of 16" in err(L)
+    assert L.mxmoe_tc_rate_probe(264, 0, 1, 10, 1, ctypes.byref(f), None) == EINVAL
+    assert L.mxmoe_tc_rate_probe(256, 0, 2, 10, 1, ctypes.byref(f), None) == EINVAL and "random_operands" in err(L)
+    assert L.mxmoe_tc_rate_probe(256, 0, 1, 0, 1, ctypes.byref(f), None) == EINVAL and "iters" in err(L)
+    assert L.mxmoe_tc_rate_probe(256, 0, 1, 10, 0, ctypes.byref(f), None) == EINVAL and "ctas" in err(L)

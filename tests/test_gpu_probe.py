@@ -8,10 +8,10 @@ import torch
 pytestmark = pytest.mark.gpu
 
 
-def _rate(B, n, copy, iters=4000):
+def _rate(B, n, copy, iters=4000, random_operands=True):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    f = B.mxmoe_tc_rate_probe(n, copy, iters)
+    f = B.mxmoe_tc_rate_probe(n, copy, iters, random_operands=random_operands)
     e1.record()
     torch.cuda.synchronize()
     B.mxmoe_check()
@@ -32,3 +32,6 @@ def test_rate_probe_runs_and_reports_its_flops():
     # the scale copy only takes pipe time (and N = 240 does 15/16 of the work per MMA); the
     # margin is the SM clock's drift between timed runs under the power cap
     assert 0.0 < tf_copy < tf * 1.15
+    # zero operands: the same FLOPs, a rate in the same physical range
+    fz, tz = max((_rate(B, 256, False, random_operands=False) for _ in range(3)), key=lambda r: r[1])
+    assert fz == f and 0.2 * 16384 * sms * 1.0e9 / 1e12 < tz < 16384 * sms * 2.1e9 / 1e12 * 1.05
