@@ -330,7 +330,8 @@ int run_layer(const LayerArgs& a, const float* act_scale, uint16_t* out, float* 
                    tc_gemm_supported(a.H, a.I, a.gu_blocks, a.d_blocks, a.gu_scales, a.d_scales);
   // a handful of tokens: the whole layer in one launch
   const bool dlay = !tc && !tcb && !calib_out && a.T <= kDecodeLayerMaxT &&
-                    decode_layer_supported(a.H, a.I, a.T, a.E, a.k, a.gu_blocks, a.d_blocks, a.gu_scales, a.d_scales);
+                    decode_layer_supported(a.H, a.I, a.T, a.E, a.k, ws->sms, a.gu_blocks, a.d_blocks, a.gu_scales,
+                                           a.d_scales);
   const bool dtc = !tc && !tcb && !dlay && !calib_out &&
                    decode_tc_supported(a.H, a.I, a.T, a.gu_blocks, a.d_blocks, a.gu_scales, a.d_scales);
   // routing: one fused launch for small batches; else the router GEMM (on the tensor cores

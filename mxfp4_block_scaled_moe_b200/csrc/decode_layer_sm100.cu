@@ -1046,10 +1046,17 @@ int down_pieces_max(int H, int G) {
 
 }  // namespace
 
-bool decode_layer_supported(int H, int I, int T, int E, int k, const void* gu_blocks, const void* d_blocks,
+bool decode_layer_supported(int H, int I, int T, int E, int k, int sms, const void* gu_blocks, const void* d_blocks,
                             const void* gu_scales, const void* d_scales) {
   if (T < 1 || T > dl::kMaxT || E > dl::kMaxE || k > dl::kMaxK) return false;
   if (H % 64 || I % 64 || H < 64 || I < 64 || H > dl::kMaxHI || I > dl::kMaxHI) return false;
+  if (sms < 1 || sms > dl::kMaxGrid) return false;
+  // a CTA's pieces of one GEMM are at most ceil(tiles / grid) + 2 under every work-list
+  // mode (whole tiles, stream-K, hybrid); keep that within the per-CTA list (on a B200's
+  // 148 SMs the bound is 30 at the largest shapes)
+  const int na_max = std::min(E, T * k);
+  const int tiles = na_max * std::max((I + dl::BM - 1) / dl::BM, (H + 2 * dl::BM - 1) / (2 * dl::BM));
+  if ((tiles + sms - 1) / sms + 2 > dl::kMaxPieces) return false;
   if ((reinterpret_cast<uintptr_t>(gu_blocks) | reinterpret_cast<uintptr_t>(d_blocks)) & 15u) return false;
   // the weight-scale converters read the e8m0 bytes as 16-bit words
   if ((reinterpret_cast<uintptr_t>(gu_scales) | reinterpret_cast<uintptr_t>(d_scales)) & 1u) return false;

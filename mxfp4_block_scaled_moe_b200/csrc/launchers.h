@@ -150,7 +150,7 @@ struct DecodeLayerArgs {
   uint16_t* out;                // (T, H) bf16
   int* err;
 };
-bool decode_layer_supported(int H, int I, int T, int E, int k, const void* gu_blocks, const void* d_blocks,
+bool decode_layer_supported(int H, int I, int T, int E, int k, int sms, const void* gu_blocks, const void* d_blocks,
                             const void* gu_scales, const void* d_scales);
 cudaError_t decode_layer_prepare();
 DecodeLayerSizes decode_layer_sizes(int T, int H, int I, int sms);
