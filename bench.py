@@ -357,6 +357,23 @@ def oracle_tokens_per_s(lay, d, act, budget_s, host_weights=None):
     return n / dt, n, dt, hw
 
 
+def oracle_one_token(lay, d, act):
+    """The oracle on one token of the workload: its layer loop gives each token one thread,
+    so this is the one-thread figure (tokens/s) beside the all-core cpu_baseline."""
+    import oracle
+    hw = {n: d[n].cpu().numpy() for n in ("gu_blocks", "gu_scales", "gu_bias", "d_blocks", "d_scales", "d_bias")}
+    xb = inputs.bits(d["x"])
+    rw = inputs.bits(d["router_w"])
+    rb = None if d["router_b"] is None else inputs.bits(d["router_b"])
+    w = (hw["gu_blocks"], hw["gu_scales"], hw["gu_bias"], hw["d_blocks"], hw["d_scales"], hw["d_bias"])
+    oracle.moe_forward(xb[:1], rw, rb, *w, lay.k, act_scale=act)   # page the weights in
+    t0 = time.perf_counter()
+    oracle.moe_forward(xb[:1], rw, rb, *w, lay.k, act_scale=act)
+    dt = time.perf_counter() - t0
+    return {"value": round(1.0 / dt, 4), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"token 0 of the {lay.name} workload, {dt * 1e3:.0f} ms"}
+
+
 # ------------------------------------------------------------------------ main ----
 
 class L2Flush:
@@ -631,6 +648,8 @@ def run_ours(args, world, rank):
             lay2, d2, act2 = build_layer(name, "cuda", cache)
             r = measure_layer(B, name, lay2, d2, act2, args, world, flusher, pk, pk_kind, tpk, False)
             r["metric"], r["unit"] = METRIC, "tokens/s"
+            if name == "decode1" and rank == 0 and world == 1 and not args.no_cpu_baseline:
+                r["cpu_baseline_1thread"] = oracle_one_token(lay2, d2, act2)
             res["other_configs"][name] = r
             del lay2, d2
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

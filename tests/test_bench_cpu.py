@@ -90,3 +90,12 @@ def test_cpulist_and_numa_fallback(monkeypatch):
 
     monkeypatch.setattr(bench.torch.cuda, "get_device_properties", lambda dev: Props())
     assert bench.gpu_numa_cpus(0) == (None, None)
+
+
+def test_one_token_oracle_figure_on_cpu_tensors():
+    from helpers import pack, to_device
+    from mxfp4_block_scaled_moe_b200 import inputs
+    lay = inputs.small_layer(E=8, k=2, T=2, H=128, I=128, seed=1)
+    d = to_device(pack(lay), device="cpu")
+    r = bench.oracle_one_token(lay, d, None)
+    assert r["cores"] == 1 and r["kind"] == "oracle" and r["value"] > 0 and lay.name in r["sample"]
