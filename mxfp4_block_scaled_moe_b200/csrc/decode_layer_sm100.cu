@@ -15,16 +15,21 @@
 //      grid meets at one counter;
 //   2. every CTA reads all logits and runs the same top-k, so every CTA knows the routed
 //      experts without another exchange;
-//   3. gate_up, then down, as stream-K work lists: the (expert, 128-row tile, 256-deep K
-//      stage) units of a GEMM are cut into one contiguous range per CTA, so every SM
-//      streams the same number of weight bytes whatever the expert count. A tile cut
-//      between CTAs is finished by the last of them (a ticket), which adds the fp32
-//      partials in CTA order;
-//   4. a down tile of expert a waits (a per-expert counter) for the 4 * (I / 128) gate_up
-//      warps that write its input; its weights are in flight before that, so the ring
-//      fills across the gate_up -> down boundary;
-//   5. the last expert to finish a 32-row slice of the output combines that slice for
-//      every token, in ascending expert order.
+//   3. gate_up, then down, as work lists of (expert, tile, 256-deep K stage) units (a
+//      gate_up tile: 128 rows of gate and the matching 128 of up; a down tile: two
+//      consecutive 128-row tiles): whole tiles per CTA, stream-K (one contiguous range of
+//      stages per CTA, so
+//      every SM streams the same weight bytes) or a hybrid of the two, chosen on the
+//      device from the tile count (down is always stream-K). A gate_up tile cut between
+//      CTAs is finished by the last of them (a ticket), which adds the fp32 partials in
+//      CTA order;
+//   4. down's token operand for one 256-deep stage of expert a waits (a counter per
+//      expert and stage) for the gate_up warps that write those 256 intermediate rows; its
+//      weights are in flight before that, so the ring fills across the boundary;
+//   5. every down piece parks its fp32 partial; after a second meeting of the grid, every
+//      warp of the grid takes (32-row slice, token) items of the output: each token's
+//      experts in ascending id, each expert's pieces in CTA order, scaled, biased and
+//      weighted by the token's softmax gate.
 //
 // Operands of every MMA (tcgen05.mma kind::mxf4 block_scale, M = 128, K = 64):
 //   A = weight rows, the checkpoint's packed e2m1 bytes by TMA, with their e8m0 scales;
