@@ -27,9 +27,10 @@
 // memory per weight byte (no 8-bit containers), which doubles the bytes in flight.
 //
 // Persistent schedule. One CTA per SM walks the work units u = blockIdx.x, +gridDim.x, ...
-// of the list (row group, 128-row tile, K split), so the TMA ring stays full across unit
-// boundaries and two TMEM accumulator slots let the epilogue of one unit overlap the MMAs
-// of the next. Few units (one token) are split along K so that every SM streams: each
+// of the list (row group, unit rows, K split; a unit is 128 rows of gate with the matching
+// 128 of up, or 256 rows of down_proj), so the TMA ring stays full across unit boundaries
+// and two TMEM accumulator slots let the epilogue of one unit overlap the MMAs of the
+// next. Few units are split along K so that every SM streams: each
 // split writes its fp32 partial accumulator, and the last split of a 32-row slice (an
 // atomic ticket) adds the partials in split order, so results do not depend on which CTA
 // finishes last.
