@@ -196,7 +196,8 @@ int moe_fp8_quantize(const uint16_t* x, int64_t n, float s, uint8_t* q, void* st
  *    e4m3 parts under per-32-value block scales: exact except for elements about 2^14 or
  *    more below their block's largest, which keep an error under ~2^-21 of it. With
  *    T <= 64 the tensor-core decode path expands each activation into four e2m1 parts,
- *    which moves a 2880-long dot product by about 2e-4 of the largest output.)
+ *    which moves a 2880-long dot product by about 2e-4 of the largest output; at most 8
+ *    tokens run as one kernel launch, routing through the combine.)
  *  - act_scale != NULL: HOST pointer to two floats {s0, s1} (static per-tensor scales
  *    read during the call); xin = e4m3(x / s0), ain = e4m3(a / s1).
  * x: device bf16 (T, H); router_w bf16 (E, H); router_b bf16 (E) or NULL; gu_bias fp32
